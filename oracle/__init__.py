@@ -1,0 +1,239 @@
+"""CPU oracle for scaled FP8 casting -- TEST INFRASTRUCTURE ONLY.
+
+Thin ctypes wrapper over ``libfp8q_oracle.so`` (plain C, ``fp8q_oracle.c``).
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import this package; the CUDA library and its Python
+binding never touch it, and the two share no code.
+
+Functions take and return numpy arrays.  Row-structured operations accept a
+``rows=(r0, r1)`` range so that callers can sample rows or split work across
+threads (ctypes releases the GIL during each C call).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp8q_oracle.c")
+_LIB = os.path.join(_HERE, "libfp8q_oracle.so")
+
+E4M3FN, E5M2 = 0, 1
+F32, F16, BF16 = 0, 1, 2
+GRAN_TENSOR, GRAN_ROW, GRAN_GROUP, GRAN_BLOCK = 0, 1, 2, 3
+
+CFLAGS = ["-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math",
+          "-fno-finite-math-only", "-fPIC", "-shared", "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (SSE binary32, no FMA contraction)."""
+    hdr = os.path.join(_HERE, "fp8q_oracle.h")
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= max(os.path.getmtime(_SRC), os.path.getmtime(hdr))):
+        return _LIB
+    tmp = _LIB + ".tmp.%d" % os.getpid()
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            L = ctypes.CDLL(_LIB)
+            c_void, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            L.orc_fp8_max.restype = ctypes.c_float
+            L.orc_fp8_max.argtypes = [i32]
+            L.orc_fp8_encode.restype = ctypes.c_uint8
+            L.orc_fp8_encode.argtypes = [ctypes.c_float, i32]
+            L.orc_fp8_decode.restype = ctypes.c_float
+            L.orc_fp8_decode.argtypes = [ctypes.c_uint8, i32]
+            for name in ("orc_fp8_encode_n", "orc_fp8_decode_n"):
+                getattr(L, name).restype = None
+                getattr(L, name).argtypes = [c_void, i64, i32, c_void]
+            for name in ("orc_bf16_encode_n", "orc_f16_encode_n"):
+                getattr(L, name).restype = None
+                getattr(L, name).argtypes = [c_void, i64, c_void]
+            L.orc_per_token_group_quant.restype = i32
+            L.orc_per_token_group_quant.argtypes = [c_void, i32, i64, i64, i32, i32, c_void, c_void, i64, i64]
+            L.orc_cast_per_channel.restype = i32
+            L.orc_cast_per_channel.argtypes = [c_void, i32, i64, i64, i32, c_void, c_void, i64, i64]
+            L.orc_cast_per_tensor.restype = i32
+            L.orc_cast_per_tensor.argtypes = [c_void, i32, i64, i32, c_void, c_void, i64, i64]
+            L.orc_block_dequant.restype = i32
+            L.orc_block_dequant.argtypes = [c_void, i32, i64, i64, c_void, i32, i32, c_void, i64, i64]
+            L.orc_cast_from_fp8.restype = i32
+            L.orc_cast_from_fp8.argtypes = [c_void, i32, i64, i64, c_void, i32, i32, i32, c_void, i64, i64]
+            _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+_NP_OF = {F32: np.float32, F16: np.uint16, BF16: np.uint16}
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise ValueError(f"oracle {what}: rejected arguments")
+
+
+def _split(r0: int, r1: int, threads: int):
+    threads = max(1, min(threads, r1 - r0))
+    step = (r1 - r0 + threads - 1) // threads if r1 > r0 else 0
+    return [(a, min(a + step, r1)) for a in range(r0, r1, step)] if step else [(r0, r1)]
+
+
+def _run(fn, r0: int, r1: int, threads: int) -> None:
+    parts = _split(r0, r1, threads)
+    if len(parts) == 1:
+        fn(*parts[0])
+        return
+    errs = []
+
+    def work(a, b):
+        try:
+            fn(a, b)
+        except Exception as e:  # pragma: no cover - surfaced below
+            errs.append(e)
+
+    ts = [threading.Thread(target=work, args=p) for p in parts]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    if errs:
+        raise errs[0]
+
+
+# ---------------------------------------------------------------------------
+# scalar / bulk codecs
+# ---------------------------------------------------------------------------
+def fp8_max(fmt: int) -> float:
+    return float(lib().orc_fp8_max(fmt))
+
+
+def fp8_encode(v: np.ndarray, fmt: int) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_fp8_encode_n(_ptr(v), v.size, fmt, _ptr(out))
+    return out
+
+
+def fp8_decode(c: np.ndarray, fmt: int) -> np.ndarray:
+    c = np.ascontiguousarray(c, dtype=np.uint8)
+    out = np.empty(c.shape, np.float32)
+    lib().orc_fp8_decode_n(_ptr(c), c.size, fmt, _ptr(out))
+    return out
+
+
+def bf16_encode(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, np.uint16)
+    lib().orc_bf16_encode_n(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def f16_encode(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, np.uint16)
+    lib().orc_f16_encode_n(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the method
+# ---------------------------------------------------------------------------
+def per_token_group_quant(x: np.ndarray, xt: int, group: int = 128, fmt: int = E4M3FN,
+                          rows=None, out=None, threads: int = 1):
+    """DeepEP per_token_cast_to_fp8 over x[m, n]; returns (q uint8[m,n], scale_inv f32[m,n/group])."""
+    x = np.ascontiguousarray(x)
+    m, n = x.shape
+    if out is None:
+        q = np.zeros((m, n), np.uint8)
+        s = np.zeros((m, n // group if group > 0 else 0), np.float32)
+    else:
+        q, s = out
+    r0, r1 = rows if rows is not None else (0, m)
+    L = lib()
+    _run(lambda a, b: _check(L.orc_per_token_group_quant(_ptr(x), xt, m, n, group, fmt,
+                                                        _ptr(q), _ptr(s), a, b),
+                             "per_token_group_quant"), r0, r1, threads)
+    return q, s
+
+
+def cast_per_channel(x: np.ndarray, xt: int, fmt: int = E4M3FN, rows=None, out=None, threads: int = 1):
+    """ColossalAI cast_to_fp8(per_channel_scale=True) over x[rows, cols]; returns (q, scale_inv[rows])."""
+    x = np.ascontiguousarray(x)
+    R, C = x.shape
+    if out is None:
+        q = np.zeros((R, C), np.uint8)
+        s = np.zeros((max(R, 1),), np.float32)
+    else:
+        q, s = out
+    r0, r1 = rows if rows is not None else (0, R)
+    L = lib()
+    _run(lambda a, b: _check(L.orc_cast_per_channel(_ptr(x), xt, R, C, fmt, _ptr(q), _ptr(s), a, b),
+                             "cast_per_channel"), r0, r1, threads)
+    return q, s
+
+
+def cast_per_tensor(x: np.ndarray, xt: int, fmt: int = E4M3FN, elems=None, out=None, threads: int = 1):
+    """ColossalAI cast_to_fp8(per_channel_scale=False) over flat x; returns (q, scale_inv[1])."""
+    x = np.ascontiguousarray(x).reshape(-1)
+    n = x.size
+    if out is None:
+        q = np.zeros((n,), np.uint8)
+        s = np.zeros((1,), np.float32)
+    else:
+        q, s = out
+    e0, e1 = elems if elems is not None else (0, n)
+    L = lib()
+    _run(lambda a, b: _check(L.orc_cast_per_tensor(_ptr(x), xt, n, fmt, _ptr(q), _ptr(s), a, b),
+                             "cast_per_tensor"), e0, e1, threads)
+    return q, s
+
+
+def block_dequant(w: np.ndarray, s: np.ndarray, fmt: int = E4M3FN, block: int = 128, yt: int = BF16,
+                  rows=None, out=None, threads: int = 1):
+    """DeepSeek-V3 weight_dequant of w[M, N] with s[ceil(M/B), ceil(N/B)]; returns y[M, N]."""
+    w = np.ascontiguousarray(w, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    M, N = w.shape
+    y = np.zeros((M, N), _NP_OF[yt]) if out is None else out
+    r0, r1 = rows if rows is not None else (0, M)
+    L = lib()
+    _run(lambda a, b: _check(L.orc_block_dequant(_ptr(w), fmt, M, N, _ptr(s), block, yt, _ptr(y), a, b),
+                             "block_dequant"), r0, r1, threads)
+    return y
+
+
+def cast_from_fp8(q: np.ndarray, scale_inv: np.ndarray, gran: int, fmt: int = E4M3FN, gb: int = 0,
+                  yt: int = BF16, rows=None, out=None, threads: int = 1):
+    """ColossalAI cast_from_fp8 (any granularity) of q[rows, cols]; returns y[rows, cols]."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(scale_inv, dtype=np.float32)
+    R, C = q.shape
+    y = np.zeros((R, C), _NP_OF[yt]) if out is None else out
+    r0, r1 = rows if rows is not None else (0, R)
+    L = lib()
+    _run(lambda a, b: _check(L.orc_cast_from_fp8(_ptr(q), fmt, R, C, _ptr(s), gran, gb, yt, _ptr(y), a, b),
+                             "cast_from_fp8"), r0, r1, threads)
+    return y
