@@ -1,0 +1,503 @@
+#!/usr/bin/env python3
+"""Benchmark of the scaled-FP8 cast path on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole hot path over one batch of synthetic inputs
+that are resident in HBM before the timed region starts:
+
+  per-token group quant   bf16 x[4096, 7168], group 128, e4m3fn   (+ its round trip
+                          back to bf16 through cast_from_fp8, group granularity)
+  block dequant           e4m3fn W[7168, 18432], 128 x 128 scales -> bf16
+  per-channel cast        bf16 X[8192, 8192] -> e4m3fn, one scale per row
+  per-tensor cast         fp32 v[64 Mi] -> e5m2; fp16 [1 Mi] zeros -> e4m3fn
+  grouped block dequant   64 x [2048, 7168] + 8 x [7000, 1000] e4m3fn -> bf16
+
+`value` is the step's algorithmic bytes (each input read once per pass the
+method needs, each output written once) divided by the device time of the
+step, in GB/s, summed over ranks.  The step streams ~4.4 GB, far more than
+the 126 MB L2, so no operation finds its inputs in L2 from the previous step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 it runs under torchrun, one rank per GPU, each rank doing the full
+step on its own copy of the inputs (independent problems, weak scaling, no
+data-path collective); the time is the max over ranks.  `--impl reference`
+times the CPU oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "achieved HBM GB/s and % of B200 peak for per-token quant and block dequant"
+UNIT = "GB/s"
+WORKLOAD = ("scaled-fp8 cast pass: per-token quant bf16[4096,7168] g128 e4m3fn + round trip to bf16; "
+            "block dequant e4m3fn[7168,18432] B128 -> bf16; per-channel bf16[8192,8192] -> e4m3fn; "
+            "per-tensor f32[64Mi] -> e5m2 and f16[1Mi] zeros -> e4m3fn; "
+            "grouped block dequant 64x[2048,7168] + 8x[7000,1000] -> bf16")
+E4M3FN, E5M2 = 0, 1
+GRAN_GROUP = 2
+
+
+# ---------------------------------------------------------------------------
+# the workload: inputs, outputs, algorithmic bytes, and the step
+# ---------------------------------------------------------------------------
+class Op:
+    def __init__(self, name, fn, bytes_, launches, kernel):
+        self.name, self.fn, self.bytes, self.launches, self.kernel = name, fn, bytes_, launches, kernel
+
+
+class Workload:
+    """All inputs of one step on `device`, outputs preallocated, plus the op list."""
+
+    def __init__(self, device, fp8q, host_inputs=None):
+        self.device = device
+        self.fp8q = fp8q
+        h = host_inputs if host_inputs is not None else make_host_inputs()
+        self.host = h
+        d = device
+        bf16 = torch.bfloat16
+        to = lambda a, dt=None: _to_dev(a, d, dt)  # noqa: E731
+
+        m, n = workloads.C2_SHAPE
+        self.c2_x = to(h["c2_x"], bf16)
+        self.c2_q = torch.empty((m, n), dtype=torch.uint8, device=d)
+        self.c2_s = torch.empty((m, n // 128), dtype=torch.float32, device=d)
+        self.c2_y = torch.empty((m, n), dtype=bf16, device=d)
+
+        M, N = workloads.C3_SHAPE
+        self.c3_w = to(h["c3_w"])
+        self.c3_s = to(h["c3_s"])
+        self.c3_y = torch.empty((M, N), dtype=bf16, device=d)
+
+        R, C = workloads.C4A_SHAPE
+        self.c4a_x = to(h["c4a_x"], bf16)
+        self.c4a_q = torch.empty((R, C), dtype=torch.uint8, device=d)
+        self.c4a_s = torch.empty((R,), dtype=torch.float32, device=d)
+
+        self.c4b_x = to(h["c4b_v"])
+        self.c4b_q = torch.empty((workloads.C4B_NUMEL,), dtype=torch.uint8, device=d)
+        self.c4b_s = torch.empty((1,), dtype=torch.float32, device=d)
+        self.c4c_x = to(h["c4c_v"], torch.float16)
+        self.c4c_q = torch.empty((workloads.C4C_NUMEL,), dtype=torch.uint8, device=d)
+        self.c4c_s = torch.empty((1,), dtype=torch.float32, device=d)
+        self.ws = torch.empty(fp8q.fp8q_cast_per_tensor_workspace_bytes(), dtype=torch.uint8, device=d)
+
+        self.c5_w = [to(w) for w, _ in h["c5"]]
+        self.c5_s = [to(s) for _, s in h["c5"]]
+        self.c5_y = [torch.empty(w.shape, dtype=bf16, device=d) for w in self.c5_w]
+
+        c2_el = m * n
+        c2_bytes = c2_el * 2 + c2_el + c2_el // 128 * 4
+        c3_el = M * N
+        c3_bytes = c3_el + c3_el * 2 + self.c3_s.numel() * 4
+        c4a_bytes = R * C * 2 + R * C + R * 4
+        c4b_bytes = 2 * workloads.C4B_NUMEL * 4 + workloads.C4B_NUMEL + 4
+        c4c_bytes = 2 * workloads.C4C_NUMEL * 2 + workloads.C4C_NUMEL + 4
+        c5_el = sum(w.numel() for w in self.c5_w)
+        c5_bytes = c5_el * 3 + sum(s.numel() for s in self.c5_s) * 4
+        f = fp8q
+        self.ops = [
+            Op("per_token_group_quant", lambda: f.fp8q_per_token_group_quant(self.c2_x, self.c2_q, self.c2_s, 128, E4M3FN),
+               c2_bytes, 1, "per_token_vec_kernel"),
+            Op("block_dequant", lambda: f.fp8q_block_dequant(self.c3_w, self.c3_s, self.c3_y, 128, E4M3FN),
+               c3_bytes, 1, "dequant_kernel"),
+            # the round trip reads q after the block dequant has streamed ~400 MB
+            # through L2, so it finds no q bytes left in L2
+            Op("cast_from_fp8_group", lambda: f.fp8q_cast_from_fp8(self.c2_q, self.c2_s, self.c2_y, GRAN_GROUP, 128, E4M3FN),
+               c2_bytes, 1, "dequant_kernel"),
+            Op("cast_per_channel", lambda: f.fp8q_cast_per_channel(self.c4a_x, self.c4a_q, self.c4a_s, E4M3FN),
+               c4a_bytes, 1, "per_channel_vec_kernel"),
+            Op("cast_per_tensor_f32_e5m2", lambda: f.fp8q_cast_per_tensor(self.c4b_x, self.c4b_q, self.c4b_s, self.ws, E5M2),
+               c4b_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel"),
+            Op("cast_per_tensor_f16_zero", lambda: f.fp8q_cast_per_tensor(self.c4c_x, self.c4c_q, self.c4c_s, self.ws, E4M3FN),
+               c4c_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel"),
+            Op("block_dequant_grouped", lambda: f.fp8q_block_dequant_grouped(self.c5_w, self.c5_s, self.c5_y, 128, E4M3FN),
+               c5_bytes, 1, "dequant_kernel"),
+        ]
+        self.step_bytes = sum(o.bytes for o in self.ops)
+        self.launches_per_step = sum(o.launches for o in self.ops)
+
+    def step(self, events=None):
+        for i, op in enumerate(self.ops):
+            if events is not None:
+                events[i][0].record()
+            op.fn()
+            if events is not None:
+                events[i][1].record()
+
+    # host<->device traffic of one end-to-end step
+    def inputs(self):
+        return [self.c2_x, self.c3_w, self.c3_s, self.c4a_x, self.c4b_x, self.c4c_x, *self.c5_w, *self.c5_s]
+
+    def outputs(self):
+        return [self.c2_q, self.c2_s, self.c2_y, self.c3_y, self.c4a_q, self.c4a_s, self.c4b_q, self.c4b_s,
+                self.c4c_q, self.c4c_s, *self.c5_y]
+
+
+def _to_dev(a, device, dt=None):
+    a = np.ascontiguousarray(a)
+    t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+    if dt is not None:
+        t = t.view(dt)
+    return t.to(device)
+
+
+def make_host_inputs():
+    c3_w, c3_s = workloads.c3_w_s()
+    return {
+        "c2_x": workloads.c2_x(),
+        "c3_w": c3_w, "c3_s": c3_s,
+        "c4a_x": workloads.c4a_x(),
+        "c4b_v": workloads.c4b_v(),
+        "c4c_v": workloads.c4c_v(),
+        "c5": [workloads.c5_weight(i) for i in range(len(workloads.C5_SHAPES))],
+    }
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons, self.max_mhz, self.ok = [], set(), None, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for k, bit in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(k)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            if not self.samples:
+                try:
+                    self._sample()
+                except Exception:
+                    pass
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# roofline helpers
+# ---------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def source_fingerprint() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dequantisation_fp8q_token_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(op_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernels."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_fingerprint") != source_fingerprint():
+        return None
+    e = d.get("ops", {}).get(op_name)
+    return None if e is None else e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline; never on the product path)
+# ---------------------------------------------------------------------------
+def oracle_sample_pass(orc, h, frac: float, threads: int):
+    """Run every op of the step on the oracle over a `frac` sample of its rows /
+    elements; returns the algorithmic bytes of the sample."""
+    nbytes = 0
+    m, n = workloads.C2_SHAPE
+    r = max(1, int(m * frac))
+    q, s = orc.per_token_group_quant(h["c2_x"][:r], orc.BF16, 128, orc.E4M3FN, threads=threads)
+    nbytes += r * n * 3 + r * (n // 128) * 4
+    orc.cast_from_fp8(q, s, orc.GRAN_GROUP, orc.E4M3FN, 128, orc.BF16, threads=threads)
+    nbytes += r * n * 3 + r * (n // 128) * 4
+    M, N = workloads.C3_SHAPE
+    r = max(1, int(M * frac))
+    orc.block_dequant(h["c3_w"], h["c3_s"], orc.E4M3FN, 128, orc.BF16, rows=(0, r), threads=threads)
+    nbytes += r * N * 3
+    R, C = workloads.C4A_SHAPE
+    r = max(1, int(R * frac))
+    orc.cast_per_channel(h["c4a_x"][:r], orc.BF16, orc.E4M3FN, threads=threads)
+    nbytes += r * C * 3 + r * 4
+    k = max(1, int(workloads.C4B_NUMEL * frac))
+    orc.cast_per_tensor(h["c4b_v"][:k], orc.F32, orc.E5M2, threads=threads)
+    nbytes += k * 9
+    k = max(1, int(workloads.C4C_NUMEL * frac))
+    orc.cast_per_tensor(h["c4c_v"][:k], orc.F16, orc.E4M3FN, threads=threads)
+    nbytes += k * 5
+    for w, sc in h["c5"]:
+        M, N = w.shape
+        r = max(1, int(M * frac))
+        orc.block_dequant(w, sc, orc.E4M3FN, 128, orc.BF16, rows=(0, r), threads=threads)
+        nbytes += r * N * 3
+    return nbytes
+
+
+def cpu_baseline(h, budget_s: float = 15.0):
+    import oracle as orc
+    orc.build()
+    threads = os.cpu_count() or 1
+    frac = 1.0 / 2048
+    t0 = time.perf_counter()
+    b = oracle_sample_pass(orc, h, frac, threads)
+    dt = time.perf_counter() - t0
+    # scale the sample so that the measured pass takes about `budget_s`
+    frac = min(1.0, frac * max(1.0, budget_s / max(dt, 1e-3)))
+    t0 = time.perf_counter()
+    b = oracle_sample_pass(orc, h, frac, threads)
+    dt = time.perf_counter() - t0
+    return {"value": round(b / dt / 1e9, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"the first {frac:.5f} of the rows / elements of every op of the step "
+                      f"({b / 1e6:.1f} MB algorithmic), plain C oracle on {threads} threads",
+            "seconds": round(dt, 2)}
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
+def dist_setup(ngpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    world, rank, local = dist_setup(args.gpus)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import dequantisation_fp8q_token_b200 as fp8q
+    fp8q.lib()
+    h = make_host_inputs()
+    wl = Workload(device, fp8q, h)
+    torch.cuda.synchronize()
+
+    nops = len(wl.ops)
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nops)]
+              for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start.record()
+        for k in range(args.steps):
+            wl.step(events[k])
+        t_end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_local = t_start.elapsed_time(t_end)
+    ms_total = max_over_ranks(ms_local, world, device)
+    ms_step = ms_total / args.steps
+    per_op_ms = [statistics.mean(events[k][i][0].elapsed_time(events[k][i][1]) for k in range(args.steps))
+                 for i in range(nops)]
+
+    # end to end: pinned host inputs -> device, the step, outputs -> pinned host
+    h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wl.inputs()]
+    for a, t in zip(h_in, wl.inputs()):
+        a.copy_(t)
+    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wl.outputs()]
+    e2e_steps = max(1, min(args.steps, 5))
+    bi = sum(t.numel() * t.element_size() for t in h_in)
+    bo = sum(t.numel() * t.element_size() for t in h_out)
+
+    def e2e_step():
+        for a, t in zip(h_in, wl.inputs()):
+            t.copy_(a, non_blocking=True)
+        wl.step()
+        for a, t in zip(h_out, wl.outputs()):
+            a.copy_(t, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / e2e_steps
+
+    if rank != 0:
+        _finish(world)
+        return
+    peak, peak_kind = measured_peaks()
+    kernels = {}
+    for op, ms in zip(wl.ops, per_op_ms):
+        gbs = op.bytes / (ms * 1e-3) / 1e9
+        kernels[op.name] = {"us": round(ms * 1e3, 2), "bytes": op.bytes, "gb_s": round(gbs, 1),
+                            "frac": round(gbs / peak, 4), "launches": op.launches}
+    dom = max(range(nops), key=lambda i: per_op_ms[i])
+    dop = wl.ops[dom]
+    dgbs = dop.bytes / (per_op_ms[dom] * 1e-3) / 1e9
+    value = world * wl.step_bytes / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp32 -> fp8 (u8)",
+        "data": "synthetic (seeded generators; shapes and value mixes of the pages' workloads)",
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "config": {"workload": WORKLOAD, "step_bytes": wl.step_bytes, "parallelism": f"replicas x{world}",
+                   "l2": "no flush: each step streams ~4.4 GB through the 126 MB L2, so every op's inputs are cold"},
+        "roofline": {"bound": "hbm", "kernel": dop.kernel, "op": dop.name, "achieved": round(dgbs, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dgbs / peak, 4),
+                     "bytes_per_launch": dop.bytes, "traffic": recorded_traffic(dop.name)},
+        "kernels": kernels,
+        "clocks": clk.summary(),
+        "e2e": {"value": round(world * wl.step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+                "steps": e2e_steps},
+        "gpu_launches": wl.launches_per_step * args.steps,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(h)
+    print(json.dumps(line), flush=True)
+    _finish(world)
+
+
+def _finish(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, timed as it stands on this host."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as orc
+    orc.build()
+    threads = os.cpu_count() or 1
+    h = make_host_inputs()
+    frac = 1.0 / 512
+    for _ in range(args.warmup):
+        oracle_sample_pass(orc, h, frac, threads)
+    t0 = time.perf_counter()
+    b = 0
+    for _ in range(args.steps):
+        b += oracle_sample_pass(orc, h, frac, threads)
+    dt = time.perf_counter() - t0
+    value = b / dt / 1e9
+    sample = (f"each step: the first {frac:.5f} of the rows / elements of every op of the GPU step "
+              f"({b / args.steps / 1e6:.1f} MB algorithmic), plain C oracle on {threads} threads")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp32 -> fp8 (u8)",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "kind": "oracle", "cores": threads,
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="leave out the CPU oracle timing (it runs after the GPU timing)")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)   # the timing rules want at least 3 untimed steps
+    args.steps = max(1, args.steps)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,362 @@
+"""Scaled FP8 casting on NVIDIA B200 (sm_100a): Python binding of libfp8q.
+
+The compute path is the C-ABI library ``libfp8q.so`` (hand-written CUDA
+kernels, declared in ``include/fp8q.h``).  This module only marshals
+arguments: it turns torch tensors into device pointers, sizes, dtype codes and
+the current CUDA stream, checks that output buffers are large enough and on
+the same device, and raises :class:`Fp8qError` on a non-zero status.  torch
+is used for device memory and streams only.  There is no CPU fallback: if the
+library is missing or a tensor is not on a CUDA device, the call fails.
+
+Entry points with the C names (caller-provided outputs, nothing allocated):
+    fp8q_per_token_group_quant, fp8q_cast_per_channel, fp8q_cast_per_tensor,
+    fp8q_block_dequant, fp8q_block_dequant_grouped, fp8q_cast_from_fp8
+
+Allocating helpers named after the functions on the pages:
+    per_token_cast_to_fp8   (DeepEP "5 Utils")
+    per_token_cast_back     (DeepEP "5 Utils", the named inverse)
+    cast_to_fp8, cast_from_fp8   (ColossalAI colossalai/quantization/fp8.py)
+    weight_dequant          (DeepSeek-V3 fp8_cast_bf16 blog)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+__all__ = [
+    "E4M3FN", "E5M2", "F32", "F16", "BF16",
+    "GRAN_TENSOR", "GRAN_ROW", "GRAN_GROUP", "GRAN_BLOCK",
+    "Fp8qError", "lib", "lib_path",
+    "fp8q_per_token_group_quant", "fp8q_cast_per_channel", "fp8q_cast_per_tensor",
+    "fp8q_cast_per_tensor_workspace_bytes", "fp8q_block_dequant", "fp8q_block_dequant_grouped",
+    "fp8q_cast_from_fp8", "fp8q_status_string", "fp8q_version",
+    "per_token_cast_to_fp8", "per_token_cast_back", "cast_to_fp8", "cast_from_fp8", "weight_dequant",
+]
+
+E4M3FN, E5M2 = 0, 1
+F32, F16, BF16 = 0, 1, 2
+GRAN_TENSOR, GRAN_ROW, GRAN_GROUP, GRAN_BLOCK = 0, 1, 2, 3
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libfp8q.so")
+
+_DTYPE_CODE = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+_CODE_DTYPE = {v: k for k, v in _DTYPE_CODE.items()}
+_FP8_DTYPES = {torch.float8_e4m3fn: E4M3FN, torch.float8_e5m2: E5M2}
+_FMT_DTYPE = {E4M3FN: torch.float8_e4m3fn, E5M2: torch.float8_e5m2}
+
+
+class Fp8qError(RuntimeError):
+    """A libfp8q call returned a non-zero fp8q_status."""
+
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {fp8q_status_string(status)}")
+
+
+class _BlockDesc(ctypes.Structure):
+    _fields_ = [("w", ctypes.c_void_p), ("scale_inv", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("M", ctypes.c_int64), ("N", ctypes.c_int64)]
+
+
+_lock = threading.Lock()
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfp8q.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise ImportError(
+                    f"libfp8q.so not found at {_LIB_PATH}; build it with "
+                    "`python -m dequantisation_fp8q_token_b200.build` (needs nvcc)")
+            L = ctypes.CDLL(_LIB_PATH)
+            p, i64, i32, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int
+            L.fp8q_status_string.restype = ctypes.c_char_p
+            L.fp8q_status_string.argtypes = [st]
+            L.fp8q_version.restype = i32
+            L.fp8q_version.argtypes = []
+            L.fp8q_per_token_group_quant.restype = st
+            L.fp8q_per_token_group_quant.argtypes = [p, i32, i64, i64, i32, i32, p, p, p]
+            L.fp8q_cast_per_channel.restype = st
+            L.fp8q_cast_per_channel.argtypes = [p, i32, i64, i64, i32, p, p, p]
+            L.fp8q_cast_per_tensor_workspace_bytes.restype = ctypes.c_size_t
+            L.fp8q_cast_per_tensor_workspace_bytes.argtypes = []
+            L.fp8q_cast_per_tensor.restype = st
+            L.fp8q_cast_per_tensor.argtypes = [p, i32, i64, i32, p, p, p, ctypes.c_size_t, p]
+            L.fp8q_block_dequant.restype = st
+            L.fp8q_block_dequant.argtypes = [p, i32, i64, i64, p, i32, i32, p, p]
+            L.fp8q_block_dequant_grouped.restype = st
+            L.fp8q_block_dequant_grouped.argtypes = [ctypes.POINTER(_BlockDesc), i32, i32, i32, i32, p]
+            L.fp8q_cast_from_fp8.restype = st
+            L.fp8q_cast_from_fp8.argtypes = [p, i32, i64, i64, p, i32, i32, i32, p, p]
+            _lib = L
+    return _lib
+
+
+def fp8q_status_string(status: int) -> str:
+    return lib().fp8q_status_string(int(status)).decode()
+
+
+def fp8q_version() -> int:
+    return int(lib().fp8q_version())
+
+
+def fp8q_cast_per_tensor_workspace_bytes() -> int:
+    return int(lib().fp8q_cast_per_tensor_workspace_bytes())
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise Fp8qError(status, what)
+
+
+def _dev_ptr(t: Optional[torch.Tensor], name: str, device=None) -> Optional[int]:
+    """Device pointer of a contiguous CUDA tensor (None for an empty tensor)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libfp8q takes device pointers)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dtype_code(t: torch.Tensor, name: str) -> int:
+    if t.dtype not in _DTYPE_CODE:
+        raise TypeError(f"{name}: only float32, float16 and bfloat16 are allowed, got {t.dtype}")
+    return _DTYPE_CODE[t.dtype]
+
+
+def _is_byte_tensor(t: torch.Tensor) -> bool:
+    return t.dtype == torch.uint8 or t.dtype in _FP8_DTYPES
+
+
+def _need(t: torch.Tensor, numel: int, name: str, byte: bool = False, dtype=None) -> None:
+    if byte and not _is_byte_tensor(t):
+        raise TypeError(f"{name} must be uint8 or a float8 dtype, got {t.dtype}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs {numel}")
+
+
+def _fmt_of(fmt) -> int:
+    if isinstance(fmt, str):
+        return {"e4m3": E4M3FN, "e4m3fn": E4M3FN, "e5m2": E5M2}[fmt]
+    if isinstance(fmt, torch.dtype):
+        return _FP8_DTYPES[fmt]
+    return int(fmt)
+
+
+# ---------------------------------------------------------------------------
+# C entry points (caller-provided outputs)
+# ---------------------------------------------------------------------------
+def fp8q_per_token_group_quant(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
+                               group: int = 128, fmt=E4M3FN, stream=None) -> None:
+    """DeepEP per_token_cast_to_fp8 into q[m, n] (uint8/fp8) and scale_inv[m, n/group] (fp32)."""
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [m, n]")
+    m, n = x.shape
+    dev = x.device
+    if group > 0 and n % group == 0:
+        _need(q, m * n, "q", byte=True)
+        _need(scale_inv, m * (n // group), "scale_inv", dtype=torch.float32)
+    _check(lib().fp8q_per_token_group_quant(
+        _dev_ptr(x, "x"), _dtype_code(x, "x"), m, n, group, _fmt_of(fmt),
+        _dev_ptr(q, "q", dev), _dev_ptr(scale_inv, "scale_inv", dev), _stream(stream, dev)),
+        "fp8q_per_token_group_quant")
+
+
+def fp8q_cast_per_channel(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
+                          fmt=E4M3FN, stream=None) -> None:
+    """ColossalAI cast_to_fp8(per_channel_scale=True): one scale per row of x[rows, cols]."""
+    x2 = x.reshape(-1, x.shape[-1]) if x.dim() != 2 else x
+    rows, cols = x2.shape
+    dev = x.device
+    _need(q, rows * cols, "q", byte=True)
+    _need(scale_inv, max(rows, 1), "scale_inv", dtype=torch.float32)
+    _check(lib().fp8q_cast_per_channel(
+        _dev_ptr(x2, "x"), _dtype_code(x, "x"), rows, cols, _fmt_of(fmt),
+        _dev_ptr(q, "q", dev), _dev_ptr(scale_inv, "scale_inv", dev), _stream(stream, dev)),
+        "fp8q_cast_per_channel")
+
+
+def fp8q_cast_per_tensor(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
+                         workspace: torch.Tensor, fmt=E4M3FN, stream=None) -> None:
+    """ColossalAI cast_to_fp8 per-tensor branch; workspace of fp8q_cast_per_tensor_workspace_bytes()."""
+    dev = x.device
+    n = x.numel()
+    _need(q, n, "q", byte=True)
+    _need(scale_inv, 1, "scale_inv", dtype=torch.float32)
+    wbytes = workspace.numel() * workspace.element_size()
+    _check(lib().fp8q_cast_per_tensor(
+        _dev_ptr(x, "x"), _dtype_code(x, "x"), n, _fmt_of(fmt), _dev_ptr(q, "q", dev),
+        _dev_ptr(scale_inv, "scale_inv", dev), _dev_ptr(workspace, "workspace", dev), wbytes,
+        _stream(stream, dev)), "fp8q_cast_per_tensor")
+
+
+def fp8q_block_dequant(w: torch.Tensor, scale_inv: torch.Tensor, y: torch.Tensor, block: int = 128,
+                       fmt=E4M3FN, stream=None) -> None:
+    """DeepSeek-V3 weight_dequant of w[M, N] with scale_inv[ceil(M/B), ceil(N/B)] into y[M, N]."""
+    if w.dim() != 2:
+        raise ValueError("w must be 2-D [M, N]")
+    M, N = w.shape
+    dev = w.device
+    if block > 0:
+        _need(w, M * N, "w", byte=True)
+        _need(scale_inv, -(-M // block) * -(-N // block), "scale_inv", dtype=torch.float32)
+        _need(y, M * N, "y")
+    _check(lib().fp8q_block_dequant(
+        _dev_ptr(w, "w"), _fmt_of(fmt), M, N, _dev_ptr(scale_inv, "scale_inv", dev), block,
+        _dtype_code(y, "y"), _dev_ptr(y, "y", dev), _stream(stream, dev)), "fp8q_block_dequant")
+
+
+def fp8q_block_dequant_grouped(ws: Sequence[torch.Tensor], scale_invs: Sequence[torch.Tensor],
+                               ys: Sequence[torch.Tensor], block: int = 128, fmt=E4M3FN,
+                               stream=None) -> None:
+    """Many block dequantisations in one launch (shared block, format and output dtype)."""
+    n = len(ws)
+    if not (len(scale_invs) == len(ys) == n):
+        raise ValueError("ws, scale_invs and ys must have the same length")
+    if n == 0:
+        return
+    dev = ws[0].device
+    yt = _dtype_code(ys[0], "y")
+    arr = (_BlockDesc * n)()
+    for i, (w, s, y) in enumerate(zip(ws, scale_invs, ys)):
+        if w.dim() != 2:
+            raise ValueError("each w must be 2-D")
+        M, N = w.shape
+        if _dtype_code(y, "y") != yt:
+            raise TypeError("all outputs must share one dtype")
+        if block > 0:
+            _need(w, M * N, "w", byte=True)
+            _need(s, -(-M // block) * -(-N // block), "scale_inv", dtype=torch.float32)
+            _need(y, M * N, "y")
+        arr[i] = _BlockDesc(_dev_ptr(w, "w", dev), _dev_ptr(s, "scale_inv", dev), _dev_ptr(y, "y", dev), M, N)
+    _check(lib().fp8q_block_dequant_grouped(arr, n, _fmt_of(fmt), block, yt, _stream(stream, dev)),
+           "fp8q_block_dequant_grouped")
+
+
+def _granule_count(gran: int, rows: int, cols: int, gb: int) -> int:
+    if gran == GRAN_TENSOR:
+        return 1
+    if gran == GRAN_ROW:
+        return rows
+    if gran == GRAN_GROUP:
+        return rows * (cols // gb) if gb > 0 else 0
+    return -(-rows // gb) * -(-cols // gb) if gb > 0 else 0
+
+
+def fp8q_cast_from_fp8(q: torch.Tensor, scale_inv: torch.Tensor, y: torch.Tensor, gran: int,
+                       group_or_block: int = 0, fmt=None, stream=None) -> None:
+    """ColossalAI cast_from_fp8 / DeepEP per_token_cast_back into y (dtype of y)."""
+    if fmt is None:
+        fmt = _FP8_DTYPES.get(q.dtype, E4M3FN)
+    q2 = q.reshape(-1, q.shape[-1]) if q.dim() != 2 else q
+    rows, cols = q2.shape if q.dim() > 0 else (1, 1)
+    dev = q.device
+    _need(q, rows * cols, "q", byte=True)
+    _need(y, rows * cols, "y")
+    if gran in (GRAN_TENSOR, GRAN_ROW, GRAN_GROUP, GRAN_BLOCK):
+        _need(scale_inv, _granule_count(gran, rows, cols, group_or_block), "scale_inv", dtype=torch.float32)
+    _check(lib().fp8q_cast_from_fp8(
+        _dev_ptr(q2, "q"), _fmt_of(fmt), rows, cols, _dev_ptr(scale_inv, "scale_inv", dev), gran,
+        group_or_block, _dtype_code(y, "y"), _dev_ptr(y, "y", dev), _stream(stream, dev)),
+        "fp8q_cast_from_fp8")
+
+
+# ---------------------------------------------------------------------------
+# allocating helpers named after the pages' functions
+# ---------------------------------------------------------------------------
+_ws_cache = {}
+
+
+def _workspace(device: torch.device) -> torch.Tensor:
+    key = (device.type, device.index)
+    w = _ws_cache.get(key)
+    if w is None:
+        w = torch.empty(fp8q_cast_per_tensor_workspace_bytes(), dtype=torch.uint8, device=device)
+        _ws_cache[key] = w
+    return w
+
+
+def per_token_cast_to_fp8(x: torch.Tensor, group: int = 128, fmt=E4M3FN) -> Tuple[torch.Tensor, torch.Tensor]:
+    """DeepEP per_token_cast_to_fp8: returns (q [m, n] float8, scale_inv [m, n/group] fp32)."""
+    m, n = x.shape
+    f = _fmt_of(fmt)
+    q = torch.empty((m, n), dtype=_FMT_DTYPE[f], device=x.device)
+    s = torch.empty((m, n // group if group > 0 else 0), dtype=torch.float32, device=x.device)
+    fp8q_per_token_group_quant(x, q, s, group, f)
+    return q, s
+
+
+def per_token_cast_back(q: torch.Tensor, scale_inv: torch.Tensor, dtype=torch.bfloat16,
+                        group: int = 128) -> torch.Tensor:
+    """Inverse of per_token_cast_to_fp8: y = dtype(scale_inv[r, c/group] * float(q))."""
+    y = torch.empty(q.shape, dtype=dtype, device=q.device)
+    fp8q_cast_from_fp8(q, scale_inv, y, GRAN_GROUP, group)
+    return y
+
+
+def cast_to_fp8(inp: torch.Tensor, fp8_format: str = "e4m3", per_channel_scale: bool = False
+                ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """ColossalAI cast_to_fp8: (q with inp's shape, scale_inv).  scale_inv has shape [rows]
+    (per-channel; [1] for an empty input) or [1] (per-tensor)."""
+    f = _fmt_of(fp8_format)
+    q = torch.empty(inp.shape, dtype=_FMT_DTYPE[f], device=inp.device)
+    if per_channel_scale:
+        rows = inp.numel() // inp.shape[-1] if inp.dim() > 0 and inp.shape[-1] > 0 else 0
+        s = torch.empty((max(rows, 1) if inp.numel() == 0 else rows,), dtype=torch.float32, device=inp.device)
+        fp8q_cast_per_channel(inp.reshape(-1, inp.shape[-1]) if inp.dim() != 2 else inp, q, s, f)
+    else:
+        s = torch.empty((1,), dtype=torch.float32, device=inp.device)
+        fp8q_cast_per_tensor(inp, q, s, _workspace(inp.device), f)
+    return q, s
+
+
+def cast_from_fp8(inp: torch.Tensor, scale_inv: torch.Tensor, ret_type: torch.dtype,
+                  per_channel_scale: bool = False) -> torch.Tensor:
+    """ColossalAI cast_from_fp8 (row r scaled by scale_inv[r] in the per-channel case)."""
+    if inp.dtype not in _FP8_DTYPES:
+        raise TypeError("Only float8_e4m3fn and float8_e5m2 are allowed.")
+    y = torch.empty(inp.shape, dtype=ret_type, device=inp.device)
+    fp8q_cast_from_fp8(inp, scale_inv, y, GRAN_ROW if per_channel_scale else GRAN_TENSOR, 0,
+                       _FP8_DTYPES[inp.dtype])
+    return y
+
+
+def weight_dequant(x: torch.Tensor, s: torch.Tensor, block_size: int = 128,
+                   dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """DeepSeek-V3 weight_dequant: y[M, N] = dtype(float(x) * s[i/B, j/B])."""
+    if not (x.is_contiguous() and s.is_contiguous()):
+        raise ValueError("Input tensors must be contiguous")
+    if x.dim() != 2 or s.dim() != 2:
+        raise ValueError("Input tensors must have 2 dimensions")
+    y = torch.empty(x.shape, dtype=dtype, device=x.device)
+    fp8q_block_dequant(x, s, y, block_size, _FP8_DTYPES.get(x.dtype, E4M3FN))
+    return y

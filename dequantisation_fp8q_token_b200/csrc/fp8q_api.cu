@@ -1,0 +1,181 @@
+// fp8q_api.cu -- the extern "C" entry points of libfp8q: argument checks on
+// the host (enums, then shapes, then null pointers, then alignment), then the
+// launchers.  Nothing is enqueued when a check fails.
+#include <atomic>
+
+#include "fp8q.h"
+#include "fp8q_device.cuh"
+#include "fp8q_internal.h"
+
+namespace fp8q {
+
+int sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64) {
+        const int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+namespace {
+
+bool fmt_ok(int f) { return f == FP8Q_E4M3FN || f == FP8Q_E5M2; }
+bool dtype_ok(int t) { return t == FP8Q_F32 || t == FP8Q_F16 || t == FP8Q_BF16; }
+int dtype_bytes(int t) { return t == FP8Q_F32 ? 4 : 2; }
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// product of two non-negative sizes, or -1 when it would not fit in int64
+int64_t checked_mul(int64_t a, int64_t b) {
+    if (a == 0 || b == 0) return 0;
+    if (a > INT64_MAX / b) return -1;
+    return a * b;
+}
+
+}  // namespace
+}  // namespace fp8q
+
+using namespace fp8q;
+
+extern "C" {
+
+const char* fp8q_status_string(fp8q_status status) {
+    switch (status) {
+    case FP8Q_OK: return "FP8Q_OK";
+    case FP8Q_ERR_NULL_POINTER: return "FP8Q_ERR_NULL_POINTER: a non-empty tensor pointer is NULL";
+    case FP8Q_ERR_BAD_DTYPE: return "FP8Q_ERR_BAD_DTYPE: only float32, float16 and bfloat16 are allowed";
+    case FP8Q_ERR_BAD_FORMAT: return "FP8Q_ERR_BAD_FORMAT: only float8_e4m3fn and float8_e5m2 are allowed";
+    case FP8Q_ERR_BAD_SHAPE: return "FP8Q_ERR_BAD_SHAPE: size, group or block edge not allowed";
+    case FP8Q_ERR_MISALIGNED: return "FP8Q_ERR_MISALIGNED: pointer not aligned to its element size";
+    case FP8Q_ERR_WORKSPACE: return "FP8Q_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case FP8Q_ERR_CUDA: return "FP8Q_ERR_CUDA: the CUDA runtime refused a launch";
+    case FP8Q_ERR_BAD_GRANULARITY: return "FP8Q_ERR_BAD_GRANULARITY: unknown scale granularity";
+    case FP8Q_ERR_TOO_MANY: return "FP8Q_ERR_TOO_MANY: descriptor count out of range";
+    }
+    return "FP8Q_ERR_UNKNOWN";
+}
+
+int fp8q_version(void) { return 10000; }
+
+fp8q_status fp8q_per_token_group_quant(const void* x, fp8q_dtype xt, int64_t m, int64_t n, int group,
+                                       fp8q_format fmt, uint8_t* q, float* scale_inv,
+                                       fp8q_stream_t stream) {
+    if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
+    if (m < 0 || n < 0 || group < 1 || n % group != 0) return FP8Q_ERR_BAD_SHAPE;
+    const int64_t numel = checked_mul(m, n);
+    if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    if (numel == 0) return FP8Q_OK;
+    if (!x || !q || !scale_inv) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(x, dtype_bytes(xt)) || !aligned(scale_inv, 4)) return FP8Q_ERR_MISALIGNED;
+    return launch_per_token(x, xt, m, n, group, fmt, q, scale_inv, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp8q_status fp8q_cast_per_channel(const void* x, fp8q_dtype xt, int64_t rows, int64_t cols,
+                                  fp8q_format fmt, uint8_t* q, float* scale_inv, fp8q_stream_t stream) {
+    if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
+    if (rows < 0 || cols < 0 || rows > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
+    const int64_t numel = checked_mul(rows, cols);
+    if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!scale_inv) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(scale_inv, 4)) return FP8Q_ERR_MISALIGNED;
+    if (numel == 0) return launch_fill(scale_inv, rows > 0 ? rows : 1, 1.0f, s);
+    if (!x || !q) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(x, dtype_bytes(xt))) return FP8Q_ERR_MISALIGNED;
+    return launch_per_channel(x, xt, rows, cols, fmt, q, scale_inv, s);
+}
+
+size_t fp8q_cast_per_tensor_workspace_bytes(void) { return kPerTensorWorkspaceBytes; }
+
+fp8q_status fp8q_cast_per_tensor(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt,
+                                 uint8_t* q, float* scale_inv, void* workspace, size_t workspace_bytes,
+                                 fp8q_stream_t stream) {
+    if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
+    if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!scale_inv) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(scale_inv, 4)) return FP8Q_ERR_MISALIGNED;
+    if (numel == 0) return launch_fill(scale_inv, 1, 1.0f, s);
+    if (!x || !q) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(x, dtype_bytes(xt))) return FP8Q_ERR_MISALIGNED;
+    if (!workspace || workspace_bytes < kPerTensorWorkspaceBytes || !aligned(workspace, 16))
+        return FP8Q_ERR_WORKSPACE;
+    return launch_per_tensor(x, xt, numel, fmt, q, scale_inv, static_cast<uint32_t*>(workspace), s);
+}
+
+fp8q_status fp8q_block_dequant(const uint8_t* w, fp8q_format fmt, int64_t M, int64_t N,
+                               const float* scale_inv, int block, fp8q_dtype yt, void* y,
+                               fp8q_stream_t stream) {
+    fp8q_block_desc d = {w, scale_inv, y, M, N};
+    return fp8q_block_dequant_grouped(&d, 1, fmt, block, yt, stream);
+}
+
+fp8q_status fp8q_block_dequant_grouped(const fp8q_block_desc* descs, int count, fp8q_format fmt, int block,
+                                       fp8q_dtype yt, fp8q_stream_t stream) {
+    if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
+    if (!dtype_ok(yt)) return FP8Q_ERR_BAD_DTYPE;
+    if (count < 0) return FP8Q_ERR_TOO_MANY;
+    if (block < 1) return FP8Q_ERR_BAD_SHAPE;
+    if (count == 0) return FP8Q_OK;
+    if (!descs) return FP8Q_ERR_NULL_POINTER;
+    for (int i = 0; i < count; ++i) {
+        const fp8q_block_desc& d = descs[i];
+        if (d.M < 0 || d.N < 0 || d.M > 0x7FFFFFFFLL || d.N > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
+        const int64_t numel = checked_mul(d.M, d.N);
+        if (numel < 0 || checked_mul(numel, dtype_bytes(yt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    }
+    for (int i = 0; i < count; ++i) {
+        const fp8q_block_desc& d = descs[i];
+        if (d.M * d.N == 0) continue;
+        if (!d.w || !d.scale_inv || !d.y) return FP8Q_ERR_NULL_POINTER;
+    }
+    for (int i = 0; i < count; ++i) {
+        const fp8q_block_desc& d = descs[i];
+        if (d.M * d.N == 0) continue;
+        if (!aligned(d.scale_inv, 4) || !aligned(d.y, dtype_bytes(yt))) return FP8Q_ERR_MISALIGNED;
+    }
+    // problems on the stack in batches; each batch is one launch
+    constexpr int kBatch = 96;
+    DequantProblem probs[kBatch];
+    for (int i = 0; i < count; i += kBatch) {
+        const int nb = count - i < kBatch ? count - i : kBatch;
+        for (int j = 0; j < nb; ++j) {
+            const fp8q_block_desc& d = descs[i + j];
+            probs[j] = DequantProblem{d.w, d.scale_inv, d.y, d.M, d.N};
+        }
+        fp8q_status st = launch_dequant(probs, nb, fmt, kGranBlock, block, yt,
+                                        reinterpret_cast<cudaStream_t>(stream));
+        if (st != FP8Q_OK) return st;
+    }
+    return FP8Q_OK;
+}
+
+fp8q_status fp8q_cast_from_fp8(const uint8_t* q, fp8q_format fmt, int64_t rows, int64_t cols,
+                               const float* scale_inv, fp8q_granularity gran, int group_or_block,
+                               fp8q_dtype yt, void* y, fp8q_stream_t stream) {
+    if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
+    if (!dtype_ok(yt)) return FP8Q_ERR_BAD_DTYPE;
+    if (gran < FP8Q_GRAN_TENSOR || gran > FP8Q_GRAN_BLOCK) return FP8Q_ERR_BAD_GRANULARITY;
+    if (rows < 0 || cols < 0 || rows > 0x7FFFFFFFLL || cols > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
+    const bool sized = gran == FP8Q_GRAN_GROUP || gran == FP8Q_GRAN_BLOCK;
+    if (sized && group_or_block < 1) return FP8Q_ERR_BAD_SHAPE;
+    if (gran == FP8Q_GRAN_GROUP && cols % group_or_block != 0) return FP8Q_ERR_BAD_SHAPE;
+    const int64_t numel = checked_mul(rows, cols);
+    if (numel < 0 || checked_mul(numel, dtype_bytes(yt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    if (numel == 0) return FP8Q_OK;
+    if (!q || !scale_inv || !y) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(scale_inv, 4) || !aligned(y, dtype_bytes(yt))) return FP8Q_ERR_MISALIGNED;
+    DequantProblem p{q, scale_inv, y, rows, cols};
+    return launch_dequant(&p, 1, fmt, gran, sized ? group_or_block : 1, yt,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

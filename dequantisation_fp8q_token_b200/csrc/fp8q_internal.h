@@ -1,0 +1,39 @@
+// fp8q_internal.h -- host-side launchers behind the C ABI (validated arguments only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fp8q.h"
+
+namespace fp8q {
+
+// per-CTA partial maxima of the per-tensor amax pass
+constexpr int kMaxPartials = 2048;
+constexpr size_t kPerTensorWorkspaceBytes = kMaxPartials * sizeof(uint32_t);
+
+// number of SMs of the current device (cached per device)
+int sm_count();
+
+fp8q_status launch_per_token(const void* x, int xt, int64_t m, int64_t n, int group, int fmt,
+                             uint8_t* q, float* sinv, cudaStream_t s);
+fp8q_status launch_per_channel(const void* x, int xt, int64_t rows, int64_t cols, int fmt,
+                               uint8_t* q, float* sinv, cudaStream_t s);
+fp8q_status launch_per_tensor(const void* x, int xt, int64_t numel, int fmt, uint8_t* q,
+                              float* sinv, uint32_t* partials, cudaStream_t s);
+fp8q_status launch_fill(float* dst, int64_t count, float value, cudaStream_t s);
+
+// one dequantisation problem: y = T(scale(r, c) * float(q)), validated shapes
+struct DequantProblem {
+    const uint8_t* q;
+    const float* s;
+    void* y;
+    int64_t rows;
+    int64_t cols;
+};
+fp8q_status launch_dequant(const DequantProblem* probs, int count, int fmt, int gran, int gb,
+                           int yt, cudaStream_t s);
+
+inline fp8q_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA; }
+
+}  // namespace fp8q

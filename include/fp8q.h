@@ -1,0 +1,195 @@
+/*
+ * fp8q.h -- C ABI of libfp8q, scaled FP8 casting on NVIDIA B200 (sm_100a).
+ *
+ * Operations (each entry point cites the passage that defines it):
+ *   fp8q_per_token_group_quant  DeepEP "5 Utils", per_token_cast_to_fp8
+ *   fp8q_cast_per_channel       ColossalAI colossalai/quantization/fp8.py,
+ *                               cast_to_fp8 (per_channel_scale=True)
+ *   fp8q_cast_per_tensor        ColossalAI cast_to_fp8 (per-tensor branch)
+ *   fp8q_block_dequant(_grouped) DeepSeek-V3 fp8_cast_bf16 blog,
+ *                               weight_dequant / weight_dequant_kernel
+ *   fp8q_cast_from_fp8          ColossalAI cast_from_fp8; DeepEP
+ *                               per_token_cast_back
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors are caller-owned DEVICE pointers to contiguous row-major data.
+ *   fp8 tensors are raw bytes (uint8_t codes); high-precision tensors are
+ *   fp32, fp16 or bf16 as named by an fp8q_dtype argument.
+ * - The library never allocates or frees memory, never synchronises, keeps
+ *   no state between calls and enqueues all work on the given stream (NULL =
+ *   the legacy default stream).  Calls on different streams are independent.
+ *   Calls return as soon as the work is enqueued; outputs are valid once the
+ *   stream reaches that point.
+ * - Arithmetic is IEEE binary32 with round-to-nearest-even: scales are
+ *   computed with true division (fl(FMAX / amax)), products are single
+ *   fp32 multiplies, narrowing to fp8 / bf16 / fp16 rounds to nearest-even.
+ *   The fp8 cast does not saturate: a magnitude that rounds above the
+ *   format's maximum becomes NaN (e4m3fn) or Inf (e5m2), as torch's
+ *   .to(float8_*) does.  Denormals are kept (no flush to zero).
+ *   FMAX is 448 (e4m3fn) or 57344 (e5m2).
+ * - Every argument is validated on the host before anything is enqueued, in
+ *   this order: enums, sizes and shape rules, null pointers, alignment.  A
+ *   pointer may be NULL only when its tensor has no elements.  On any error
+ *   nothing is enqueued.  Errors reported by the CUDA runtime while
+ *   enqueueing map to FP8Q_ERR_CUDA.  The library never aborts and never
+ *   traps on the device.
+ * - Alignment: each pointer must be aligned to its element size
+ *   (FP8Q_ERR_MISALIGNED otherwise).  16-byte aligned pointers and row
+ *   strides take the vectorised paths; other layouts are still accepted and
+ *   take narrower loads.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA include. */
+typedef struct CUstream_st* fp8q_stream_t;
+
+typedef enum {
+    FP8Q_E4M3FN = 0, /* float8_e4m3fn: bias 7, 3 mantissa bits, no Inf, max 448 */
+    FP8Q_E5M2 = 1    /* float8_e5m2:   bias 15, 2 mantissa bits, max 57344 */
+} fp8q_format;
+
+typedef enum { FP8Q_F32 = 0, FP8Q_F16 = 1, FP8Q_BF16 = 2 } fp8q_dtype;
+
+typedef enum {
+    FP8Q_GRAN_TENSOR = 0, /* one scale for the whole tensor: scale_inv[0] */
+    FP8Q_GRAN_ROW = 1,    /* one scale per row: scale_inv[r] */
+    FP8Q_GRAN_GROUP = 2,  /* 1 x G groups along a row: scale_inv[r * (cols/G) + c/G] */
+    FP8Q_GRAN_BLOCK = 3   /* B x B blocks: scale_inv[(r/B) * ceil(cols/B) + c/B] */
+} fp8q_granularity;
+
+typedef enum {
+    FP8Q_OK = 0,
+    FP8Q_ERR_NULL_POINTER = 1,    /* a non-empty tensor was given as NULL */
+    FP8Q_ERR_BAD_DTYPE = 2,       /* dtype not fp32/fp16/bf16 (the pages' TypeError) */
+    FP8Q_ERR_BAD_FORMAT = 3,      /* format not e4m3fn/e5m2 (the pages' TypeError) */
+    FP8Q_ERR_BAD_SHAPE = 4,       /* negative size, n % group != 0, bad group/block edge */
+    FP8Q_ERR_MISALIGNED = 5,      /* pointer not aligned to its element size */
+    FP8Q_ERR_WORKSPACE = 6,       /* workspace missing or too small */
+    FP8Q_ERR_CUDA = 7,            /* the CUDA runtime refused a launch */
+    FP8Q_ERR_BAD_GRANULARITY = 8, /* granularity enum out of range */
+    FP8Q_ERR_TOO_MANY = 9         /* grouped call: count < 0 */
+} fp8q_status;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* fp8q_status_string(fp8q_status status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int fp8q_version(void);
+
+/*
+ * Per-token group quantisation -- DeepEP "5 Utils", per_token_cast_to_fp8:
+ *   for each row r and group g of `group` consecutive elements,
+ *     amax      = max(max_k |float(x[r][g*group + k])|, fl32(1e-4))  (clamp)
+ *     scale     = fl(FMAX / amax)
+ *     q[r][c]   = fp8(fl(float(x[r][c]) * scale))
+ *     scale_inv[r][g] = fl(amax / FMAX)
+ *   A NaN in a group makes its amax, scales and codes NaN (torch's amax and
+ *   clamp keep NaN).  The pages fix group = 128 and e4m3fn; any group that
+ *   divides n is accepted (powers of two from 16 to 1024 take the vector path).
+ * x:         [m][n] elements of type xt (fp32, fp16 or bf16).
+ * q:         [m][n] fp8 codes (output).
+ * scale_inv: [m][n/group] fp32 (output).
+ * Errors: n % group != 0 or group < 1 -> FP8Q_ERR_BAD_SHAPE (the page's
+ *   assert on x.size(1) % 128).  m == 0 or n == 0 writes nothing.
+ */
+fp8q_status fp8q_per_token_group_quant(const void* x, fp8q_dtype xt, int64_t m, int64_t n,
+                                       int group, fp8q_format fmt, uint8_t* q,
+                                       float* scale_inv, fp8q_stream_t stream);
+
+/*
+ * Per-channel cast -- ColossalAI cast_to_fp8 with per_channel_scale=True:
+ *   amax[r]      = max_c |x[r][c]|, then amax[r] := amax[r] > 0 ? amax[r] : 1
+ *                  (a NaN amax fails the test and becomes 1)
+ *   scale[r]     = fl(FMAX / amax[r]);  scale_inv[r] = fl(amax[r] / FMAX)
+ *   q[r][c]      = fp8(fl(float(x[r][c]) * scale[r]))
+ *   Row r dequantises with scale_inv[r].
+ * x: [rows][cols] of type xt; q: [rows][cols]; scale_inv: [max(rows, 1)].
+ * Empty tensor (rows * cols == 0): scale_inv[0 .. max(rows,1)) = 1.0 (the
+ *   page returns tensor([1.0]) for an empty input); q is not touched.
+ */
+fp8q_status fp8q_cast_per_channel(const void* x, fp8q_dtype xt, int64_t rows, int64_t cols,
+                                  fp8q_format fmt, uint8_t* q, float* scale_inv,
+                                  fp8q_stream_t stream);
+
+/*
+ * Per-tensor cast -- ColossalAI cast_to_fp8 per-tensor branch:
+ *   amax = max |x| over all numel elements, amax := amax > 0 ? amax : 1
+ *   scale = fl(FMAX / amax);  scale_inv[0] = fl(1 / scale)
+ *   q[i] = fp8(fl(float(x[i]) * scale))
+ * Two passes over x (an amax reduction, then the scaled cast) in two kernels;
+ * the first writes per-CTA partial maxima into `workspace`, the second
+ * reduces them.  No atomics, no spin-waits, deterministic.
+ * workspace: device memory of at least fp8q_cast_per_tensor_workspace_bytes()
+ *   bytes, 16-byte aligned, owned by the caller; its contents need no
+ *   initialisation and are scratch after the call.  Calls that share one
+ *   workspace must be ordered (same stream, or synchronised).
+ * Empty tensor (numel == 0): scale_inv[0] = 1.0 is written on the stream.
+ */
+size_t fp8q_cast_per_tensor_workspace_bytes(void);
+fp8q_status fp8q_cast_per_tensor(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt,
+                                 uint8_t* q, float* scale_inv, void* workspace,
+                                 size_t workspace_bytes, fp8q_stream_t stream);
+
+/*
+ * Block dequantisation -- DeepSeek-V3 weight_dequant / weight_dequant_kernel:
+ *   y[i][j] = T(fl(float(w[i][j]) * scale_inv[i / B][j / B]))
+ *   with scale_inv row-major [ceil(M/B)][ceil(N/B)] (the kernel's
+ *   pid_m * cdiv(N, B) + pid_n index); partial edge blocks use their own
+ *   scale.  T is bf16 on the pages (the default dtype the converter sets);
+ *   fp16 and fp32 outputs are also offered.  The pages fix B = 128 and
+ *   e4m3fn weights; e5m2 weights are also accepted.
+ * w: [M][N] fp8 codes; scale_inv as above; y: [M][N] of type yt (output).
+ * Errors: block < 1 -> FP8Q_ERR_BAD_SHAPE.
+ */
+fp8q_status fp8q_block_dequant(const uint8_t* w, fp8q_format fmt, int64_t M, int64_t N,
+                               const float* scale_inv, int block, fp8q_dtype yt, void* y,
+                               fp8q_stream_t stream);
+
+/*
+ * Many block dequantisations in one launch (the converter's loop over every
+ * fp8 weight of a checkpoint, e.g. a mixture-of-experts layer).  `descs` is a
+ * HOST array of `count` descriptors, read during the call only; each entry
+ * is one fp8q_block_dequant problem with its own shape and pointers; fmt,
+ * block and yt are shared.  Bytes written are identical to calling
+ * fp8q_block_dequant once per entry.  Entries with M * N == 0 are skipped.
+ * Large counts are split into several launches internally.
+ */
+typedef struct {
+    const uint8_t* w;       /* [M][N] fp8 codes */
+    const float* scale_inv; /* [ceil(M/B)][ceil(N/B)] fp32 */
+    void* y;                /* [M][N] of the shared output type */
+    int64_t M;
+    int64_t N;
+} fp8q_block_desc;
+
+fp8q_status fp8q_block_dequant_grouped(const fp8q_block_desc* descs, int count,
+                                       fp8q_format fmt, int block, fp8q_dtype yt,
+                                       fp8q_stream_t stream);
+
+/*
+ * Dequantising cast -- ColossalAI cast_from_fp8 (ret = scale_inv * q.float(),
+ * then .to(ret_type)), and DeepEP per_token_cast_back for 1 x G groups:
+ *   y[r][c] = T(fl(scale_inv[granule(r, c)] * float(q[r][c])))
+ * granule per fp8q_granularity above; group_or_block is G (GROUP) or B
+ * (BLOCK) and is ignored for TENSOR and ROW.  For a per-channel cast the
+ * intended row scaling is used (row r by scale_inv[r]).
+ * q: [rows][cols] codes; scale_inv: granule-count fp32; y: [rows][cols] of yt.
+ * Errors: GROUP with cols % G != 0, or G / B < 1 -> FP8Q_ERR_BAD_SHAPE.
+ */
+fp8q_status fp8q_cast_from_fp8(const uint8_t* q, fp8q_format fmt, int64_t rows, int64_t cols,
+                               const float* scale_inv, fp8q_granularity gran, int group_or_block,
+                               fp8q_dtype yt, void* y, fp8q_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP8Q_H */

@@ -23,3 +23,15 @@ def orc():
     oracle.build()
     oracle.lib()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def fp8q():
+    """The CUDA library's Python binding, built for sm_100a (rebuilt if stale)."""
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from dequantisation_fp8q_token_b200 import build as _build
+    _build.build()
+    import dequantisation_fp8q_token_b200 as m
+    m.lib()
+    return m
