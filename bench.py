@@ -176,7 +176,7 @@ class ClockSampler:
     REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.005):
         self.index, self.period = index, period_s
         self.samples, self.reasons, self.max_mhz, self.ok = [], set(), None, False
         self._stop = threading.Event()
@@ -303,15 +303,16 @@ def cpu_baseline(h, budget_s: float = 15.0):
     import oracle as orc
     orc.build()
     threads = os.cpu_count() or 1
-    frac = 1.0 / 2048
-    t0 = time.perf_counter()
-    b = oracle_sample_pass(orc, h, frac, threads)
-    dt = time.perf_counter() - t0
-    # scale the sample so that the measured pass takes about `budget_s`
-    frac = min(1.0, frac * max(1.0, budget_s / max(dt, 1e-3)))
-    t0 = time.perf_counter()
-    b = oracle_sample_pass(orc, h, frac, threads)
-    dt = time.perf_counter() - t0
+    frac = 1.0 / 4096
+    # grow the sample until one pass takes about `budget_s` (small samples are
+    # dominated by thread start-up, so grow by at most 8x per probe)
+    while True:
+        t0 = time.perf_counter()
+        b = oracle_sample_pass(orc, h, frac, threads)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 2 or frac >= 1.0:
+            break
+        frac = min(1.0, frac * min(8.0, max(1.5, budget_s / max(dt, 1e-3))))
     return {"value": round(b / dt / 1e9, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"the first {frac:.5f} of the rows / elements of every op of the step "
                       f"({b / 1e6:.1f} MB algorithmic), plain C oracle on {threads} threads",
@@ -485,8 +486,8 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="leave out the CPU oracle timing (it runs after the GPU timing)")
