@@ -57,8 +57,12 @@ GRAN_GROUP = 2
 # the workload: inputs, outputs, algorithmic bytes, and the step
 # ---------------------------------------------------------------------------
 class Op:
-    def __init__(self, name, fn, bytes_, launches, kernel):
+    """One call of the step: `ins` are the tensors it reads that come from the
+    host in an end-to-end run, `outs` the tensors it writes."""
+
+    def __init__(self, name, fn, bytes_, launches, kernel, ins=(), outs=()):
         self.name, self.fn, self.bytes, self.launches, self.kernel = name, fn, bytes_, launches, kernel
+        self.ins, self.outs = list(ins), list(outs)
 
 
 class Workload:
@@ -113,21 +117,21 @@ class Workload:
         f = fp8q
         self.ops = [
             Op("per_token_group_quant", lambda: f.fp8q_per_token_group_quant(self.c2_x, self.c2_q, self.c2_s, 128, E4M3FN),
-               c2_bytes, 1, "per_token_vec_kernel"),
+               c2_bytes, 1, "per_token_vec_kernel", [self.c2_x], [self.c2_q, self.c2_s]),
             Op("block_dequant", lambda: f.fp8q_block_dequant(self.c3_w, self.c3_s, self.c3_y, 128, E4M3FN),
-               c3_bytes, 1, "dequant_kernel"),
+               c3_bytes, 1, "dequant_kernel", [self.c3_w, self.c3_s], [self.c3_y]),
             # the round trip reads q after the block dequant has streamed ~400 MB
             # through L2, so it finds no q bytes left in L2
             Op("cast_from_fp8_group", lambda: f.fp8q_cast_from_fp8(self.c2_q, self.c2_s, self.c2_y, GRAN_GROUP, 128, E4M3FN),
-               c2_bytes, 1, "dequant_kernel"),
+               c2_bytes, 1, "dequant_kernel", [], [self.c2_y]),
             Op("cast_per_channel", lambda: f.fp8q_cast_per_channel(self.c4a_x, self.c4a_q, self.c4a_s, E4M3FN),
-               c4a_bytes, 1, "per_channel_vec_kernel"),
+               c4a_bytes, 1, "per_channel_vec_kernel", [self.c4a_x], [self.c4a_q, self.c4a_s]),
             Op("cast_per_tensor_f32_e5m2", lambda: f.fp8q_cast_per_tensor(self.c4b_x, self.c4b_q, self.c4b_s, self.ws, E5M2),
-               c4b_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel"),
+               c4b_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel", [self.c4b_x], [self.c4b_q, self.c4b_s]),
             Op("cast_per_tensor_f16_zero", lambda: f.fp8q_cast_per_tensor(self.c4c_x, self.c4c_q, self.c4c_s, self.ws, E4M3FN),
-               c4c_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel"),
+               c4c_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel", [self.c4c_x], [self.c4c_q, self.c4c_s]),
             Op("block_dequant_grouped", lambda: f.fp8q_block_dequant_grouped(self.c5_w, self.c5_s, self.c5_y, 128, E4M3FN),
-               c5_bytes, 1, "dequant_kernel"),
+               c5_bytes, 1, "dequant_kernel", [*self.c5_w, *self.c5_s], self.c5_y),
         ]
         self.step_bytes = sum(o.bytes for o in self.ops)
         self.launches_per_step = sum(o.launches for o in self.ops)
@@ -142,11 +146,71 @@ class Workload:
 
     # host<->device traffic of one end-to-end step
     def inputs(self):
-        return [self.c2_x, self.c3_w, self.c3_s, self.c4a_x, self.c4b_x, self.c4c_x, *self.c5_w, *self.c5_s]
+        return [t for op in self.ops for t in op.ins]
 
     def outputs(self):
-        return [self.c2_q, self.c2_s, self.c2_y, self.c3_y, self.c4a_q, self.c4a_s, self.c4b_q, self.c4b_s,
-                self.c4c_q, self.c4c_s, *self.c5_y]
+        return [t for op in self.ops for t in op.outs]
+
+
+class EndToEnd:
+    """The step from pinned host memory to pinned host memory.  Each op's inputs
+    go host->device on a copy-in stream, the op runs on the compute stream, its
+    outputs go device->host on a copy-out stream; events order each op's three
+    parts and keep the next step from overwriting a buffer still in use, so the
+    upload of one op overlaps the compute and download of the ones before it
+    (PCIe carries both directions at once)."""
+
+    def __init__(self, wl: Workload):
+        self.wl = wl
+        self.h_in = {id(t): torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wl.inputs()}
+        for t in wl.inputs():
+            self.h_in[id(t)].copy_(t)
+        self.h_out = {id(t): torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wl.outputs()}
+        self.s_in, self.s_comp, self.s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        n = len(wl.ops)
+        self.done_comp = [None] * n
+        self.done_out = [None] * n
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in wl.inputs())
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in wl.outputs())
+
+    def step(self):
+        for i, op in enumerate(self.wl.ops):
+            with torch.cuda.stream(self.s_in):
+                if self.done_comp[i] is not None:
+                    self.s_in.wait_event(self.done_comp[i])      # previous step's op i has read its inputs
+                for t in op.ins:
+                    t.copy_(self.h_in[id(t)], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(self.s_in)
+            with torch.cuda.stream(self.s_comp):
+                self.s_comp.wait_event(ev_in)
+                if self.done_out[i] is not None:
+                    self.s_comp.wait_event(self.done_out[i])     # previous step's outputs are on the host
+                op.fn()
+                ev_c = torch.cuda.Event()
+                ev_c.record(self.s_comp)
+                self.done_comp[i] = ev_c
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(ev_c)
+                for t in op.outs:
+                    self.h_out[id(t)].copy_(t, non_blocking=True)
+                ev_o = torch.cuda.Event()
+                ev_o.record(self.s_out)
+                self.done_out[i] = ev_o
+
+    def time(self, steps: int) -> float:
+        """Milliseconds per step on the device clock (first upload to last download)."""
+        self.step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.s_in)
+        for _ in range(steps):
+            self.step()
+        self.s_out.wait_stream(self.s_comp)
+        self.s_out.wait_stream(self.s_in)
+        e1.record(self.s_out)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
 
 
 def _to_dev(a, device, dt=None):
@@ -383,31 +447,11 @@ def run_ours(args):
                  for i in range(nops)]
 
     # end to end: pinned host inputs -> device, the step, outputs -> pinned host
-    h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wl.inputs()]
-    for a, t in zip(h_in, wl.inputs()):
-        a.copy_(t)
-    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wl.outputs()]
+    e2e = EndToEnd(wl)
     e2e_steps = max(1, min(args.steps, 5))
-    bi = sum(t.numel() * t.element_size() for t in h_in)
-    bo = sum(t.numel() * t.element_size() for t in h_out)
-
-    def e2e_step():
-        for a, t in zip(h_in, wl.inputs()):
-            t.copy_(a, non_blocking=True)
-        wl.step()
-        for a, t in zip(h_out, wl.outputs()):
-            a.copy_(t, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
     barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / e2e_steps
+    e2e_ms = max_over_ranks(e2e.time(e2e_steps), world, device)
+    bi, bo = e2e.h2d_bytes, e2e.d2h_bytes
 
     if rank != 0:
         _finish(world)
@@ -483,6 +527,64 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# single-op cases for profiler captures (ncu -k <kernel> -c <n>): one op, a few
+# launches, inputs larger than L2 and a few GB on the device at most
+# ---------------------------------------------------------------------------
+def _profile_case(name, fp8q, device):
+    g = np.random.default_rng(20261299)
+    bf16 = torch.bfloat16
+    if name in ("per_token_4x", "cast_from_fp8_4x"):
+        m, n = 4 * workloads.C2_SHAPE[0], workloads.C2_SHAPE[1]   # bf16 [16384, 7168]: 235 MB
+        x = _to_dev(workloads.to_bf16_bits(g.standard_normal((m, n), dtype=np.float32)), device, bf16)
+        q = torch.empty((m, n), dtype=torch.uint8, device=device)
+        s = torch.empty((m, n // 128), dtype=torch.float32, device=device)
+        y = torch.empty((m, n), dtype=bf16, device=device)
+        fp8q.fp8q_per_token_group_quant(x, q, s, 128, E4M3FN)
+        if name == "per_token_4x":
+            return lambda: fp8q.fp8q_per_token_group_quant(x, q, s, 128, E4M3FN)
+        return lambda: fp8q.fp8q_cast_from_fp8(q, s, y, GRAN_GROUP, 128, E4M3FN)
+    if name == "block_dequant":
+        w, sc = workloads.c3_w_s()
+        w, sc = _to_dev(w, device), _to_dev(sc, device)
+        y = torch.empty(w.shape, dtype=bf16, device=device)
+        return lambda: fp8q.fp8q_block_dequant(w, sc, y, 128, E4M3FN)
+    if name == "grouped_16":
+        idx = list(range(8)) + list(range(64, 72))                 # 8 big + 8 ragged experts: 174 MB in
+        ws, ss = zip(*[workloads.c5_weight(i) for i in idx])
+        ws = [_to_dev(w, device) for w in ws]
+        ss = [_to_dev(s_, device) for s_ in ss]
+        ys = [torch.empty(w.shape, dtype=bf16, device=device) for w in ws]
+        return lambda: fp8q.fp8q_block_dequant_grouped(ws, ss, ys, 128, E4M3FN)
+    if name == "per_channel":
+        x = _to_dev(workloads.c4a_x(), device, bf16)
+        q = torch.empty(x.shape, dtype=torch.uint8, device=device)
+        s = torch.empty((x.shape[0],), dtype=torch.float32, device=device)
+        return lambda: fp8q.fp8q_cast_per_channel(x, q, s, E4M3FN)
+    if name == "per_tensor":
+        x = _to_dev(workloads.c4b_v(), device)
+        q = torch.empty(x.shape, dtype=torch.uint8, device=device)
+        s = torch.empty((1,), dtype=torch.float32, device=device)
+        ws = torch.empty(fp8q.fp8q_cast_per_tensor_workspace_bytes(), dtype=torch.uint8, device=device)
+        return lambda: fp8q.fp8q_cast_per_tensor(x, q, s, ws, E5M2)
+    raise SystemExit(f"unknown profile case {name}")
+
+
+PROFILE_CASES = ["per_token_4x", "cast_from_fp8_4x", "block_dequant", "grouped_16", "per_channel", "per_tensor"]
+
+
+def run_profile_case(name, iters):
+    """Run one op `iters` times after one untimed launch; prints no bench line."""
+    device = torch.device("cuda", 0)
+    import dequantisation_fp8q_token_b200 as fp8q
+    fn = _profile_case(name, fp8q, device)
+    torch.cuda.synchronize()
+    for _ in range(iters):
+        fn()
+    torch.cuda.synchronize()
+    print(f"profile case {name}: {iters} launches done")
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -491,7 +593,13 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="leave out the CPU oracle timing (it runs after the GPU timing)")
+    ap.add_argument("--profile", choices=PROFILE_CASES,
+                    help="run one op of a fixed case --iters times for a profiler capture (no timing)")
+    ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args(argv)
+    if args.profile:
+        run_profile_case(args.profile, args.iters)
+        return
     args.warmup = max(3, args.warmup)   # the timing rules want at least 3 untimed steps
     args.steps = max(1, args.steps)
     if args.impl == "reference":
