@@ -32,7 +32,7 @@ __all__ = [
     "GRAN_TENSOR", "GRAN_ROW", "GRAN_GROUP", "GRAN_BLOCK",
     "Fp8qError", "lib", "lib_path",
     "fp8q_per_token_group_quant", "fp8q_cast_per_channel", "fp8q_cast_per_tensor",
-    "fp8q_cast_per_tensor_workspace_bytes", "fp8q_block_dequant", "fp8q_block_dequant_grouped",
+    "fp8q_cast_per_tensor_workspace_bytes", "fp8q_cast_per_tensor_noalloc", "fp8q_block_dequant", "fp8q_block_dequant_grouped",
     "fp8q_cast_from_fp8", "fp8q_status_string", "fp8q_version",
     "per_token_cast_to_fp8", "per_token_cast_back", "cast_to_fp8", "cast_from_fp8", "weight_dequant",
 ]
@@ -217,6 +217,26 @@ def fp8q_cast_per_tensor(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tens
         _dev_ptr(x, "x"), _dtype_code(x, "x"), n, _fmt_of(fmt), _dev_ptr(q, "q", dev),
         _dev_ptr(scale_inv, "scale_inv", dev), _dev_ptr(workspace, "workspace", dev), wbytes,
         _stream(stream, dev)), "fp8q_cast_per_tensor")
+
+
+def fp8q_cast_per_tensor_noalloc(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
+                                 fmt=E4M3FN, stream=None) -> None:
+    """Per-tensor cast with the library's own static scratch (no workspace argument).
+
+    For callers that cannot allocate device memory.  Calls that overlap on the
+    GPU share the scratch and race; the first call on a device sets it up."""
+    L = lib()
+    f = L.fp8q_cast_per_tensor_noalloc
+    if f.argtypes is None:
+        p = ctypes.c_void_p
+        f.restype = ctypes.c_int
+        f.argtypes = [p, ctypes.c_int, ctypes.c_int64, ctypes.c_int, p, p, p]
+    dev = x.device
+    n = x.numel()
+    _need(q, n, "q", byte=True)
+    _need(scale_inv, 1, "scale_inv", dtype=torch.float32)
+    _check(f(_dev_ptr(x, "x"), _dtype_code(x, "x"), n, _fmt_of(fmt), _dev_ptr(q, "q", dev),
+             _dev_ptr(scale_inv, "scale_inv", dev), _stream(stream, dev)), "fp8q_cast_per_tensor_noalloc")
 
 
 def fp8q_block_dequant(w: torch.Tensor, scale_inv: torch.Tensor, y: torch.Tensor, block: int = 128,

@@ -140,6 +140,31 @@ fp8q_status fp8q_cast_per_tensor(const void* x, fp8q_dtype xt, int64_t numel, fp
                                  size_t workspace_bytes, fp8q_stream_t stream);
 
 /*
+ * Per-tensor cast without a caller workspace.  The paper has no counterpart:
+ * this entry point is a convenience of this library, not part of the method.
+ * Same computation and bytes as fp8q_cast_per_tensor, for callers that
+ * cannot allocate device memory -- for example code running under an
+ * allocator that owns all of the GPU's memory, or code that must not call
+ * cudaMalloc because that call may synchronise the device.  The scratch for
+ * the amax pass lives in a file-scope __device__ array inside the library:
+ * 8 KiB (2048 per-CTA partial maxima), present on every GPU that loads the
+ * library until the process exits.  Every tensor size fits, because the
+ * amax pass never uses more than 2048 CTAs; a launch that would need more
+ * slots than the array holds is refused with FP8Q_ERR_WORKSPACE.
+ * - The call allocates nothing (no cudaMalloc / cudaFree).  The first call on
+ *   a device looks up the array's device address on that device (with it
+ *   current) and caches it; make that first call before any stream capture.
+ * - All calls share the one array per device, and it keeps the last call's
+ *   contents; nothing needs clearing, since each call writes every slot it
+ *   reads.  Calls whose work overlaps on the GPU (different streams, no
+ *   ordering between them) race on the array and may give wrong results;
+ *   order them on one stream or synchronise.
+ * Arguments, errors and empty-tensor rule as fp8q_cast_per_tensor.
+ */
+fp8q_status fp8q_cast_per_tensor_noalloc(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt,
+                                         uint8_t* q, float* scale_inv, fp8q_stream_t stream);
+
+/*
  * Block dequantisation -- DeepSeek-V3 weight_dequant / weight_dequant_kernel:
  *   y[i][j] = T(fl(float(w[i][j]) * scale_inv[i / B][j / B]))
  *   with scale_inv row-major [ceil(M/B)][ceil(N/B)] (the kernel's
