@@ -1,0 +1,111 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point that include/fp8q.h declares, and rejects bad arguments on the host
+before any CUDA call (no compute is attempted here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8q.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8q_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from dequantisation_fp8q_token_b200 import build
+    build.build()
+    import dequantisation_fp8q_token_b200 as fp8q
+    return fp8q.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in fp8q.h but not exported"
+
+
+def test_binding_names_match_the_c_names():
+    import dequantisation_fp8q_token_b200 as fp8q
+    for n in declared_functions():
+        assert hasattr(fp8q, n), f"binding lacks {n}"
+
+
+def test_enum_values_match_the_binding():
+    import dequantisation_fp8q_token_b200 as fp8q
+    src = open(HEADER).read()
+    for name, val in [("FP8Q_E4M3FN", fp8q.E4M3FN), ("FP8Q_E5M2", fp8q.E5M2), ("FP8Q_F32", fp8q.F32),
+                      ("FP8Q_F16", fp8q.F16), ("FP8Q_BF16", fp8q.BF16), ("FP8Q_GRAN_TENSOR", fp8q.GRAN_TENSOR),
+                      ("FP8Q_GRAN_ROW", fp8q.GRAN_ROW), ("FP8Q_GRAN_GROUP", fp8q.GRAN_GROUP),
+                      ("FP8Q_GRAN_BLOCK", fp8q.GRAN_BLOCK)]:
+        assert re.search(rf"\b{name}\s*=\s*{val}\b", src), name
+
+
+def test_status_strings(L):
+    import dequantisation_fp8q_token_b200 as fp8q
+    for code in range(10):
+        s = fp8q.fp8q_status_string(code)
+        assert s.startswith("FP8Q_")
+    assert "UNKNOWN" in fp8q.fp8q_status_string(99)
+    assert fp8q.fp8q_version() == 10000
+    assert fp8q.fp8q_cast_per_tensor_workspace_bytes() == 8192
+
+
+# host-side validation: each of these returns before the library touches CUDA
+P = 0x1000   # a fake, never-dereferenced pointer value
+
+
+def test_per_token_validation(L):
+    f = L.fp8q_per_token_group_quant
+    assert f(P, 7, 4, 128, 128, 0, P, P, None) == 2             # dtype
+    assert f(P, 2, 4, 128, 128, 9, P, P, None) == 3             # format
+    assert f(P, 2, 4, 130, 128, 0, P, P, None) == 4             # n % group
+    assert f(P, 2, -1, 128, 128, 0, P, P, None) == 4            # negative size
+    assert f(P, 2, 4, 128, 0, 0, P, P, None) == 4               # group < 1
+    assert f(None, 2, 4, 128, 128, 0, P, P, None) == 1          # null x
+    assert f(P, 2, 4, 128, 128, 0, P, None, None) == 1          # null scale_inv
+    assert f(P + 1, 2, 4, 128, 128, 0, P, P, None) == 5         # bf16 pointer on an odd address
+    assert f(None, 2, 0, 128, 128, 0, None, None, None) == 0    # empty: nothing to do
+
+
+def test_per_channel_and_tensor_validation(L):
+    assert L.fp8q_cast_per_channel(P, 3, 4, 4, 0, P, P, None) == 2
+    assert L.fp8q_cast_per_channel(P, 0, 4, 4, 2, P, P, None) == 3
+    assert L.fp8q_cast_per_channel(P, 0, -4, 4, 0, P, P, None) == 4
+    assert L.fp8q_cast_per_channel(P, 0, 4, 4, 0, P, None, None) == 1
+    assert L.fp8q_cast_per_channel(P + 2, 0, 4, 4, 0, P, P, None) == 5
+    assert L.fp8q_cast_per_tensor(P, 0, 16, 0, P, P, None, 8192, None) == 6
+    assert L.fp8q_cast_per_tensor(P, 0, 16, 0, P, P, P, 100, None) == 6
+    assert L.fp8q_cast_per_tensor(P, 0, 16, 0, P, P, P + 4, 8192, None) == 6
+    assert L.fp8q_cast_per_tensor(P, 0, -1, 0, P, P, P, 8192, None) == 4
+    assert L.fp8q_cast_per_tensor(None, 0, 16, 0, P, P, P, 8192, None) == 1
+    f = L.fp8q_cast_per_tensor_noalloc
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    assert f(P, 5, 16, 0, P, P, None) == 2
+    assert f(P, 0, 16, 4, P, P, None) == 3
+    assert f(None, 0, 16, 0, P, P, None) == 1
+    assert f(P + 1, 0, 16, 0, P, P, None) == 5
+
+
+def test_dequant_validation(L):
+    assert L.fp8q_block_dequant(P, 2, 4, 4, P, 128, 0, P, None) == 3
+    assert L.fp8q_block_dequant(P, 0, 4, 4, P, 128, 5, P, None) == 2
+    assert L.fp8q_block_dequant(P, 0, 4, 4, P, 0, 0, P, None) == 4
+    assert L.fp8q_block_dequant(P, 0, -4, 4, P, 128, 0, P, None) == 4
+    assert L.fp8q_block_dequant(None, 0, 4, 4, P, 128, 0, P, None) == 1
+    assert L.fp8q_block_dequant(P, 0, 4, 4, P + 2, 128, 0, P, None) == 5
+    assert L.fp8q_block_dequant_grouped(None, -1, 0, 128, 2, None) == 9
+    assert L.fp8q_block_dequant_grouped(None, 0, 0, 128, 2, None) == 0
+    assert L.fp8q_block_dequant_grouped(None, 3, 0, 128, 2, None) == 1
+    assert L.fp8q_cast_from_fp8(P, 0, 4, 4, P, 4, 0, 2, P, None) == 8
+    assert L.fp8q_cast_from_fp8(P, 0, 4, 6, P, 2, 4, 2, P, None) == 4
+    assert L.fp8q_cast_from_fp8(P, 0, 4, 8, P, 3, 0, 2, P, None) == 4
+    assert L.fp8q_cast_from_fp8(P, 0, 4, 8, None, 1, 0, 2, P, None) == 1
