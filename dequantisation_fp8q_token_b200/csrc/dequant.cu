@@ -4,13 +4,14 @@
 // cast_from_fp8 / DeepEP per_token_cast_back (tensor, row and 1 x G groups).
 //
 // Work decomposition: each problem is cut into tiles of kRowsPerTile rows by
-// 32 chunks of V consecutive elements (V = 16, 8, 4, 2 or 1, the widest that
-// the row length and pointer alignment allow).  A CTA of 8 warps owns one
-// tile: warp w handles rows w, w + 8, ..., lane l the l-th chunk, so every
-// warp-wide access is 32 * V contiguous codes (512 bytes at V = 16) and the
-// bf16 stores 1 KiB.  Each thread issues its kUnroll row loads before
-// converting any of them.  Problems of one launch (a checkpoint's weights,
-// a mixture-of-experts layer) share the grid through a descriptor table in
+// 32 chunks of V consecutive elements (V = 32, 16, 8, 4, 2 or 1, the widest
+// that the row length, granule edge and pointer alignment allow).  A CTA of 8
+// warps owns one tile: warp w handles rows w, w + 8, ..., lane l the l-th
+// chunk, so at V = 32 every warp-wide load is one 256-bit access per lane
+// (1 KiB of contiguous codes) and each lane writes its 32 bf16 outputs with
+// two 256-bit stores.  Each thread issues its kUnroll row loads before
+// converting any of them.  Problems of one launch (a checkpoint's weights, a
+// mixture-of-experts layer) share the grid through a descriptor table in
 // kernel-parameter space; a CTA finds its problem by binary search over the
 // first-tile prefix, so heterogeneous shapes need no device-side metadata.
 //
@@ -24,7 +25,13 @@ namespace {
 
 constexpr int kDqThreads = 256;
 constexpr int kDqWarps = kDqThreads / 32;
-constexpr int kUnroll = 4;
+#ifndef FP8Q_DQ_UNROLL
+#define FP8Q_DQ_UNROLL 2
+#endif
+#ifndef FP8Q_DQ_V32
+#define FP8Q_DQ_V32 1  // 32-code chunks with 256-bit loads / stores where aligned
+#endif
+constexpr int kUnroll = FP8Q_DQ_UNROLL;  // rows per thread per tile
 constexpr int kRowsPerTile = kDqWarps * kUnroll;  // 32
 constexpr int kMaxGroupedDescs = 96;
 
@@ -52,26 +59,58 @@ __device__ __forceinline__ uint32_t div_gb(uint32_t a, int gb, int gb_shift) {
     return gb_shift >= 0 ? (a >> gb_shift) : a / (uint32_t)gb;
 }
 
-// load V codes (V <= 16) as up to four 32-bit words
+// V codes (V <= 32) in up to eight 32-bit words, code i in byte i
+struct Chunk {
+    uint32_t w[8];
+};
+
 template <int V>
-__device__ __forceinline__ uint4 load_codes(const uint8_t* p) {
-    if (V == 16) return ld_stream_v4(p);
-    if (V == 8) {
+__device__ __forceinline__ Chunk load_codes(const uint8_t* p) {
+    Chunk c;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c.w[i] = 0u;
+    if (V == 32) {
+        const U8x32 t = ld_stream_v8(p);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) c.w[i] = t.w[i];
+    } else if (V == 16) {
+        const uint4 t = ld_stream_v4(p);
+        c.w[0] = t.x; c.w[1] = t.y; c.w[2] = t.z; c.w[3] = t.w;
+    } else if (V == 8) {
         const uint2 t = ld_stream_v2(p);
-        return make_uint4(t.x, t.y, 0u, 0u);
+        c.w[0] = t.x; c.w[1] = t.y;
+    } else if (V == 4) {
+        c.w[0] = ld_stream_u32(p);
+    } else if (V == 2) {
+        c.w[0] = *reinterpret_cast<const uint16_t*>(p);
+    } else {
+        c.w[0] = *p;
     }
-    if (V == 4) return make_uint4(ld_stream_u32(p), 0u, 0u, 0u);
-    if (V == 2) return make_uint4(*reinterpret_cast<const uint16_t*>(p), 0u, 0u, 0u);
-    return make_uint4(*p, 0u, 0u, 0u);
+    return c;
 }
 
 // convert and store V outputs starting at element offset e of y
 template <int FMT, int YT, int V>
-__device__ __forceinline__ void convert_store(uint4 c, float sc, void* y, int64_t e) {
-    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+__device__ __forceinline__ void convert_store(const Chunk& c, float sc, void* y, int64_t e) {
+    const uint32_t* w = c.w;
     if (YT == kF32) {
         float* yf = static_cast<float*>(y) + e;
-        if (V >= 4) {
+        if (V == 32) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float2 a = dec2<FMT>(w[2 * h + i] & 0xFFFFu);
+                    const float2 b = dec2<FMT>(w[2 * h + i] >> 16);
+                    o[4 * i + 0] = __float_as_uint(__fmul_rn(a.x, sc));
+                    o[4 * i + 1] = __float_as_uint(__fmul_rn(a.y, sc));
+                    o[4 * i + 2] = __float_as_uint(__fmul_rn(b.x, sc));
+                    o[4 * i + 3] = __float_as_uint(__fmul_rn(b.y, sc));
+                }
+                st_v8(yf + 8 * h, o);
+            }
+        } else if (V >= 4) {
 #pragma unroll
             for (int i = 0; i < V / 4; ++i) {
                 const float2 a = dec2<FMT>(w[i] & 0xFFFFu);
@@ -88,7 +127,20 @@ __device__ __forceinline__ void convert_store(uint4 c, float sc, void* y, int64_
         }
     } else {
         uint16_t* yh = static_cast<uint16_t*>(y) + e;
-        if (V >= 8) {
+        if (V == 32) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 a = dec2<FMT>(w[4 * h + i] & 0xFFFFu);
+                    const float2 b = dec2<FMT>(w[4 * h + i] >> 16);
+                    o[2 * i] = pack2<YT>(__fmul_rn(a.x, sc), __fmul_rn(a.y, sc));
+                    o[2 * i + 1] = pack2<YT>(__fmul_rn(b.x, sc), __fmul_rn(b.y, sc));
+                }
+                st_v8(yh + 16 * h, o);
+            }
+        } else if (V >= 8) {
 #pragma unroll
             for (int i = 0; i < V / 8; ++i) {
                 uint32_t o[4];
@@ -127,11 +179,11 @@ __device__ __forceinline__ void dequant_tile(const DqDesc& D, int gb, int gb_shi
     const int64_t r0 = tr * kRowsPerTile + warp;
     const uint8_t* q = D.q;
     const float* s = D.s;
-    uint4 codes[kUnroll];
+    Chunk codes[kUnroll];
 #pragma unroll
     for (int k = 0; k < kUnroll; ++k) {
         const int64_t r = r0 + (int64_t)k * kDqWarps;
-        codes[k] = r < rows ? load_codes<V>(q + r * cols + c) : make_uint4(0u, 0u, 0u, 0u);
+        if (r < rows) codes[k] = load_codes<V>(q + r * cols + c);
     }
     // scale index pieces that do not depend on the row
     int64_t s_cols = 0, s_col = 0;
@@ -158,6 +210,7 @@ __device__ __forceinline__ void dequant_tile(const DqDesc& D, int gb, int gb_shi
 
 template <int FMT, int YT, int GRAN, int N>
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(const __grid_constant__ DqParams<N> p) {
+    pdl_begin();
     const int64_t tile = blockIdx.x;
     int lo = 0;
     if (N > 1) {
@@ -173,6 +226,9 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(const __grid_consta
     const int64_t tr = t / D.tiles_per_row;
     const int tc = (int)(t - tr * D.tiles_per_row);
     switch (D.vshift) {
+#if FP8Q_DQ_V32
+    case 5: dequant_tile<FMT, YT, GRAN, 32>(D, p.gb, p.gb_shift, tr, tc); break;
+#endif
     case 4: dequant_tile<FMT, YT, GRAN, 16>(D, p.gb, p.gb_shift, tr, tc); break;
     case 3: dequant_tile<FMT, YT, GRAN, 8>(D, p.gb, p.gb_shift, tr, tc); break;
     case 2: dequant_tile<FMT, YT, GRAN, 4>(D, p.gb, p.gb_shift, tr, tc); break;
@@ -184,12 +240,13 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(const __grid_consta
 // widest chunk V such that rows start V-aligned, the chunk never crosses a
 // granule, and loads / stores of the chunk are naturally aligned
 int choose_vshift(const DequantProblem& P, int gran, int gb, int ybytes) {
-    for (int vs = 4; vs > 0; --vs) {
+    for (int vs = FP8Q_DQ_V32 ? 5 : 4; vs > 0; --vs) {
         const int V = 1 << vs;
         if (P.cols % V) continue;
         if ((gran == kGranGroup || gran == kGranBlock) && gb % V) continue;
         if ((uintptr_t)P.q % V) continue;
-        const int ystore = V * ybytes < 16 ? V * ybytes : 16;
+        const int widest = V == 32 ? 32 : 16;  // 256-bit stores only at V = 32
+        const int ystore = V * ybytes < widest ? V * ybytes : widest;
         if ((uintptr_t)P.y % ystore) continue;
         return vs;
     }
@@ -226,19 +283,26 @@ fp8q_status run_batch(const DequantProblem* probs, int count, int gb, cudaStream
     }
     if (p.count == 0) return FP8Q_OK;
     if (tiles > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
-    dequant_kernel<FMT, YT, GRAN, N><<<(unsigned)tiles, kDqThreads, 0, s>>>(p);
-    return cuda_status(cudaGetLastError());
+    const cudaError_t err = launch_kernel(dequant_kernel<FMT, YT, GRAN, N>, dim3((unsigned)tiles), dim3(kDqThreads), s, p);
+    return cuda_status(err);
 }
 
 template <int FMT, int YT, int GRAN>
 fp8q_status run_all(const DequantProblem* probs, int count, int gb, cudaStream_t s) {
-    if (count == 1) return run_batch<FMT, YT, GRAN, 1>(probs, 1, gb, s);
-    for (int i = 0; i < count; i += kMaxGroupedDescs) {
-        const int n = count - i < kMaxGroupedDescs ? count - i : kMaxGroupedDescs;
-        fp8q_status st = run_batch<FMT, YT, GRAN, kMaxGroupedDescs>(probs + i, n, gb, s);
-        if (st != FP8Q_OK) return st;
+    if constexpr (GRAN != kGranBlock) {
+        // only block dequant takes several problems per call
+        fp8q_status st = FP8Q_OK;
+        for (int i = 0; i < count && st == FP8Q_OK; ++i) st = run_batch<FMT, YT, GRAN, 1>(probs + i, 1, gb, s);
+        return st;
+    } else {
+        if (count == 1) return run_batch<FMT, YT, GRAN, 1>(probs, 1, gb, s);
+        for (int i = 0; i < count; i += kMaxGroupedDescs) {
+            const int n = count - i < kMaxGroupedDescs ? count - i : kMaxGroupedDescs;
+            fp8q_status st = run_batch<FMT, YT, GRAN, kMaxGroupedDescs>(probs + i, n, gb, s);
+            if (st != FP8Q_OK) return st;
+        }
+        return FP8Q_OK;
     }
-    return FP8Q_OK;
 }
 
 template <int FMT, int YT>

@@ -16,6 +16,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#ifndef FP8Q_PDL
+#define FP8Q_PDL 0
+#endif
+
 namespace fp8q {
 
 enum : int { kE4M3 = 0, kE5M2 = 1 };
@@ -26,6 +30,21 @@ template <int XT> struct ElemBytes { static constexpr int value = XT == kF32 ? 4
 
 template <int FMT> __device__ __forceinline__ float fp8_max() {
     return FMT == kE4M3 ? 448.0f : 57344.0f;
+}
+
+// ---------------------------------------------------------------------------
+// programmatic dependent launch.  Every kernel calls pdl_begin() before it
+// touches global memory: it lets the next kernel on the stream be scheduled
+// once all of this grid's CTAs have started (so the next grid only fills SMs
+// that this one's tail leaves idle), then waits until the previous grid on
+// the stream has completed and its writes are visible.  Without a
+// programmatic predecessor the wait returns at once.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_begin() {
+#if FP8Q_PDL
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
 }
 
 // ---------------------------------------------------------------------------
@@ -47,6 +66,39 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
     uint32_t r;
     asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
     return r;
+}
+// L2 eviction-priority policies (createpolicy) and a streaming load that
+// carries one: evict_last keeps a line in L2 ahead of normal traffic,
+// evict_first lets it go first.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint4 ld_stream_v4_policy(const void* p, uint64_t policy) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p), "l"(policy));
+    return r;
+}
+// 256-bit accesses (sm_100): 32 contiguous bytes per thread, 32-byte aligned
+struct U8x32 { uint32_t w[8]; };
+__device__ __forceinline__ U8x32 ld_stream_v8(const void* p) {
+    U8x32 r;
+    asm("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]),
+          "=r"(r.w[4]), "=r"(r.w[5]), "=r"(r.w[6]), "=r"(r.w[7]) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ void st_v8(void* p, const uint32_t (&w)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :: "l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]),
+                    "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]) : "memory");
 }
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};"
@@ -139,6 +191,39 @@ template <int FMT> __device__ __forceinline__ uint32_t enc2(float lo, float hi) 
     return r;
 }
 
+// four fp32 -> four fp8 codes in one word, a in bits 0..7 ... d in bits 24..31
+template <int FMT> __device__ __forceinline__ uint32_t enc4(float a, float b, float c, float d) {
+    uint32_t r;
+    if (FMT == kE4M3)
+        asm("{\n.reg .b16 lo, hi;\n"
+            "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n"
+            "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n"
+            "mov.b32 %0, {lo, hi};\n}"
+            : "=r"(r) : "f"(a), "f"(b), "f"(c), "f"(d));
+    else
+        asm("{\n.reg .b16 lo, hi;\n"
+            "cvt.rn.satfinite.e5m2x2.f32 lo, %2, %1;\n"
+            "cvt.rn.satfinite.e5m2x2.f32 hi, %4, %3;\n"
+            "mov.b32 %0, {lo, hi};\n}"
+            : "=r"(r) : "f"(a), "f"(b), "f"(c), "f"(d));
+    return r;
+}
+
+// Magnitude maxima that propagate NaN, on packed 16-bit pairs or fp32:
+// max.NaN.xorsign.abs returns max(|a|, |b|) (NaN if either is NaN) with a
+// sign bit we discard, so callers mask the result with 0x7FFF7FFF / 0x7FFFFFFF.
+template <int XT> __device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    if (XT == kBF16)
+        asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    else if (XT == kF16)
+        asm("max.NaN.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    else
+        asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(*reinterpret_cast<float*>(&d))
+            : "f"(__uint_as_float(a)), "f"(__uint_as_float(b)));
+    return d;
+}
+
 // non-saturating semantics for one value given the hardware code c:
 //   NaN -> NaN code (sign kept); e4m3fn: |v| > 464 (incl. Inf) -> NaN;
 //   e5m2: |v| >= 61440 (incl. Inf) -> Inf.
@@ -187,6 +272,90 @@ template <int YT> __device__ __forceinline__ uint32_t pack2(float lo, float hi) 
         __half2 h = __floats2half2_rn(lo, hi);
         return *reinterpret_cast<uint32_t*>(&h);
     }
+}
+
+// ---------------------------------------------------------------------------
+// VB-byte vectors of high-precision elements (VB = 16 or 32)
+// ---------------------------------------------------------------------------
+template <int VB>
+struct Vec {
+    uint32_t w[VB / 4];
+};
+
+template <int VB>
+__device__ __forceinline__ Vec<VB> load_vec(const uint8_t* p) {
+    Vec<VB> v;
+    if constexpr (VB == 32) {
+        const U8x32 t = ld_stream_v8(p);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v.w[i] = t.w[i];
+    } else {
+        const uint4 t = ld_stream_v4(p);
+        v.w[0] = t.x; v.w[1] = t.y; v.w[2] = t.z; v.w[3] = t.w;
+    }
+    return v;
+}
+
+template <int VB>
+__device__ __forceinline__ Vec<VB> load_vec_policy(const uint8_t* p, uint64_t policy) {
+    Vec<VB> v;
+    if constexpr (VB == 32) {
+        asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
+            : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]),
+              "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7]) : "l"(p), "l"(policy));
+    } else {
+        const uint4 t = ld_stream_v4_policy(p, policy);
+        v.w[0] = t.x; v.w[1] = t.y; v.w[2] = t.z; v.w[3] = t.w;
+    }
+    return v;
+}
+
+// unmasked NaN-propagating magnitude maximum over a vector (see absmax2)
+template <int XT, int VB>
+__device__ __forceinline__ uint32_t vec_absmax(const Vec<VB>& v) {
+    uint32_t t = absmax2<XT>(v.w[0], v.w[1]);
+#pragma unroll
+    for (int i = 2; i < VB / 4; ++i) t = absmax2<XT>(t, v.w[i]);
+    return t;
+}
+
+// result of absmax2 reductions -> fp32 magnitude bits
+template <int XT>
+__device__ __forceinline__ uint32_t absmax_bits(uint32_t m) {
+    if (XT == kF32) return m & 0x7FFFFFFFu;
+    return packed16_to_f32bits<XT>(m & 0x7FFF7FFFu);
+}
+
+// codes of one vector scaled by `scale`, stored in one access of VB / ES bytes;
+// FIX applies the non-saturating NaN / Inf rules to every element
+template <int XT, int FMT, int VB, bool FIX>
+__device__ __forceinline__ void encode_store_vec(const Vec<VB>& v, float scale, uint8_t* dst) {
+    constexpr int WPV = VB / 4;
+    constexpr int NC = XT == kF32 ? WPV / 4 : WPV / 2;  // 32-bit words of codes
+    uint32_t c[NC];
+    if (XT == kF32) {
+#pragma unroll
+        for (int i = 0; i < NC; ++i) {
+            const float a = __fmul_rn(__uint_as_float(v.w[4 * i]), scale);
+            const float b = __fmul_rn(__uint_as_float(v.w[4 * i + 1]), scale);
+            const float d = __fmul_rn(__uint_as_float(v.w[4 * i + 2]), scale);
+            const float e = __fmul_rn(__uint_as_float(v.w[4 * i + 3]), scale);
+            c[i] = FIX ? (enc2_sem<FMT, true>(a, b) | (enc2_sem<FMT, true>(d, e) << 16)) : enc4<FMT>(a, b, d, e);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < NC; ++i) {
+            float a0, a1, b0, b1;
+            widen2<XT>(v.w[2 * i], a0, a1);
+            widen2<XT>(v.w[2 * i + 1], b0, b1);
+            const float a = __fmul_rn(a0, scale), b = __fmul_rn(a1, scale);
+            const float d = __fmul_rn(b0, scale), e = __fmul_rn(b1, scale);
+            c[i] = FIX ? (enc2_sem<FMT, true>(a, b) | (enc2_sem<FMT, true>(d, e) << 16)) : enc4<FMT>(a, b, d, e);
+        }
+    }
+    if constexpr (NC == 4) st_v4(dst, make_uint4(c[0], c[1], c[2], c[3]));
+    else if constexpr (NC == 2) st_v2(dst, make_uint2(c[0], c[1]));
+    else st_u32(dst, c[0]);
 }
 
 __host__ __device__ constexpr int ilog2c(int v) { return v <= 1 ? 0 : 1 + ilog2c(v / 2); }

@@ -6,6 +6,10 @@
 
 #include "fp8q.h"
 
+#ifndef FP8Q_PDL
+#define FP8Q_PDL 0
+#endif
+
 namespace fp8q {
 
 // per-CTA partial maxima of the per-tensor amax pass
@@ -14,6 +18,38 @@ constexpr size_t kPerTensorWorkspaceBytes = kMaxPartials * sizeof(uint32_t);
 
 // number of SMs of the current device (cached per device)
 int sm_count();
+
+// CTAs of `kernel` with `threads` threads that fit on one SM at once (>= 1)
+template <typename Kernel>
+int resident_blocks_per_sm(Kernel kernel, int threads) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1) n = 1;
+    return n;
+}
+
+// Launch `kernel` on `s`; with FP8Q_PDL the launch may overlap the previous
+// kernel's tail (programmatic stream serialization: the kernel's own
+// pdl_begin() waits for that kernel to finish before touching memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+#if FP8Q_PDL
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+#else
+    (void)attr;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+#endif
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 fp8q_status launch_per_token(const void* x, int xt, int64_t m, int64_t n, int group, int fmt,
                              uint8_t* q, float* sinv, cudaStream_t s);

@@ -6,14 +6,21 @@
 // elements [g*G, (g+1)*G) of x and q and owns scale_inv[g]; the kernel walks
 // groups as one flat sequence.
 //
-// Vector kernel: a group is held by LANES = min(32, G / EPV) consecutive
-// lanes, each with VPL 16-byte vectors (EPV elements per vector).  For the
-// pages' bf16 G = 128 that is a half warp with one 16-byte load per lane:
-// every warp-wide load covers 512 contiguous bytes.  Each thread keeps
-// kTokUnroll groups' loads in flight before reducing, the amax is an
-// integer max on magnitude bits (NaN-propagating) finished with xor
-// shuffles inside the lane segment, and each lane stores its EPV codes in
-// one store.
+// Vector kernel: a group is held by LANES consecutive lanes, each with VPL
+// vectors of VB bytes (EPV elements each); vector j of lane l covers
+// elements (j * LANES + l) * EPV .. + EPV of its group, so every warp-wide
+// load is LANES * VB contiguous bytes per group and uses whole sectors.  For
+// the pages' bf16 G = 128 with 256-bit loads (VB = 32) that is 8 lanes x one
+// vector: a warp holds 4 groups, each warp-wide load 4 x 256 contiguous bytes.
+//   - amax: NaN-propagating magnitude max (packed for 16-bit types), then
+//     xor shuffles inside the lane segment;
+//   - scales: the warp's SEGS amaxes are gathered into lanes 0..SEGS-1, so
+//     the two IEEE divisions run once per warp for all its groups; each lane
+//     then fetches its group's scale, and lanes 0..SEGS-1 store SEGS
+//     consecutive scale_inv values in one coalesced store;
+//   - encode: four fp32 products -> one 32-bit word of codes, one store per
+//     vector.
+// Each CTA loads kTokUnroll batches of GPB groups before converting any.
 #include "fp8q_device.cuh"
 #include "fp8q_internal.h"
 
@@ -21,97 +28,97 @@ namespace fp8q {
 namespace {
 
 constexpr int kTokThreads = 256;
-constexpr int kTokUnroll = 4;
+#ifndef FP8Q_TOK_UNROLL
+#define FP8Q_TOK_UNROLL 2
+#endif
+#ifndef FP8Q_TOK_VPL
+#define FP8Q_TOK_VPL 1
+#endif
+#ifndef FP8Q_TOK_V32
+#define FP8Q_TOK_V32 1  // 32-byte vectors (256-bit loads) where the pointers allow
+#endif
+constexpr int kTokUnroll = FP8Q_TOK_UNROLL;  // batches per CTA
+constexpr int kTokVpl = FP8Q_TOK_VPL;        // target vectors per lane per group
 
-template <int XT, int G>
+template <int XT, int G, int VB>
 struct TokCfg {
     static constexpr int ES = ElemBytes<XT>::value;
-    static constexpr int EPV = 16 / ES;
-    static constexpr int LANES = (G / EPV) < 32 ? (G / EPV) : 32;
-    static constexpr int VPL = G / (EPV * LANES);
-    static constexpr int SEGS = 32 / LANES;
-    static constexpr int GPI = (kTokThreads / 32) * SEGS;  // groups per CTA iteration
-    static constexpr int GPC = GPI * kTokUnroll;            // groups per CTA
+    static constexpr int EPV = VB / ES;                    // elements per vector (VB bytes)
+    static constexpr int NV = G / EPV;                     // vectors per group
+    static constexpr int LANES = NV / kTokVpl < 1 ? 1 : (NV / kTokVpl > 32 ? 32 : NV / kTokVpl);
+    static constexpr int VPL = NV / LANES;                 // vectors per lane
+    static constexpr int SEGS = 32 / LANES;                // groups per warp
+    static constexpr int GPB = (kTokThreads / 32) * SEGS;  // groups per CTA batch
+    static constexpr int WPV = VB / 4;                     // 32-bit words per vector
 };
 
-// encode one 16-byte input vector (already widened on the fly) and store its codes
-template <int XT, int FMT, bool FIX>
-__device__ __forceinline__ void encode_store_vec(uint4 v, float scale, uint8_t* dst) {
-    if (XT == kF32) {
-        const float f0 = __fmul_rn(__uint_as_float(v.x), scale);
-        const float f1 = __fmul_rn(__uint_as_float(v.y), scale);
-        const float f2 = __fmul_rn(__uint_as_float(v.z), scale);
-        const float f3 = __fmul_rn(__uint_as_float(v.w), scale);
-        st_u32(dst, enc2_sem<FMT, FIX>(f0, f1) | (enc2_sem<FMT, FIX>(f2, f3) << 16));
-    } else {
-        float a0, a1, b0, b1, c0, c1, d0, d1;
-        widen2<XT>(v.x, a0, a1);
-        widen2<XT>(v.y, b0, b1);
-        widen2<XT>(v.z, c0, c1);
-        widen2<XT>(v.w, d0, d1);
-        const uint32_t w0 = enc2_sem<FMT, FIX>(__fmul_rn(a0, scale), __fmul_rn(a1, scale)) |
-                            (enc2_sem<FMT, FIX>(__fmul_rn(b0, scale), __fmul_rn(b1, scale)) << 16);
-        const uint32_t w1 = enc2_sem<FMT, FIX>(__fmul_rn(c0, scale), __fmul_rn(c1, scale)) |
-                            (enc2_sem<FMT, FIX>(__fmul_rn(d0, scale), __fmul_rn(d1, scale)) << 16);
-        st_v2(dst, make_uint2(w0, w1));
+template <int XT, int G, int VB>
+__device__ __forceinline__ void load_batch(const uint8_t* __restrict__ x, int64_t ngroups, int64_t bt,
+                                           int gw, int sl, Vec<VB> (&v)[TokCfg<XT, G, VB>::VPL]) {
+    using C = TokCfg<XT, G, VB>;
+    const int64_t g = bt * C::GPB + gw;
+#pragma unroll
+    for (int j = 0; j < C::VPL; ++j) {
+        const int64_t e = g * G + (int64_t)(j * C::LANES + sl) * C::EPV;
+        if (g < ngroups) v[j] = load_vec<VB>(x + e * C::ES);
+        else
+#pragma unroll
+            for (int i = 0; i < C::WPV; ++i) v[j].w[i] = 0u;
     }
 }
 
-template <int XT, int FMT, int G>
+template <int XT, int FMT, int G, int VB>
+__device__ __forceinline__ void process_batch(const Vec<VB> (&v)[TokCfg<XT, G, VB>::VPL], uint8_t* __restrict__ q,
+                                              float* __restrict__ sinv, int64_t ngroups, int64_t bt,
+                                              int seg, int sl, int lane, int warp) {
+    using C = TokCfg<XT, G, VB>;
+    // magnitude maximum of this lane's elements
+    uint32_t m = vec_absmax<XT, VB>(v[0]);
+#pragma unroll
+    for (int j = 1; j < C::VPL; ++j) m = absmax2<XT>(m, vec_absmax<XT, VB>(v[j]));
+#pragma unroll
+    for (int off = C::LANES / 2; off > 0; off >>= 1) m = absmax2<XT>(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    const uint32_t bits = absmax_bits<XT>(m);
+    // the warp's SEGS scales, one group per lane, computed once
+    float amax = __uint_as_float(__shfl_sync(0xFFFFFFFFu, bits, (lane % C::SEGS) * C::LANES));
+    if (amax < 1e-4f) amax = 1e-4f;  // clamp(1e-4); a NaN amax stays NaN
+    const float scale_l = __fdiv_rn(fp8_max<FMT>(), amax);
+    const float sinv_l = __fdiv_rn(amax, fp8_max<FMT>());
+    const float scale = __shfl_sync(0xFFFFFFFFu, scale_l, seg);
+    const int64_t gbase = bt * C::GPB + (int64_t)warp * C::SEGS;
+    if (lane < C::SEGS && gbase + lane < ngroups) sinv[gbase + lane] = sinv_l;
+    // finite x with a finite scale never overflows, and NaN/Inf inputs give
+    // NaN or zero products: the hardware codes are already final
+    const int64_t g = gbase + seg;
+    if (g < ngroups) {
+#pragma unroll
+        for (int j = 0; j < C::VPL; ++j) {
+            const int64_t e = g * G + (int64_t)(j * C::LANES + sl) * C::EPV;
+            encode_store_vec<XT, FMT, VB, false>(v[j], scale, q + e);
+        }
+    }
+}
+
+// one CTA per kTokUnroll consecutive batches: all their loads are issued
+// before any batch is converted
+template <int XT, int FMT, int G, int VB>
 __global__ void __launch_bounds__(kTokThreads)
 per_token_vec_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
-                     float* __restrict__ sinv, int64_t ngroups) {
-    using C = TokCfg<XT, G>;
-    constexpr int U = kTokUnroll;
+                     float* __restrict__ sinv, int64_t ngroups, int64_t nbatch) {
+    pdl_begin();
+    using C = TokCfg<XT, G, VB>;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int seg = lane / C::LANES;
     const int sl = lane % C::LANES;
-    const int64_t g0 = (int64_t)blockIdx.x * C::GPC + warp * C::SEGS + seg;
-
-    uint4 v[U][C::VPL];
+    const int gw = warp * C::SEGS + seg;
+    Vec<VB> v[kTokUnroll][C::VPL];
+    const int64_t b0 = (int64_t)blockIdx.x * kTokUnroll;
 #pragma unroll
-    for (int k = 0; k < U; ++k) {
-        const int64_t g = g0 + (int64_t)k * C::GPI;
+    for (int u = 0; u < kTokUnroll; ++u) load_batch<XT, G, VB>(x, ngroups, b0 + u, gw, sl, v[u]);
 #pragma unroll
-        for (int j = 0; j < C::VPL; ++j) {
-            const int64_t e = g * G + (int64_t)(j * C::LANES + sl) * C::EPV;
-            v[k][j] = g < ngroups ? ld_stream_v4(x + e * C::ES) : make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
-
-#pragma unroll
-    for (int k = 0; k < U; ++k) {
-        const int64_t g = g0 + (int64_t)k * C::GPI;
-        uint32_t m;
-        if (XT == kF32) {
-            m = 0u;
-#pragma unroll
-            for (int j = 0; j < C::VPL; ++j) m = max(m, vec_absmax_bits<kF32>(v[k][j]));
-        } else {
-            uint32_t p = 0u;
-#pragma unroll
-            for (int j = 0; j < C::VPL; ++j) p = max_u16x2(p, vec_absmax_packed16(v[k][j]));
-            m = packed16_to_f32bits<XT>(p);
-        }
-#pragma unroll
-        for (int off = C::LANES / 2; off > 0; off >>= 1)
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-
-        float amax = __uint_as_float(m);
-        if (amax < 1e-4f) amax = 1e-4f;  // clamp(1e-4); a NaN amax stays NaN
-        const float scale = __fdiv_rn(fp8_max<FMT>(), amax);
-        if (g < ngroups) {
-            if (sl == 0) sinv[g] = __fdiv_rn(amax, fp8_max<FMT>());
-            // finite x with a finite scale never overflows, and NaN/Inf inputs
-            // give NaN or zero products: the hardware codes are already final
-#pragma unroll
-            for (int j = 0; j < C::VPL; ++j) {
-                const int64_t e = g * G + (int64_t)(j * C::LANES + sl) * C::EPV;
-                encode_store_vec<XT, FMT, false>(v[k][j], scale, q + e);
-            }
-        }
-    }
+    for (int u = 0; u < kTokUnroll; ++u)
+        if (b0 + u < nbatch) process_batch<XT, FMT, G, VB>(v[u], q, sinv, ngroups, b0 + u, seg, sl, lane, warp);
 }
 
 // any group size dividing n, any element-aligned pointers: one warp per group
@@ -119,6 +126,7 @@ template <int XT, int FMT>
 __global__ void __launch_bounds__(256)
 per_token_generic_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
                          float* __restrict__ sinv, int64_t ngroups, int G) {
+    pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
     const int lane = threadIdx.x & 31;
     const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -140,14 +148,15 @@ per_token_generic_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
     }
 }
 
-template <int XT, int FMT, int G>
+template <int XT, int FMT, int G, int VB>
 fp8q_status run_vec(const void* x, uint8_t* q, float* sinv, int64_t ngroups, cudaStream_t s) {
-    using C = TokCfg<XT, G>;
-    const int64_t blocks = (ngroups + C::GPC - 1) / C::GPC;
-    if (blocks > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
-    per_token_vec_kernel<XT, FMT, G><<<(unsigned)blocks, kTokThreads, 0, s>>>(
-        static_cast<const uint8_t*>(x), q, sinv, ngroups);
-    return cuda_status(cudaGetLastError());
+    using C = TokCfg<XT, G, VB>;
+    const int64_t nbatch = (ngroups + C::GPB - 1) / C::GPB;
+    const int64_t grid = (nbatch + kTokUnroll - 1) / kTokUnroll;
+    if (grid > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
+    const cudaError_t err = launch_kernel(per_token_vec_kernel<XT, FMT, G, VB>, dim3((unsigned)grid), dim3(kTokThreads), s,
+                                          static_cast<const uint8_t*>(x), q, sinv, ngroups, nbatch);
+    return cuda_status(err);
 }
 
 template <int XT, int FMT>
@@ -155,34 +164,42 @@ fp8q_status run_generic(const void* x, uint8_t* q, float* sinv, int64_t ngroups,
                         cudaStream_t s) {
     const int64_t want = (ngroups + 7) / 8;
     const int blocks = (int)(want < (int64_t)sm_count() * 16 ? want : (int64_t)sm_count() * 16);
-    per_token_generic_kernel<XT, FMT><<<blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), q, sinv,
-                                                            ngroups, group);
-    return cuda_status(cudaGetLastError());
+    const cudaError_t err = launch_kernel(per_token_generic_kernel<XT, FMT>, dim3(blocks), dim3(256), s,
+                                          static_cast<const uint8_t*>(x), q, sinv, ngroups, group);
+    return cuda_status(err);
 }
 
-template <int XT, int FMT>
+template <int XT, int FMT, int VB>
 fp8q_status dispatch_group(const void* x, uint8_t* q, float* sinv, int64_t ngroups, int group,
                            cudaStream_t s) {
     switch (group) {
-    case 16: return run_vec<XT, FMT, 16>(x, q, sinv, ngroups, s);
-    case 32: return run_vec<XT, FMT, 32>(x, q, sinv, ngroups, s);
-    case 64: return run_vec<XT, FMT, 64>(x, q, sinv, ngroups, s);
-    case 128: return run_vec<XT, FMT, 128>(x, q, sinv, ngroups, s);
-    case 256: return run_vec<XT, FMT, 256>(x, q, sinv, ngroups, s);
-    case 512: return run_vec<XT, FMT, 512>(x, q, sinv, ngroups, s);
-    case 1024: return run_vec<XT, FMT, 1024>(x, q, sinv, ngroups, s);
+    case 16: return run_vec<XT, FMT, 16, VB>(x, q, sinv, ngroups, s);
+    case 32: return run_vec<XT, FMT, 32, VB>(x, q, sinv, ngroups, s);
+    case 64: return run_vec<XT, FMT, 64, VB>(x, q, sinv, ngroups, s);
+    case 128: return run_vec<XT, FMT, 128, VB>(x, q, sinv, ngroups, s);
+    case 256: return run_vec<XT, FMT, 256, VB>(x, q, sinv, ngroups, s);
+    case 512: return run_vec<XT, FMT, 512, VB>(x, q, sinv, ngroups, s);
+    case 1024: return run_vec<XT, FMT, 1024, VB>(x, q, sinv, ngroups, s);
     default: return run_generic<XT, FMT>(x, q, sinv, ngroups, group, s);
     }
 }
 
+// vb: 32 or 16 (vector bytes the pointers allow), 0 for the generic kernel
+template <int XT, int FMT>
+fp8q_status dispatch_vb(const void* x, uint8_t* q, float* sinv, int64_t ngroups, int group, int vb,
+                        cudaStream_t s) {
+#if FP8Q_TOK_V32
+    if (vb == 32) return dispatch_group<XT, FMT, 32>(x, q, sinv, ngroups, group, s);
+#endif
+    if (vb >= 16) return dispatch_group<XT, FMT, 16>(x, q, sinv, ngroups, group, s);
+    return run_generic<XT, FMT>(x, q, sinv, ngroups, group, s);
+}
+
 template <int XT>
 fp8q_status dispatch_fmt(const void* x, int fmt, uint8_t* q, float* sinv, int64_t ngroups,
-                         int group, bool vec, cudaStream_t s) {
-    if (fmt == kE4M3)
-        return vec ? dispatch_group<XT, kE4M3>(x, q, sinv, ngroups, group, s)
-                   : run_generic<XT, kE4M3>(x, q, sinv, ngroups, group, s);
-    return vec ? dispatch_group<XT, kE5M2>(x, q, sinv, ngroups, group, s)
-               : run_generic<XT, kE5M2>(x, q, sinv, ngroups, group, s);
+                         int group, int vb, cudaStream_t s) {
+    if (fmt == kE4M3) return dispatch_vb<XT, kE4M3>(x, q, sinv, ngroups, group, vb, s);
+    return dispatch_vb<XT, kE5M2>(x, q, sinv, ngroups, group, vb, s);
 }
 
 }  // namespace
@@ -192,14 +209,15 @@ fp8q_status launch_per_token(const void* x, int xt, int64_t m, int64_t n, int gr
     const int64_t ngroups = m * (n / group);
     if (ngroups == 0) return FP8Q_OK;
     const int es = xt == kF32 ? 4 : 2;
-    const int epv = 16 / es;
     const bool pow2 = group >= 16 && group <= 1024 && (group & (group - 1)) == 0;
-    // vector path: 16-byte aligned input, codes stored epv bytes at a time
-    const bool vec = pow2 && ((uintptr_t)x % 16 == 0) && ((uintptr_t)q % epv == 0);
+    // vector paths: VB-byte aligned input, codes stored VB / es bytes at a time
+    int vb = 0;
+    if (pow2 && (uintptr_t)x % 32 == 0 && (uintptr_t)q % (32 / es) == 0) vb = 32;
+    else if (pow2 && (uintptr_t)x % 16 == 0 && (uintptr_t)q % (16 / es) == 0) vb = 16;
     switch (xt) {
-    case kF32: return dispatch_fmt<kF32>(x, fmt, q, sinv, ngroups, group, vec, s);
-    case kF16: return dispatch_fmt<kF16>(x, fmt, q, sinv, ngroups, group, vec, s);
-    default: return dispatch_fmt<kBF16>(x, fmt, q, sinv, ngroups, group, vec, s);
+    case kF32: return dispatch_fmt<kF32>(x, fmt, q, sinv, ngroups, group, vb, s);
+    case kF16: return dispatch_fmt<kF16>(x, fmt, q, sinv, ngroups, group, vb, s);
+    default: return dispatch_fmt<kBF16>(x, fmt, q, sinv, ngroups, group, vb, s);
     }
 }
 

@@ -12,17 +12,25 @@
 // Per-tensor: two kernels, no grid barrier and no atomics.  Pass 1 writes one
 // magnitude-bits maximum per CTA into the caller's workspace; pass 2 has
 // every CTA reduce those partials (a few KiB from L2), derive the scale and
-// cast.  Pass 2 walks the tensor from the end, so its first reads hit the
-// part of x that pass 1 left in L2.
+// cast.  Pass 1 reads the last kL2KeepBytes of x with an L2 evict_last policy
+// (the rest evict_first), and pass 2 walks the tensor from the end, so the
+// second read of that tail comes from L2 instead of HBM.
 #include "fp8q_device.cuh"
 #include "fp8q_internal.h"
 
 namespace fp8q {
 namespace {
 
+#ifndef FP8Q_SCALED_V32
+#define FP8Q_SCALED_V32 1  // 32-byte vectors (256-bit loads) where the pointers allow
+#endif
 constexpr int kChThreads = 256;
 constexpr int kPtThreads = 256;
 constexpr int kPtUnroll = 4;
+#ifndef FP8Q_PT_L2_KEEP_MB
+#define FP8Q_PT_L2_KEEP_MB 80
+#endif
+constexpr int64_t kL2KeepBytes = (int64_t)FP8Q_PT_L2_KEEP_MB << 20;  // well inside the 126 MB L2
 
 __device__ __forceinline__ uint32_t block_max_u32(uint32_t m, uint32_t* sh) {
 #pragma unroll
@@ -34,28 +42,6 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t m, uint32_t* sh) {
     const int nw = blockDim.x >> 5;
     for (int w = 0; w < nw; ++w) m = max(m, sh[w]);
     return m;
-}
-
-template <int XT, int FMT, bool FIX>
-__device__ __forceinline__ void encode_store(uint4 v, float scale, uint8_t* dst) {
-    if (XT == kF32) {
-        const float f0 = __fmul_rn(__uint_as_float(v.x), scale);
-        const float f1 = __fmul_rn(__uint_as_float(v.y), scale);
-        const float f2 = __fmul_rn(__uint_as_float(v.z), scale);
-        const float f3 = __fmul_rn(__uint_as_float(v.w), scale);
-        st_u32(dst, enc2_sem<FMT, FIX>(f0, f1) | (enc2_sem<FMT, FIX>(f2, f3) << 16));
-    } else {
-        float a0, a1, b0, b1, c0, c1, d0, d1;
-        widen2<XT>(v.x, a0, a1);
-        widen2<XT>(v.y, b0, b1);
-        widen2<XT>(v.z, c0, c1);
-        widen2<XT>(v.w, d0, d1);
-        const uint32_t w0 = enc2_sem<FMT, FIX>(__fmul_rn(a0, scale), __fmul_rn(a1, scale)) |
-                            (enc2_sem<FMT, FIX>(__fmul_rn(b0, scale), __fmul_rn(b1, scale)) << 16);
-        const uint32_t w1 = enc2_sem<FMT, FIX>(__fmul_rn(c0, scale), __fmul_rn(c1, scale)) |
-                            (enc2_sem<FMT, FIX>(__fmul_rn(d0, scale), __fmul_rn(d1, scale)) << 16);
-        st_v2(dst, make_uint2(w0, w1));
-    }
 }
 
 template <int FMT, bool FIX>
@@ -80,87 +66,89 @@ __device__ __forceinline__ float colossal_scale(uint32_t amax_bits, float& amax_
 // ---------------------------------------------------------------------------
 // per-channel
 // ---------------------------------------------------------------------------
-template <int XT, int FMT, int K>
+template <int XT, int FMT, int K, int VB>
 __global__ void __launch_bounds__(kChThreads)
 per_channel_vec_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
                        float* __restrict__ sinv, int64_t cols) {
+    pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
-    constexpr int EPV = 16 / ES;
+    constexpr int EPV = VB / ES;
     __shared__ uint32_t sh[kChThreads / 32];
     const int64_t row = blockIdx.x;
     const int64_t nvec = cols / EPV;
     const uint8_t* xr = x + row * cols * ES;
     uint8_t* qr = q + row * cols;
 
-    uint4 v[K];
+    Vec<VB> v[K];
+    uint32_t m = 0u;
 #pragma unroll
     for (int k = 0; k < K; ++k) {
         const int64_t i = threadIdx.x + (int64_t)k * kChThreads;
-        v[k] = i < nvec ? ld_stream_v4(xr + i * 16) : make_uint4(0u, 0u, 0u, 0u);
+        if (i < nvec) v[k] = load_vec<VB>(xr + i * VB);
     }
-    uint32_t m;
-    if (XT == kF32) {
-        m = 0u;
 #pragma unroll
-        for (int k = 0; k < K; ++k) m = max(m, vec_absmax_bits<kF32>(v[k]));
-    } else {
-        uint32_t p = 0u;
-#pragma unroll
-        for (int k = 0; k < K; ++k) p = max_u16x2(p, vec_absmax_packed16(v[k]));
-        m = packed16_to_f32bits<XT>(p);
+    for (int k = 0; k < K; ++k) {
+        const int64_t i = threadIdx.x + (int64_t)k * kChThreads;
+        if (i < nvec) m = absmax2<XT>(m, vec_absmax<XT, VB>(v[k]));
     }
-    m = block_max_u32(m, sh);
+    const uint32_t bits = block_max_u32(absmax_bits<XT>(m), sh);
     float amax;
     bool fix;
-    const float scale = colossal_scale<FMT>(m, amax, fix);
+    const float scale = colossal_scale<FMT>(bits, amax, fix);
     if (threadIdx.x == 0) sinv[row] = __fdiv_rn(amax, fp8_max<FMT>());
     if (!fix) {
 #pragma unroll
         for (int k = 0; k < K; ++k) {
             const int64_t i = threadIdx.x + (int64_t)k * kChThreads;
-            if (i < nvec) encode_store<XT, FMT, false>(v[k], scale, qr + i * EPV);
+            if (i < nvec) encode_store_vec<XT, FMT, VB, false>(v[k], scale, qr + i * EPV);
         }
     } else {
 #pragma unroll
         for (int k = 0; k < K; ++k) {
             const int64_t i = threadIdx.x + (int64_t)k * kChThreads;
-            if (i < nvec) encode_store<XT, FMT, true>(v[k], scale, qr + i * EPV);
+            if (i < nvec) encode_store_vec<XT, FMT, VB, true>(v[k], scale, qr + i * EPV);
         }
     }
 }
 
 // rows too long for registers, or layouts the vector path cannot take:
-// reduce over the row, then re-read it for the cast.  VEC selects 16-byte
-// accesses (row stride and base 16-byte aligned) or scalar accesses.
-template <int XT, int FMT, bool VEC>
+// reduce over the row, then re-read it for the cast.  VB = 16 / 32 selects
+// vector accesses (row stride and base VB-aligned), VB = 0 scalar accesses.
+template <int XT, int FMT, int VB>
 __global__ void __launch_bounds__(kChThreads)
 per_channel_loop_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
                         float* __restrict__ sinv, int64_t cols) {
+    pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
-    constexpr int EPV = 16 / ES;
+    constexpr int EPV = VB > 0 ? VB / ES : 1;
     __shared__ uint32_t sh[kChThreads / 32];
     const int64_t row = blockIdx.x;
     const uint8_t* xr = x + row * cols * ES;
     uint8_t* qr = q + row * cols;
-    uint32_t m = 0u;
-    if (VEC) {
+    uint32_t bits;
+    if constexpr (VB > 0) {
+        uint32_t m = 0u;
         const int64_t nvec = cols / EPV;
         for (int64_t i = threadIdx.x; i < nvec; i += kChThreads)
-            m = max(m, vec_absmax_bits<XT>(ld_stream_v4(xr + i * 16)));
+            m = absmax2<XT>(m, vec_absmax<XT, VB>(load_vec<VB>(xr + i * VB)));
+        bits = absmax_bits<XT>(m);
     } else {
-        for (int64_t c = threadIdx.x; c < cols; c += kChThreads) m = max(m, elem_abs_bits<XT>(xr + c * ES));
+        bits = 0u;
+        for (int64_t c = threadIdx.x; c < cols; c += kChThreads) bits = max(bits, elem_abs_bits<XT>(xr + c * ES));
     }
-    m = block_max_u32(m, sh);
+    bits = block_max_u32(bits, sh);
     float amax;
     bool fix;
-    const float scale = colossal_scale<FMT>(m, amax, fix);
+    const float scale = colossal_scale<FMT>(bits, amax, fix);
     if (threadIdx.x == 0) sinv[row] = __fdiv_rn(amax, fp8_max<FMT>());
-    if (VEC) {
+    if constexpr (VB > 0) {
         const int64_t nvec = cols / EPV;
         for (int64_t i = threadIdx.x; i < nvec; i += kChThreads) {
-            const uint4 v = *reinterpret_cast<const uint4*>(xr + i * 16);
-            if (fix) encode_store<XT, FMT, true>(v, scale, qr + i * EPV);
-            else encode_store<XT, FMT, false>(v, scale, qr + i * EPV);
+            Vec<VB> v;
+#pragma unroll
+            for (int w = 0; w < VB / 4; ++w) v.w[w] = reinterpret_cast<const uint32_t*>(xr + i * VB)[w];
+            if (fix) encode_store_vec<XT, FMT, VB, true>(v, scale, qr + i * EPV);
+            else encode_store_vec<XT, FMT, VB, false>(v, scale, qr + i * EPV);
         }
     } else {
         for (int64_t c = threadIdx.x; c < cols; c += kChThreads) {
@@ -173,54 +161,51 @@ per_channel_loop_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
 // ---------------------------------------------------------------------------
 // per-tensor
 // ---------------------------------------------------------------------------
-// pass 1: per-CTA magnitude-bits maximum over 16-byte vectors (plus the
-// scalar tail of numel % EPV elements, taken by the first threads of CTA 0)
-template <int XT, bool VEC>
+// pass 1: per-CTA magnitude-bits maximum over VB-byte vectors (plus the scalar
+// tail of numel % EPV elements, taken by the first threads of CTA 0); VB = 0
+// is the scalar path for unaligned tensors
+template <int XT, int VB>
 __global__ void __launch_bounds__(kPtThreads)
 tensor_amax_kernel(const uint8_t* __restrict__ x, int64_t numel, uint32_t* __restrict__ partials) {
+    pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
-    constexpr int EPV = VEC ? 16 / ES : 1;
+    constexpr int EPV = VB > 0 ? VB / ES : 1;
     __shared__ uint32_t sh[kPtThreads / 32];
     const int64_t nvec = numel / EPV;
     const int64_t stride = (int64_t)gridDim.x * kPtThreads;
     int64_t i = (int64_t)blockIdx.x * kPtThreads + threadIdx.x;
-    uint32_t m = 0u;
-    if (VEC) {
-        if (XT == kF32) {
-            for (; i + 3 * stride < nvec; i += 4 * stride) {
-                const uint4 a = ld_stream_v4(x + i * 16), b = ld_stream_v4(x + (i + stride) * 16);
-                const uint4 c = ld_stream_v4(x + (i + 2 * stride) * 16), d = ld_stream_v4(x + (i + 3 * stride) * 16);
-                m = max(m, max(max(vec_absmax_bits<kF32>(a), vec_absmax_bits<kF32>(b)),
-                               max(vec_absmax_bits<kF32>(c), vec_absmax_bits<kF32>(d))));
-            }
-            for (; i < nvec; i += stride) m = max(m, vec_absmax_bits<kF32>(ld_stream_v4(x + i * 16)));
-        } else {
-            uint32_t p = 0u;
-            for (; i + 3 * stride < nvec; i += 4 * stride) {
-                const uint4 a = ld_stream_v4(x + i * 16), b = ld_stream_v4(x + (i + stride) * 16);
-                const uint4 c = ld_stream_v4(x + (i + 2 * stride) * 16), d = ld_stream_v4(x + (i + 3 * stride) * 16);
-                p = max_u16x2(p, max_u16x2(max_u16x2(vec_absmax_packed16(a), vec_absmax_packed16(b)),
-                                           max_u16x2(vec_absmax_packed16(c), vec_absmax_packed16(d))));
-            }
-            for (; i < nvec; i += stride) p = max_u16x2(p, vec_absmax_packed16(ld_stream_v4(x + i * 16)));
-            m = packed16_to_f32bits<XT>(p);
+    uint32_t bits;
+    if constexpr (VB > 0) {
+        // vectors from keep_from on stay in L2 for pass 2
+        const int64_t keep_from = nvec - kL2KeepBytes / VB;
+        const uint64_t keep = l2_evict_last_policy(), drop = l2_evict_first_policy();
+        auto ld = [&](int64_t j) { return load_vec_policy<VB>(x + j * VB, j >= keep_from ? keep : drop); };
+        uint32_t m = 0u;
+        for (; i + 3 * stride < nvec; i += 4 * stride) {
+            const Vec<VB> a = ld(i), b = ld(i + stride), c = ld(i + 2 * stride), d = ld(i + 3 * stride);
+            m = absmax2<XT>(m, absmax2<XT>(absmax2<XT>(vec_absmax<XT, VB>(a), vec_absmax<XT, VB>(b)),
+                                           absmax2<XT>(vec_absmax<XT, VB>(c), vec_absmax<XT, VB>(d))));
         }
+        for (; i < nvec; i += stride) m = absmax2<XT>(m, vec_absmax<XT, VB>(ld(i)));
+        bits = absmax_bits<XT>(m);
         if (blockIdx.x == 0 && threadIdx.x < numel - nvec * EPV)
-            m = max(m, elem_abs_bits<XT>(x + (nvec * EPV + threadIdx.x) * ES));
+            bits = max(bits, elem_abs_bits<XT>(x + (nvec * EPV + threadIdx.x) * ES));
     } else {
-        for (; i < numel; i += stride) m = max(m, elem_abs_bits<XT>(x + i * ES));
+        bits = 0u;
+        for (; i < numel; i += stride) bits = max(bits, elem_abs_bits<XT>(x + i * ES));
     }
-    m = block_max_u32(m, sh);
-    if (threadIdx.x == 0) partials[blockIdx.x] = m;
+    bits = block_max_u32(bits, sh);
+    if (threadIdx.x == 0) partials[blockIdx.x] = bits;
 }
 
 // pass 2: reduce the partials, derive the scale, cast (walking from the end)
-template <int XT, int FMT, bool VEC>
+template <int XT, int FMT, int VB>
 __global__ void __launch_bounds__(kPtThreads)
 tensor_cast_kernel(const uint8_t* __restrict__ x, int64_t numel, uint8_t* __restrict__ q,
                    float* __restrict__ sinv, const uint32_t* __restrict__ partials, int nparts) {
+    pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
-    constexpr int EPV = VEC ? 16 / ES : 1;
+    constexpr int EPV = VB > 0 ? VB / ES : 1;
     __shared__ uint32_t sh;
     if (threadIdx.x < 32) {
         uint32_t m = 0u;
@@ -237,23 +222,27 @@ tensor_cast_kernel(const uint8_t* __restrict__ x, int64_t numel, uint8_t* __rest
     const int64_t nvec = numel / EPV;
     const int64_t stride = (int64_t)gridDim.x * kPtThreads;
     const int64_t t0 = (int64_t)blockIdx.x * kPtThreads + threadIdx.x;
-    if (VEC) {
-        // vector j = nvec - 1 - t, t = t0, t0 + stride, ...; four in flight
+    if constexpr (VB > 0) {
+        // vector j = nvec - 1 - t, t = t0, t0 + stride, ...; four in flight;
+        // x is not needed again, so its lines go first
+        const uint64_t drop = l2_evict_first_policy();
         int64_t t = t0;
         if (!fix) {
             for (; t + 3 * stride < nvec; t += 4 * stride) {
-                uint4 v[4];
+                Vec<VB> v[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) v[u] = ld_stream_v4(x + (nvec - 1 - (t + u * stride)) * 16);
+                for (int u = 0; u < 4; ++u) v[u] = load_vec_policy<VB>(x + (nvec - 1 - (t + u * stride)) * VB, drop);
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    encode_store<XT, FMT, false>(v[u], scale, q + (nvec - 1 - (t + u * stride)) * EPV);
+                    encode_store_vec<XT, FMT, VB, false>(v[u], scale, q + (nvec - 1 - (t + u * stride)) * EPV);
             }
             for (; t < nvec; t += stride)
-                encode_store<XT, FMT, false>(ld_stream_v4(x + (nvec - 1 - t) * 16), scale, q + (nvec - 1 - t) * EPV);
+                encode_store_vec<XT, FMT, VB, false>(load_vec_policy<VB>(x + (nvec - 1 - t) * VB, drop), scale,
+                                                     q + (nvec - 1 - t) * EPV);
         } else {
             for (; t < nvec; t += stride)
-                encode_store<XT, FMT, true>(ld_stream_v4(x + (nvec - 1 - t) * 16), scale, q + (nvec - 1 - t) * EPV);
+                encode_store_vec<XT, FMT, VB, true>(load_vec_policy<VB>(x + (nvec - 1 - t) * VB, drop), scale,
+                                                    q + (nvec - 1 - t) * EPV);
         }
         if (blockIdx.x == 0 && threadIdx.x < numel - nvec * EPV) {
             const int64_t e = nvec * EPV + threadIdx.x;
@@ -269,56 +258,81 @@ tensor_cast_kernel(const uint8_t* __restrict__ x, int64_t numel, uint8_t* __rest
 }
 
 __global__ void fill_kernel(float* __restrict__ dst, int64_t count, float value) {
+    pdl_begin();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
          i += (int64_t)gridDim.x * blockDim.x)
         dst[i] = value;
+}
+
+// widest vector (32 or 16 bytes) that a base pointer, a row stride in bytes
+// and the matching code pointer allow; 0 when neither does
+int vector_bytes(const void* x, int64_t stride_bytes, const void* q, int es) {
+#if FP8Q_SCALED_V32
+    if ((uintptr_t)x % 32 == 0 && stride_bytes % 32 == 0 && (uintptr_t)q % (32 / es) == 0) return 32;
+#endif
+    if ((uintptr_t)x % 16 == 0 && stride_bytes % 16 == 0 && (uintptr_t)q % (16 / es) == 0) return 16;
+    return 0;
+}
+
+template <int XT, int FMT, int VB>
+cudaError_t per_channel_launch(const uint8_t* x, uint8_t* q, float* sinv, int64_t rows, int64_t cols, cudaStream_t s) {
+    constexpr int ES = ElemBytes<XT>::value;
+    const unsigned grid = (unsigned)rows;
+    cudaError_t err;
+    const int64_t nvec = cols * ES / VB;
+    if (nvec <= 1 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 1, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
+    else if (nvec <= 2 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 2, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
+    else if (nvec <= 4 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 4, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
+    else if constexpr (VB == 16) {
+        if (nvec <= 8 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 8, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
+        else err = launch_kernel(per_channel_loop_kernel<XT, FMT, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
+    } else {
+        err = launch_kernel(per_channel_loop_kernel<XT, FMT, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
+    }
+    return err;
 }
 
 template <int XT, int FMT>
 fp8q_status run_per_channel(const uint8_t* x, uint8_t* q, float* sinv, int64_t rows, int64_t cols,
                             cudaStream_t s) {
     constexpr int ES = ElemBytes<XT>::value;
-    constexpr int EPV = 16 / ES;
     if (rows > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
-    const bool vec = ((uintptr_t)x % 16 == 0) && ((cols * ES) % 16 == 0) && ((uintptr_t)q % EPV == 0);
-    const unsigned grid = (unsigned)rows;
-    if (vec) {
-        const int64_t nvec = cols / EPV;
-        if (nvec <= 1 * kChThreads) per_channel_vec_kernel<XT, FMT, 1><<<grid, kChThreads, 0, s>>>(x, q, sinv, cols);
-        else if (nvec <= 2 * kChThreads) per_channel_vec_kernel<XT, FMT, 2><<<grid, kChThreads, 0, s>>>(x, q, sinv, cols);
-        else if (nvec <= 4 * kChThreads) per_channel_vec_kernel<XT, FMT, 4><<<grid, kChThreads, 0, s>>>(x, q, sinv, cols);
-        else if (nvec <= 8 * kChThreads) per_channel_vec_kernel<XT, FMT, 8><<<grid, kChThreads, 0, s>>>(x, q, sinv, cols);
-        else per_channel_loop_kernel<XT, FMT, true><<<grid, kChThreads, 0, s>>>(x, q, sinv, cols);
-    } else {
-        per_channel_loop_kernel<XT, FMT, false><<<grid, kChThreads, 0, s>>>(x, q, sinv, cols);
-    }
-    return cuda_status(cudaGetLastError());
+    const int vb = vector_bytes(x, cols * ES, q, ES);
+    cudaError_t err;
+    if (vb == 32) err = per_channel_launch<XT, FMT, 32>(x, q, sinv, rows, cols, s);
+    else if (vb == 16) err = per_channel_launch<XT, FMT, 16>(x, q, sinv, rows, cols, s);
+    else err = launch_kernel(per_channel_loop_kernel<XT, FMT, 0>, dim3((unsigned)rows), dim3(kChThreads), s, x, q, sinv, cols);
+    return cuda_status(err);
+}
+
+template <int XT, int FMT, int VB>
+fp8q_status per_tensor_launch(const uint8_t* x, int64_t numel, uint8_t* q, float* sinv, uint32_t* partials,
+                              cudaStream_t s) {
+    constexpr int ES = ElemBytes<XT>::value;
+    const int64_t units = VB > 0 ? numel * ES / VB : numel;
+    int64_t want = (units + kPtThreads * kPtUnroll - 1) / (kPtThreads * kPtUnroll);
+    // one wave: both passes grid-stride over the tensor with every CTA resident
+    static const int per_sm = min(resident_blocks_per_sm(tensor_amax_kernel<XT, VB>, kPtThreads),
+                                  resident_blocks_per_sm(tensor_cast_kernel<XT, FMT, VB>, kPtThreads));
+    int64_t cap = (int64_t)sm_count() * min(per_sm, 8);
+    if (cap > kMaxPartials) cap = kMaxPartials;
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    const int grid = (int)want;
+    cudaError_t err = launch_kernel(tensor_amax_kernel<XT, VB>, dim3(grid), dim3(kPtThreads), s, x, numel, partials);
+    if (err != cudaSuccess) return FP8Q_ERR_CUDA;
+    err = launch_kernel(tensor_cast_kernel<XT, FMT, VB>, dim3(grid), dim3(kPtThreads), s, x, numel, q, sinv, partials, grid);
+    return cuda_status(err);
 }
 
 template <int XT, int FMT>
 fp8q_status run_per_tensor(const uint8_t* x, int64_t numel, uint8_t* q, float* sinv, uint32_t* partials,
                            cudaStream_t s) {
     constexpr int ES = ElemBytes<XT>::value;
-    constexpr int EPV = 16 / ES;
-    const bool vec = ((uintptr_t)x % 16 == 0) && ((uintptr_t)q % EPV == 0);
-    const int64_t units = vec ? numel / EPV : numel;
-    int64_t want = (units + kPtThreads * kPtUnroll - 1) / (kPtThreads * kPtUnroll);
-    const int64_t cap = (int64_t)sm_count() * 8 < kMaxPartials ? (int64_t)sm_count() * 8 : kMaxPartials;
-    if (want > cap) want = cap;
-    if (want < 1) want = 1;
-    const int grid = (int)want;
-    if (vec) {
-        tensor_amax_kernel<XT, true><<<grid, kPtThreads, 0, s>>>(x, numel, partials);
-        fp8q_status st = cuda_status(cudaGetLastError());
-        if (st != FP8Q_OK) return st;
-        tensor_cast_kernel<XT, FMT, true><<<grid, kPtThreads, 0, s>>>(x, numel, q, sinv, partials, grid);
-    } else {
-        tensor_amax_kernel<XT, false><<<grid, kPtThreads, 0, s>>>(x, numel, partials);
-        fp8q_status st = cuda_status(cudaGetLastError());
-        if (st != FP8Q_OK) return st;
-        tensor_cast_kernel<XT, FMT, false><<<grid, kPtThreads, 0, s>>>(x, numel, q, sinv, partials, grid);
-    }
-    return cuda_status(cudaGetLastError());
+    const int vb = vector_bytes(x, 0, q, ES);
+    if (vb == 32) return per_tensor_launch<XT, FMT, 32>(x, numel, q, sinv, partials, s);
+    if (vb == 16) return per_tensor_launch<XT, FMT, 16>(x, numel, q, sinv, partials, s);
+    return per_tensor_launch<XT, FMT, 0>(x, numel, q, sinv, partials, s);
 }
 
 template <int XT>
@@ -341,8 +355,8 @@ fp8q_status launch_fill(float* dst, int64_t count, float value, cudaStream_t s) 
     if (count <= 0) return FP8Q_OK;
     const int64_t want = (count + 255) / 256;
     const int grid = (int)(want < 1024 ? want : 1024);
-    fill_kernel<<<grid, 256, 0, s>>>(dst, count, value);
-    return cuda_status(cudaGetLastError());
+    const cudaError_t err = launch_kernel(fill_kernel, dim3(grid), dim3(256), s, dst, count, value);
+    return cuda_status(err);
 }
 
 fp8q_status launch_per_channel(const void* x, int xt, int64_t rows, int64_t cols, int fmt,
