@@ -492,7 +492,7 @@ def run_ours(args):
                 "steps": e2e_steps},
         "gpu_launches": wl.launches_per_step * args.steps,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1:
         line["cpu_baseline"] = cpu_baseline(h)
     print(json.dumps(line), flush=True)
     _finish(world)
@@ -566,8 +566,9 @@ def _profile_case(name, fp8q, device):
         w, sc = _to_dev(w, device), _to_dev(sc, device)
         y = torch.empty(w.shape, dtype=bf16, device=device)
         return lambda: fp8q.fp8q_block_dequant(w, sc, y, 128, E4M3FN)
-    if name == "grouped_16":
-        idx = list(range(8)) + list(range(64, 72))                 # 8 big + 8 ragged experts: 174 MB in
+    if name in ("grouped_16", "grouped_72"):
+        # 8 big + 8 ragged experts (174 MB in), or all 72 of the bench step (1 GB in, 2 GB out)
+        idx = list(range(8)) + list(range(64, 72)) if name == "grouped_16" else list(range(72))
         ws, ss = zip(*[workloads.c5_weight(i) for i in idx])
         ws = [_to_dev(w, device) for w in ws]
         ss = [_to_dev(s_, device) for s_ in ss]
@@ -587,7 +588,8 @@ def _profile_case(name, fp8q, device):
     raise SystemExit(f"unknown profile case {name}")
 
 
-PROFILE_CASES = ["per_token_4x", "cast_from_fp8_4x", "block_dequant", "grouped_16", "per_channel", "per_tensor"]
+PROFILE_CASES = ["per_token_4x", "cast_from_fp8_4x", "block_dequant", "grouped_16", "grouped_72", "per_channel",
+                 "per_tensor"]
 
 
 def run_profile_case(name, iters):
@@ -613,8 +615,6 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--no-cpu-baseline", action="store_true",
-                    help="leave out the CPU oracle timing (it runs after the GPU timing)")
     ap.add_argument("--profile", choices=PROFILE_CASES,
                     help="run one op of a fixed case --iters times for a profiler capture (no timing)")
     ap.add_argument("--iters", type=int, default=3)

@@ -17,7 +17,7 @@
 #include <stdint.h>
 
 #ifndef FP8Q_PDL
-#define FP8Q_PDL 0
+#define FP8Q_PDL 1
 #endif
 
 namespace fp8q {

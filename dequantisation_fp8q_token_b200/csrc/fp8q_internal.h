@@ -7,7 +7,7 @@
 #include "fp8q.h"
 
 #ifndef FP8Q_PDL
-#define FP8Q_PDL 0
+#define FP8Q_PDL 1
 #endif
 
 namespace fp8q {
