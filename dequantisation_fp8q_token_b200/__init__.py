@@ -29,9 +29,10 @@ import torch
 
 __all__ = [
     "E4M3FN", "E5M2", "F32", "F16", "BF16",
-    "GRAN_TENSOR", "GRAN_ROW", "GRAN_GROUP", "GRAN_BLOCK",
+    "GRAN_TENSOR", "GRAN_ROW", "GRAN_GROUP", "GRAN_BLOCK", "SCALE_IEEE", "SCALE_TORCH",
     "Fp8qError", "lib", "lib_path",
     "fp8q_per_token_group_quant", "fp8q_cast_per_channel", "fp8q_cast_per_tensor",
+    "fp8q_per_token_group_quant_ex", "fp8q_cast_per_channel_ex", "fp8q_cast_per_tensor_ex",
     "fp8q_cast_per_tensor_workspace_bytes", "fp8q_cast_per_tensor_noalloc", "fp8q_block_dequant", "fp8q_block_dequant_grouped",
     "fp8q_cast_from_fp8", "fp8q_status_string", "fp8q_version",
     "per_token_cast_to_fp8", "per_token_cast_back", "cast_to_fp8", "cast_from_fp8", "weight_dequant",
@@ -40,6 +41,7 @@ __all__ = [
 E4M3FN, E5M2 = 0, 1
 F32, F16, BF16 = 0, 1, 2
 GRAN_TENSOR, GRAN_ROW, GRAN_GROUP, GRAN_BLOCK = 0, 1, 2, 3
+SCALE_IEEE, SCALE_TORCH = 0, 1
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libfp8q.so")
@@ -100,6 +102,12 @@ def lib() -> ctypes.CDLL:
             L.fp8q_block_dequant_grouped.argtypes = [ctypes.POINTER(_BlockDesc), i32, i32, i32, i32, p]
             L.fp8q_cast_from_fp8.restype = st
             L.fp8q_cast_from_fp8.argtypes = [p, i32, i64, i64, p, i32, i32, i32, p, p]
+            L.fp8q_per_token_group_quant_ex.restype = st
+            L.fp8q_per_token_group_quant_ex.argtypes = [p, i32, i64, i64, i32, i32, p, p, i32, p]
+            L.fp8q_cast_per_channel_ex.restype = st
+            L.fp8q_cast_per_channel_ex.argtypes = [p, i32, i64, i64, i32, p, p, i32, p]
+            L.fp8q_cast_per_tensor_ex.restype = st
+            L.fp8q_cast_per_tensor_ex.argtypes = [p, i32, i64, i32, p, p, p, ctypes.c_size_t, i32, p]
             _lib = L
     return _lib
 
@@ -164,6 +172,12 @@ def _need(t: torch.Tensor, numel: int, name: str, byte: bool = False, dtype=None
         raise ValueError(f"{name} holds {t.numel()} elements, needs {numel}")
 
 
+def _rule_of(rule) -> int:
+    if isinstance(rule, str):
+        return {"ieee": SCALE_IEEE, "torch": SCALE_TORCH}[rule]
+    return int(rule)
+
+
 def _fmt_of(fmt) -> int:
     if isinstance(fmt, str):
         return {"e4m3": E4M3FN, "e4m3fn": E4M3FN, "e5m2": E5M2}[fmt]
@@ -178,6 +192,12 @@ def _fmt_of(fmt) -> int:
 def fp8q_per_token_group_quant(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
                                group: int = 128, fmt=E4M3FN, stream=None) -> None:
     """DeepEP per_token_cast_to_fp8 into q[m, n] (uint8/fp8) and scale_inv[m, n/group] (fp32)."""
+    fp8q_per_token_group_quant_ex(x, q, scale_inv, group, fmt, SCALE_IEEE, stream)
+
+
+def fp8q_per_token_group_quant_ex(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
+                                  group: int = 128, fmt=E4M3FN, rule=SCALE_IEEE, stream=None) -> None:
+    """fp8q_per_token_group_quant with a scale rule ("ieee" or "torch")."""
     if x.dim() != 2:
         raise ValueError("x must be 2-D [m, n]")
     m, n = x.shape
@@ -185,38 +205,50 @@ def fp8q_per_token_group_quant(x: torch.Tensor, q: torch.Tensor, scale_inv: torc
     if group > 0 and n % group == 0:
         _need(q, m * n, "q", byte=True)
         _need(scale_inv, m * (n // group), "scale_inv", dtype=torch.float32)
-    _check(lib().fp8q_per_token_group_quant(
+    _check(lib().fp8q_per_token_group_quant_ex(
         _dev_ptr(x, "x"), _dtype_code(x, "x"), m, n, group, _fmt_of(fmt),
-        _dev_ptr(q, "q", dev), _dev_ptr(scale_inv, "scale_inv", dev), _stream(stream, dev)),
+        _dev_ptr(q, "q", dev), _dev_ptr(scale_inv, "scale_inv", dev), _rule_of(rule), _stream(stream, dev)),
         "fp8q_per_token_group_quant")
 
 
 def fp8q_cast_per_channel(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
                           fmt=E4M3FN, stream=None) -> None:
     """ColossalAI cast_to_fp8(per_channel_scale=True): one scale per row of x[rows, cols]."""
+    fp8q_cast_per_channel_ex(x, q, scale_inv, fmt, SCALE_IEEE, stream)
+
+
+def fp8q_cast_per_channel_ex(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
+                             fmt=E4M3FN, rule=SCALE_IEEE, stream=None) -> None:
+    """fp8q_cast_per_channel with a scale rule ("ieee" or "torch")."""
     x2 = x.reshape(-1, x.shape[-1]) if x.dim() != 2 else x
     rows, cols = x2.shape
     dev = x.device
     _need(q, rows * cols, "q", byte=True)
     _need(scale_inv, max(rows, 1), "scale_inv", dtype=torch.float32)
-    _check(lib().fp8q_cast_per_channel(
+    _check(lib().fp8q_cast_per_channel_ex(
         _dev_ptr(x2, "x"), _dtype_code(x, "x"), rows, cols, _fmt_of(fmt),
-        _dev_ptr(q, "q", dev), _dev_ptr(scale_inv, "scale_inv", dev), _stream(stream, dev)),
+        _dev_ptr(q, "q", dev), _dev_ptr(scale_inv, "scale_inv", dev), _rule_of(rule), _stream(stream, dev)),
         "fp8q_cast_per_channel")
 
 
 def fp8q_cast_per_tensor(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
                          workspace: torch.Tensor, fmt=E4M3FN, stream=None) -> None:
     """ColossalAI cast_to_fp8 per-tensor branch; workspace of fp8q_cast_per_tensor_workspace_bytes()."""
+    fp8q_cast_per_tensor_ex(x, q, scale_inv, workspace, fmt, SCALE_IEEE, stream)
+
+
+def fp8q_cast_per_tensor_ex(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
+                            workspace: torch.Tensor, fmt=E4M3FN, rule=SCALE_IEEE, stream=None) -> None:
+    """fp8q_cast_per_tensor with a scale rule ("ieee" or "torch")."""
     dev = x.device
     n = x.numel()
     _need(q, n, "q", byte=True)
     _need(scale_inv, 1, "scale_inv", dtype=torch.float32)
     wbytes = workspace.numel() * workspace.element_size()
-    _check(lib().fp8q_cast_per_tensor(
+    _check(lib().fp8q_cast_per_tensor_ex(
         _dev_ptr(x, "x"), _dtype_code(x, "x"), n, _fmt_of(fmt), _dev_ptr(q, "q", dev),
         _dev_ptr(scale_inv, "scale_inv", dev), _dev_ptr(workspace, "workspace", dev), wbytes,
-        _stream(stream, dev)), "fp8q_cast_per_tensor")
+        _rule_of(rule), _stream(stream, dev)), "fp8q_cast_per_tensor")
 
 
 def fp8q_cast_per_tensor_noalloc(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor,
@@ -325,13 +357,15 @@ def _workspace(device: torch.device) -> torch.Tensor:
     return w
 
 
-def per_token_cast_to_fp8(x: torch.Tensor, group: int = 128, fmt=E4M3FN) -> Tuple[torch.Tensor, torch.Tensor]:
-    """DeepEP per_token_cast_to_fp8: returns (q [m, n] float8, scale_inv [m, n/group] fp32)."""
+def per_token_cast_to_fp8(x: torch.Tensor, group: int = 128, fmt=E4M3FN, rule=SCALE_IEEE
+                          ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """DeepEP per_token_cast_to_fp8: returns (q [m, n] float8, scale_inv [m, n/group] fp32).
+    rule="torch" reproduces the bytes torch itself computes for the page's code on a GPU."""
     m, n = x.shape
     f = _fmt_of(fmt)
     q = torch.empty((m, n), dtype=_FMT_DTYPE[f], device=x.device)
     s = torch.empty((m, n // group if group > 0 else 0), dtype=torch.float32, device=x.device)
-    fp8q_per_token_group_quant(x, q, s, group, f)
+    fp8q_per_token_group_quant_ex(x, q, s, group, f, rule)
     return q, s
 
 
@@ -343,8 +377,8 @@ def per_token_cast_back(q: torch.Tensor, scale_inv: torch.Tensor, dtype=torch.bf
     return y
 
 
-def cast_to_fp8(inp: torch.Tensor, fp8_format: str = "e4m3", per_channel_scale: bool = False
-                ) -> Tuple[torch.Tensor, torch.Tensor]:
+def cast_to_fp8(inp: torch.Tensor, fp8_format: str = "e4m3", per_channel_scale: bool = False,
+                rule=SCALE_IEEE) -> Tuple[torch.Tensor, torch.Tensor]:
     """ColossalAI cast_to_fp8: (q with inp's shape, scale_inv).  scale_inv has shape [rows]
     (per-channel; [1] for an empty input) or [1] (per-tensor)."""
     f = _fmt_of(fp8_format)
@@ -352,10 +386,10 @@ def cast_to_fp8(inp: torch.Tensor, fp8_format: str = "e4m3", per_channel_scale: 
     if per_channel_scale:
         rows = inp.numel() // inp.shape[-1] if inp.dim() > 0 and inp.shape[-1] > 0 else 0
         s = torch.empty((max(rows, 1) if inp.numel() == 0 else rows,), dtype=torch.float32, device=inp.device)
-        fp8q_cast_per_channel(inp.reshape(-1, inp.shape[-1]) if inp.dim() != 2 else inp, q, s, f)
+        fp8q_cast_per_channel_ex(inp.reshape(-1, inp.shape[-1]) if inp.dim() != 2 else inp, q, s, f, rule)
     else:
         s = torch.empty((1,), dtype=torch.float32, device=inp.device)
-        fp8q_cast_per_tensor(inp, q, s, _workspace(inp.device), f)
+        fp8q_cast_per_tensor_ex(inp, q, s, _workspace(inp.device), f, rule)
     return q, s
 
 

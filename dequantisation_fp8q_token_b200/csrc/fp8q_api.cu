@@ -26,6 +26,7 @@ int sm_count() {
 namespace {
 
 bool fmt_ok(int f) { return f == FP8Q_E4M3FN || f == FP8Q_E5M2; }
+bool rule_ok(int r) { return r == FP8Q_SCALE_IEEE || r == FP8Q_SCALE_TORCH; }
 bool dtype_ok(int t) { return t == FP8Q_F32 || t == FP8Q_F16 || t == FP8Q_BF16; }
 int dtype_bytes(int t) { return t == FP8Q_F32 ? 4 : 2; }
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
@@ -56,16 +57,24 @@ const char* fp8q_status_string(fp8q_status status) {
     case FP8Q_ERR_CUDA: return "FP8Q_ERR_CUDA: the CUDA runtime refused a launch";
     case FP8Q_ERR_BAD_GRANULARITY: return "FP8Q_ERR_BAD_GRANULARITY: unknown scale granularity";
     case FP8Q_ERR_TOO_MANY: return "FP8Q_ERR_TOO_MANY: descriptor count out of range";
+    case FP8Q_ERR_BAD_RULE: return "FP8Q_ERR_BAD_RULE: unknown scale rule";
     }
     return "FP8Q_ERR_UNKNOWN";
 }
 
-int fp8q_version(void) { return 10000; }
+int fp8q_version(void) { return 10100; }
 
 fp8q_status fp8q_per_token_group_quant(const void* x, fp8q_dtype xt, int64_t m, int64_t n, int group,
                                        fp8q_format fmt, uint8_t* q, float* scale_inv,
                                        fp8q_stream_t stream) {
+    return fp8q_per_token_group_quant_ex(x, xt, m, n, group, fmt, q, scale_inv, FP8Q_SCALE_IEEE, stream);
+}
+
+fp8q_status fp8q_per_token_group_quant_ex(const void* x, fp8q_dtype xt, int64_t m, int64_t n, int group,
+                                          fp8q_format fmt, uint8_t* q, float* scale_inv,
+                                          fp8q_scale_rule rule, fp8q_stream_t stream) {
     if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!rule_ok(rule)) return FP8Q_ERR_BAD_RULE;
     if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
     if (m < 0 || n < 0 || group < 1 || n % group != 0) return FP8Q_ERR_BAD_SHAPE;
     const int64_t numel = checked_mul(m, n);
@@ -73,12 +82,19 @@ fp8q_status fp8q_per_token_group_quant(const void* x, fp8q_dtype xt, int64_t m, 
     if (numel == 0) return FP8Q_OK;
     if (!x || !q || !scale_inv) return FP8Q_ERR_NULL_POINTER;
     if (!aligned(x, dtype_bytes(xt)) || !aligned(scale_inv, 4)) return FP8Q_ERR_MISALIGNED;
-    return launch_per_token(x, xt, m, n, group, fmt, q, scale_inv, reinterpret_cast<cudaStream_t>(stream));
+    return launch_per_token(x, xt, m, n, group, fmt, q, scale_inv, rule, reinterpret_cast<cudaStream_t>(stream));
 }
 
 fp8q_status fp8q_cast_per_channel(const void* x, fp8q_dtype xt, int64_t rows, int64_t cols,
                                   fp8q_format fmt, uint8_t* q, float* scale_inv, fp8q_stream_t stream) {
+    return fp8q_cast_per_channel_ex(x, xt, rows, cols, fmt, q, scale_inv, FP8Q_SCALE_IEEE, stream);
+}
+
+fp8q_status fp8q_cast_per_channel_ex(const void* x, fp8q_dtype xt, int64_t rows, int64_t cols,
+                                     fp8q_format fmt, uint8_t* q, float* scale_inv, fp8q_scale_rule rule,
+                                     fp8q_stream_t stream) {
     if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!rule_ok(rule)) return FP8Q_ERR_BAD_RULE;
     if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
     if (rows < 0 || cols < 0 || rows > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
     const int64_t numel = checked_mul(rows, cols);
@@ -89,7 +105,7 @@ fp8q_status fp8q_cast_per_channel(const void* x, fp8q_dtype xt, int64_t rows, in
     if (numel == 0) return launch_fill(scale_inv, rows > 0 ? rows : 1, 1.0f, s);
     if (!x || !q) return FP8Q_ERR_NULL_POINTER;
     if (!aligned(x, dtype_bytes(xt))) return FP8Q_ERR_MISALIGNED;
-    return launch_per_channel(x, xt, rows, cols, fmt, q, scale_inv, s);
+    return launch_per_channel(x, xt, rows, cols, fmt, q, scale_inv, rule, s);
 }
 
 size_t fp8q_cast_per_tensor_workspace_bytes(void) { return kPerTensorWorkspaceBytes; }
@@ -97,7 +113,15 @@ size_t fp8q_cast_per_tensor_workspace_bytes(void) { return kPerTensorWorkspaceBy
 fp8q_status fp8q_cast_per_tensor(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt,
                                  uint8_t* q, float* scale_inv, void* workspace, size_t workspace_bytes,
                                  fp8q_stream_t stream) {
+    return fp8q_cast_per_tensor_ex(x, xt, numel, fmt, q, scale_inv, workspace, workspace_bytes, FP8Q_SCALE_IEEE,
+                                   stream);
+}
+
+fp8q_status fp8q_cast_per_tensor_ex(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt,
+                                    uint8_t* q, float* scale_inv, void* workspace, size_t workspace_bytes,
+                                    fp8q_scale_rule rule, fp8q_stream_t stream) {
     if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!rule_ok(rule)) return FP8Q_ERR_BAD_RULE;
     if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
     if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -108,7 +132,7 @@ fp8q_status fp8q_cast_per_tensor(const void* x, fp8q_dtype xt, int64_t numel, fp
     if (!aligned(x, dtype_bytes(xt))) return FP8Q_ERR_MISALIGNED;
     if (!workspace || workspace_bytes < kPerTensorWorkspaceBytes || !aligned(workspace, 16))
         return FP8Q_ERR_WORKSPACE;
-    return launch_per_tensor(x, xt, numel, fmt, q, scale_inv, static_cast<uint32_t*>(workspace), s);
+    return launch_per_tensor(x, xt, numel, fmt, q, scale_inv, static_cast<uint32_t*>(workspace), rule, s);
 }
 
 fp8q_status fp8q_block_dequant(const uint8_t* w, fp8q_format fmt, int64_t M, int64_t N,

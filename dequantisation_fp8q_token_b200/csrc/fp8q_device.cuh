@@ -48,6 +48,20 @@ __device__ __forceinline__ void pdl_begin() {
 }
 
 // ---------------------------------------------------------------------------
+// scale rules: rule 0 divides once (fl(FMAX / amax), fl(amax / FMAX)); rule 1
+// reproduces torch's evaluation of the same expressions on a CUDA tensor
+// (fl(fl(1 / amax) * FMAX) and fl(amax * fl(1 / FMAX))).
+// ---------------------------------------------------------------------------
+template <int FMT> __device__ __forceinline__ float scale_from_amax(float amax, int rule) {
+    if (rule) return __fmul_rn(__fdiv_rn(1.0f, amax), FMT == 0 ? 448.0f : 57344.0f);
+    return __fdiv_rn(FMT == 0 ? 448.0f : 57344.0f, amax);
+}
+template <int FMT> __device__ __forceinline__ float scale_inv_from_amax(float amax, int rule) {
+    if (rule) return __fmul_rn(amax, __fdiv_rn(1.0f, FMT == 0 ? 448.0f : 57344.0f));
+    return __fdiv_rn(amax, FMT == 0 ? 448.0f : 57344.0f);
+}
+
+// ---------------------------------------------------------------------------
 // global memory access
 // ---------------------------------------------------------------------------
 // Streaming 16-byte load through the non-coherent path, not kept in L1.

@@ -51,12 +51,13 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaS
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// `rule` is an fp8q_scale_rule: 0 one IEEE division, 1 torch's evaluation order
 fp8q_status launch_per_token(const void* x, int xt, int64_t m, int64_t n, int group, int fmt,
-                             uint8_t* q, float* sinv, cudaStream_t s);
+                             uint8_t* q, float* sinv, int rule, cudaStream_t s);
 fp8q_status launch_per_channel(const void* x, int xt, int64_t rows, int64_t cols, int fmt,
-                               uint8_t* q, float* sinv, cudaStream_t s);
+                               uint8_t* q, float* sinv, int rule, cudaStream_t s);
 fp8q_status launch_per_tensor(const void* x, int xt, int64_t numel, int fmt, uint8_t* q,
-                              float* sinv, uint32_t* partials, cudaStream_t s);
+                              float* sinv, uint32_t* partials, int rule, cudaStream_t s);
 fp8q_status launch_fill(float* dst, int64_t count, float value, cudaStream_t s);
 
 // one dequantisation problem: y = T(scale(r, c) * float(q)), validated shapes

@@ -77,5 +77,5 @@ extern "C" fp8q_status fp8q_cast_per_tensor_noalloc(const void* x, fp8q_dtype xt
     if (st != FP8Q_OK) return st;
     // Every slot the cast pass reads is written by the amax pass of the same
     // call, so nothing left over from an earlier call needs clearing.
-    return launch_per_tensor(x, xt, numel, fmt, q, scale_inv, scratch, s);
+    return launch_per_tensor(x, xt, numel, fmt, q, scale_inv, scratch, FP8Q_SCALE_IEEE, s);
 }

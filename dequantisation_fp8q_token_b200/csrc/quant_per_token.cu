@@ -70,7 +70,7 @@ __device__ __forceinline__ void load_batch(const uint8_t* __restrict__ x, int64_
 template <int XT, int FMT, int G, int VB>
 __device__ __forceinline__ void process_batch(const Vec<VB> (&v)[TokCfg<XT, G, VB>::VPL], uint8_t* __restrict__ q,
                                               float* __restrict__ sinv, int64_t ngroups, int64_t bt,
-                                              int seg, int sl, int lane, int warp) {
+                                              int seg, int sl, int lane, int warp, int rule) {
     using C = TokCfg<XT, G, VB>;
     // magnitude maximum of this lane's elements
     uint32_t m = vec_absmax<XT, VB>(v[0]);
@@ -82,8 +82,8 @@ __device__ __forceinline__ void process_batch(const Vec<VB> (&v)[TokCfg<XT, G, V
     // the warp's SEGS scales, one group per lane, computed once
     float amax = __uint_as_float(__shfl_sync(0xFFFFFFFFu, bits, (lane % C::SEGS) * C::LANES));
     if (amax < 1e-4f) amax = 1e-4f;  // clamp(1e-4); a NaN amax stays NaN
-    const float scale_l = __fdiv_rn(fp8_max<FMT>(), amax);
-    const float sinv_l = __fdiv_rn(amax, fp8_max<FMT>());
+    const float scale_l = scale_from_amax<FMT>(amax, rule);
+    const float sinv_l = scale_inv_from_amax<FMT>(amax, rule);
     const float scale = __shfl_sync(0xFFFFFFFFu, scale_l, seg);
     const int64_t gbase = bt * C::GPB + (int64_t)warp * C::SEGS;
     if (lane < C::SEGS && gbase + lane < ngroups) sinv[gbase + lane] = sinv_l;
@@ -104,7 +104,7 @@ __device__ __forceinline__ void process_batch(const Vec<VB> (&v)[TokCfg<XT, G, V
 template <int XT, int FMT, int G, int VB>
 __global__ void __launch_bounds__(kTokThreads)
 per_token_vec_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
-                     float* __restrict__ sinv, int64_t ngroups, int64_t nbatch) {
+                     float* __restrict__ sinv, int64_t ngroups, int64_t nbatch, int rule) {
     pdl_begin();
     using C = TokCfg<XT, G, VB>;
     const int lane = threadIdx.x & 31;
@@ -118,14 +118,14 @@ per_token_vec_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
     for (int u = 0; u < kTokUnroll; ++u) load_batch<XT, G, VB>(x, ngroups, b0 + u, gw, sl, v[u]);
 #pragma unroll
     for (int u = 0; u < kTokUnroll; ++u)
-        if (b0 + u < nbatch) process_batch<XT, FMT, G, VB>(v[u], q, sinv, ngroups, b0 + u, seg, sl, lane, warp);
+        if (b0 + u < nbatch) process_batch<XT, FMT, G, VB>(v[u], q, sinv, ngroups, b0 + u, seg, sl, lane, warp, rule);
 }
 
 // any group size dividing n, any element-aligned pointers: one warp per group
 template <int XT, int FMT>
 __global__ void __launch_bounds__(256)
 per_token_generic_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
-                         float* __restrict__ sinv, int64_t ngroups, int G) {
+                         float* __restrict__ sinv, int64_t ngroups, int G, int rule) {
     pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
     const int lane = threadIdx.x & 31;
@@ -139,8 +139,8 @@ per_token_generic_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
         for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
         float amax = __uint_as_float(m);
         if (amax < 1e-4f) amax = 1e-4f;
-        const float scale = __fdiv_rn(fp8_max<FMT>(), amax);
-        if (lane == 0) sinv[g] = __fdiv_rn(amax, fp8_max<FMT>());
+        const float scale = scale_from_amax<FMT>(amax, rule);
+        if (lane == 0) sinv[g] = scale_inv_from_amax<FMT>(amax, rule);
         for (int k = lane; k < G; k += 32) {
             const float f = __fmul_rn(elem_load<XT>(x + (base + k) * ES), scale);
             q[base + k] = (uint8_t)(enc2<FMT>(f, 0.0f) & 0xFFu);
@@ -149,63 +149,63 @@ per_token_generic_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
 }
 
 template <int XT, int FMT, int G, int VB>
-fp8q_status run_vec(const void* x, uint8_t* q, float* sinv, int64_t ngroups, cudaStream_t s) {
+fp8q_status run_vec(const void* x, uint8_t* q, float* sinv, int64_t ngroups, int rule, cudaStream_t s) {
     using C = TokCfg<XT, G, VB>;
     const int64_t nbatch = (ngroups + C::GPB - 1) / C::GPB;
     const int64_t grid = (nbatch + kTokUnroll - 1) / kTokUnroll;
     if (grid > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
     const cudaError_t err = launch_kernel(per_token_vec_kernel<XT, FMT, G, VB>, dim3((unsigned)grid), dim3(kTokThreads), s,
-                                          static_cast<const uint8_t*>(x), q, sinv, ngroups, nbatch);
+                                          static_cast<const uint8_t*>(x), q, sinv, ngroups, nbatch, rule);
     return cuda_status(err);
 }
 
 template <int XT, int FMT>
-fp8q_status run_generic(const void* x, uint8_t* q, float* sinv, int64_t ngroups, int group,
+fp8q_status run_generic(const void* x, uint8_t* q, float* sinv, int64_t ngroups, int group, int rule,
                         cudaStream_t s) {
     const int64_t want = (ngroups + 7) / 8;
     const int blocks = (int)(want < (int64_t)sm_count() * 16 ? want : (int64_t)sm_count() * 16);
     const cudaError_t err = launch_kernel(per_token_generic_kernel<XT, FMT>, dim3(blocks), dim3(256), s,
-                                          static_cast<const uint8_t*>(x), q, sinv, ngroups, group);
+                                          static_cast<const uint8_t*>(x), q, sinv, ngroups, group, rule);
     return cuda_status(err);
 }
 
 template <int XT, int FMT, int VB>
-fp8q_status dispatch_group(const void* x, uint8_t* q, float* sinv, int64_t ngroups, int group,
+fp8q_status dispatch_group(const void* x, uint8_t* q, float* sinv, int64_t ngroups, int group, int rule,
                            cudaStream_t s) {
     switch (group) {
-    case 16: return run_vec<XT, FMT, 16, VB>(x, q, sinv, ngroups, s);
-    case 32: return run_vec<XT, FMT, 32, VB>(x, q, sinv, ngroups, s);
-    case 64: return run_vec<XT, FMT, 64, VB>(x, q, sinv, ngroups, s);
-    case 128: return run_vec<XT, FMT, 128, VB>(x, q, sinv, ngroups, s);
-    case 256: return run_vec<XT, FMT, 256, VB>(x, q, sinv, ngroups, s);
-    case 512: return run_vec<XT, FMT, 512, VB>(x, q, sinv, ngroups, s);
-    case 1024: return run_vec<XT, FMT, 1024, VB>(x, q, sinv, ngroups, s);
-    default: return run_generic<XT, FMT>(x, q, sinv, ngroups, group, s);
+    case 16: return run_vec<XT, FMT, 16, VB>(x, q, sinv, ngroups, rule, s);
+    case 32: return run_vec<XT, FMT, 32, VB>(x, q, sinv, ngroups, rule, s);
+    case 64: return run_vec<XT, FMT, 64, VB>(x, q, sinv, ngroups, rule, s);
+    case 128: return run_vec<XT, FMT, 128, VB>(x, q, sinv, ngroups, rule, s);
+    case 256: return run_vec<XT, FMT, 256, VB>(x, q, sinv, ngroups, rule, s);
+    case 512: return run_vec<XT, FMT, 512, VB>(x, q, sinv, ngroups, rule, s);
+    case 1024: return run_vec<XT, FMT, 1024, VB>(x, q, sinv, ngroups, rule, s);
+    default: return run_generic<XT, FMT>(x, q, sinv, ngroups, group, rule, s);
     }
 }
 
 // vb: 32 or 16 (vector bytes the pointers allow), 0 for the generic kernel
 template <int XT, int FMT>
-fp8q_status dispatch_vb(const void* x, uint8_t* q, float* sinv, int64_t ngroups, int group, int vb,
+fp8q_status dispatch_vb(const void* x, uint8_t* q, float* sinv, int64_t ngroups, int group, int vb, int rule,
                         cudaStream_t s) {
 #if FP8Q_TOK_V32
-    if (vb == 32) return dispatch_group<XT, FMT, 32>(x, q, sinv, ngroups, group, s);
+    if (vb == 32) return dispatch_group<XT, FMT, 32>(x, q, sinv, ngroups, group, rule, s);
 #endif
-    if (vb >= 16) return dispatch_group<XT, FMT, 16>(x, q, sinv, ngroups, group, s);
-    return run_generic<XT, FMT>(x, q, sinv, ngroups, group, s);
+    if (vb >= 16) return dispatch_group<XT, FMT, 16>(x, q, sinv, ngroups, group, rule, s);
+    return run_generic<XT, FMT>(x, q, sinv, ngroups, group, rule, s);
 }
 
 template <int XT>
 fp8q_status dispatch_fmt(const void* x, int fmt, uint8_t* q, float* sinv, int64_t ngroups,
-                         int group, int vb, cudaStream_t s) {
-    if (fmt == kE4M3) return dispatch_vb<XT, kE4M3>(x, q, sinv, ngroups, group, vb, s);
-    return dispatch_vb<XT, kE5M2>(x, q, sinv, ngroups, group, vb, s);
+                         int group, int vb, int rule, cudaStream_t s) {
+    if (fmt == kE4M3) return dispatch_vb<XT, kE4M3>(x, q, sinv, ngroups, group, vb, rule, s);
+    return dispatch_vb<XT, kE5M2>(x, q, sinv, ngroups, group, vb, rule, s);
 }
 
 }  // namespace
 
 fp8q_status launch_per_token(const void* x, int xt, int64_t m, int64_t n, int group, int fmt,
-                             uint8_t* q, float* sinv, cudaStream_t s) {
+                             uint8_t* q, float* sinv, int rule, cudaStream_t s) {
     const int64_t ngroups = m * (n / group);
     if (ngroups == 0) return FP8Q_OK;
     const int es = xt == kF32 ? 4 : 2;
@@ -215,9 +215,9 @@ fp8q_status launch_per_token(const void* x, int xt, int64_t m, int64_t n, int gr
     if (pow2 && (uintptr_t)x % 32 == 0 && (uintptr_t)q % (32 / es) == 0) vb = 32;
     else if (pow2 && (uintptr_t)x % 16 == 0 && (uintptr_t)q % (16 / es) == 0) vb = 16;
     switch (xt) {
-    case kF32: return dispatch_fmt<kF32>(x, fmt, q, sinv, ngroups, group, vb, s);
-    case kF16: return dispatch_fmt<kF16>(x, fmt, q, sinv, ngroups, group, vb, s);
-    default: return dispatch_fmt<kBF16>(x, fmt, q, sinv, ngroups, group, vb, s);
+    case kF32: return dispatch_fmt<kF32>(x, fmt, q, sinv, ngroups, group, vb, rule, s);
+    case kF16: return dispatch_fmt<kF16>(x, fmt, q, sinv, ngroups, group, vb, rule, s);
+    default: return dispatch_fmt<kBF16>(x, fmt, q, sinv, ngroups, group, vb, rule, s);
     }
 }
 

@@ -54,10 +54,10 @@ __device__ __forceinline__ uint8_t encode_one(float f) {
 // reference: a NaN amax (replaced by 1, so NaN/Inf elements and overflow can
 // occur) or a scale that overflowed to Inf (amax < FMAX / FLT_MAX).
 template <int FMT>
-__device__ __forceinline__ float colossal_scale(uint32_t amax_bits, float& amax_out, bool& fix) {
+__device__ __forceinline__ float colossal_scale(uint32_t amax_bits, float& amax_out, bool& fix, int rule) {
     const float a = __uint_as_float(amax_bits);
     const float amax = a > 0.0f ? a : 1.0f;
-    const float scale = __fdiv_rn(fp8_max<FMT>(), amax);
+    const float scale = scale_from_amax<FMT>(amax, rule);
     fix = (amax_bits > 0x7F800000u) || isinf(scale);
     amax_out = amax;
     return scale;
@@ -69,7 +69,7 @@ __device__ __forceinline__ float colossal_scale(uint32_t amax_bits, float& amax_
 template <int XT, int FMT, int K, int VB>
 __global__ void __launch_bounds__(kChThreads)
 per_channel_vec_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
-                       float* __restrict__ sinv, int64_t cols) {
+                       float* __restrict__ sinv, int64_t cols, int rule) {
     pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
     constexpr int EPV = VB / ES;
@@ -94,8 +94,8 @@ per_channel_vec_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
     const uint32_t bits = block_max_u32(absmax_bits<XT>(m), sh);
     float amax;
     bool fix;
-    const float scale = colossal_scale<FMT>(bits, amax, fix);
-    if (threadIdx.x == 0) sinv[row] = __fdiv_rn(amax, fp8_max<FMT>());
+    const float scale = colossal_scale<FMT>(bits, amax, fix, rule);
+    if (threadIdx.x == 0) sinv[row] = scale_inv_from_amax<FMT>(amax, rule);
     if (!fix) {
 #pragma unroll
         for (int k = 0; k < K; ++k) {
@@ -117,7 +117,7 @@ per_channel_vec_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
 template <int XT, int FMT, int VB>
 __global__ void __launch_bounds__(kChThreads)
 per_channel_loop_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
-                        float* __restrict__ sinv, int64_t cols) {
+                        float* __restrict__ sinv, int64_t cols, int rule) {
     pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
     constexpr int EPV = VB > 0 ? VB / ES : 1;
@@ -139,8 +139,8 @@ per_channel_loop_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
     bits = block_max_u32(bits, sh);
     float amax;
     bool fix;
-    const float scale = colossal_scale<FMT>(bits, amax, fix);
-    if (threadIdx.x == 0) sinv[row] = __fdiv_rn(amax, fp8_max<FMT>());
+    const float scale = colossal_scale<FMT>(bits, amax, fix, rule);
+    if (threadIdx.x == 0) sinv[row] = scale_inv_from_amax<FMT>(amax, rule);
     if constexpr (VB > 0) {
         const int64_t nvec = cols / EPV;
         for (int64_t i = threadIdx.x; i < nvec; i += kChThreads) {
@@ -202,7 +202,7 @@ tensor_amax_kernel(const uint8_t* __restrict__ x, int64_t numel, uint32_t* __res
 template <int XT, int FMT, int VB>
 __global__ void __launch_bounds__(kPtThreads)
 tensor_cast_kernel(const uint8_t* __restrict__ x, int64_t numel, uint8_t* __restrict__ q,
-                   float* __restrict__ sinv, const uint32_t* __restrict__ partials, int nparts) {
+                   float* __restrict__ sinv, const uint32_t* __restrict__ partials, int nparts, int rule) {
     pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
     constexpr int EPV = VB > 0 ? VB / ES : 1;
@@ -217,7 +217,7 @@ tensor_cast_kernel(const uint8_t* __restrict__ x, int64_t numel, uint8_t* __rest
     __syncthreads();
     float amax;
     bool fix;
-    const float scale = colossal_scale<FMT>(sh, amax, fix);
+    const float scale = colossal_scale<FMT>(sh, amax, fix, rule);
     if (blockIdx.x == 0 && threadIdx.x == 0) sinv[0] = __fdiv_rn(1.0f, scale);
     const int64_t nvec = numel / EPV;
     const int64_t stride = (int64_t)gridDim.x * kPtThreads;
@@ -275,39 +275,40 @@ int vector_bytes(const void* x, int64_t stride_bytes, const void* q, int es) {
 }
 
 template <int XT, int FMT, int VB>
-cudaError_t per_channel_launch(const uint8_t* x, uint8_t* q, float* sinv, int64_t rows, int64_t cols, cudaStream_t s) {
+cudaError_t per_channel_launch(const uint8_t* x, uint8_t* q, float* sinv, int64_t rows, int64_t cols, int rule,
+                               cudaStream_t s) {
     constexpr int ES = ElemBytes<XT>::value;
     const unsigned grid = (unsigned)rows;
     cudaError_t err;
     const int64_t nvec = cols * ES / VB;
-    if (nvec <= 1 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 1, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
-    else if (nvec <= 2 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 2, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
-    else if (nvec <= 4 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 4, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
+    if (nvec <= 1 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 1, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols, rule);
+    else if (nvec <= 2 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 2, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols, rule);
+    else if (nvec <= 4 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 4, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols, rule);
     else if constexpr (VB == 16) {
-        if (nvec <= 8 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 8, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
-        else err = launch_kernel(per_channel_loop_kernel<XT, FMT, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
+        if (nvec <= 8 * kChThreads) err = launch_kernel(per_channel_vec_kernel<XT, FMT, 8, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols, rule);
+        else err = launch_kernel(per_channel_loop_kernel<XT, FMT, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols, rule);
     } else {
-        err = launch_kernel(per_channel_loop_kernel<XT, FMT, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols);
+        err = launch_kernel(per_channel_loop_kernel<XT, FMT, VB>, dim3(grid), dim3(kChThreads), s, x, q, sinv, cols, rule);
     }
     return err;
 }
 
 template <int XT, int FMT>
-fp8q_status run_per_channel(const uint8_t* x, uint8_t* q, float* sinv, int64_t rows, int64_t cols,
+fp8q_status run_per_channel(const uint8_t* x, uint8_t* q, float* sinv, int64_t rows, int64_t cols, int rule,
                             cudaStream_t s) {
     constexpr int ES = ElemBytes<XT>::value;
     if (rows > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
     const int vb = vector_bytes(x, cols * ES, q, ES);
     cudaError_t err;
-    if (vb == 32) err = per_channel_launch<XT, FMT, 32>(x, q, sinv, rows, cols, s);
-    else if (vb == 16) err = per_channel_launch<XT, FMT, 16>(x, q, sinv, rows, cols, s);
-    else err = launch_kernel(per_channel_loop_kernel<XT, FMT, 0>, dim3((unsigned)rows), dim3(kChThreads), s, x, q, sinv, cols);
+    if (vb == 32) err = per_channel_launch<XT, FMT, 32>(x, q, sinv, rows, cols, rule, s);
+    else if (vb == 16) err = per_channel_launch<XT, FMT, 16>(x, q, sinv, rows, cols, rule, s);
+    else err = launch_kernel(per_channel_loop_kernel<XT, FMT, 0>, dim3((unsigned)rows), dim3(kChThreads), s, x, q, sinv, cols, rule);
     return cuda_status(err);
 }
 
 template <int XT, int FMT, int VB>
 fp8q_status per_tensor_launch(const uint8_t* x, int64_t numel, uint8_t* q, float* sinv, uint32_t* partials,
-                              cudaStream_t s) {
+                              int rule, cudaStream_t s) {
     constexpr int ES = ElemBytes<XT>::value;
     const int64_t units = VB > 0 ? numel * ES / VB : numel;
     int64_t want = (units + kPtThreads * kPtUnroll - 1) / (kPtThreads * kPtUnroll);
@@ -321,32 +322,32 @@ fp8q_status per_tensor_launch(const uint8_t* x, int64_t numel, uint8_t* q, float
     const int grid = (int)want;
     cudaError_t err = launch_kernel(tensor_amax_kernel<XT, VB>, dim3(grid), dim3(kPtThreads), s, x, numel, partials);
     if (err != cudaSuccess) return FP8Q_ERR_CUDA;
-    err = launch_kernel(tensor_cast_kernel<XT, FMT, VB>, dim3(grid), dim3(kPtThreads), s, x, numel, q, sinv, partials, grid);
+    err = launch_kernel(tensor_cast_kernel<XT, FMT, VB>, dim3(grid), dim3(kPtThreads), s, x, numel, q, sinv, partials, grid, rule);
     return cuda_status(err);
 }
 
 template <int XT, int FMT>
 fp8q_status run_per_tensor(const uint8_t* x, int64_t numel, uint8_t* q, float* sinv, uint32_t* partials,
-                           cudaStream_t s) {
+                           int rule, cudaStream_t s) {
     constexpr int ES = ElemBytes<XT>::value;
     const int vb = vector_bytes(x, 0, q, ES);
-    if (vb == 32) return per_tensor_launch<XT, FMT, 32>(x, numel, q, sinv, partials, s);
-    if (vb == 16) return per_tensor_launch<XT, FMT, 16>(x, numel, q, sinv, partials, s);
-    return per_tensor_launch<XT, FMT, 0>(x, numel, q, sinv, partials, s);
+    if (vb == 32) return per_tensor_launch<XT, FMT, 32>(x, numel, q, sinv, partials, rule, s);
+    if (vb == 16) return per_tensor_launch<XT, FMT, 16>(x, numel, q, sinv, partials, rule, s);
+    return per_tensor_launch<XT, FMT, 0>(x, numel, q, sinv, partials, rule, s);
 }
 
 template <int XT>
 fp8q_status per_channel_fmt(const uint8_t* x, int fmt, uint8_t* q, float* sinv, int64_t rows, int64_t cols,
-                            cudaStream_t s) {
-    return fmt == kE4M3 ? run_per_channel<XT, kE4M3>(x, q, sinv, rows, cols, s)
-                        : run_per_channel<XT, kE5M2>(x, q, sinv, rows, cols, s);
+                            int rule, cudaStream_t s) {
+    return fmt == kE4M3 ? run_per_channel<XT, kE4M3>(x, q, sinv, rows, cols, rule, s)
+                        : run_per_channel<XT, kE5M2>(x, q, sinv, rows, cols, rule, s);
 }
 
 template <int XT>
 fp8q_status per_tensor_fmt(const uint8_t* x, int fmt, int64_t numel, uint8_t* q, float* sinv,
-                           uint32_t* partials, cudaStream_t s) {
-    return fmt == kE4M3 ? run_per_tensor<XT, kE4M3>(x, numel, q, sinv, partials, s)
-                        : run_per_tensor<XT, kE5M2>(x, numel, q, sinv, partials, s);
+                           uint32_t* partials, int rule, cudaStream_t s) {
+    return fmt == kE4M3 ? run_per_tensor<XT, kE4M3>(x, numel, q, sinv, partials, rule, s)
+                        : run_per_tensor<XT, kE5M2>(x, numel, q, sinv, partials, rule, s);
 }
 
 }  // namespace
@@ -360,22 +361,22 @@ fp8q_status launch_fill(float* dst, int64_t count, float value, cudaStream_t s) 
 }
 
 fp8q_status launch_per_channel(const void* x, int xt, int64_t rows, int64_t cols, int fmt,
-                               uint8_t* q, float* sinv, cudaStream_t s) {
+                               uint8_t* q, float* sinv, int rule, cudaStream_t s) {
     const uint8_t* xb = static_cast<const uint8_t*>(x);
     switch (xt) {
-    case kF32: return per_channel_fmt<kF32>(xb, fmt, q, sinv, rows, cols, s);
-    case kF16: return per_channel_fmt<kF16>(xb, fmt, q, sinv, rows, cols, s);
-    default: return per_channel_fmt<kBF16>(xb, fmt, q, sinv, rows, cols, s);
+    case kF32: return per_channel_fmt<kF32>(xb, fmt, q, sinv, rows, cols, rule, s);
+    case kF16: return per_channel_fmt<kF16>(xb, fmt, q, sinv, rows, cols, rule, s);
+    default: return per_channel_fmt<kBF16>(xb, fmt, q, sinv, rows, cols, rule, s);
     }
 }
 
 fp8q_status launch_per_tensor(const void* x, int xt, int64_t numel, int fmt, uint8_t* q,
-                              float* sinv, uint32_t* partials, cudaStream_t s) {
+                              float* sinv, uint32_t* partials, int rule, cudaStream_t s) {
     const uint8_t* xb = static_cast<const uint8_t*>(x);
     switch (xt) {
-    case kF32: return per_tensor_fmt<kF32>(xb, fmt, numel, q, sinv, partials, s);
-    case kF16: return per_tensor_fmt<kF16>(xb, fmt, numel, q, sinv, partials, s);
-    default: return per_tensor_fmt<kBF16>(xb, fmt, numel, q, sinv, partials, s);
+    case kF32: return per_tensor_fmt<kF32>(xb, fmt, numel, q, sinv, partials, rule, s);
+    case kF16: return per_tensor_fmt<kF16>(xb, fmt, numel, q, sinv, partials, rule, s);
+    default: return per_tensor_fmt<kBF16>(xb, fmt, numel, q, sinv, partials, rule, s);
     }
 }
 

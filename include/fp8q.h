@@ -66,6 +66,22 @@ typedef enum {
     FP8Q_GRAN_BLOCK = 3   /* B x B blocks: scale_inv[(r/B) * ceil(cols/B) + c/B] */
 } fp8q_granularity;
 
+/*
+ * How the scale and scale_inv divisions are rounded (the pages write them as
+ * `FMAX / amax` and `amax / FMAX` without saying more):
+ *   FP8Q_SCALE_IEEE   one IEEE binary32 division each: scale = fl(FMAX / amax),
+ *                     scale_inv = fl(amax / FMAX).  The default of every call.
+ *   FP8Q_SCALE_TORCH  the order in which torch evaluates those expressions on
+ *                     a CUDA tensor, for byte parity with outputs torch
+ *                     produced: a Python number divided by a tensor is the
+ *                     tensor's reciprocal times the number, scale =
+ *                     fl(fl(1 / amax) * FMAX); a CUDA tensor divided by a
+ *                     Python number is a multiply by the number's reciprocal,
+ *                     scale_inv = fl(amax * fl(1 / FMAX)).  The per-tensor
+ *                     scale_inv = fl(1 / scale) is the same under both rules.
+ */
+typedef enum { FP8Q_SCALE_IEEE = 0, FP8Q_SCALE_TORCH = 1 } fp8q_scale_rule;
+
 typedef enum {
     FP8Q_OK = 0,
     FP8Q_ERR_NULL_POINTER = 1,    /* a non-empty tensor was given as NULL */
@@ -76,7 +92,8 @@ typedef enum {
     FP8Q_ERR_WORKSPACE = 6,       /* workspace missing or too small */
     FP8Q_ERR_CUDA = 7,            /* the CUDA runtime refused a launch */
     FP8Q_ERR_BAD_GRANULARITY = 8, /* granularity enum out of range */
-    FP8Q_ERR_TOO_MANY = 9         /* grouped call: count < 0 */
+    FP8Q_ERR_TOO_MANY = 9,        /* grouped call: count < 0 */
+    FP8Q_ERR_BAD_RULE = 10        /* scale rule enum out of range */
 } fp8q_status;
 
 /* Human-readable name of a status code (static storage; never NULL). */
@@ -105,6 +122,12 @@ fp8q_status fp8q_per_token_group_quant(const void* x, fp8q_dtype xt, int64_t m, 
                                        int group, fp8q_format fmt, uint8_t* q,
                                        float* scale_inv, fp8q_stream_t stream);
 
+/* The same with an explicit scale rule (fp8q_scale_rule). */
+fp8q_status fp8q_per_token_group_quant_ex(const void* x, fp8q_dtype xt, int64_t m, int64_t n,
+                                          int group, fp8q_format fmt, uint8_t* q,
+                                          float* scale_inv, fp8q_scale_rule rule,
+                                          fp8q_stream_t stream);
+
 /*
  * Per-channel cast -- ColossalAI cast_to_fp8 with per_channel_scale=True:
  *   amax[r]      = max_c |x[r][c]|, then amax[r] := amax[r] > 0 ? amax[r] : 1
@@ -119,6 +142,11 @@ fp8q_status fp8q_per_token_group_quant(const void* x, fp8q_dtype xt, int64_t m, 
 fp8q_status fp8q_cast_per_channel(const void* x, fp8q_dtype xt, int64_t rows, int64_t cols,
                                   fp8q_format fmt, uint8_t* q, float* scale_inv,
                                   fp8q_stream_t stream);
+
+/* The same with an explicit scale rule (fp8q_scale_rule). */
+fp8q_status fp8q_cast_per_channel_ex(const void* x, fp8q_dtype xt, int64_t rows, int64_t cols,
+                                     fp8q_format fmt, uint8_t* q, float* scale_inv,
+                                     fp8q_scale_rule rule, fp8q_stream_t stream);
 
 /*
  * Per-tensor cast -- ColossalAI cast_to_fp8 per-tensor branch:
@@ -138,6 +166,11 @@ size_t fp8q_cast_per_tensor_workspace_bytes(void);
 fp8q_status fp8q_cast_per_tensor(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt,
                                  uint8_t* q, float* scale_inv, void* workspace,
                                  size_t workspace_bytes, fp8q_stream_t stream);
+/* The same with an explicit scale rule (fp8q_scale_rule). */
+fp8q_status fp8q_cast_per_tensor_ex(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt,
+                                    uint8_t* q, float* scale_inv, void* workspace,
+                                    size_t workspace_bytes, fp8q_scale_rule rule,
+                                    fp8q_stream_t stream);
 
 /*
  * Per-tensor cast without a caller workspace.  The paper has no counterpart:

@@ -25,6 +25,7 @@ _LIB = os.path.join(_HERE, "libfp8q_oracle.so")
 E4M3FN, E5M2 = 0, 1
 F32, F16, BF16 = 0, 1, 2
 GRAN_TENSOR, GRAN_ROW, GRAN_GROUP, GRAN_BLOCK = 0, 1, 2, 3
+RULE_IEEE, RULE_TORCH = 0, 1
 
 CFLAGS = ["-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math",
           "-fno-finite-math-only", "-fPIC", "-shared", "-Wall", "-Wextra"]
@@ -71,6 +72,16 @@ def lib() -> ctypes.CDLL:
             L.orc_cast_per_channel.argtypes = [c_void, i32, i64, i64, i32, c_void, c_void, i64, i64]
             L.orc_cast_per_tensor.restype = i32
             L.orc_cast_per_tensor.argtypes = [c_void, i32, i64, i32, c_void, c_void, i64, i64]
+            L.orc_per_token_group_quant_rule.restype = i32
+            L.orc_per_token_group_quant_rule.argtypes = [c_void, i32, i64, i64, i32, i32, c_void, c_void, i64, i64, i32]
+            L.orc_cast_per_channel_rule.restype = i32
+            L.orc_cast_per_channel_rule.argtypes = [c_void, i32, i64, i64, i32, c_void, c_void, i64, i64, i32]
+            L.orc_cast_per_tensor_rule.restype = i32
+            L.orc_cast_per_tensor_rule.argtypes = [c_void, i32, i64, i32, c_void, c_void, i64, i64, i32]
+            L.orc_cast_pipeline.restype = i32
+            L.orc_cast_pipeline.argtypes = [c_void, i32, i64, c_void, c_void, c_void, i32, i64, i64]
+            L.orc_cast_from_pipeline.restype = i32
+            L.orc_cast_from_pipeline.argtypes = [c_void, i32, i64, c_void, i32, c_void, i64, i64]
             L.orc_block_dequant.restype = i32
             L.orc_block_dequant.argtypes = [c_void, i32, i64, i64, c_void, i32, i32, c_void, i64, i64]
             L.orc_cast_from_fp8.restype = i32
@@ -162,7 +173,7 @@ def f16_encode(v: np.ndarray) -> np.ndarray:
 # the method
 # ---------------------------------------------------------------------------
 def per_token_group_quant(x: np.ndarray, xt: int, group: int = 128, fmt: int = E4M3FN,
-                          rows=None, out=None, threads: int = 1):
+                          rows=None, out=None, threads: int = 1, rule: int = RULE_IEEE):
     """DeepEP per_token_cast_to_fp8 over x[m, n]; returns (q uint8[m,n], scale_inv f32[m,n/group])."""
     x = np.ascontiguousarray(x)
     m, n = x.shape
@@ -173,13 +184,14 @@ def per_token_group_quant(x: np.ndarray, xt: int, group: int = 128, fmt: int = E
         q, s = out
     r0, r1 = rows if rows is not None else (0, m)
     L = lib()
-    _run(lambda a, b: _check(L.orc_per_token_group_quant(_ptr(x), xt, m, n, group, fmt,
-                                                        _ptr(q), _ptr(s), a, b),
+    _run(lambda a, b: _check(L.orc_per_token_group_quant_rule(_ptr(x), xt, m, n, group, fmt,
+                                                             _ptr(q), _ptr(s), a, b, rule),
                              "per_token_group_quant"), r0, r1, threads)
     return q, s
 
 
-def cast_per_channel(x: np.ndarray, xt: int, fmt: int = E4M3FN, rows=None, out=None, threads: int = 1):
+def cast_per_channel(x: np.ndarray, xt: int, fmt: int = E4M3FN, rows=None, out=None, threads: int = 1,
+                     rule: int = RULE_IEEE):
     """ColossalAI cast_to_fp8(per_channel_scale=True) over x[rows, cols]; returns (q, scale_inv[rows])."""
     x = np.ascontiguousarray(x)
     R, C = x.shape
@@ -190,12 +202,13 @@ def cast_per_channel(x: np.ndarray, xt: int, fmt: int = E4M3FN, rows=None, out=N
         q, s = out
     r0, r1 = rows if rows is not None else (0, R)
     L = lib()
-    _run(lambda a, b: _check(L.orc_cast_per_channel(_ptr(x), xt, R, C, fmt, _ptr(q), _ptr(s), a, b),
+    _run(lambda a, b: _check(L.orc_cast_per_channel_rule(_ptr(x), xt, R, C, fmt, _ptr(q), _ptr(s), a, b, rule),
                              "cast_per_channel"), r0, r1, threads)
     return q, s
 
 
-def cast_per_tensor(x: np.ndarray, xt: int, fmt: int = E4M3FN, elems=None, out=None, threads: int = 1):
+def cast_per_tensor(x: np.ndarray, xt: int, fmt: int = E4M3FN, elems=None, out=None, threads: int = 1,
+                    rule: int = RULE_IEEE):
     """ColossalAI cast_to_fp8(per_channel_scale=False) over flat x; returns (q, scale_inv[1])."""
     x = np.ascontiguousarray(x).reshape(-1)
     n = x.size
@@ -206,9 +219,33 @@ def cast_per_tensor(x: np.ndarray, xt: int, fmt: int = E4M3FN, elems=None, out=N
         q, s = out
     e0, e1 = elems if elems is not None else (0, n)
     L = lib()
-    _run(lambda a, b: _check(L.orc_cast_per_tensor(_ptr(x), xt, n, fmt, _ptr(q), _ptr(s), a, b),
+    _run(lambda a, b: _check(L.orc_cast_per_tensor_rule(_ptr(x), xt, n, fmt, _ptr(q), _ptr(s), a, b, rule),
                              "cast_per_tensor"), e0, e1, threads)
     return q, s
+
+
+def cast_pipeline(x: np.ndarray, xt: int, rule: int = RULE_IEEE, elems=None, threads: int = 1):
+    """ColossalAI cast_to_fp8_pipeline over flat x; returns (q, scale_inv[1], fmt)."""
+    x = np.ascontiguousarray(x).reshape(-1)
+    n = x.size
+    q = np.zeros((n,), np.uint8)
+    s = np.zeros((1,), np.float32)
+    f = np.zeros((1,), np.int32)
+    e0, e1 = elems if elems is not None else (0, n)
+    L = lib()
+    _run(lambda a, b: _check(L.orc_cast_pipeline(_ptr(x), xt, n, _ptr(q), _ptr(s), _ptr(f), rule, a, b),
+                             "cast_pipeline"), e0, e1, threads)
+    return q, s, int(f[0])
+
+
+def cast_from_pipeline(q: np.ndarray, fmt: int, scale_inv: np.ndarray, yt: int = BF16):
+    """ColossalAI cast_from_fp8_pipeline; returns y with q's size in output type yt."""
+    q = np.ascontiguousarray(q, dtype=np.uint8).reshape(-1)
+    s = np.ascontiguousarray(scale_inv, dtype=np.float32)
+    y = np.zeros((q.size,), _NP_OF[yt])
+    _check(lib().orc_cast_from_pipeline(_ptr(q), fmt, q.size, _ptr(s), yt, _ptr(y), 0, q.size),
+           "cast_from_pipeline")
+    return y
 
 
 def block_dequant(w: np.ndarray, s: np.ndarray, fmt: int = E4M3FN, block: int = 128, yt: int = BF16,

@@ -235,6 +235,37 @@ static float abs_max(const void* x, int xt, int64_t i0, int64_t count)
 }
 
 /* ------------------------------------------------------------------------
+ * Scale rules: how FMAX / amax and amax / FMAX are rounded.
+ *   ORC_RULE_IEEE  one IEEE binary32 division each (the reading used by
+ *                  every operation unless a rule is given).
+ *   ORC_RULE_TORCH the order in which torch evaluates the pages' own
+ *                  expressions on a CUDA tensor: a Python number divided by
+ *                  a tensor is the tensor's reciprocal times the number,
+ *                  fl(fl(1 / amax) * FMAX); a tensor divided by a Python
+ *                  number on the GPU is a multiply by the number's
+ *                  reciprocal, fl(amax * fl(1 / FMAX)).
+ * ---------------------------------------------------------------------- */
+static float scale_of(float amax, float fmax, int rule)
+{
+    if (rule == ORC_RULE_TORCH) {
+        float r = 1.0f / amax;
+        return r * fmax;
+    }
+    return fmax / amax;
+}
+
+static float scale_inv_of(float amax, float fmax, int rule)
+{
+    if (rule == ORC_RULE_TORCH) {
+        float inv = 1.0f / fmax;
+        return amax * inv;
+    }
+    return amax / fmax;
+}
+
+static int valid_rule(int rule) { return rule == ORC_RULE_IEEE || rule == ORC_RULE_TORCH; }
+
+/* ------------------------------------------------------------------------
  * [DEP] per_token_cast_to_fp8.
  *   view x[m][n] as x[m][n/G][G];
  *   amax[r][g]      = clamp(max_k |float(x[r][g][k])|, min = 1e-4)
@@ -249,7 +280,15 @@ int orc_per_token_group_quant(const void* x, int xt, int64_t m, int64_t n,
                               int group, int fmt, uint8_t* q, float* scale_inv,
                               int64_t r0, int64_t r1)
 {
-    if (!valid_fmt(fmt) || !valid_dt(xt) || group <= 0 || m < 0 || n < 0 ||
+    return orc_per_token_group_quant_rule(x, xt, m, n, group, fmt, q, scale_inv, r0, r1,
+                                          ORC_RULE_IEEE);
+}
+
+int orc_per_token_group_quant_rule(const void* x, int xt, int64_t m, int64_t n,
+                                   int group, int fmt, uint8_t* q, float* scale_inv,
+                                   int64_t r0, int64_t r1, int rule)
+{
+    if (!valid_rule(rule) || !valid_fmt(fmt) || !valid_dt(xt) || group <= 0 || m < 0 || n < 0 ||
         n % group != 0 || r0 < 0 || r1 > m || r0 > r1)
         return -1;
     const float fmax     = orc_fp8_max(fmt);
@@ -261,8 +300,8 @@ int orc_per_token_group_quant(const void* x, int xt, int64_t m, int64_t n,
             float amax = abs_max(x, xt, base, group);
             if (amax < clampmin)
                 amax = clampmin;
-            float scale = fmax / amax;
-            scale_inv[r * G + g] = amax / fmax;
+            float scale = scale_of(amax, fmax, rule);
+            scale_inv[r * G + g] = scale_inv_of(amax, fmax, rule);
             for (int64_t k = 0; k < group; ++k) {
                 float v = load_elem(x, xt, base + k) * scale;
                 q[base + k] = orc_fp8_encode(v, fmt);
@@ -284,7 +323,14 @@ int orc_cast_per_channel(const void* x, int xt, int64_t rows, int64_t cols,
                          int fmt, uint8_t* q, float* scale_inv,
                          int64_t r0, int64_t r1)
 {
-    if (!valid_fmt(fmt) || !valid_dt(xt) || rows < 0 || cols < 0 ||
+    return orc_cast_per_channel_rule(x, xt, rows, cols, fmt, q, scale_inv, r0, r1, ORC_RULE_IEEE);
+}
+
+int orc_cast_per_channel_rule(const void* x, int xt, int64_t rows, int64_t cols,
+                              int fmt, uint8_t* q, float* scale_inv,
+                              int64_t r0, int64_t r1, int rule)
+{
+    if (!valid_rule(rule) || !valid_fmt(fmt) || !valid_dt(xt) || rows < 0 || cols < 0 ||
         r0 < 0 || r1 > rows || r0 > r1)
         return -1;
     const float fmax = orc_fp8_max(fmt);
@@ -297,8 +343,8 @@ int orc_cast_per_channel(const void* x, int xt, int64_t rows, int64_t cols,
     for (int64_t r = r0; r < r1; ++r) {
         float amax = abs_max(x, xt, r * cols, cols);
         amax = amax > 0.0f ? amax : 1.0f;
-        float scale = fmax / amax;
-        scale_inv[r] = amax / fmax;
+        float scale = scale_of(amax, fmax, rule);
+        scale_inv[r] = scale_inv_of(amax, fmax, rule);
         for (int64_t c = 0; c < cols; ++c) {
             float v = load_elem(x, xt, r * cols + c) * scale;
             q[r * cols + c] = orc_fp8_encode(v, fmt);
@@ -317,7 +363,13 @@ int orc_cast_per_channel(const void* x, int xt, int64_t rows, int64_t cols,
 int orc_cast_per_tensor(const void* x, int xt, int64_t numel, int fmt,
                         uint8_t* q, float* scale_inv, int64_t e0, int64_t e1)
 {
-    if (!valid_fmt(fmt) || !valid_dt(xt) || numel < 0 || e0 < 0 ||
+    return orc_cast_per_tensor_rule(x, xt, numel, fmt, q, scale_inv, e0, e1, ORC_RULE_IEEE);
+}
+
+int orc_cast_per_tensor_rule(const void* x, int xt, int64_t numel, int fmt,
+                             uint8_t* q, float* scale_inv, int64_t e0, int64_t e1, int rule)
+{
+    if (!valid_rule(rule) || !valid_fmt(fmt) || !valid_dt(xt) || numel < 0 || e0 < 0 ||
         e1 > numel || e0 > e1)
         return -1;
     if (numel == 0) {
@@ -327,11 +379,54 @@ int orc_cast_per_tensor(const void* x, int xt, int64_t numel, int fmt,
     const float fmax = orc_fp8_max(fmt);
     float amax = abs_max(x, xt, 0, numel);
     amax = amax > 0.0f ? amax : 1.0f;
-    float scale = fmax / amax;
-    scale_inv[0] = 1.0f / scale;
+    float scale = scale_of(amax, fmax, rule);
+    scale_inv[0] = 1.0f / scale;   /* `1.0 / scale` is one rounding under both rules */
     for (int64_t i = e0; i < e1; ++i) {
         float v = load_elem(x, xt, i) * scale;
         q[i] = orc_fp8_encode(v, fmt);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * [CAI] cast_to_fp8_pipeline: per-tensor cast whose fp8 format is chosen by
+ * the amax, for activations sent between pipeline stages.
+ *   amax  = max |x|  (the page takes max(|min|, |max|) from aminmax; NaN
+ *           propagates)
+ *   fmt   = amax > 448 (the e4m3fn maximum) ? e5m2 : e4m3fn
+ *           (a NaN amax fails the test and gives e4m3fn)
+ *   scale = amax == 0 ? 1 : FMAX(fmt) / amax       (scale rule as above)
+ *   q     = fp8_fmt(fl(float(x) * scale)); scale_inv[0] = fl(1 / scale)
+ *           (the page keeps scale.reciprocal()); *fmt_out = fmt
+ * Only q[e0..e1) is written; amax is always over all numel elements.
+ * ---------------------------------------------------------------------- */
+int orc_cast_pipeline(const void* x, int xt, int64_t numel, uint8_t* q, float* scale_inv,
+                      int* fmt_out, int rule, int64_t e0, int64_t e1)
+{
+    if (!valid_rule(rule) || !valid_dt(xt) || numel < 0 || e0 < 0 || e1 > numel || e0 > e1)
+        return -1;
+    float amax = abs_max(x, xt, 0, numel);
+    int fmt = amax > orc_fp8_max(ORC_E4M3FN) ? ORC_E5M2 : ORC_E4M3FN;
+    float scale = amax == 0.0f ? 1.0f : scale_of(amax, orc_fp8_max(fmt), rule);
+    scale_inv[0] = 1.0f / scale;
+    *fmt_out = fmt;
+    for (int64_t i = e0; i < e1; ++i) {
+        float v = load_elem(x, xt, i) * scale;
+        q[i] = orc_fp8_encode(v, fmt);
+    }
+    return 0;
+}
+
+/* [CAI] cast_from_fp8_pipeline: y = T(fl(float(q) * scale_inv[0])), the
+ * codes read in the format the tag names. */
+int orc_cast_from_pipeline(const uint8_t* q, int fmt, int64_t numel, const float* scale_inv,
+                           int yt, void* y, int64_t e0, int64_t e1)
+{
+    if (!valid_fmt(fmt) || !valid_dt(yt) || numel < 0 || e0 < 0 || e1 > numel || e0 > e1)
+        return -1;
+    for (int64_t i = e0; i < e1; ++i) {
+        float v = orc_fp8_decode(q[i], fmt) * scale_inv[0];
+        store_elem(y, yt, i, v);
     }
     return 0;
 }

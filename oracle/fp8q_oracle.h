@@ -45,6 +45,9 @@ extern "C" {
 enum { ORC_E4M3FN = 0, ORC_E5M2 = 1 };
 /* element types of high-precision tensors */
 enum { ORC_F32 = 0, ORC_F16 = 1, ORC_BF16 = 2 };
+/* scale rules (see fp8q_oracle.c): one IEEE division, or torch's evaluation
+ * order for the pages' expressions on a CUDA tensor */
+enum { ORC_RULE_IEEE = 0, ORC_RULE_TORCH = 1 };
 /* scale granularity for the dequantising cast */
 enum { ORC_GRAN_TENSOR = 0, ORC_GRAN_ROW = 1, ORC_GRAN_GROUP = 2, ORC_GRAN_BLOCK = 3 };
 
@@ -77,17 +80,38 @@ int orc_per_token_group_quant(const void* x, int xt, int64_t m, int64_t n,
                               int group, int fmt, uint8_t* q, float* scale_inv,
                               int64_t r0, int64_t r1);
 
+int orc_per_token_group_quant_rule(const void* x, int xt, int64_t m, int64_t n,
+                                   int group, int fmt, uint8_t* q, float* scale_inv,
+                                   int64_t r0, int64_t r1, int rule);
+
 /* [CAI] cast_to_fp8, per-channel branch: one scale per row of x[rows][cols].
  * scale_inv[rows]. */
 int orc_cast_per_channel(const void* x, int xt, int64_t rows, int64_t cols,
                          int fmt, uint8_t* q, float* scale_inv,
                          int64_t r0, int64_t r1);
 
+int orc_cast_per_channel_rule(const void* x, int xt, int64_t rows, int64_t cols,
+                              int fmt, uint8_t* q, float* scale_inv,
+                              int64_t r0, int64_t r1, int rule);
+
 /* [CAI] cast_to_fp8, per-tensor branch over numel elements.  The amax is
  * always taken over all numel elements; only q[e0..e1) is written.
  * scale_inv[0]. */
 int orc_cast_per_tensor(const void* x, int xt, int64_t numel, int fmt,
                         uint8_t* q, float* scale_inv, int64_t e0, int64_t e1);
+
+int orc_cast_per_tensor_rule(const void* x, int xt, int64_t numel, int fmt,
+                             uint8_t* q, float* scale_inv, int64_t e0, int64_t e1, int rule);
+
+/* [CAI] cast_to_fp8_pipeline: per-tensor cast with the format chosen by the
+ * amax (e5m2 above 448, else e4m3fn); scale 1 for an all-zero tensor;
+ * scale_inv[0] = 1 / scale; *fmt_out = the chosen format. */
+int orc_cast_pipeline(const void* x, int xt, int64_t numel, uint8_t* q, float* scale_inv,
+                      int* fmt_out, int rule, int64_t e0, int64_t e1);
+
+/* [CAI] cast_from_fp8_pipeline: y = T(float(q) * scale_inv[0]) in format fmt. */
+int orc_cast_from_pipeline(const uint8_t* q, int fmt, int64_t numel, const float* scale_inv,
+                           int yt, void* y, int64_t e0, int64_t e1);
 
 /* [DSV3] weight_dequant: w[M][N] codes, s[ceil(M/B)][ceil(N/B)] fp32,
  * y[M][N] in yt. */

@@ -104,8 +104,22 @@ def _amax_nan(a: np.ndarray, axis) -> np.ndarray:
     return np.where(np.isnan(a).any(axis=axis), np.nan, m)
 
 
+def _scale(F, amax, rule):
+    """fl(F / amax), or torch's fl(fl(1 / amax) * F)."""
+    if rule == 1:
+        return fl(fl(1.0 / amax).astype(np.float64) * F).astype(np.float64)
+    return fl(F / amax).astype(np.float64)
+
+
+def _scale_inv(F, amax, rule):
+    """fl(amax / F), or torch's GPU form fl(amax * fl(1 / F))."""
+    if rule == 1:
+        return fl(amax * float(fl(1.0 / F)))
+    return fl(amax / F)
+
+
 @np.errstate(all="ignore")
-def per_token_group_quant(x, xt, group, fmt):
+def per_token_group_quant(x, xt, group, fmt, rule=0):
     xf = widen(x, xt).astype(np.float64)
     m, n = xf.shape
     g = xf.reshape(m, n // group, group)
@@ -114,24 +128,24 @@ def per_token_group_quant(x, xt, group, fmt):
     amax = np.where(amax < lo, lo, amax)           # clamp; NaN stays NaN
     amax = fl(amax).astype(np.float64)
     F = fmax(fmt)
-    scale = fl(F / amax).astype(np.float64)
-    sinv = fl(amax / F)
+    scale = _scale(F, amax, rule)
+    sinv = _scale_inv(F, amax, rule)
     q = encode(fl(g * scale[:, :, None]), fmt).reshape(m, n)
     return q, sinv
 
 
 @np.errstate(all="ignore")
-def cast_per_channel(x, xt, fmt):
+def cast_per_channel(x, xt, fmt, rule=0):
     xf = widen(x, xt).astype(np.float64)
     amax = _amax_nan(xf, 1)
     amax = np.where(amax > 0, amax, 1.0)           # NaN fails > 0
     F = fmax(fmt)
-    scale = fl(F / amax).astype(np.float64)
-    sinv = fl(amax / F)
+    scale = _scale(F, amax, rule)
+    sinv = _scale_inv(F, amax, rule)
     return encode(fl(xf * scale[:, None]), fmt), sinv
 
 
-def cast_per_tensor(x, xt, fmt):
+def cast_per_tensor(x, xt, fmt, rule=0):
     xf = widen(x, xt).astype(np.float64).reshape(-1)
     if xf.size == 0:
         return np.zeros(0, np.uint8), np.array([1.0], np.float32)
@@ -139,7 +153,7 @@ def cast_per_tensor(x, xt, fmt):
     amax = amax if amax > 0 else np.float64(1.0)
     F = np.float64(fmax(fmt))
     with np.errstate(all="ignore"):
-        scale = np.float64(fl(F / amax))
+        scale = np.float64(_scale(F, amax, rule))
         sinv = fl(np.float64(1.0) / scale).reshape(1)
         return encode(fl(xf * scale), fmt), sinv
 
@@ -170,3 +184,19 @@ def cast_from_fp8(q, scale_inv, gran, fmt, gb, yt):
     else:
         sc = s[(r // gb) * ((C + gb - 1) // gb) + c // gb]
     return narrow(fl(decode(q, fmt) * sc), yt)
+
+
+@np.errstate(all="ignore")
+def cast_pipeline(x, xt, rule=0):
+    """Format by amax (e5m2 above 448), scale 1 for an all-zero tensor."""
+    xf = widen(x, xt).astype(np.float64).reshape(-1)
+    amax = np.float64(_amax_nan(xf, 0)) if xf.size else np.float64(0.0)
+    fmt = E5M2 if amax > 448.0 else E4M3FN
+    scale = np.float64(1.0) if amax == 0 else np.float64(_scale(fmax(fmt), amax, rule))
+    sinv = fl(np.float64(1.0) / scale).reshape(1)
+    return encode(fl(xf * scale), fmt), sinv, fmt
+
+
+@np.errstate(all="ignore")
+def cast_from_pipeline(q, fmt, scale_inv, yt):
+    return narrow(fl(decode(q, fmt) * np.float64(np.float32(scale_inv[0]))), yt)

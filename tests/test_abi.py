@@ -41,7 +41,8 @@ def test_binding_names_match_the_c_names():
 def test_enum_values_match_the_binding():
     import dequantisation_fp8q_token_b200 as fp8q
     src = open(HEADER).read()
-    for name, val in [("FP8Q_E4M3FN", fp8q.E4M3FN), ("FP8Q_E5M2", fp8q.E5M2), ("FP8Q_F32", fp8q.F32),
+    for name, val in [("FP8Q_SCALE_IEEE", fp8q.SCALE_IEEE), ("FP8Q_SCALE_TORCH", fp8q.SCALE_TORCH),
+                      ("FP8Q_E4M3FN", fp8q.E4M3FN), ("FP8Q_E5M2", fp8q.E5M2), ("FP8Q_F32", fp8q.F32),
                       ("FP8Q_F16", fp8q.F16), ("FP8Q_BF16", fp8q.BF16), ("FP8Q_GRAN_TENSOR", fp8q.GRAN_TENSOR),
                       ("FP8Q_GRAN_ROW", fp8q.GRAN_ROW), ("FP8Q_GRAN_GROUP", fp8q.GRAN_GROUP),
                       ("FP8Q_GRAN_BLOCK", fp8q.GRAN_BLOCK)]:
@@ -50,11 +51,11 @@ def test_enum_values_match_the_binding():
 
 def test_status_strings(L):
     import dequantisation_fp8q_token_b200 as fp8q
-    for code in range(10):
+    for code in range(11):
         s = fp8q.fp8q_status_string(code)
         assert s.startswith("FP8Q_")
     assert "UNKNOWN" in fp8q.fp8q_status_string(99)
-    assert fp8q.fp8q_version() == 10000
+    assert fp8q.fp8q_version() == 10100
     assert fp8q.fp8q_cast_per_tensor_workspace_bytes() == 8192
 
 
@@ -93,6 +94,23 @@ def test_per_channel_and_tensor_validation(L):
     assert f(P, 0, 16, 4, P, P, None) == 3
     assert f(None, 0, 16, 0, P, P, None) == 1
     assert f(P + 1, 0, 16, 0, P, P, None) == 5
+
+
+def test_scale_rule_validation(L):
+    f = L.fp8q_per_token_group_quant_ex
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    assert f(P, 2, 4, 128, 128, 0, P, P, 2, None) == 10
+    assert f(P, 2, 4, 128, 128, 0, P, P, -1, None) == 10
+    assert f(P, 2, 4, 130, 128, 0, P, P, 1, None) == 4
+    g = L.fp8q_cast_per_channel_ex
+    g.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    assert g(P, 0, 4, 4, 0, P, P, 7, None) == 10
+    h = L.fp8q_cast_per_tensor_ex
+    h.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+    assert h(P, 0, 16, 0, P, P, P, 8192, 3, None) == 10
 
 
 def test_dequant_validation(L):
