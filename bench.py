@@ -115,7 +115,13 @@ class Workload:
         c5_el = sum(w.numel() for w in self.c5_w)
         c5_bytes = c5_el * 3 + sum(s.numel() for s in self.c5_s) * 4
         f = fp8q
+        # Each op pays for the dirty L2 lines (up to ~60 MB) the op before it
+        # left; the tiny fp16 zero-tensor cast follows the 3 GB grouped dequant
+        # of the previous step, so that write-back lands on it rather than on
+        # the per-token quant.  The step total does not depend on the order.
         self.ops = [
+            Op("cast_per_tensor_f16_zero", lambda: f.fp8q_cast_per_tensor(self.c4c_x, self.c4c_q, self.c4c_s, self.ws, E4M3FN),
+               c4c_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel", [self.c4c_x], [self.c4c_q, self.c4c_s]),
             Op("per_token_group_quant", lambda: f.fp8q_per_token_group_quant(self.c2_x, self.c2_q, self.c2_s, 128, E4M3FN),
                c2_bytes, 1, "per_token_vec_kernel", [self.c2_x], [self.c2_q, self.c2_s]),
             Op("block_dequant", lambda: f.fp8q_block_dequant(self.c3_w, self.c3_s, self.c3_y, 128, E4M3FN),
@@ -128,8 +134,6 @@ class Workload:
                c4a_bytes, 1, "per_channel_vec_kernel", [self.c4a_x], [self.c4a_q, self.c4a_s]),
             Op("cast_per_tensor_f32_e5m2", lambda: f.fp8q_cast_per_tensor(self.c4b_x, self.c4b_q, self.c4b_s, self.ws, E5M2),
                c4b_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel", [self.c4b_x], [self.c4b_q, self.c4b_s]),
-            Op("cast_per_tensor_f16_zero", lambda: f.fp8q_cast_per_tensor(self.c4c_x, self.c4c_q, self.c4c_s, self.ws, E4M3FN),
-               c4c_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel", [self.c4c_x], [self.c4c_q, self.c4c_s]),
             Op("block_dequant_grouped", lambda: f.fp8q_block_dequant_grouped(self.c5_w, self.c5_s, self.c5_y, 128, E4M3FN),
                c5_bytes, 1, "dequant_kernel", [*self.c5_w, *self.c5_s], self.c5_y),
         ]
@@ -305,27 +309,40 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def source_fingerprint() -> str:
+# kernel sources each op's device code depends on (the launch wrappers are host code)
+OP_SOURCES = {
+    "per_token_group_quant": ["quant_per_token.cu", "fp8q_device.cuh"],
+    "block_dequant": ["dequant.cu", "fp8q_device.cuh"],
+    "cast_from_fp8_group": ["dequant.cu", "fp8q_device.cuh"],
+    "block_dequant_grouped": ["dequant.cu", "fp8q_device.cuh"],
+    "cast_per_channel": ["quant_scaled.cu", "fp8q_device.cuh"],
+    "cast_per_tensor_f32_e5m2": ["quant_scaled.cu", "fp8q_device.cuh"],
+    "cast_per_tensor_f16_zero": ["quant_scaled.cu", "fp8q_device.cuh"],
+}
+
+
+def source_fingerprint(files) -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dequantisation_fp8q_token_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in sorted(files):
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(op_name: str):
-    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernels."""
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the kernel sources the op runs now (else None)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    if d.get("source_fingerprint") != source_fingerprint():
-        return None
     e = d.get("ops", {}).get(op_name)
-    return None if e is None else e.get("dram_bytes_per_launch")
+    if e is None or e.get("source_fingerprint") != source_fingerprint(OP_SOURCES[op_name]):
+        return None
+    return e.get("dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------
@@ -549,6 +566,7 @@ def run_reference(args):
 # launches, inputs larger than L2 and a few GB on the device at most
 # ---------------------------------------------------------------------------
 def _profile_case(name, fp8q, device):
+    """Returns (one call of the op, its algorithmic bytes)."""
     g = np.random.default_rng(20261299)
     bf16 = torch.bfloat16
     if name in ("per_token_4x", "cast_from_fp8_4x"):
@@ -558,14 +576,15 @@ def _profile_case(name, fp8q, device):
         s = torch.empty((m, n // 128), dtype=torch.float32, device=device)
         y = torch.empty((m, n), dtype=bf16, device=device)
         fp8q.fp8q_per_token_group_quant(x, q, s, 128, E4M3FN)
+        nbytes = m * n * 3 + m * (n // 128) * 4
         if name == "per_token_4x":
-            return lambda: fp8q.fp8q_per_token_group_quant(x, q, s, 128, E4M3FN)
-        return lambda: fp8q.fp8q_cast_from_fp8(q, s, y, GRAN_GROUP, 128, E4M3FN)
+            return (lambda: fp8q.fp8q_per_token_group_quant(x, q, s, 128, E4M3FN)), nbytes
+        return (lambda: fp8q.fp8q_cast_from_fp8(q, s, y, GRAN_GROUP, 128, E4M3FN)), nbytes
     if name == "block_dequant":
         w, sc = workloads.c3_w_s()
         w, sc = _to_dev(w, device), _to_dev(sc, device)
         y = torch.empty(w.shape, dtype=bf16, device=device)
-        return lambda: fp8q.fp8q_block_dequant(w, sc, y, 128, E4M3FN)
+        return (lambda: fp8q.fp8q_block_dequant(w, sc, y, 128, E4M3FN)), w.numel() * 3 + sc.numel() * 4
     if name in ("grouped_16", "grouped_72"):
         # 8 big + 8 ragged experts (174 MB in), or all 72 of the bench step (1 GB in, 2 GB out)
         idx = list(range(8)) + list(range(64, 72)) if name == "grouped_16" else list(range(72))
@@ -573,23 +592,43 @@ def _profile_case(name, fp8q, device):
         ws = [_to_dev(w, device) for w in ws]
         ss = [_to_dev(s_, device) for s_ in ss]
         ys = [torch.empty(w.shape, dtype=bf16, device=device) for w in ws]
-        return lambda: fp8q.fp8q_block_dequant_grouped(ws, ss, ys, 128, E4M3FN)
+        nbytes = sum(w.numel() * 3 for w in ws) + sum(s_.numel() * 4 for s_ in ss)
+        return (lambda: fp8q.fp8q_block_dequant_grouped(ws, ss, ys, 128, E4M3FN)), nbytes
     if name == "per_channel":
         x = _to_dev(workloads.c4a_x(), device, bf16)
         q = torch.empty(x.shape, dtype=torch.uint8, device=device)
         s = torch.empty((x.shape[0],), dtype=torch.float32, device=device)
-        return lambda: fp8q.fp8q_cast_per_channel(x, q, s, E4M3FN)
+        return (lambda: fp8q.fp8q_cast_per_channel(x, q, s, E4M3FN)), x.numel() * 3 + x.shape[0] * 4
     if name == "per_tensor":
         x = _to_dev(workloads.c4b_v(), device)
         q = torch.empty(x.shape, dtype=torch.uint8, device=device)
         s = torch.empty((1,), dtype=torch.float32, device=device)
         ws = torch.empty(fp8q.fp8q_cast_per_tensor_workspace_bytes(), dtype=torch.uint8, device=device)
-        return lambda: fp8q.fp8q_cast_per_tensor(x, q, s, ws, E5M2)
+        return (lambda: fp8q.fp8q_cast_per_tensor(x, q, s, ws, E5M2)), x.numel() * 9 + 4
+    if name in ("records_pack", "records_unpack"):
+        # the fp8 all-gather's device work for 8 ranks of 16 Mi bf16 each
+        # (32 MiB per rank): pack = each rank's per-tensor cast into its
+        # record (amax pass + cast pass); unpack = all 8 records dequantised
+        W, n = 8, 1 << 24
+        R = fp8q.record_bytes(n)
+        xs = [_to_dev(workloads.to_bf16_bits(g.standard_normal(n, dtype=np.float32)), device, bf16)
+              for _ in range(W)]
+        rec = torch.empty((W * R,), dtype=torch.uint8, device=device)
+        y = torch.empty((W * n,), dtype=bf16, device=device)
+        ws = torch.empty(fp8q.fp8q_cast_per_tensor_workspace_bytes(), dtype=torch.uint8, device=device)
+
+        def pack():
+            for r in range(W):
+                fp8q.fp8q_pack_record(xs[r], rec[r * R:(r + 1) * R], ws, E5M2)
+        pack()
+        if name == "records_pack":
+            return pack, W * (n * 2 * 2 + R)
+        return (lambda: fp8q.fp8q_unpack_records(rec, W, n, y, E5M2)), W * (R + n * 2)
     raise SystemExit(f"unknown profile case {name}")
 
 
 PROFILE_CASES = ["per_token_4x", "cast_from_fp8_4x", "block_dequant", "grouped_16", "grouped_72", "per_channel",
-                 "per_tensor"]
+                 "per_tensor", "records_pack", "records_unpack"]
 
 
 def run_profile_case(name, iters):
@@ -597,7 +636,7 @@ def run_profile_case(name, iters):
     time per launch (CUDA events, back to back); prints no bench line."""
     device = torch.device("cuda", 0)
     import dequantisation_fp8q_token_b200 as fp8q
-    fn = _profile_case(name, fp8q, device)
+    fn, nbytes = _profile_case(name, fp8q, device)
     fn()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -606,7 +645,9 @@ def run_profile_case(name, iters):
         fn()
     e1.record()
     torch.cuda.synchronize()
-    print(f"profile case {name}: {iters} launches, {e0.elapsed_time(e1) * 1e3 / max(iters, 1):.2f} us per launch")
+    us = e0.elapsed_time(e1) * 1e3 / max(iters, 1)
+    print(f"profile case {name}: {iters} calls, {us:.2f} us per call, "
+          f"{nbytes / (us * 1e-6) / 1e9 if iters else 0.0:.1f} GB/s algorithmic")
 
 
 def main(argv=None):

@@ -12,6 +12,11 @@ Entry points with the C names (caller-provided outputs, nothing allocated):
     fp8q_per_token_group_quant, fp8q_cast_per_channel, fp8q_cast_per_tensor,
     fp8q_block_dequant, fp8q_block_dequant_grouped, fp8q_cast_from_fp8
 
+fp8-compressed collectives (ColossalAI all_gather_fp8 / all_to_all_fp8 /
+all_to_all_single_fp8): each rank packs [scale_inv | fp8 payload] records
+with libfp8q, torch.distributed moves the bytes, and libfp8q dequantises
+every received record; no arithmetic runs outside the library.
+
 Allocating helpers named after the functions on the pages:
     per_token_cast_to_fp8   (DeepEP "5 Utils")
     per_token_cast_back     (DeepEP "5 Utils", the named inverse)
@@ -34,8 +39,12 @@ __all__ = [
     "fp8q_per_token_group_quant", "fp8q_cast_per_channel", "fp8q_cast_per_tensor",
     "fp8q_per_token_group_quant_ex", "fp8q_cast_per_channel_ex", "fp8q_cast_per_tensor_ex",
     "fp8q_cast_per_tensor_workspace_bytes", "fp8q_cast_per_tensor_noalloc", "fp8q_block_dequant", "fp8q_block_dequant_grouped",
-    "fp8q_cast_from_fp8", "fp8q_status_string", "fp8q_version",
+    "fp8q_cast_from_fp8", "fp8q_cast_pipeline", "fp8q_cast_from_pipeline", "fp8q_status_string", "fp8q_version",
+    "fp8q_tensor_amax", "fp8q_cast_per_tensor_with_amax", "allreduce_amax_bits", "cast_to_fp8_sharded",
     "per_token_cast_to_fp8", "per_token_cast_back", "cast_to_fp8", "cast_from_fp8", "weight_dequant",
+    "cast_to_fp8_pipeline", "cast_from_fp8_pipeline",
+    "RECORD_HEADER_BYTES", "record_bytes", "fp8q_record_bytes", "fp8q_pack_record", "fp8q_unpack_records",
+    "exchange_records", "exchange_records_all_to_all", "exchange_payload_all_to_all", "all_gather_fp8", "all_to_all_fp8", "all_to_all_single_fp8",
 ]
 
 E4M3FN, E5M2 = 0, 1
@@ -102,12 +111,26 @@ def lib() -> ctypes.CDLL:
             L.fp8q_block_dequant_grouped.argtypes = [ctypes.POINTER(_BlockDesc), i32, i32, i32, i32, p]
             L.fp8q_cast_from_fp8.restype = st
             L.fp8q_cast_from_fp8.argtypes = [p, i32, i64, i64, p, i32, i32, i32, p, p]
+            L.fp8q_tensor_amax.restype = st
+            L.fp8q_tensor_amax.argtypes = [p, i32, i64, p, p, ctypes.c_size_t, p]
+            L.fp8q_cast_per_tensor_with_amax.restype = st
+            L.fp8q_cast_per_tensor_with_amax.argtypes = [p, i32, i64, i32, p, p, p, i32, p]
+            L.fp8q_cast_pipeline.restype = st
+            L.fp8q_cast_pipeline.argtypes = [p, i32, i64, p, p, p, p, ctypes.c_size_t, i32, p]
+            L.fp8q_cast_from_pipeline.restype = st
+            L.fp8q_cast_from_pipeline.argtypes = [p, i64, p, p, i32, p, p]
             L.fp8q_per_token_group_quant_ex.restype = st
             L.fp8q_per_token_group_quant_ex.argtypes = [p, i32, i64, i64, i32, i32, p, p, i32, p]
             L.fp8q_cast_per_channel_ex.restype = st
             L.fp8q_cast_per_channel_ex.argtypes = [p, i32, i64, i64, i32, p, p, i32, p]
             L.fp8q_cast_per_tensor_ex.restype = st
             L.fp8q_cast_per_tensor_ex.argtypes = [p, i32, i64, i32, p, p, p, ctypes.c_size_t, i32, p]
+            L.fp8q_record_bytes.restype = ctypes.c_size_t
+            L.fp8q_record_bytes.argtypes = [i64]
+            L.fp8q_pack_record.restype = st
+            L.fp8q_pack_record.argtypes = [p, i32, i64, i32, p, p, ctypes.c_size_t, i32, p]
+            L.fp8q_unpack_records.restype = st
+            L.fp8q_unpack_records.argtypes = [p, i32, i64, i32, i32, p, p]
             _lib = L
     return _lib
 
@@ -271,6 +294,87 @@ def fp8q_cast_per_tensor_noalloc(x: torch.Tensor, q: torch.Tensor, scale_inv: to
              _dev_ptr(scale_inv, "scale_inv", dev), _stream(stream, dev)), "fp8q_cast_per_tensor_noalloc")
 
 
+def fp8q_tensor_amax(x: torch.Tensor, amax_bits: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    """amax_bits[0] (int32) = fp32 bit pattern of max |x| over this tensor (a shard)."""
+    dev = x.device
+    _need(amax_bits, 1, "amax_bits", dtype=torch.int32)
+    wbytes = workspace.numel() * workspace.element_size()
+    _check(lib().fp8q_tensor_amax(_dev_ptr(x, "x"), _dtype_code(x, "x"), x.numel(),
+                                  _dev_ptr(amax_bits, "amax_bits", dev), _dev_ptr(workspace, "workspace", dev),
+                                  wbytes, _stream(stream, dev)), "fp8q_tensor_amax")
+
+
+def fp8q_cast_per_tensor_with_amax(x: torch.Tensor, amax_bits: torch.Tensor, q: torch.Tensor,
+                                   scale_inv: torch.Tensor, fmt=E4M3FN, rule=SCALE_IEEE, stream=None) -> None:
+    """Per-tensor cast of x with the amax given as fp32 bits in amax_bits[0] (device int32)."""
+    dev = x.device
+    n = x.numel()
+    _need(q, n, "q", byte=True)
+    _need(scale_inv, 1, "scale_inv", dtype=torch.float32)
+    _need(amax_bits, 1, "amax_bits", dtype=torch.int32)
+    _check(lib().fp8q_cast_per_tensor_with_amax(
+        _dev_ptr(x, "x"), _dtype_code(x, "x"), n, _fmt_of(fmt), _dev_ptr(amax_bits, "amax_bits", dev),
+        _dev_ptr(q, "q", dev), _dev_ptr(scale_inv, "scale_inv", dev), _rule_of(rule), _stream(stream, dev)),
+        "fp8q_cast_per_tensor_with_amax")
+
+
+def allreduce_amax_bits(amax_bits: torch.Tensor, group=None) -> None:
+    """The exchange step of a sharded per-tensor cast: an integer MAX of the
+    ranks' amax bit patterns (int32, sign bit clear), in place.  Integer max
+    orders fp32 magnitudes and keeps a NaN from any rank, whatever the
+    backend's float max would do with NaN.  A no-op without a process group."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(amax_bits, op=dist.ReduceOp.MAX, group=group)
+
+
+def cast_to_fp8_sharded(x_local: torch.Tensor, fp8_format: str = "e4m3", group=None,
+                        rule=SCALE_IEEE) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-tensor cast of a tensor whose shards live on the ranks of `group`:
+    local amax, a 4-byte all-reduce (MAX) across ranks, then the cast with the
+    global amax.  Each rank gets its slice of the one-tensor cast's bytes and
+    the shared scale_inv."""
+    f = _fmt_of(fp8_format)
+    dev = x_local.device
+    amax = torch.empty((1,), dtype=torch.int32, device=dev)
+    ws = _workspace(dev)
+    fp8q_tensor_amax(x_local, amax, ws)
+    allreduce_amax_bits(amax, group)
+    q = torch.empty(x_local.shape, dtype=_FMT_DTYPE[f], device=dev)
+    s = torch.empty((1,), dtype=torch.float32, device=dev)
+    fp8q_cast_per_tensor_with_amax(x_local, amax, q, s, f, rule)
+    return q, s
+
+
+def fp8q_cast_pipeline(x: torch.Tensor, q: torch.Tensor, scale_inv: torch.Tensor, fmt_tag: torch.Tensor,
+                       workspace: torch.Tensor, rule=SCALE_IEEE, stream=None) -> None:
+    """ColossalAI cast_to_fp8_pipeline: format chosen by the amax, written to fmt_tag (int32 [1])."""
+    dev = x.device
+    n = x.numel()
+    _need(q, n, "q", byte=True)
+    _need(scale_inv, 1, "scale_inv", dtype=torch.float32)
+    _need(fmt_tag, 1, "fmt_tag", dtype=torch.int32)
+    wbytes = workspace.numel() * workspace.element_size()
+    _check(lib().fp8q_cast_pipeline(
+        _dev_ptr(x, "x"), _dtype_code(x, "x"), n, _dev_ptr(q, "q", dev), _dev_ptr(scale_inv, "scale_inv", dev),
+        _dev_ptr(fmt_tag, "fmt_tag", dev), _dev_ptr(workspace, "workspace", dev), wbytes, _rule_of(rule),
+        _stream(stream, dev)), "fp8q_cast_pipeline")
+
+
+def fp8q_cast_from_pipeline(q: torch.Tensor, scale_inv: torch.Tensor, fmt_tag: torch.Tensor, y: torch.Tensor,
+                            stream=None) -> None:
+    """ColossalAI cast_from_fp8_pipeline into y (its dtype), reading the format tag on the device."""
+    dev = q.device
+    n = q.numel()
+    _need(q, n, "q", byte=True)
+    _need(y, n, "y")
+    _need(scale_inv, 1, "scale_inv", dtype=torch.float32)
+    _need(fmt_tag, 1, "fmt_tag", dtype=torch.int32)
+    _check(lib().fp8q_cast_from_pipeline(
+        _dev_ptr(q, "q"), n, _dev_ptr(scale_inv, "scale_inv", dev), _dev_ptr(fmt_tag, "fmt_tag", dev),
+        _dtype_code(y, "y"), _dev_ptr(y, "y", dev), _stream(stream, dev)), "fp8q_cast_from_pipeline")
+
+
 def fp8q_block_dequant(w: torch.Tensor, scale_inv: torch.Tensor, y: torch.Tensor, block: int = 128,
                        fmt=E4M3FN, stream=None) -> None:
     """DeepSeek-V3 weight_dequant of w[M, N] with scale_inv[ceil(M/B), ceil(N/B)] into y[M, N]."""
@@ -414,3 +518,197 @@ def weight_dequant(x: torch.Tensor, s: torch.Tensor, block_size: int = 128,
     y = torch.empty(x.shape, dtype=dtype, device=x.device)
     fp8q_block_dequant(x, s, y, block_size, _FP8_DTYPES.get(x.dtype, E4M3FN))
     return y
+
+
+def cast_to_fp8_pipeline(x: torch.Tensor, rule=SCALE_IEEE) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """ColossalAI cast_to_fp8_pipeline: returns (codes uint8 with x's shape, scale_inv [1], fmt_tag int32 [1])."""
+    q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    s = torch.empty((1,), dtype=torch.float32, device=x.device)
+    tag = torch.empty((1,), dtype=torch.int32, device=x.device)
+    fp8q_cast_pipeline(x, q, s, tag, _workspace(x.device), rule)
+    return q, s, tag
+
+
+def cast_from_fp8_pipeline(q: torch.Tensor, scale_inv: torch.Tensor, fmt_tag: torch.Tensor,
+                           dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """ColossalAI cast_from_fp8_pipeline: y = dtype(scale_inv * float(q)) in the tagged format."""
+    y = torch.empty(q.shape, dtype=dtype, device=q.device)
+    fp8q_cast_from_pipeline(q, scale_inv, fmt_tag, y)
+    return y
+
+
+# ---------------------------------------------------------------------------
+# fp8-compressed collectives: [scale_inv | fp8 payload] records
+# ---------------------------------------------------------------------------
+RECORD_HEADER_BYTES = 16
+
+
+def record_bytes(numel: int) -> int:
+    """Size of one record: a 16-byte header (fp32 scale_inv, then zeros) and
+    the fp8 payload padded with zeros to a multiple of 16 bytes.  The same
+    arithmetic as fp8q_record_bytes, on the host, so that buffers can be sized
+    without loading the library."""
+    if numel < 0:
+        raise ValueError("numel must be >= 0")
+    return RECORD_HEADER_BYTES + -(-numel // 16) * 16
+
+
+def fp8q_record_bytes(numel: int) -> int:
+    return int(lib().fp8q_record_bytes(int(numel)))
+
+
+def fp8q_pack_record(x: torch.Tensor, record: torch.Tensor, workspace: torch.Tensor, fmt=E5M2,
+                     rule=SCALE_IEEE, stream=None) -> None:
+    """Per-tensor cast of x into one record (uint8, record_bytes(x.numel()) bytes)."""
+    dev = x.device
+    n = x.numel()
+    _need(record, record_bytes(n), "record", byte=True)
+    wbytes = workspace.numel() * workspace.element_size()
+    _check(lib().fp8q_pack_record(
+        _dev_ptr(x, "x"), _dtype_code(x, "x"), n, _fmt_of(fmt), _dev_ptr(record, "record", dev),
+        _dev_ptr(workspace, "workspace", dev), wbytes, _rule_of(rule), _stream(stream, dev)), "fp8q_pack_record")
+
+
+def fp8q_unpack_records(records: torch.Tensor, count: int, numel: int, y: torch.Tensor, fmt=E5M2,
+                        stream=None) -> None:
+    """Dequantise `count` back-to-back records of `numel` codes into y[count * numel] (dtype of y)."""
+    dev = records.device
+    _need(records, count * record_bytes(numel), "records", byte=True)
+    _need(y, count * numel, "y")
+    _check(lib().fp8q_unpack_records(
+        _dev_ptr(records, "records"), int(count), int(numel), _fmt_of(fmt), _dtype_code(y, "y"),
+        _dev_ptr(y, "y", dev), _stream(stream, dev)), "fp8q_unpack_records")
+
+
+def exchange_records(combined: torch.Tensor, group=None) -> None:
+    """The all-gather step: combined is uint8 [world * R]; this rank's record
+    sits at slot `rank` and every other slot is filled from its rank, in
+    place.  Only bytes move; a no-op without a process group."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return
+    world = dist.get_world_size(group)
+    if world == 1:
+        return
+    slots = combined.view(world, -1)
+    mine = slots[dist.get_rank(group)]
+    dist.all_gather_into_tensor(combined, mine, group=group)
+
+
+def exchange_records_all_to_all(recv: torch.Tensor, send: torch.Tensor, group=None) -> None:
+    """The all-to-all step: send is uint8 [world * R] with the record for rank
+    j at slot j; afterwards recv slot i holds rank i's record for this rank.
+    Needs an initialised process group."""
+    import torch.distributed as dist
+    dist.all_to_all_single(recv, send, group=group)
+
+
+def exchange_payload_all_to_all(recv_q: torch.Tensor, q: torch.Tensor, scales: torch.Tensor,
+                                scale_inv: torch.Tensor, group=None) -> None:
+    """The exchange of all_to_all_single_fp8: equal chunks of this rank's
+    codes q go to the ranks (recv_q chunk i from rank i), and every rank's
+    one scale_inv is all-gathered into scales[world].  Needs an initialised
+    process group."""
+    import torch.distributed as dist
+    dist.all_to_all_single(recv_q, q, group=group)
+    dist.all_gather_into_tensor(scales, scale_inv, group=group)
+
+
+def _world_rank(group):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        return dist.get_world_size(group), dist.get_rank(group)
+    return 1, 0
+
+
+def all_gather_fp8(output_list, input_: torch.Tensor, group=None, fp8_format: str = "e5m2",
+                   rule=SCALE_IEEE) -> None:
+    """ColossalAI all_gather_fp8 (and all_gather_fp8_lagacy): every rank casts
+    its tensor with its own per-tensor scale into a record, one all-gather
+    moves the records, and each output_list[r] receives rank r's tensor
+    dequantised with rank r's scale, in input_'s dtype.  output_list may
+    also be one contiguous tensor [world, *input_.shape]."""
+    world, rank = _world_rank(group)
+    dev = input_.device
+    n = input_.numel()
+    f = _fmt_of(fp8_format)
+    R = record_bytes(n)
+    combined = torch.empty(world * R, dtype=torch.uint8, device=dev)
+    fp8q_pack_record(input_, combined[rank * R:(rank + 1) * R], _workspace(dev), f, rule)
+    exchange_records(combined, group)
+    if isinstance(output_list, torch.Tensor):
+        if output_list.numel() != world * n or not output_list.is_contiguous():
+            raise ValueError("the output tensor must be contiguous with world * input_.numel() elements")
+        fp8q_unpack_records(combined, world, n, output_list, f)
+        return
+    if len(output_list) != world:
+        raise ValueError(f"output_list has {len(output_list)} tensors, the group has {world} ranks")
+    for r, out in enumerate(output_list):
+        fp8q_unpack_records(combined[r * R:(r + 1) * R], 1, n, out, f)
+
+
+def all_to_all_fp8(output_list, input_list, group=None, fp8_format: str = "e5m2", rule=SCALE_IEEE) -> None:
+    """ColossalAI all_to_all_fp8: input_list[j] (for rank j) is cast with its
+    own per-tensor scale; output_list[i] receives rank i's tensor for this
+    rank, dequantised with the scale rank i used.  All tensors have one
+    numel and dtype."""
+    world, _ = _world_rank(group)
+    if len(input_list) != world or len(output_list) != world:
+        raise ValueError("input_list and output_list need one tensor per rank")
+    n = input_list[0].numel()
+    if any(t.numel() != n for t in input_list) or any(t.numel() != n for t in output_list):
+        raise ValueError("every tensor must have the same numel")
+    dev = input_list[0].device
+    f = _fmt_of(fp8_format)
+    R = record_bytes(n)
+    send = torch.empty(world * R, dtype=torch.uint8, device=dev)
+    ws = _workspace(dev)
+    for j, t in enumerate(input_list):
+        fp8q_pack_record(t, send[j * R:(j + 1) * R], ws, f, rule)
+    recv = send
+    if world > 1:
+        recv = torch.empty_like(send)
+        exchange_records_all_to_all(recv, send, group)
+    for i, out in enumerate(output_list):
+        fp8q_unpack_records(recv[i * R:(i + 1) * R], 1, n, out, f)
+
+
+def all_to_all_single_fp8(output: torch.Tensor, input: torch.Tensor, group=None, fp8_format: str = "e5m2",
+                          rule=SCALE_IEEE) -> None:
+    """ColossalAI all_to_all_single_fp8 with equal splits: the whole input is
+    cast with ONE per-tensor scale, its world equal chunks along dim 0 go to
+    the ranks, the scales are all-gathered, and chunk i of output is rank
+    i's chunk dequantised with rank i's scale, in input's dtype."""
+    world, _ = _world_rank(group)
+    if input.shape[0] % world:
+        raise ValueError("dim 0 must split evenly across the ranks")
+    if output.shape != input.shape or output.dtype != input.dtype or not output.is_contiguous():
+        raise ValueError("output must be a contiguous tensor of input's shape and dtype")
+    dev = input.device
+    f = _fmt_of(fp8_format)
+    n = input.numel()
+    c = n // world
+    q = torch.empty(n, dtype=torch.uint8, device=dev)
+    s = torch.empty(1, dtype=torch.float32, device=dev)
+    fp8q_cast_per_tensor_ex(input, q, s, _workspace(dev), f, rule)
+    qr, scales = q, s
+    if world > 1:
+        qr = torch.empty_like(q)
+        scales = torch.empty(world, dtype=torch.float32, device=dev)
+        exchange_payload_all_to_all(qr, q, scales, s, group)
+    # chunk i with scale i: a block edge above any size gives one scale per chunk
+    ws_, ss, ys = [], [], []
+    flat = output.view(-1)
+    cols = 4096
+    for i in range(world):
+        body, tail = divmod(c, cols)
+        base = i * c
+        if body:
+            ws_.append(qr[base:base + body * cols].view(body, cols))
+            ss.append(scales[i:i + 1])
+            ys.append(flat[base:base + body * cols])
+        if tail:
+            ws_.append(qr[base + body * cols:base + c].view(1, tail))
+            ss.append(scales[i:i + 1])
+            ys.append(flat[base + body * cols:base + c])
+    fp8q_block_dequant_grouped(ws_, ss, ys, block=1 << 30, fmt=f)

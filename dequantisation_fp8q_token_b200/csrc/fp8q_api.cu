@@ -135,6 +135,126 @@ fp8q_status fp8q_cast_per_tensor_ex(const void* x, fp8q_dtype xt, int64_t numel,
     return launch_per_tensor(x, xt, numel, fmt, q, scale_inv, static_cast<uint32_t*>(workspace), rule, s);
 }
 
+fp8q_status fp8q_tensor_amax(const void* x, fp8q_dtype xt, int64_t numel, uint32_t* amax_bits, void* workspace,
+                             size_t workspace_bytes, fp8q_stream_t stream) {
+    if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!amax_bits) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(amax_bits, 4)) return FP8Q_ERR_MISALIGNED;
+    if (numel == 0) return cuda_status(cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t), s));
+    if (!x) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(x, dtype_bytes(xt))) return FP8Q_ERR_MISALIGNED;
+    if (!workspace || workspace_bytes < kPerTensorWorkspaceBytes || !aligned(workspace, 16))
+        return FP8Q_ERR_WORKSPACE;
+    return launch_tensor_amax(x, xt, numel, static_cast<uint32_t*>(workspace), amax_bits, s);
+}
+
+fp8q_status fp8q_cast_per_tensor_with_amax(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt,
+                                           const uint32_t* amax_bits, uint8_t* q, float* scale_inv,
+                                           fp8q_scale_rule rule, fp8q_stream_t stream) {
+    if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!rule_ok(rule)) return FP8Q_ERR_BAD_RULE;
+    if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
+    if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!scale_inv || !amax_bits) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(scale_inv, 4) || !aligned(amax_bits, 4)) return FP8Q_ERR_MISALIGNED;
+    // an empty shard still takes the shared scale from the global amax
+    if (numel > 0 && (!x || !q)) return FP8Q_ERR_NULL_POINTER;
+    if (numel > 0 && !aligned(x, dtype_bytes(xt))) return FP8Q_ERR_MISALIGNED;
+    return launch_cast_with_amax(x, xt, numel, fmt, amax_bits, q, scale_inv, rule, s);
+}
+
+fp8q_status fp8q_cast_pipeline(const void* x, fp8q_dtype xt, int64_t numel, uint8_t* q, float* scale_inv,
+                               int32_t* fmt_tag, void* workspace, size_t workspace_bytes, fp8q_scale_rule rule,
+                               fp8q_stream_t stream) {
+    if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!rule_ok(rule)) return FP8Q_ERR_BAD_RULE;
+    if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!scale_inv || !fmt_tag) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(scale_inv, 4) || !aligned(fmt_tag, 4)) return FP8Q_ERR_MISALIGNED;
+    if (numel == 0) {
+        fp8q_status st = launch_fill(scale_inv, 1, 1.0f, s);
+        if (st != FP8Q_OK) return st;
+        return cuda_status(cudaMemsetAsync(fmt_tag, 0, sizeof(int32_t), s));
+    }
+    if (!x || !q) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(x, dtype_bytes(xt))) return FP8Q_ERR_MISALIGNED;
+    if (!workspace || workspace_bytes < kPerTensorWorkspaceBytes || !aligned(workspace, 16))
+        return FP8Q_ERR_WORKSPACE;
+    return launch_cast_pipeline(x, xt, numel, q, scale_inv, fmt_tag, static_cast<uint32_t*>(workspace), rule, s);
+}
+
+fp8q_status fp8q_cast_from_pipeline(const uint8_t* q, int64_t numel, const float* scale_inv,
+                                    const int32_t* fmt_tag, fp8q_dtype yt, void* y, fp8q_stream_t stream) {
+    if (!dtype_ok(yt)) return FP8Q_ERR_BAD_DTYPE;
+    if (numel < 0 || checked_mul(numel, dtype_bytes(yt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    if (numel == 0) return FP8Q_OK;
+    if (!q || !scale_inv || !fmt_tag || !y) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(scale_inv, 4) || !aligned(fmt_tag, 4) || !aligned(y, dtype_bytes(yt))) return FP8Q_ERR_MISALIGNED;
+    return launch_cast_from_pipeline(q, numel, scale_inv, fmt_tag, yt, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fp8q_record_bytes(int64_t numel) {
+    if (numel < 0) return 0;
+    return (size_t)(16 + ((numel + 15) / 16) * 16);
+}
+
+fp8q_status fp8q_pack_record(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt, uint8_t* record,
+                             void* workspace, size_t workspace_bytes, fp8q_scale_rule rule, fp8q_stream_t stream) {
+    if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!rule_ok(rule)) return FP8Q_ERR_BAD_RULE;
+    if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
+    if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    if (!record) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(record, 16)) return FP8Q_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // header padding and the payload's last partial 16-byte block start at zero
+    if (cudaMemsetAsync(record, 0, 16, s) != cudaSuccess) return FP8Q_ERR_CUDA;
+    if (numel % 16 && cudaMemsetAsync(record + 16 + (numel / 16) * 16, 0, 16, s) != cudaSuccess)
+        return FP8Q_ERR_CUDA;
+    return fp8q_cast_per_tensor_ex(x, xt, numel, fmt, record + 16, reinterpret_cast<float*>(record), workspace,
+                                   workspace_bytes, rule, stream);
+}
+
+fp8q_status fp8q_unpack_records(const uint8_t* records, int count, int64_t numel, fp8q_format fmt, fp8q_dtype yt,
+                                void* y, fp8q_stream_t stream) {
+    if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
+    if (!dtype_ok(yt)) return FP8Q_ERR_BAD_DTYPE;
+    if (count < 0) return FP8Q_ERR_TOO_MANY;
+    if (numel < 0 || checked_mul(checked_mul(numel, count), dtype_bytes(yt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    if (count == 0 || numel == 0) return FP8Q_OK;
+    if (!records || !y) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(records, 16) || !aligned(y, dtype_bytes(yt))) return FP8Q_ERR_MISALIGNED;
+    // each record's payload as a [numel / 4096][4096] matrix plus a one-row
+    // tail, both with the header's single scale: a block edge above any size
+    // makes every element's scale index 0
+    constexpr int64_t kCols = 4096;
+    const int64_t body_rows = numel / kCols, tail = numel % kCols;
+    const size_t rec = fp8q_record_bytes(numel);
+    const int yb = dtype_bytes(yt);
+    // up to 48 records (96 problems) per launch; nothing is allocated
+    constexpr int kBatch = 96;
+    DequantProblem probs[kBatch];
+    int n = 0;
+    for (int r = 0; r < count; ++r) {
+        const uint8_t* base = records + (size_t)r * rec;
+        const float* sc = reinterpret_cast<const float*>(base);
+        uint8_t* yr = static_cast<uint8_t*>(y) + (size_t)r * numel * yb;
+        if (body_rows) probs[n++] = DequantProblem{base + 16, sc, yr, body_rows, kCols};
+        if (tail) probs[n++] = DequantProblem{base + 16 + body_rows * kCols, sc, yr + body_rows * kCols * yb, 1, tail};
+        if (n > kBatch - 2 || r == count - 1) {
+            const fp8q_status st = launch_dequant(probs, n, fmt, kGranBlock, 1 << 30, yt,
+                                                  reinterpret_cast<cudaStream_t>(stream));
+            if (st != FP8Q_OK) return st;
+            n = 0;
+        }
+    }
+    return FP8Q_OK;
+}
+
 fp8q_status fp8q_block_dequant(const uint8_t* w, fp8q_format fmt, int64_t M, int64_t N,
                                const float* scale_inv, int block, fp8q_dtype yt, void* y,
                                fp8q_stream_t stream) {

@@ -59,6 +59,14 @@ fp8q_status launch_per_channel(const void* x, int xt, int64_t rows, int64_t cols
 fp8q_status launch_per_tensor(const void* x, int xt, int64_t numel, int fmt, uint8_t* q,
                               float* sinv, uint32_t* partials, int rule, cudaStream_t s);
 fp8q_status launch_fill(float* dst, int64_t count, float value, cudaStream_t s);
+fp8q_status launch_cast_pipeline(const void* x, int xt, int64_t numel, uint8_t* q, float* sinv,
+                                 int32_t* fmt_out, uint32_t* partials, int rule, cudaStream_t s);
+fp8q_status launch_tensor_amax(const void* x, int xt, int64_t numel, uint32_t* partials, uint32_t* amax_bits,
+                               cudaStream_t s);
+fp8q_status launch_cast_with_amax(const void* x, int xt, int64_t numel, int fmt, const uint32_t* amax_bits,
+                                  uint8_t* q, float* sinv, int rule, cudaStream_t s);
+fp8q_status launch_cast_from_pipeline(const uint8_t* q, int64_t numel, const float* sinv, const int32_t* fmt_in,
+                                      int yt, void* y, cudaStream_t s);
 
 // one dequantisation problem: y = T(scale(r, c) * float(q)), validated shapes
 struct DequantProblem {

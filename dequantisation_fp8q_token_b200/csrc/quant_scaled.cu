@@ -198,27 +198,27 @@ tensor_amax_kernel(const uint8_t* __restrict__ x, int64_t numel, uint32_t* __res
     if (threadIdx.x == 0) partials[blockIdx.x] = bits;
 }
 
-// pass 2: reduce the partials, derive the scale, cast (walking from the end)
-template <int XT, int FMT, int VB>
-__global__ void __launch_bounds__(kPtThreads)
-tensor_cast_kernel(const uint8_t* __restrict__ x, int64_t numel, uint8_t* __restrict__ q,
-                   float* __restrict__ sinv, const uint32_t* __restrict__ partials, int nparts, int rule) {
-    pdl_begin();
-    constexpr int ES = ElemBytes<XT>::value;
-    constexpr int EPV = VB > 0 ? VB / ES : 1;
-    __shared__ uint32_t sh;
+// magnitude-bits maximum of the amax pass's partials (every thread gets it)
+__device__ __forceinline__ uint32_t reduce_partials(const uint32_t* __restrict__ partials, int nparts,
+                                                    uint32_t* sh) {
     if (threadIdx.x < 32) {
         uint32_t m = 0u;
         for (int p = threadIdx.x; p < nparts; p += 32) m = max(m, __ldcg(partials + p));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-        if (threadIdx.x == 0) sh = m;
+        if (threadIdx.x == 0) *sh = m;
     }
     __syncthreads();
-    float amax;
-    bool fix;
-    const float scale = colossal_scale<FMT>(sh, amax, fix, rule);
-    if (blockIdx.x == 0 && threadIdx.x == 0) sinv[0] = __fdiv_rn(1.0f, scale);
+    return *sh;
+}
+
+// the cast pass over the whole tensor with a known scale, walking from the
+// end so the part of x the amax pass kept in L2 is read first
+template <int XT, int FMT, int VB>
+__device__ __forceinline__ void cast_tensor_body(const uint8_t* __restrict__ x, int64_t numel,
+                                                 uint8_t* __restrict__ q, float scale, bool fix) {
+    constexpr int ES = ElemBytes<XT>::value;
+    constexpr int EPV = VB > 0 ? VB / ES : 1;
     const int64_t nvec = numel / EPV;
     const int64_t stride = (int64_t)gridDim.x * kPtThreads;
     const int64_t t0 = (int64_t)blockIdx.x * kPtThreads + threadIdx.x;
@@ -255,6 +255,121 @@ tensor_cast_kernel(const uint8_t* __restrict__ x, int64_t numel, uint8_t* __rest
             q[e] = fix ? encode_one<FMT, true>(f) : encode_one<FMT, false>(f);
         }
     }
+}
+
+// pass 2: reduce the partials, derive the scale, cast
+template <int XT, int FMT, int VB>
+__global__ void __launch_bounds__(kPtThreads)
+tensor_cast_kernel(const uint8_t* __restrict__ x, int64_t numel, uint8_t* __restrict__ q,
+                   float* __restrict__ sinv, const uint32_t* __restrict__ partials, int nparts, int rule) {
+    pdl_begin();
+    __shared__ uint32_t sh;
+    const uint32_t bits = reduce_partials(partials, nparts, &sh);
+    float amax;
+    bool fix;
+    const float scale = colossal_scale<FMT>(bits, amax, fix, rule);
+    if (blockIdx.x == 0 && threadIdx.x == 0) sinv[0] = __fdiv_rn(1.0f, scale);
+    cast_tensor_body<XT, FMT, VB>(x, numel, q, scale, fix);
+}
+
+// ColossalAI cast_to_fp8_pipeline, pass 2: the format follows the amax
+// (e5m2 above the e4m3fn maximum of 448, else e4m3fn; a NaN amax fails the
+// test), the scale is 1 for an all-zero tensor; writes the format tag and
+// scale_inv = 1 / scale
+template <int XT, int VB>
+__global__ void __launch_bounds__(kPtThreads)
+pipeline_cast_kernel(const uint8_t* __restrict__ x, int64_t numel, uint8_t* __restrict__ q,
+                     float* __restrict__ sinv, int32_t* __restrict__ fmt_out,
+                     const uint32_t* __restrict__ partials, int nparts, int rule) {
+    pdl_begin();
+    __shared__ uint32_t sh;
+    const float amax = __uint_as_float(reduce_partials(partials, nparts, &sh));
+    const bool e5 = amax > 448.0f;
+    const float scale = amax == 0.0f ? 1.0f
+                        : (e5 ? scale_from_amax<kE5M2>(amax, rule) : scale_from_amax<kE4M3>(amax, rule));
+    // finite amax > 0 with a finite scale cannot overflow, and a NaN amax
+    // makes every product NaN; only an overflowed scale needs the fix-up
+    const bool fix = isinf(scale);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        sinv[0] = __fdiv_rn(1.0f, scale);
+        fmt_out[0] = e5 ? kE5M2 : kE4M3;
+    }
+    if (e5) cast_tensor_body<XT, kE5M2, VB>(x, numel, q, scale, fix);
+    else cast_tensor_body<XT, kE4M3, VB>(x, numel, q, scale, fix);
+}
+
+// ColossalAI cast_from_fp8_pipeline: y = T(fl(float(q) * scale_inv[0])) in
+// the format the tag names (1 = e5m2, anything else e4m3fn); 16 codes per
+// thread when q and y allow 16-byte accesses (VEC), else one
+template <int FMT, int YT>
+__device__ __forceinline__ void decode16(uint4 c, float sc, void* y, int64_t e) {
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    if (YT == kF32) {
+        float* yf = static_cast<float*>(y) + e;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 a = dec2<FMT>(w[i] & 0xFFFFu), b = dec2<FMT>(w[i] >> 16);
+            st_v4(yf + 4 * i, make_uint4(__float_as_uint(__fmul_rn(a.x, sc)), __float_as_uint(__fmul_rn(a.y, sc)),
+                                         __float_as_uint(__fmul_rn(b.x, sc)), __float_as_uint(__fmul_rn(b.y, sc))));
+        }
+    } else {
+        uint16_t* yh = static_cast<uint16_t*>(y) + e;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float2 a = dec2<FMT>(w[2 * h + i] & 0xFFFFu), b = dec2<FMT>(w[2 * h + i] >> 16);
+                o[2 * i] = pack2<YT>(__fmul_rn(a.x, sc), __fmul_rn(a.y, sc));
+                o[2 * i + 1] = pack2<YT>(__fmul_rn(b.x, sc), __fmul_rn(b.y, sc));
+            }
+            st_v4(yh + 8 * h, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    }
+}
+
+template <int FMT, int YT>
+__device__ __forceinline__ void decode_one(uint8_t c, float sc, void* y, int64_t e) {
+    const float v = __fmul_rn(dec2<FMT>(c).x, sc);
+    if (YT == kF32) static_cast<float*>(y)[e] = v;
+    else static_cast<uint16_t*>(y)[e] = (uint16_t)(pack2<YT>(v, 0.0f) & 0xFFFFu);
+}
+
+template <int FMT, int YT, bool VEC>
+__device__ __forceinline__ void decode_body(const uint8_t* __restrict__ q, int64_t numel, float sc, void* y) {
+    const int64_t stride = (int64_t)gridDim.x * kPtThreads;
+    const int64_t t0 = (int64_t)blockIdx.x * kPtThreads + threadIdx.x;
+    if (VEC) {
+        const int64_t nch = numel / 16;
+        for (int64_t t = t0; t < nch; t += stride) decode16<FMT, YT>(ld_stream_v4(q + t * 16), sc, y, t * 16);
+        if (blockIdx.x == 0 && threadIdx.x < numel - nch * 16) {
+            const int64_t e = nch * 16 + threadIdx.x;
+            decode_one<FMT, YT>(q[e], sc, y, e);
+        }
+    } else {
+        for (int64_t e = t0; e < numel; e += stride) decode_one<FMT, YT>(q[e], sc, y, e);
+    }
+}
+
+template <int YT, bool VEC>
+__global__ void __launch_bounds__(kPtThreads)
+pipeline_decode_kernel(const uint8_t* __restrict__ q, int64_t numel, const float* __restrict__ sinv,
+                       const int32_t* __restrict__ fmt_in, void* __restrict__ y) {
+    pdl_begin();
+    const float sc = __ldg(sinv);
+    if (__ldg(fmt_in) == kE5M2) decode_body<kE5M2, YT, VEC>(q, numel, sc, y);
+    else decode_body<kE4M3, YT, VEC>(q, numel, sc, y);
+}
+
+// the amax of a tensor as fp32 magnitude bits, from the amax pass's partials
+// (one CTA); ranks holding shards of one tensor combine these words with an
+// integer MAX, which orders magnitudes and propagates NaN like the kernels
+__global__ void __launch_bounds__(kPtThreads)
+amax_finish_kernel(const uint32_t* __restrict__ partials, int nparts, uint32_t* __restrict__ amax_bits) {
+    pdl_begin();
+    __shared__ uint32_t sh;
+    const uint32_t bits = reduce_partials(partials, nparts, &sh);
+    if (threadIdx.x == 0) amax_bits[0] = bits;
 }
 
 __global__ void fill_kernel(float* __restrict__ dst, int64_t count, float value) {
@@ -360,6 +475,54 @@ fp8q_status launch_fill(float* dst, int64_t count, float value, cudaStream_t s) 
     return cuda_status(err);
 }
 
+// the pipeline cast: the amax pass, then the format-selecting cast pass
+template <int XT, int VB>
+fp8q_status pipeline_launch(const uint8_t* x, int64_t numel, uint8_t* q, float* sinv, int32_t* fmt_out,
+                            uint32_t* partials, int rule, cudaStream_t s) {
+    constexpr int ES = ElemBytes<XT>::value;
+    const int64_t units = VB > 0 ? numel * ES / VB : numel;
+    int64_t want = (units + kPtThreads * kPtUnroll - 1) / (kPtThreads * kPtUnroll);
+    static const int per_sm = min(resident_blocks_per_sm(tensor_amax_kernel<XT, VB>, kPtThreads),
+                                  resident_blocks_per_sm(pipeline_cast_kernel<XT, VB>, kPtThreads));
+    int64_t cap = (int64_t)sm_count() * min(per_sm, 8);
+    if (cap > kMaxPartials) cap = kMaxPartials;
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    const int grid = (int)want;
+    cudaError_t err = launch_kernel(tensor_amax_kernel<XT, VB>, dim3(grid), dim3(kPtThreads), s, x, numel, partials);
+    if (err != cudaSuccess) return FP8Q_ERR_CUDA;
+    err = launch_kernel(pipeline_cast_kernel<XT, VB>, dim3(grid), dim3(kPtThreads), s, x, numel, q, sinv, fmt_out,
+                        partials, grid, rule);
+    return cuda_status(err);
+}
+
+template <int XT>
+fp8q_status run_pipeline(const uint8_t* x, int64_t numel, uint8_t* q, float* sinv, int32_t* fmt_out,
+                         uint32_t* partials, int rule, cudaStream_t s) {
+    constexpr int ES = ElemBytes<XT>::value;
+    const int vb = vector_bytes(x, 0, q, ES);
+    if (vb == 32) return pipeline_launch<XT, 32>(x, numel, q, sinv, fmt_out, partials, rule, s);
+    if (vb == 16) return pipeline_launch<XT, 16>(x, numel, q, sinv, fmt_out, partials, rule, s);
+    return pipeline_launch<XT, 0>(x, numel, q, sinv, fmt_out, partials, rule, s);
+}
+
+template <int YT>
+fp8q_status run_pipeline_decode(const uint8_t* q, int64_t numel, const float* sinv, const int32_t* fmt_in,
+                                void* y, cudaStream_t s) {
+    const int ys = YT == kF32 ? 4 : 2;
+    const bool vec = (uintptr_t)q % 16 == 0 && (uintptr_t)y % 16 == 0;
+    const int64_t units = vec ? numel / 16 : numel;
+    int64_t want = (units + kPtThreads * 4 - 1) / (kPtThreads * 4);
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    (void)ys;
+    const cudaError_t err = vec
+        ? launch_kernel(pipeline_decode_kernel<YT, true>, dim3((unsigned)want), dim3(kPtThreads), s, q, numel, sinv, fmt_in, y)
+        : launch_kernel(pipeline_decode_kernel<YT, false>, dim3((unsigned)want), dim3(kPtThreads), s, q, numel, sinv, fmt_in, y);
+    return cuda_status(err);
+}
+
 fp8q_status launch_per_channel(const void* x, int xt, int64_t rows, int64_t cols, int fmt,
                                uint8_t* q, float* sinv, int rule, cudaStream_t s) {
     const uint8_t* xb = static_cast<const uint8_t*>(x);
@@ -377,6 +540,107 @@ fp8q_status launch_per_tensor(const void* x, int xt, int64_t numel, int fmt, uin
     case kF32: return per_tensor_fmt<kF32>(xb, fmt, numel, q, sinv, partials, rule, s);
     case kF16: return per_tensor_fmt<kF16>(xb, fmt, numel, q, sinv, partials, rule, s);
     default: return per_tensor_fmt<kBF16>(xb, fmt, numel, q, sinv, partials, rule, s);
+    }
+}
+
+// amax pass + finish: amax_bits[0] = magnitude bits of max |x|
+template <int XT, int VB>
+fp8q_status tensor_amax_launch(const uint8_t* x, int64_t numel, uint32_t* partials, uint32_t* amax_bits,
+                               cudaStream_t s) {
+    constexpr int ES = ElemBytes<XT>::value;
+    const int64_t units = VB > 0 ? numel * ES / VB : numel;
+    int64_t want = (units + kPtThreads * kPtUnroll - 1) / (kPtThreads * kPtUnroll);
+    static const int per_sm = resident_blocks_per_sm(tensor_amax_kernel<XT, VB>, kPtThreads);
+    int64_t cap = (int64_t)sm_count() * min(per_sm, 8);
+    if (cap > kMaxPartials) cap = kMaxPartials;
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    const int grid = (int)want;
+    cudaError_t err = launch_kernel(tensor_amax_kernel<XT, VB>, dim3(grid), dim3(kPtThreads), s, x, numel, partials);
+    if (err != cudaSuccess) return FP8Q_ERR_CUDA;
+    err = launch_kernel(amax_finish_kernel, dim3(1), dim3(kPtThreads), s, (const uint32_t*)partials, grid, amax_bits);
+    return cuda_status(err);
+}
+
+// the cast pass with an amax given on the device (one "partial")
+template <int XT, int FMT, int VB>
+fp8q_status cast_with_amax_launch(const uint8_t* x, int64_t numel, uint8_t* q, float* sinv,
+                                  const uint32_t* amax_bits, int rule, cudaStream_t s) {
+    constexpr int ES = ElemBytes<XT>::value;
+    const int64_t units = VB > 0 ? numel * ES / VB : numel;
+    int64_t want = (units + kPtThreads * kPtUnroll - 1) / (kPtThreads * kPtUnroll);  // >= 1 CTA even when empty
+    static const int per_sm = resident_blocks_per_sm(tensor_cast_kernel<XT, FMT, VB>, kPtThreads);
+    const int64_t cap = (int64_t)sm_count() * min(per_sm, 8);
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    const cudaError_t err = launch_kernel(tensor_cast_kernel<XT, FMT, VB>, dim3((unsigned)want), dim3(kPtThreads), s,
+                                          x, numel, q, sinv, amax_bits, 1, rule);
+    return cuda_status(err);
+}
+
+template <int XT>
+fp8q_status run_tensor_amax(const uint8_t* x, int64_t numel, uint32_t* partials, uint32_t* amax_bits,
+                            cudaStream_t s) {
+    // the amax pass only reads x: its own alignment picks the vector width
+    const int vb = vector_bytes(x, 0, x, 1);
+    if (vb == 32) return tensor_amax_launch<XT, 32>(x, numel, partials, amax_bits, s);
+    if (vb == 16) return tensor_amax_launch<XT, 16>(x, numel, partials, amax_bits, s);
+    return tensor_amax_launch<XT, 0>(x, numel, partials, amax_bits, s);
+}
+
+template <int XT, int FMT>
+fp8q_status run_cast_with_amax(const uint8_t* x, int64_t numel, uint8_t* q, float* sinv, const uint32_t* amax_bits,
+                               int rule, cudaStream_t s) {
+    constexpr int ES = ElemBytes<XT>::value;
+    const int vb = vector_bytes(x, 0, q, ES);
+    if (vb == 32) return cast_with_amax_launch<XT, FMT, 32>(x, numel, q, sinv, amax_bits, rule, s);
+    if (vb == 16) return cast_with_amax_launch<XT, FMT, 16>(x, numel, q, sinv, amax_bits, rule, s);
+    return cast_with_amax_launch<XT, FMT, 0>(x, numel, q, sinv, amax_bits, rule, s);
+}
+
+fp8q_status launch_cast_pipeline(const void* x, int xt, int64_t numel, uint8_t* q, float* sinv,
+                                 int32_t* fmt_out, uint32_t* partials, int rule, cudaStream_t s) {
+    const uint8_t* xb = static_cast<const uint8_t*>(x);
+    switch (xt) {
+    case kF32: return run_pipeline<kF32>(xb, numel, q, sinv, fmt_out, partials, rule, s);
+    case kF16: return run_pipeline<kF16>(xb, numel, q, sinv, fmt_out, partials, rule, s);
+    default: return run_pipeline<kBF16>(xb, numel, q, sinv, fmt_out, partials, rule, s);
+    }
+}
+
+fp8q_status launch_cast_from_pipeline(const uint8_t* q, int64_t numel, const float* sinv, const int32_t* fmt_in,
+                                      int yt, void* y, cudaStream_t s) {
+    switch (yt) {
+    case kF32: return run_pipeline_decode<kF32>(q, numel, sinv, fmt_in, y, s);
+    case kF16: return run_pipeline_decode<kF16>(q, numel, sinv, fmt_in, y, s);
+    default: return run_pipeline_decode<kBF16>(q, numel, sinv, fmt_in, y, s);
+    }
+}
+
+fp8q_status launch_tensor_amax(const void* x, int xt, int64_t numel, uint32_t* partials, uint32_t* amax_bits,
+                               cudaStream_t s) {
+    const uint8_t* xb = static_cast<const uint8_t*>(x);
+    switch (xt) {
+    case kF32: return run_tensor_amax<kF32>(xb, numel, partials, amax_bits, s);
+    case kF16: return run_tensor_amax<kF16>(xb, numel, partials, amax_bits, s);
+    default: return run_tensor_amax<kBF16>(xb, numel, partials, amax_bits, s);
+    }
+}
+
+fp8q_status launch_cast_with_amax(const void* x, int xt, int64_t numel, int fmt, const uint32_t* amax_bits,
+                                  uint8_t* q, float* sinv, int rule, cudaStream_t s) {
+    const uint8_t* xb = static_cast<const uint8_t*>(x);
+    if (fmt == kE4M3) {
+        switch (xt) {
+        case kF32: return run_cast_with_amax<kF32, kE4M3>(xb, numel, q, sinv, amax_bits, rule, s);
+        case kF16: return run_cast_with_amax<kF16, kE4M3>(xb, numel, q, sinv, amax_bits, rule, s);
+        default: return run_cast_with_amax<kBF16, kE4M3>(xb, numel, q, sinv, amax_bits, rule, s);
+        }
+    }
+    switch (xt) {
+    case kF32: return run_cast_with_amax<kF32, kE5M2>(xb, numel, q, sinv, amax_bits, rule, s);
+    case kF16: return run_cast_with_amax<kF16, kE5M2>(xb, numel, q, sinv, amax_bits, rule, s);
+    default: return run_cast_with_amax<kBF16, kE5M2>(xb, numel, q, sinv, amax_bits, rule, s);
     }
 }
 

@@ -198,6 +198,94 @@ fp8q_status fp8q_cast_per_tensor_noalloc(const void* x, fp8q_dtype xt, int64_t n
                                          uint8_t* q, float* scale_inv, fp8q_stream_t stream);
 
 /*
+ * Per-tensor cast of a tensor sharded across ranks, in two calls with a
+ * 4-byte exchange between them -- the pattern of ColossalAI
+ * fp8_compress_fsdp_params_comm_hook (all_reduce(MAX) of the per-tensor max,
+ * then scale = fp8_max / max on every rank):
+ *   fp8q_tensor_amax:   amax_bits[0] = fp32 bit pattern of max |x| over this
+ *                       rank's numel elements (0 for an empty shard).  The
+ *                       sign bit is clear, so as int32 the words of all
+ *                       ranks order like the magnitudes and every NaN lies
+ *                       above +Inf: an integer MAX over ranks (e.g. NCCL
+ *                       all_reduce MAX on int32) gives the amax of the whole
+ *                       tensor with NaN propagating.
+ *   fp8q_cast_per_tensor_with_amax: the per-tensor cast of this shard with the
+ *                       amax read from amax_bits[0] (zero or NaN replaced by
+ *                       1, scale and scale_inv as in fp8q_cast_per_tensor).
+ * Every rank then holds the bytes the one-tensor cast gives for its slice,
+ * and every rank -- one with an empty shard too -- the same scale_inv, derived
+ * from the global amax.  (The one-tensor calls return scale_inv = 1.0 for an
+ * empty tensor; a sharded tensor that is empty on every rank has amax 0,
+ * which becomes 1 as for any zero tensor, so its scale_inv is fl(1 / FMAX).)
+ * amax_bits: device uint32 [1]; workspace as fp8q_cast_per_tensor.
+ */
+fp8q_status fp8q_tensor_amax(const void* x, fp8q_dtype xt, int64_t numel, uint32_t* amax_bits,
+                             void* workspace, size_t workspace_bytes, fp8q_stream_t stream);
+fp8q_status fp8q_cast_per_tensor_with_amax(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt,
+                                           const uint32_t* amax_bits, uint8_t* q, float* scale_inv,
+                                           fp8q_scale_rule rule, fp8q_stream_t stream);
+
+/*
+ * Pipeline cast -- ColossalAI cast_to_fp8_pipeline: a per-tensor cast whose
+ * fp8 format follows the data, for activations sent between pipeline stages.
+ *   amax  = max |x| over all numel elements (NaN propagates)
+ *   fmt   = amax > 448 (the e4m3fn maximum) ? e5m2 : e4m3fn
+ *           (a NaN amax fails the test and gives e4m3fn)
+ *   scale = amax == 0 ? 1 : FMAX(fmt) / amax        (rounded per `rule`)
+ *   q[i]  = fmt(fl(float(x[i]) * scale)); scale_inv[0] = fl(1 / scale)
+ *   fmt_tag[0] = the chosen fp8q_format (0 e4m3fn, 1 e5m2)
+ * The page carries the format in the view dtype of the payload; here it is
+ * a device int32 written on the stream, so the call needs no host round
+ * trip and the decode reads it on the device.  Two kernels, as
+ * fp8q_cast_per_tensor, with the same workspace rules.
+ * Empty tensor (numel == 0): scale_inv[0] = 1.0 and fmt_tag[0] = e4m3fn.
+ */
+fp8q_status fp8q_cast_pipeline(const void* x, fp8q_dtype xt, int64_t numel, uint8_t* q,
+                               float* scale_inv, int32_t* fmt_tag, void* workspace,
+                               size_t workspace_bytes, fp8q_scale_rule rule, fp8q_stream_t stream);
+
+/*
+ * Pipeline decode -- ColossalAI cast_from_fp8_pipeline:
+ *   y[i] = T(fl(float(q[i]) * scale_inv[0])), the codes read in the format
+ *   fmt_tag[0] names (a device int32 as fp8q_cast_pipeline writes it: 1 is
+ *   e5m2, any other value e4m3fn).
+ * q: numel codes; scale_inv: [1]; y: numel elements of yt (output).
+ */
+fp8q_status fp8q_cast_from_pipeline(const uint8_t* q, int64_t numel, const float* scale_inv,
+                                    const int32_t* fmt_tag, fp8q_dtype yt, void* y,
+                                    fp8q_stream_t stream);
+
+/*
+ * fp8-compressed all-gather records -- ColossalAI all_gather_fp8_lagacy (and
+ * _all_gather_fp8): every rank casts its tensor with its own per-tensor
+ * scale and sends [scale | fp8 payload]; every rank then dequantises each
+ * received chunk with the scale in its header.  A record here is
+ *   bytes [0, 4)            fp32 scale_inv (fl(1 / scale) of the per-tensor cast)
+ *   bytes [4, 16)           zero
+ *   bytes [16, 16 + numel)  fp8 codes, then zero padding to a multiple of 16
+ * (the page uses a 4-byte header; 16 keeps the payload 16-byte aligned), so
+ * records of equal numel can be gathered back to back by any byte-level
+ * all-gather (NCCL all_gather_into_tensor on uint8).
+ *   fp8q_record_bytes:   the record size for numel codes.
+ *   fp8q_pack_record:    the per-tensor cast of x into `record` (scale rule as
+ *                        fp8q_cast_per_tensor_ex; workspace likewise).
+ *   fp8q_unpack_records: `count` records of numel codes each, laid out
+ *                        back to back (records 16-byte aligned), dequantised
+ *                        into y[count][numel] (type yt, element-aligned):
+ *                        y[r][i] = T(fl(float(code) * scale_inv of record r)),
+ *                        one launch per 48 records.  count == 0 or numel == 0
+ *                        enqueues nothing.
+ * Ownership and errors as for the calls above: caller-owned device buffers,
+ * host-side checks before any launch, nothing allocated.
+ */
+size_t fp8q_record_bytes(int64_t numel);
+fp8q_status fp8q_pack_record(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt, uint8_t* record,
+                             void* workspace, size_t workspace_bytes, fp8q_scale_rule rule,
+                             fp8q_stream_t stream);
+fp8q_status fp8q_unpack_records(const uint8_t* records, int count, int64_t numel, fp8q_format fmt,
+                                fp8q_dtype yt, void* y, fp8q_stream_t stream);
+
+/*
  * Block dequantisation -- DeepSeek-V3 weight_dequant / weight_dequant_kernel:
  *   y[i][j] = T(fl(float(w[i][j]) * scale_inv[i / B][j / B]))
  *   with scale_inv row-major [ceil(M/B)][ceil(N/B)] (the kernel's

@@ -274,3 +274,68 @@ def cast_from_fp8(q: np.ndarray, scale_inv: np.ndarray, gran: int, fmt: int = E4
     _run(lambda a, b: _check(L.orc_cast_from_fp8(_ptr(q), fmt, R, C, _ptr(s), gran, gb, yt, _ptr(y), a, b),
                              "cast_from_fp8"), r0, r1, threads)
     return y
+
+
+# ---------------------------------------------------------------------------
+# fp8-compressed collectives (ColossalAI colossalai/quantization/fp8.py:
+# all_gather_fp8, all_gather_fp8_lagacy, all_to_all_fp8, all_to_all_single_fp8).
+# Each is the per-tensor cast of what a rank sends, the bytes moved as they
+# are, and cast_from_fp8 with the sender's scale_inv on receipt; the ranks
+# are plain Python lists here.  The record is the sender's
+# [fp32 scale_inv | fp8 codes] buffer of all_gather_fp8_lagacy, with a
+# 16-byte header (scale_inv in bytes 0..3, zeros after) and the payload
+# zero-padded to a multiple of 16 bytes.
+# ---------------------------------------------------------------------------
+RECORD_HEADER = 16
+
+
+def record_size(numel: int) -> int:
+    return RECORD_HEADER + ((numel + 15) // 16) * 16
+
+
+def record(x: np.ndarray, xt: int, fmt: int, rule: int = RULE_IEEE) -> np.ndarray:
+    """The sender's record for tensor x: its per-tensor cast, header first."""
+    q, s = cast_per_tensor(x, xt, fmt, rule=rule)
+    r = np.zeros((record_size(q.size),), np.uint8)
+    r[0:4] = np.frombuffer(s.astype("<f4").tobytes(), np.uint8)
+    r[RECORD_HEADER:RECORD_HEADER + q.size] = q
+    return r
+
+
+def record_decode(r: np.ndarray, numel: int, fmt: int, yt: int) -> np.ndarray:
+    """The receiver's step: cast_from_fp8 of the payload with the header's scale_inv."""
+    s = np.frombuffer(r[0:4].tobytes(), "<f4").astype(np.float32)
+    q = r[RECORD_HEADER:RECORD_HEADER + numel].reshape(1, numel)
+    return cast_from_fp8(q, s, GRAN_TENSOR, fmt, yt=yt).reshape(-1)
+
+
+def all_gather_fp8(xs, xt: int, fmt: int, rule: int = RULE_IEEE):
+    """xs[r] = rank r's tensor; returns out[r], which every rank receives:
+    rank r's tensor cast with rank r's own scale and cast back to xt."""
+    return [record_decode(record(x, xt, fmt, rule), np.asarray(x).size, fmt, xt) for x in xs]
+
+
+def all_to_all_fp8(inputs, xt: int, fmt: int, rule: int = RULE_IEEE):
+    """inputs[j][i] = what rank j sends to rank i (each with its own scale);
+    returns outputs[i][j] = what rank i receives from rank j."""
+    W = len(inputs)
+    return [[record_decode(record(inputs[j][i], xt, fmt, rule), np.asarray(inputs[j][i]).size, fmt, xt)
+             for j in range(W)] for i in range(W)]
+
+
+def all_to_all_single_fp8(inputs, xt: int, fmt: int, rule: int = RULE_IEEE):
+    """inputs[j] = rank j's whole tensor (flat, numel divisible by the rank
+    count), cast with ONE scale; rank i receives chunk i of every sender's
+    codes and decodes each with that sender's scale_inv.  Returns
+    outputs[i], the concatenation over senders j."""
+    W = len(inputs)
+    casts = [cast_per_tensor(x, xt, fmt, rule=rule) for x in inputs]
+    out = []
+    for i in range(W):
+        parts = []
+        for j in range(W):
+            q, s = casts[j]
+            c = q.size // W
+            parts.append(cast_from_fp8(q[i * c:(i + 1) * c].reshape(1, c), s, GRAN_TENSOR, fmt, yt=xt).reshape(-1))
+        out.append(np.concatenate(parts))
+    return out

@@ -22,6 +22,10 @@ Workloads (shapes and value mixes of the pages' use cases):
   Seed 20261241.
 * ``c4b`` per-tensor: fp32 v[64 Mi] ~ N(0, sigma = 1e-2).  Seed 20261242.
 * ``c4c`` per-tensor zero: fp16 [1 Mi] all +0.  Seed 20261243 (unused).
+* ``device_normal`` / ``device_codes``: inputs above 2^32 elements (the
+  64-bit indexing cases), drawn on the device by torch's seeded CUDA
+  generator in chunks, because the host cannot draw them in seconds.  The
+  tests copy sampled rows back for the oracle.
 * ``c5`` ragged MoE dequant: 64 weights [2048, 7168] then 8 weights
   [7000, 1000]; codes uniform over the finite e4m3fn codes; ceil-sized
   scales exp(N(-8, 1)).  Weight i draws from seed (20261205, i) so any
@@ -141,3 +145,48 @@ def c5_weight(i: int):
     w = uniform_codes(g, (M, N), finite_e4m3fn_codes())
     s = lognormal_scales(g, scale_shape(M, N))
     return w, s
+
+
+# ---------------------------------------------------------------------------
+# device-side draws for the largest sizes
+# ---------------------------------------------------------------------------
+_CHUNK = 1 << 27
+
+
+def device_normal(shape, seed: int, dtype=torch.bfloat16, device="cuda", row_scale: bool = True,
+                  std: float = 1.0) -> torch.Tensor:
+    """N(0, std) draws of `shape` stored as `dtype`, made on the device by a
+    torch.Generator seeded with `seed`, 128 Mi elements at a time.  With
+    row_scale (2-D shapes), row r is multiplied by 2^((r mod 17) - 8), so
+    that rows far apart differ in magnitude and an index that wraps lands
+    on visibly different data."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    out = torch.empty(shape, dtype=dtype, device=device)
+    flat = out.view(-1)
+    n = flat.numel()
+    cols = shape[-1] if len(shape) == 2 else n
+    for a in range(0, n, _CHUNK):
+        b = min(n, a + _CHUNK)
+        v = torch.randn(b - a, generator=g, device=device, dtype=torch.float32) * std
+        if row_scale and len(shape) == 2:
+            r = torch.arange(a, b, device=device, dtype=torch.int64) // cols
+            v *= torch.exp2((r % 17 - 8).to(torch.float32))
+        flat[a:b] = v.to(dtype)
+    return out
+
+
+def device_codes(shape, seed: int, device="cuda") -> torch.Tensor:
+    """fp8 e4m3fn codes uniform over the 254 finite codes, drawn on the
+    device by a torch.Generator seeded with `seed`."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    out = torch.empty(shape, dtype=torch.uint8, device=device)
+    flat = out.view(-1)
+    n = flat.numel()
+    for a in range(0, n, _CHUNK):
+        b = min(n, a + _CHUNK)
+        k = torch.randint(0, 254, (b - a,), generator=g, device=device, dtype=torch.int32)
+        k = k + (k >= 0x7F).to(torch.int32)               # skip 0x7F; 0xFF is never reached
+        flat[a:b] = k.to(torch.uint8)
+    return out
