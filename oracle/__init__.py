@@ -86,6 +86,9 @@ def lib() -> ctypes.CDLL:
             L.orc_block_dequant.argtypes = [c_void, i32, i64, i64, c_void, i32, i32, c_void, i64, i64]
             L.orc_cast_from_fp8.restype = i32
             L.orc_cast_from_fp8.argtypes = [c_void, i32, i64, i64, c_void, i32, i32, i32, c_void, i64, i64]
+            L.orc_scaled_mm.restype = i32
+            L.orc_scaled_mm.argtypes = [c_void, i32, c_void, i32, i64, i64, i64, ctypes.c_float, ctypes.c_float,
+                                        c_void, c_void, i64, i64]
             _lib = L
     return _lib
 
@@ -338,4 +341,28 @@ def all_to_all_single_fp8(inputs, xt: int, fmt: int, rule: int = RULE_IEEE):
             c = q.size // W
             parts.append(cast_from_fp8(q[i * c:(i + 1) * c].reshape(1, c), s, GRAN_TENSOR, fmt, yt=xt).reshape(-1))
         out.append(np.concatenate(parts))
+    return out
+
+
+def scaled_mm(a: np.ndarray, fa: int, b: np.ndarray, fb: int, sa: float, sb: float, bias=None, rows=None,
+              threads: int = 1) -> np.ndarray:
+    """ColossalAI linear_fp8 forward (torch._scaled_mm with per-tensor scales):
+    a[M, K] and b[N, K] fp8 codes; returns out[M, N] in float64 (rows outside
+    `rows` are zero)."""
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    M, K = a.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError("a and b need the same K")
+    out = np.zeros((M, N), np.float64)
+    bp = None
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float64)
+        bp = ctypes.c_void_p(bias.ctypes.data)
+    r0, r1 = rows if rows is not None else (0, M)
+    L = lib()
+    _run(lambda x, y: _check(L.orc_scaled_mm(_ptr(a), fa, _ptr(b), fb, M, N, K, ctypes.c_float(sa),
+                                             ctypes.c_float(sb), bp, _ptr(out), x, y), "scaled_mm"),
+         r0, r1, threads)
     return out

@@ -491,3 +491,39 @@ int orc_cast_from_fp8(const uint8_t* q, int fmt, int64_t rows, int64_t cols,
     }
     return 0;
 }
+
+/*
+ * [CAI] linear_fp8 forward (_LinearFp8.forward): both operands are cast to
+ * fp8 with per-tensor scales and multiplied by torch._scaled_mm(x_fp8,
+ * w_fp8.t(), scale_a = scale_inv of x, scale_b = scale_inv of w, bias):
+ *     out[m][n] = (sum over k of dec(a[m][k]) * dec(b[n][k])) * sa * sb + bias[n]
+ * a is [M][K] (the activations), b is [N][K] (the weight, as stored; the
+ * product uses its transpose).  Evaluated in binary64: every product of two
+ * fp8 values is exact, and for e4m3fn operands every partial sum is exact
+ * too (products span 2^-18 .. 2^17.6 with 8 significant bits, and K < 2^20
+ * keeps the sums inside 53 bits), so for e4m3fn the sum is the exact one.
+ * bias may be NULL.  Only rows [r0, r1) of out are written.
+ */
+int orc_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
+                  float sa, float sb, const double* bias, double* out, int64_t r0, int64_t r1)
+{
+    if (!valid_fmt(fa) || !valid_fmt(fb) || M < 0 || N < 0 || K < 0 || r0 < 0 || r1 > M || r0 > r1)
+        return -1;
+    double da[256], db[256];
+    for (int c = 0; c < 256; ++c) {
+        da[c] = (double)orc_fp8_decode((uint8_t)c, fa);
+        db[c] = (double)orc_fp8_decode((uint8_t)c, fb);
+    }
+    for (int64_t m = r0; m < r1; ++m) {
+        const uint8_t* ar = a + m * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t* br = b + n * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += da[ar[k]] * db[br[k]];
+            double v = acc * (double)sa * (double)sb;
+            if (bias) v += bias[n];
+            out[m * N + n] = v;
+        }
+    }
+    return 0;
+}

@@ -126,6 +126,13 @@ int orc_cast_from_fp8(const uint8_t* q, int fmt, int64_t rows, int64_t cols,
                       const float* scale_inv, int gran, int gb, int yt,
                       void* y, int64_t r0, int64_t r1);
 
+/* [CAI] linear_fp8 forward, torch._scaled_mm with per-tensor scales:
+ * out[m][n] = (sum_k dec(a[m][k]) * dec(b[n][k])) * sa * sb + bias[n], in
+ * binary64 (exact sums for e4m3fn operands); a [M][K], b [N][K]; bias NULL
+ * or [N]; rows [r0, r1) of out[M][N]. */
+int orc_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
+                  float sa, float sb, const double* bias, double* out, int64_t r0, int64_t r1);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,98 @@
+"""Pins for the oracle's scaled fp8 matrix product (CPU only).
+
+ColossalAI colossalai/quantization/fp8.py, _LinearFp8.forward:
+torch._scaled_mm(x_fp8, w_fp8.t(), scale_a, scale_b, bias) with the
+per-tensor scale_inv of each operand, i.e.
+    out[m][n] = (sum_k dec(a[m][k]) * dec(b[n][k])) * sa * sb + bias[n].
+
+Pinned by: closed forms (constant operands), an identity operand that
+returns the other operand transposed (a transposed or swapped operand fails),
+exact integer arithmetic (every e4m3fn value is a multiple of 2^-9, so the
+exact sum is an integer count of 2^-18 units), numpy's float64 product of the
+decoded operands, and the row range.
+"""
+import numpy as np
+import pytest
+
+E4M3FN, E5M2 = 0, 1
+ONE = {E4M3FN: 0x38, E5M2: 0x3C}          # the code of 1.0
+
+
+def _finite_codes(g, shape, fmt):
+    import workloads
+    codes = workloads.finite_e4m3fn_codes() if fmt == E4M3FN else workloads.finite_e5m2_codes()
+    c = workloads.uniform_codes(g, shape, codes)
+    if fmt == E5M2:
+        c[(c & 0x7F) == 0x7C] = 0                # no infinities in the random operands
+    return c
+
+
+def test_closed_form_constants(orc):
+    for fa, fb in ((E4M3FN, E4M3FN), (E5M2, E4M3FN), (E4M3FN, E5M2)):
+        M, N, K = 3, 5, 96
+        a = np.full((M, K), ONE[fa], np.uint8)                 # 1.0
+        b = np.full((N, K), ONE[fb] + (4 if fb == E4M3FN else 2), np.uint8)   # 1.5
+        bias = np.arange(N, dtype=np.float64) - 2.0
+        out = orc.scaled_mm(a, fa, b, fb, 0.5, 0.25, bias=bias)
+        np.testing.assert_array_equal(out, np.tile(K * 1.5 * 0.125 + bias, (M, 1)))
+        # negative codes flip the sign; no bias
+        out = orc.scaled_mm(a | 0x80, fa, b, fb, 2.0, 1.0)
+        np.testing.assert_array_equal(out, np.full((M, N), -K * 1.5 * 2.0))
+
+
+@pytest.mark.parametrize("fmt", [E4M3FN, E5M2])
+def test_identity_operand_gives_the_other_transposed(orc, fmt):
+    g = np.random.default_rng(11 + fmt)
+    K, N = 48, 7
+    a = np.zeros((K, K), np.uint8)
+    a[np.arange(K), np.arange(K)] = ONE[fmt]
+    b = _finite_codes(g, (N, K), fmt)
+    out = orc.scaled_mm(a, fmt, b, fmt, 1.0, 1.0)
+    np.testing.assert_array_equal(out, orc.fp8_decode(b, fmt).astype(np.float64).T)
+    # and as the right operand: out = dec(a_rand) (b = identity, stored [N][K])
+    out = orc.scaled_mm(b, fmt, a, fmt, 1.0, 1.0)
+    np.testing.assert_array_equal(out, orc.fp8_decode(b, fmt).astype(np.float64))
+
+
+def test_e4m3_sum_is_exact(orc):
+    """Every e4m3fn value is an integer multiple of 2^-9: the exact sum,
+    counted in 2^-18 units with Python integers, equals the oracle's."""
+    g = np.random.default_rng(5)
+    M, N, K = 4, 6, 1000
+    a = _finite_codes(g, (M, K), E4M3FN)
+    b = _finite_codes(g, (N, K), E4M3FN)
+    out = orc.scaled_mm(a, E4M3FN, b, E4M3FN, 1.0, 1.0)
+    ia = (orc.fp8_decode(a, E4M3FN).astype(np.float64) * 512).astype(np.int64)
+    ib = (orc.fp8_decode(b, E4M3FN).astype(np.float64) * 512).astype(np.int64)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(int(x) * int(y) for x, y in zip(ia[m], ib[n]))
+            assert out[m, n] == exact / float(1 << 18)
+
+
+@pytest.mark.parametrize("fa,fb", [(E4M3FN, E4M3FN), (E5M2, E5M2), (E5M2, E4M3FN)])
+def test_matches_numpy_float64_product(orc, fa, fb):
+    g = np.random.default_rng(7 + fa + 2 * fb)
+    M, N, K = 33, 17, 256
+    a = _finite_codes(g, (M, K), fa)
+    b = _finite_codes(g, (N, K), fb)
+    sa, sb = np.float32(0.0123), np.float32(3.5)
+    bias = g.standard_normal(N)
+    out = orc.scaled_mm(a, fa, b, fb, float(sa), float(sb), bias=bias)
+    ref = (orc.fp8_decode(a, fa).astype(np.float64) @ orc.fp8_decode(b, fb).astype(np.float64).T)
+    ref = ref * float(sa) * float(sb) + bias
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_row_range_and_empty(orc):
+    g = np.random.default_rng(3)
+    a = _finite_codes(g, (10, 32), E4M3FN)
+    b = _finite_codes(g, (4, 32), E4M3FN)
+    full = orc.scaled_mm(a, E4M3FN, b, E4M3FN, 1.0, 1.0)
+    part = orc.scaled_mm(a, E4M3FN, b, E4M3FN, 1.0, 1.0, rows=(3, 7))
+    np.testing.assert_array_equal(part[3:7], full[3:7])
+    assert not part[:3].any() and not part[7:].any()
+    # K = 0: the sum is empty, so out is the bias alone
+    out = orc.scaled_mm(np.zeros((2, 0), np.uint8), E4M3FN, np.zeros((3, 0), np.uint8), E4M3FN, 1.0, 1.0,
+                        bias=np.array([1.0, -2.0, 0.5]))
+    np.testing.assert_array_equal(out, np.array([[1.0, -2.0, 0.5]] * 2))
