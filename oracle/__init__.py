@@ -89,6 +89,9 @@ def lib() -> ctypes.CDLL:
             L.orc_scaled_mm.restype = i32
             L.orc_scaled_mm.argtypes = [c_void, i32, c_void, i32, i64, i64, i64, ctypes.c_float, ctypes.c_float,
                                         c_void, c_void, i64, i64]
+            L.orc_scaled_mm_blockwise.restype = i32
+            L.orc_scaled_mm_blockwise.argtypes = [c_void, i32, c_void, i64, c_void, i32, c_void, i64,
+                                                  i64, i64, i64, c_void, c_void, i64, i64]
             _lib = L
     return _lib
 
@@ -364,5 +367,34 @@ def scaled_mm(a: np.ndarray, fa: int, b: np.ndarray, fb: int, sa: float, sb: flo
     L = lib()
     _run(lambda x, y: _check(L.orc_scaled_mm(_ptr(a), fa, _ptr(b), fb, M, N, K, ctypes.c_float(sa),
                                              ctypes.c_float(sb), bp, _ptr(out), x, y), "scaled_mm"),
+         r0, r1, threads)
+    return out
+
+
+def scaled_mm_blockwise(a: np.ndarray, fa: int, sa: np.ndarray, b: np.ndarray, fb: int, sb: np.ndarray,
+                        group: int = 128, block: int = 128, bias=None, rows=None, threads: int = 1) -> np.ndarray:
+    """DeepEP per-token activations times a DeepSeek-V3 block-scaled weight:
+    a[M, K] codes with sa[M, ceil(K/group)], b[N, K] codes with
+    sb[ceil(N/block), ceil(K/block)]; returns out[M, N] in float64, the
+    product of the exactly dequantised operands (rows outside `rows` zero)."""
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    sb = np.ascontiguousarray(sb, dtype=np.float32)
+    M, K = a.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError("a and b need the same K")
+    if sa.shape != (M, -(-K // group)) or sb.shape != (-(-N // block), -(-K // block)):
+        raise ValueError("scale shapes do not match the operands")
+    out = np.zeros((M, N), np.float64)
+    bp = None
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float64)
+        bp = ctypes.c_void_p(bias.ctypes.data)
+    r0, r1 = rows if rows is not None else (0, M)
+    L = lib()
+    _run(lambda x, y: _check(L.orc_scaled_mm_blockwise(_ptr(a), fa, _ptr(sa), group, _ptr(b), fb, _ptr(sb), block,
+                                                       M, N, K, bp, _ptr(out), x, y), "scaled_mm_blockwise"),
          r0, r1, threads)
     return out

@@ -527,3 +527,50 @@ int orc_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M,
     }
     return 0;
 }
+
+/*
+ * The same product with fine-grained scales: the activations quantised by
+ * [DEP] per_token_cast_to_fp8 (one scale_inv per 1 x ga group of a row,
+ * sa[M][ceil(K/ga)]) times a weight stored as [DSV3] weight_dequant expects
+ * it (one scale_inv per bb x bb block, sb[ceil(N/bb)][ceil(K/bb)]):
+ *     out[m][n] = sum over k of (dec(a[m][k]) * sa[m][k/ga])
+ *                             * (dec(b[n][k]) * sb[n/bb][k/bb])  + bias[n]
+ * i.e. the product of the two dequantised operands, each element taken at
+ * its exact value (no rounding to bf16 in between).  Evaluated in binary64,
+ * k ascending: each dequantised element is exact in binary64 (4 + 24
+ * significant bits), so only the products and the running sum round, each
+ * at 2^-53 relative.  bias may be NULL.  Only rows [r0, r1) are written.
+ */
+int orc_scaled_mm_blockwise(const uint8_t* a, int fa, const float* sa, int64_t ga,
+                            const uint8_t* b, int fb, const float* sb, int64_t bb,
+                            int64_t M, int64_t N, int64_t K, const double* bias,
+                            double* out, int64_t r0, int64_t r1)
+{
+    if (!valid_fmt(fa) || !valid_fmt(fb) || M < 0 || N < 0 || K < 0 || ga < 1 || bb < 1 ||
+        r0 < 0 || r1 > M || r0 > r1)
+        return -1;
+    double da[256], db[256];
+    for (int c = 0; c < 256; ++c) {
+        da[c] = (double)orc_fp8_decode((uint8_t)c, fa);
+        db[c] = (double)orc_fp8_decode((uint8_t)c, fb);
+    }
+    int64_t ka = (K + ga - 1) / ga;          /* groups per activation row */
+    int64_t kb = (K + bb - 1) / bb;          /* blocks per weight block-row */
+    for (int64_t m = r0; m < r1; ++m) {
+        const uint8_t* ar = a + m * K;
+        const float* sar = sa + m * ka;
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t* br = b + n * K;
+            const float* sbr = sb + (n / bb) * kb;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double x = da[ar[k]] * (double)sar[k / ga];
+                double w = db[br[k]] * (double)sbr[k / bb];
+                acc += x * w;
+            }
+            if (bias) acc += bias[n];
+            out[m * N + n] = acc;
+        }
+    }
+    return 0;
+}

@@ -133,6 +133,15 @@ int orc_cast_from_fp8(const uint8_t* q, int fmt, int64_t rows, int64_t cols,
 int orc_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
                   float sa, float sb, const double* bias, double* out, int64_t r0, int64_t r1);
 
+/* [DEP] x [DSV3] the same product with per-token-group activation scales
+ * sa[M][ceil(K/ga)] and per-block weight scales sb[ceil(N/bb)][ceil(K/bb)]:
+ * out[m][n] = sum_k (dec(a[m][k]) * sa[m][k/ga]) * (dec(b[n][k]) * sb[n/bb][k/bb])
+ *             + bias[n], in binary64; rows [r0, r1) of out[M][N]. */
+int orc_scaled_mm_blockwise(const uint8_t* a, int fa, const float* sa, int64_t ga,
+                            const uint8_t* b, int fb, const float* sb, int64_t bb,
+                            int64_t M, int64_t N, int64_t K, const double* bias,
+                            double* out, int64_t r0, int64_t r1);
+
 #ifdef __cplusplus
 }
 #endif

@@ -96,3 +96,113 @@ def test_row_range_and_empty(orc):
     out = orc.scaled_mm(np.zeros((2, 0), np.uint8), E4M3FN, np.zeros((3, 0), np.uint8), E4M3FN, 1.0, 1.0,
                         bias=np.array([1.0, -2.0, 0.5]))
     np.testing.assert_array_equal(out, np.array([[1.0, -2.0, 0.5]] * 2))
+
+
+# ---------------------------------------------------------------------------
+# fine-grained scales: DeepEP per-token activations (sa[M][K/G]) times a
+# DeepSeek-V3 block-scaled weight (sb[ceil(N/B)][ceil(K/B)])
+# ---------------------------------------------------------------------------
+def _torch_decode(codes, fmt):
+    """Exact fp8 values from torch's own fp8 -> float64 conversion."""
+    import torch
+    dt = torch.float8_e4m3fn if fmt == E4M3FN else torch.float8_e5m2
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(dt).to(torch.float64).numpy()
+
+
+def _golden(name):
+    import os
+    p = os.path.join(os.path.dirname(__file__), "golden", name)
+    d = {}
+    for line in open(p):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            k, v = (s.strip() for s in line.split("=", 1))
+            d[k] = v
+    return d
+
+
+def test_blockwise_hand_worked(orc):
+    d = _golden("scaled_mm_blockwise_small.txt")
+    M, N, K, G, B = (int(d[k]) for k in ("M", "N", "K", "group", "block"))
+    a = np.array([int(t, 16) for t in d["a"].split()], np.uint8).reshape(M, K)
+    b = np.array([int(t, 16) for t in d["b"].split()], np.uint8).reshape(N, K)
+    sa = np.array(d["sa"].split(), np.float32).reshape(M, -(-K // G))
+    sb = np.array(d["sb"].split(), np.float32).reshape(-(-N // B), -(-K // B))
+    bias = np.array(d["bias"].split(), np.float64)
+    want = np.array(d["out"].split(), np.float64).reshape(M, N)
+    out = orc.scaled_mm_blockwise(a, E4M3FN, sa, b, E4M3FN, sb, group=G, block=B, bias=bias)
+    np.testing.assert_array_equal(out, want)
+
+
+@pytest.mark.parametrize("fa,fb,M,N,K", [(E4M3FN, E4M3FN, 37, 300, 384), (E5M2, E4M3FN, 5, 129, 256),
+                                         (E4M3FN, E5M2, 130, 17, 200)])
+def test_blockwise_matches_dequantise_then_matmul(orc, fa, fb, M, N, K):
+    """The definition with library routines: decode with torch, scale every
+    element by its group / block scale, numpy float64 matmul.  Non-square
+    scale grids, a partial last weight block-row (N % 128) and a partial last
+    K group make a transposed or shifted scale index fail."""
+    g = np.random.default_rng(100 + M)
+    G = B = 128
+    a = _finite_codes(g, (M, K), fa)
+    b = _finite_codes(g, (N, K), fb)
+    sa = np.exp(g.normal(-4, 2, (M, -(-K // G)))).astype(np.float32)
+    sb = np.exp(g.normal(-8, 1, (-(-N // B), -(-K // B)))).astype(np.float32)
+    bias = g.standard_normal(N)
+    out = orc.scaled_mm_blockwise(a, fa, sa, b, fb, sb, bias=bias)
+    A = _torch_decode(a, fa) * np.repeat(sa.astype(np.float64), G, axis=1)[:, :K]
+    W = _torch_decode(b, fb) * np.repeat(np.repeat(sb.astype(np.float64), B, axis=0), B, axis=1)[:N, :K]
+    ref = A @ W.T + bias
+    mag = np.abs(A) @ np.abs(W).T + np.abs(bias)
+    assert np.all(np.abs(out - ref) <= 1e-13 * mag)
+
+
+def test_blockwise_power_of_two_scales_are_exact(orc):
+    """With power-of-two scales every dequantised product is a multiple of a
+    fixed power of two: the exact sum, in Python integers, equals the
+    oracle's value exactly."""
+    from fractions import Fraction
+    g = np.random.default_rng(9)
+    M, N, K = 3, 130, 256
+    a = _finite_codes(g, (M, K), E4M3FN)
+    b = _finite_codes(g, (N, K), E4M3FN)
+    ea = g.integers(-6, 7, (M, 2))
+    eb = g.integers(-6, 7, (2, 2))
+    sa = np.ldexp(1.0, ea).astype(np.float32)
+    sb = np.ldexp(1.0, eb).astype(np.float32)
+    out = orc.scaled_mm_blockwise(a, E4M3FN, sa, b, E4M3FN, sb)
+    va = (_torch_decode(a, E4M3FN) * 512).astype(np.int64)     # integer multiples of 2^-9
+    vb = (_torch_decode(b, E4M3FN) * 512).astype(np.int64)
+    for m in range(M):
+        for n in (0, 1, 127, 128, 129):
+            exact = Fraction(0)
+            for k in range(K):
+                exact += Fraction(int(va[m, k]) * int(vb[n, k]), 1 << 18) * \
+                    Fraction(2) ** int(ea[m, k // 128]) * Fraction(2) ** int(eb[n // 128, k // 128])
+            assert Fraction(out[m, n]) == exact, (m, n)
+
+
+def test_blockwise_uniform_scales_reduce_to_per_tensor(orc):
+    g = np.random.default_rng(4)
+    M, N, K = 9, 140, 256
+    a = _finite_codes(g, (M, K), E4M3FN)
+    b = _finite_codes(g, (N, K), E4M3FN)
+    sa = np.full((M, 2), 0.375, np.float32)
+    sb = np.full((2, 2), 2.0 ** -7, np.float32)
+    out = orc.scaled_mm_blockwise(a, E4M3FN, sa, b, E4M3FN, sb)
+    np.testing.assert_array_equal(out, orc.scaled_mm(a, E4M3FN, b, E4M3FN, 0.375, 2.0 ** -7))
+
+
+def test_blockwise_rows_and_empty(orc):
+    g = np.random.default_rng(8)
+    a = _finite_codes(g, (10, 128), E4M3FN)
+    b = _finite_codes(g, (4, 128), E4M3FN)
+    sa = np.ones((10, 1), np.float32)
+    sb = np.ones((1, 1), np.float32)
+    full = orc.scaled_mm_blockwise(a, E4M3FN, sa, b, E4M3FN, sb)
+    part = orc.scaled_mm_blockwise(a, E4M3FN, sa, b, E4M3FN, sb, rows=(2, 5))
+    np.testing.assert_array_equal(part[2:5], full[2:5])
+    assert not part[:2].any() and not part[5:].any()
+    out = orc.scaled_mm_blockwise(np.zeros((2, 0), np.uint8), E4M3FN, np.zeros((2, 0), np.float32),
+                                  np.zeros((3, 0), np.uint8), E4M3FN, np.zeros((1, 0), np.float32),
+                                  bias=np.array([1.0, -2.0, 0.5]))
+    np.testing.assert_array_equal(out, np.array([[1.0, -2.0, 0.5]] * 2))
