@@ -217,6 +217,55 @@ class EndToEnd:
         return e0.elapsed_time(e1) / steps
 
 
+def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
+    """Each op the metric names, timed alone in a steady state: the op runs
+    back to back over `sets` copies of its buffers, rotating, with the sets
+    together at least 4x the L2 size, so every launch reads cold inputs and
+    pays for the write-back of exactly one launch's outputs (its own kind).
+    Returns {op name: {"us", "gb_s", "sets"}} (mean over `launches`)."""
+    f = wl.fp8q
+    d = wl.device
+    l2 = torch.cuda.get_device_properties(d).L2_cache_size
+    need = max(4 * l2, min_footprint)
+    out = {}
+
+    def run(name, make_set, footprint, nbytes):
+        sets = [make_set(i) for i in range(max(1, -(-need // footprint)))]
+        for fn in sets:
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k in range(launches):
+            sets[k % len(sets)]()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / launches
+        out[name] = {"us": round(us, 2), "gb_s": round(nbytes / (us * 1e-6) / 1e9, 1), "sets": len(sets)}
+        del sets
+        torch.cuda.empty_cache()
+
+    m, n = wl.c2_x.shape
+    c2_bytes = m * n * 3 + m * (n // 128) * 4
+
+    def per_token_set(i):
+        x = wl.c2_x if i == 0 else wl.c2_x.clone()
+        q = torch.empty((m, n), dtype=torch.uint8, device=d)
+        s = torch.empty((m, n // 128), dtype=torch.float32, device=d)
+        return lambda: f.fp8q_per_token_group_quant(x, q, s, 128, E4M3FN)
+    run("per_token_group_quant", per_token_set, c2_bytes, c2_bytes)
+
+    M, N = wl.c3_w.shape
+    c3_bytes = M * N * 3 + wl.c3_s.numel() * 4
+
+    def dequant_set(i):
+        w = wl.c3_w if i == 0 else wl.c3_w.clone()
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=d)
+        return lambda: f.fp8q_block_dequant(w, wl.c3_s, y, 128, E4M3FN)
+    run("block_dequant", dequant_set, c3_bytes, c3_bytes)
+    return out
+
+
 def _to_dev(a, device, dt=None):
     a = np.ascontiguousarray(a)
     t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
@@ -477,6 +526,8 @@ def run_ours(args):
     barrier(world)
     e2e_ms = max_over_ranks(e2e.time(e2e_steps), world, device)
     bi, bo = e2e.h2d_bytes, e2e.d2h_bytes
+    del e2e
+    iso = isolated_timing(wl) if rank == 0 else {}
 
     if rank != 0:
         _finish(world)
@@ -503,6 +554,7 @@ def run_ours(args):
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dgbs / peak, 4),
                      "bytes_per_launch": dop.bytes, "traffic": recorded_traffic(dop.name)},
         "kernels": kernels,
+        "isolated": {k: {**v, "frac": round(v["gb_s"] / peak, 4)} for k, v in iso.items()},
         "clocks": clk.summary(),
         "e2e": {"value": round(world * wl.step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
