@@ -89,6 +89,12 @@ def lib() -> ctypes.CDLL:
             L.orc_scaled_mm.restype = i32
             L.orc_scaled_mm.argtypes = [c_void, i32, c_void, i32, i64, i64, i64, ctypes.c_float, ctypes.c_float,
                                         c_void, c_void, i64, i64]
+            L.orc_scaled_mm_rounded.restype = i32
+            L.orc_scaled_mm_rounded.argtypes = [c_void, i32, c_void, i32, i64, i64, i64, ctypes.c_float,
+                                                ctypes.c_float, c_void, i32, c_void, i64, i64]
+            L.orc_scaled_mm_blockwise_rounded.restype = i32
+            L.orc_scaled_mm_blockwise_rounded.argtypes = [c_void, i32, c_void, c_void, i32, c_void, i64, i64, i64,
+                                                          i64, c_void, i32, c_void, i64, i64]
             L.orc_scaled_mm_blockwise.restype = i32
             L.orc_scaled_mm_blockwise.argtypes = [c_void, i32, c_void, i64, c_void, i32, c_void, i64,
                                                   i64, i64, i64, c_void, c_void, i64, i64]
@@ -397,4 +403,60 @@ def scaled_mm_blockwise(a: np.ndarray, fa: int, sa: np.ndarray, b: np.ndarray, f
     _run(lambda x, y: _check(L.orc_scaled_mm_blockwise(_ptr(a), fa, _ptr(sa), group, _ptr(b), fb, _ptr(sb), block,
                                                        M, N, K, bp, _ptr(out), x, y), "scaled_mm_blockwise"),
          r0, r1, threads)
+    return out
+
+
+def _out_array(M: int, N: int, yt: int) -> np.ndarray:
+    return np.zeros((M, N), np.float32 if yt == F32 else np.uint16)
+
+
+def scaled_mm_rounded(a: np.ndarray, fa: int, b: np.ndarray, fb: int, sa: float, sb: float, bias=None,
+                      yt: int = BF16, rows=None, threads: int = 1) -> np.ndarray:
+    """The per-tensor product with the library's fp32 epilogue, d = T(fl(fl(acc * fl(sa * sb)) + bias)),
+    acc the exact sum rounded once to fp32.  bias: fp32 values or None.  Returns float32 (yt = F32) or
+    the uint16 bit patterns of bf16 / fp16."""
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b need the same K")
+    out = _out_array(M, N, yt)
+    bp = None
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float32)
+        bp = ctypes.c_void_p(bias.ctypes.data)
+    r0, r1 = rows if rows is not None else (0, M)
+    L = lib()
+    _run(lambda x, y: _check(L.orc_scaled_mm_rounded(_ptr(a), fa, _ptr(b), fb, M, N, K, ctypes.c_float(sa),
+                                                     ctypes.c_float(sb), bp, yt, _ptr(out), x, y),
+                             "scaled_mm_rounded"), r0, r1, threads)
+    return out
+
+
+def scaled_mm_blockwise_rounded(a: np.ndarray, fa: int, sa: np.ndarray, b: np.ndarray, fb: int, sb: np.ndarray,
+                                block: int = 128, bias=None, yt: int = BF16, rows=None,
+                                threads: int = 1) -> np.ndarray:
+    """The fine-grained product with the library's fp32 rounding: acc = fma(acc_kb, fl(sa * sb), acc)
+    over 128-deep k-blocks in order, d = T(fl(acc + bias)); activation groups and weight blocks are
+    both `block` wide."""
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    sb = np.ascontiguousarray(sb, dtype=np.float32)
+    M, K = a.shape
+    N = b.shape[0]
+    kb = -(-K // block)
+    if b.shape[1] != K or sa.shape != (M, kb) or sb.shape != (-(-N // block), kb):
+        raise ValueError("operand or scale shapes do not match")
+    out = _out_array(M, N, yt)
+    bp = None
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float32)
+        bp = ctypes.c_void_p(bias.ctypes.data)
+    r0, r1 = rows if rows is not None else (0, M)
+    L = lib()
+    _run(lambda x, y: _check(L.orc_scaled_mm_blockwise_rounded(_ptr(a), fa, _ptr(sa), _ptr(b), fb, _ptr(sb),
+                                                               block, M, N, K, bp, yt, _ptr(out), x, y),
+                             "scaled_mm_blockwise_rounded"), r0, r1, threads)
     return out

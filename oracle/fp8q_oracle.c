@@ -574,3 +574,76 @@ int orc_scaled_mm_blockwise(const uint8_t* a, int fa, const float* sa, int64_t g
     }
     return 0;
 }
+
+/*
+ * The two products as the library rounds them.  The pages leave the
+ * rounding inside torch._scaled_mm to the GEMM library; the reading taken
+ * here is the plainest single-precision one:
+ *   per-tensor:    d = T(fl(fl(acc * fl(sa * sb)) + bias[n]))
+ *   fine-grained:  acc = 0; for kb ascending: acc = fma(acc_kb, fl(sa[m][kb] * sb[n/bb][kb]), acc)
+ *                  d = T(fl(acc + bias[n]))
+ * where acc (per-tensor) and acc_kb (one 128-deep block) are the binary64
+ * sums above rounded once to binary32 -- the correctly rounded fp32 sum.
+ * Whenever every partial sum of the products is an fp32 number (for
+ * example all operand values multiples of 1/8 of magnitude <= 4, K <= 16384:
+ * products are multiples of 2^-6 below 2^4, sums below 2^18), any fp32
+ * accumulation order gives that same acc, so d is fixed bit for bit.
+ * Other inputs differ from the tensor cores' sum only by its own rounding.
+ * fmaf is the C library's correctly rounded fused multiply-add; bias is
+ * NULL or binary32 values (bf16 / fp16 biases widen exactly); out is yt.
+ */
+static double dot_exact(const uint8_t* ar, const uint8_t* br, const double* da, const double* db,
+                        int64_t k0, int64_t k1)
+{
+    double acc = 0.0;
+    for (int64_t k = k0; k < k1; ++k) acc += da[ar[k]] * db[br[k]];
+    return acc;
+}
+
+int orc_scaled_mm_rounded(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
+                          float sa, float sb, const float* bias, int yt, void* out, int64_t r0, int64_t r1)
+{
+    if (!valid_fmt(fa) || !valid_fmt(fb) || M < 0 || N < 0 || K < 0 || r0 < 0 || r1 > M || r0 > r1)
+        return -1;
+    double da[256], db[256];
+    for (int c = 0; c < 256; ++c) {
+        da[c] = (double)orc_fp8_decode((uint8_t)c, fa);
+        db[c] = (double)orc_fp8_decode((uint8_t)c, fb);
+    }
+    const float s = sa * sb;
+    for (int64_t m = r0; m < r1; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float acc = (float)dot_exact(a + m * K, b + n * K, da, db, 0, K);
+            float v = acc * s;
+            if (bias) v = v + bias[n];
+            store_elem(out, yt, m * N + n, v);
+        }
+    return 0;
+}
+
+int orc_scaled_mm_blockwise_rounded(const uint8_t* a, int fa, const float* sa, const uint8_t* b, int fb,
+                                    const float* sb, int64_t bb, int64_t M, int64_t N, int64_t K,
+                                    const float* bias, int yt, void* out, int64_t r0, int64_t r1)
+{
+    if (!valid_fmt(fa) || !valid_fmt(fb) || M < 0 || N < 0 || K < 0 || bb < 1 || r0 < 0 || r1 > M || r0 > r1)
+        return -1;
+    double da[256], db[256];
+    for (int c = 0; c < 256; ++c) {
+        da[c] = (double)orc_fp8_decode((uint8_t)c, fa);
+        db[c] = (double)orc_fp8_decode((uint8_t)c, fb);
+    }
+    const int64_t kb = (K + bb - 1) / bb;
+    for (int64_t m = r0; m < r1; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float acc = 0.0f;
+            for (int64_t j = 0; j < kb; ++j) {
+                const int64_t k1 = (j + 1) * bb < K ? (j + 1) * bb : K;
+                const float part = (float)dot_exact(a + m * K, b + n * K, da, db, j * bb, k1);
+                const float s = sa[m * kb + j] * sb[(n / bb) * kb + j];
+                acc = fmaf(part, s, acc);
+            }
+            if (bias) acc = acc + bias[n];
+            store_elem(out, yt, m * N + n, acc);
+        }
+    return 0;
+}

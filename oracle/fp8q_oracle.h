@@ -142,6 +142,17 @@ int orc_scaled_mm_blockwise(const uint8_t* a, int fa, const float* sa, int64_t g
                             int64_t M, int64_t N, int64_t K, const double* bias,
                             double* out, int64_t r0, int64_t r1);
 
+/* The same two products with the library's single-precision rounding:
+ * per-tensor d = T(fl(fl(acc * fl(sa * sb)) + bias[n])); fine-grained
+ * acc = fma(acc_kb, fl(sa[m][kb] * sb[n/bb][kb]), acc) over kb ascending,
+ * d = T(fl(acc + bias[n])); acc and acc_kb the exact sums rounded once to
+ * binary32.  bias NULL or fp32 [N]; out [M][N] of type yt. */
+int orc_scaled_mm_rounded(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
+                          float sa, float sb, const float* bias, int yt, void* out, int64_t r0, int64_t r1);
+int orc_scaled_mm_blockwise_rounded(const uint8_t* a, int fa, const float* sa, const uint8_t* b, int fb,
+                                    const float* sb, int64_t bb, int64_t M, int64_t N, int64_t K,
+                                    const float* bias, int yt, void* out, int64_t r0, int64_t r1);
+
 #ifdef __cplusplus
 }
 #endif

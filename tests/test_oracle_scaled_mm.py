@@ -206,3 +206,87 @@ def test_blockwise_rows_and_empty(orc):
                                   np.zeros((3, 0), np.uint8), E4M3FN, np.zeros((1, 0), np.float32),
                                   bias=np.array([1.0, -2.0, 0.5]))
     np.testing.assert_array_equal(out, np.array([[1.0, -2.0, 0.5]] * 2))
+
+
+# ---------------------------------------------------------------------------
+# the library's single-precision rounding of the two products
+# ---------------------------------------------------------------------------
+def _exact_grid_codes(g, shape, fmt):
+    """Codes whose values are multiples of 1/8 of magnitude <= 4: products are
+    multiples of 2^-6 below 16, so every partial sum of up to 2^12 of them is
+    an fp32 number and any fp32 summation order is exact."""
+    import workloads
+    codes = workloads.finite_e4m3fn_codes() if fmt == E4M3FN else workloads.finite_e5m2_codes()
+    v = _torch_decode(codes, fmt)
+    keep = codes[(np.abs(v) <= 4) & (v * 8 == np.round(v * 8))]
+    return keep[g.integers(0, keep.size, size=shape)].astype(np.uint8)
+
+
+def _torch_round(v64, yt):
+    import torch
+    dt = {0: torch.float32, 1: torch.float16, 2: torch.bfloat16}[yt]
+    t = torch.from_numpy(np.ascontiguousarray(v64)).to(dt)
+    return t.numpy() if yt == 0 else t.view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("yt", [0, 1, 2])
+def test_rounded_forms_closed_form(orc, yt):
+    """Exact-grid operands, power-of-two scales and a bias on the same grid:
+    every fp32 step is exact, so the output is the exact value rounded once to
+    T, which torch's own float64 -> T conversion gives."""
+    g = np.random.default_rng(30 + yt)
+    M, N, K = 7, 300, 1024
+    fa, fb = E4M3FN, E5M2
+    a = _exact_grid_codes(g, (M, K), fa)
+    b = _exact_grid_codes(g, (N, K), fb)
+    bias = (g.integers(-512, 512, N) / 64.0).astype(np.float32)
+    A, W = _torch_decode(a, fa), _torch_decode(b, fb)
+    exact = (A @ W.T) * 0.25 * 0.5 + bias
+    got = orc.scaled_mm_rounded(a, fa, b, fb, 0.25, 0.5, bias=bias, yt=yt)
+    np.testing.assert_array_equal(got, _torch_round(exact, yt))
+    # fine-grained: power-of-two scales 1/2 .. 2 per group / block keep every
+    # product a multiple of 2^-8 and every sum below 2^16 (24 bits)
+    kb = K // 128
+    sa = np.ldexp(1.0, g.integers(-1, 2, (M, kb))).astype(np.float32)
+    sb = np.ldexp(1.0, g.integers(-1, 2, (-(-N // 128), kb))).astype(np.float32)
+    Af = A * np.repeat(sa.astype(np.float64), 128, axis=1)
+    Wf = W * np.repeat(np.repeat(sb.astype(np.float64), 128, axis=0), 128, axis=1)[:N]
+    exact = Af @ Wf.T + bias
+    got = orc.scaled_mm_blockwise_rounded(a, fa, sa, b, fb, sb, bias=bias, yt=yt)
+    np.testing.assert_array_equal(got, _torch_round(exact, yt))
+
+
+def test_rounded_epilogue_order_hand_worked(orc):
+    d = _golden("scaled_mm_epilogue_order.txt")
+    K = int(d["K"])
+    a = np.array([int(t, 16) for t in d["a"].split()], np.uint8).reshape(1, K)
+    b = np.array([int(t, 16) for t in d["b"].split()], np.uint8).reshape(1, K)
+    s = float(np.array(int(d["scale_f32"], 16), np.uint32).view(np.float32))
+    got = orc.scaled_mm_rounded(a, E4M3FN, b, E4M3FN, s, s, yt=0)
+    assert got.view(np.uint32)[0, 0] == int(d["out_f32"], 16)
+    got = orc.scaled_mm_rounded(a, E4M3FN, b, E4M3FN, s, s, bias=np.array([float(d["bias"])]), yt=0)
+    assert got.view(np.uint32)[0, 0] == int(d["out_f32_bias"], 16)
+    got = orc.scaled_mm_rounded(a, E4M3FN, b, E4M3FN, s, s, yt=2)
+    assert got[0, 0] == int(d["out_bf16"], 16)
+
+
+def test_rounded_forms_stay_within_half_an_ulp_of_the_exact_product(orc):
+    """General operands: each fp32 step rounds once, so the fp32 result lies
+    within a few fp32 ulps of the binary64 definition (a dropped k-block, a
+    swapped scale or a wrong bias would be far outside)."""
+    g = np.random.default_rng(44)
+    M, N, K = 6, 140, 512
+    a = _finite_codes(g, (M, K), E4M3FN)
+    b = _finite_codes(g, (N, K), E4M3FN)
+    sa = np.exp(g.normal(-4, 2, (M, 4))).astype(np.float32)
+    sb = np.exp(g.normal(-8, 1, (2, 4))).astype(np.float32)
+    bias = g.standard_normal(N).astype(np.float32)
+    exact = orc.scaled_mm_blockwise(a, E4M3FN, sa, b, E4M3FN, sb, bias=bias.astype(np.float64))
+    A, W = _torch_decode(a, E4M3FN), _torch_decode(b, E4M3FN)
+    mag = (np.abs(A) * np.repeat(sa, 128, axis=1)) @ (np.abs(W) * np.repeat(np.repeat(sb, 128, 0), 128, 1)[:N]).T
+    got = orc.scaled_mm_blockwise_rounded(a, E4M3FN, sa, b, E4M3FN, sb, bias=bias, yt=0)
+    assert np.all(np.abs(got - exact) <= 2.0 ** -21 * (mag + np.abs(bias)))
+    got = orc.scaled_mm_rounded(a, E4M3FN, b, E4M3FN, 0.01, 3.0, bias=bias, yt=0)
+    exact = orc.scaled_mm(a, E4M3FN, b, E4M3FN, 0.01, 3.0, bias=bias.astype(np.float64))
+    mag = (np.abs(A) @ np.abs(W).T) * 0.03
+    assert np.all(np.abs(got - exact) <= 2.0 ** -21 * (mag + np.abs(bias)))
