@@ -17,6 +17,12 @@ all_to_all_single_fp8): each rank packs [scale_inv | fp8 payload] records
 with libfp8q, torch.distributed moves the bytes, and libfp8q dequantises
 every received record; no arithmetic runs outside the library.
 
+fp8 matrix products on the tensor cores (tcgen05):
+    fp8q_scaled_mm            ColossalAI _LinearFp8.forward (torch._scaled_mm,
+                              per-tensor scales)
+    fp8q_scaled_mm_blockwise  DeepEP per-token activations x DeepSeek-V3
+                              128 x 128 block-scaled weight
+
 Allocating helpers named after the functions on the pages:
     per_token_cast_to_fp8   (DeepEP "5 Utils")
     per_token_cast_back     (DeepEP "5 Utils", the named inverse)
@@ -45,6 +51,8 @@ __all__ = [
     "cast_to_fp8_pipeline", "cast_from_fp8_pipeline",
     "RECORD_HEADER_BYTES", "record_bytes", "fp8q_record_bytes", "fp8q_pack_record", "fp8q_unpack_records",
     "exchange_records", "exchange_records_all_to_all", "exchange_payload_all_to_all", "all_gather_fp8", "all_to_all_fp8", "all_to_all_single_fp8",
+    "fp8q_scaled_mm", "fp8q_scaled_mm_blockwise", "scaled_mm", "scaled_mm_blockwise", "linear_fp8",
+    "linear_fp8_blockwise",
 ]
 
 E4M3FN, E5M2 = 0, 1
@@ -131,6 +139,10 @@ def lib() -> ctypes.CDLL:
             L.fp8q_pack_record.argtypes = [p, i32, i64, i32, p, p, ctypes.c_size_t, i32, p]
             L.fp8q_unpack_records.restype = st
             L.fp8q_unpack_records.argtypes = [p, i32, i64, i32, i32, p, p]
+            L.fp8q_scaled_mm.restype = st
+            L.fp8q_scaled_mm.argtypes = [p, i32, p, i32, i64, i64, i64, p, p, p, i32, p, p, p]
+            L.fp8q_scaled_mm_blockwise.restype = st
+            L.fp8q_scaled_mm_blockwise.argtypes = [p, i32, p, p, i32, p, i64, i64, i64, p, i32, p, p, p]
             _lib = L
     return _lib
 
@@ -712,3 +724,108 @@ def all_to_all_single_fp8(output: torch.Tensor, input: torch.Tensor, group=None,
             ss.append(scales[i:i + 1])
             ys.append(flat[base + body * cols:base + c])
     fp8q_block_dequant_grouped(ws_, ss, ys, block=1 << 30, fmt=f)
+
+
+# ---------------------------------------------------------------------------
+# fp8 matrix products (tensor cores)
+# ---------------------------------------------------------------------------
+def _mm_operands(a: torch.Tensor, b: torch.Tensor, out: torch.Tensor, bias, fa, fb):
+    if a.dim() != 2 or b.dim() != 2:
+        raise ValueError("a must be [M, K] and b [N, K] (the weight as stored)")
+    M, K = a.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError(f"a has K = {K} but b has K = {K2}")
+    _need(a, M * K, "a", byte=True)
+    _need(b, N * K, "b", byte=True)
+    _need(out, M * N, "out")
+    if bias is not None:
+        _need(bias, N, "bias", dtype=out.dtype)
+    fa = _fmt_of(fa) if fa is not None else _FP8_DTYPES.get(a.dtype, E4M3FN)
+    fb = _fmt_of(fb) if fb is not None else _FP8_DTYPES.get(b.dtype, E4M3FN)
+    return M, N, K, fa, fb
+
+
+def fp8q_scaled_mm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
+                   out: torch.Tensor, bias: Optional[torch.Tensor] = None, fa=None, fb=None,
+                   status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ColossalAI linear_fp8 forward product, torch._scaled_mm(a, b.t(), scale_a, scale_b, bias):
+    out[M, N] = T(acc * scale_a[0] * scale_b[0] + bias) with a [M, K] and b [N, K] fp8 codes
+    (formats from their float8 dtypes, or fa / fb), scale_a / scale_b fp32 [1] on the device.
+    `status`: optional int32/uint32 [1] device word that the kernel ORs a nonzero code into if
+    one of its bounded internal waits runs out."""
+    M, N, K, fa, fb = _mm_operands(a, b, out, bias, fa, fb)
+    dev = a.device
+    _need(scale_a, 1, "scale_a", dtype=torch.float32)
+    _need(scale_b, 1, "scale_b", dtype=torch.float32)
+    _check(lib().fp8q_scaled_mm(
+        _dev_ptr(a, "a", dev), fa, _dev_ptr(b, "b", dev), fb, M, N, K,
+        _dev_ptr(scale_a, "scale_a", dev), _dev_ptr(scale_b, "scale_b", dev), _dev_ptr(bias, "bias", dev),
+        _dtype_code(out, "out"), _dev_ptr(out, "out", dev), _dev_ptr(status, "status", dev),
+        _stream(stream, dev)), "fp8q_scaled_mm")
+
+
+def fp8q_scaled_mm_blockwise(a: torch.Tensor, scale_a: torch.Tensor, b: torch.Tensor, scale_b: torch.Tensor,
+                             out: torch.Tensor, bias: Optional[torch.Tensor] = None, fa=None, fb=None,
+                             status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Per-token activations a [M, K] with scale_a [M, ceil(K/128)] (per_token_cast_to_fp8) times
+    a weight b [N, K] with scale_b [ceil(N/128), ceil(K/128)] (one scale_inv per 128 x 128 block):
+    out[M, N] = T(sum_kb scale_a[m, kb] * scale_b[n/128, kb] * acc_kb + bias)."""
+    M, N, K, fa, fb = _mm_operands(a, b, out, bias, fa, fb)
+    dev = a.device
+    kb = -(-K // 128)
+    _need(scale_a, M * kb, "scale_a", dtype=torch.float32)
+    _need(scale_b, -(-N // 128) * kb, "scale_b", dtype=torch.float32)
+    _check(lib().fp8q_scaled_mm_blockwise(
+        _dev_ptr(a, "a", dev), fa, _dev_ptr(scale_a, "scale_a", dev), _dev_ptr(b, "b", dev), fb,
+        _dev_ptr(scale_b, "scale_b", dev), M, N, K, _dev_ptr(bias, "bias", dev), _dtype_code(out, "out"),
+        _dev_ptr(out, "out", dev), _dev_ptr(status, "status", dev), _stream(stream, dev)),
+        "fp8q_scaled_mm_blockwise")
+
+
+def scaled_mm(a: torch.Tensor, b_t: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
+              bias: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """torch._scaled_mm(a, b_t, scale_a, scale_b, bias, out_dtype) as ColossalAI calls it: b_t is the
+    transpose of a row-major weight w [N, K] (w.t()), which is what the kernel reads."""
+    w = b_t.t()
+    if not w.is_contiguous():
+        raise ValueError("b_t must be the transpose of a contiguous [N, K] weight (w.t())")
+    out = torch.empty((a.shape[0], w.shape[0]), dtype=out_dtype, device=a.device)
+    fp8q_scaled_mm(a, w, scale_a, scale_b, out, bias)
+    return out
+
+
+def scaled_mm_blockwise(a: torch.Tensor, scale_a: torch.Tensor, w: torch.Tensor, scale_w: torch.Tensor,
+                        bias: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """a [M, K] fp8 with per-token-group scale_a times the weight w [N, K] fp8 with 128 x 128 block
+    scale_w; returns out [M, N] of out_dtype."""
+    out = torch.empty((a.shape[0], w.shape[0]), dtype=out_dtype, device=a.device)
+    fp8q_scaled_mm_blockwise(a, scale_a, w, scale_w, out, bias)
+    return out
+
+
+def linear_fp8(input: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """ColossalAI linear_fp8 forward: per-tensor e4m3 casts of input and weight (cast_to_fp8),
+    then the scaled product with the input's dtype as output dtype."""
+    if input.dtype not in (torch.bfloat16, torch.float16) or input.dtype != weight.dtype:
+        raise TypeError("Only float16 and bfloat16 are allowed.")
+    if bias is not None and bias.dtype != input.dtype:
+        raise TypeError("Bias should have the same dtype as input.")
+    x = input.contiguous().reshape(-1, input.shape[-1])
+    x_fp8, sx = cast_to_fp8(x, "e4m3")
+    w_fp8, sw = cast_to_fp8(weight.contiguous(), "e4m3")
+    out = torch.empty((x.shape[0], weight.shape[0]), dtype=input.dtype, device=input.device)
+    fp8q_scaled_mm(x_fp8, w_fp8, sx, sw, out, bias)
+    return out.reshape(*input.shape[:-1], weight.shape[0])
+
+
+def linear_fp8_blockwise(input: torch.Tensor, weight: torch.Tensor, weight_scale_inv: torch.Tensor,
+                         bias: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """A linear layer on a DeepSeek-V3-style fp8 weight [N, K] with its 128 x 128 block scale_inv:
+    the input is quantised per token (per_token_cast_to_fp8, 1 x 128 groups), then multiplied
+    without dequantising either operand; the output has the input's dtype."""
+    x = input.contiguous().reshape(-1, input.shape[-1])
+    q, s = per_token_cast_to_fp8(x)
+    out = torch.empty((x.shape[0], weight.shape[0]), dtype=input.dtype, device=input.device)
+    fp8q_scaled_mm_blockwise(q, s, weight, weight_scale_inv, out, bias)
+    return out.reshape(*input.shape[:-1], weight.shape[0])

@@ -323,3 +323,61 @@ fp8q_status fp8q_cast_from_fp8(const uint8_t* q, fp8q_format fmt, int64_t rows, 
 }
 
 }  // extern "C"
+
+namespace {
+
+// shared checks of the two fp8 products; returns FP8Q_OK to go on
+fp8q_status check_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
+                            const float* sa, const float* sb, const void* bias, int yt, const void* d,
+                            const uint32_t* status, bool* nothing) {
+    *nothing = false;
+    if (!dtype_ok(yt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!fmt_ok(fa) || !fmt_ok(fb)) return FP8Q_ERR_BAD_FORMAT;
+    const int64_t lim = 0x7FFFFFFFLL - 512;
+    if (M < 0 || N < 0 || K < 0 || M > lim || N > lim || K > lim || K % 16 != 0) return FP8Q_ERR_BAD_SHAPE;
+    const int64_t mn = checked_mul(M, N);
+    if (mn < 0 || checked_mul(mn, dtype_bytes(yt)) < 0 || checked_mul(M, K) < 0 || checked_mul(N, K) < 0)
+        return FP8Q_ERR_BAD_SHAPE;
+    if (mn == 0) {
+        *nothing = true;
+        return FP8Q_OK;
+    }
+    if (!d) return FP8Q_ERR_NULL_POINTER;
+    if (K > 0 && (!a || !b || !sa || !sb)) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(d, dtype_bytes(yt)) || (bias && !aligned(bias, dtype_bytes(yt))) || (status && !aligned(status, 4)))
+        return FP8Q_ERR_MISALIGNED;
+    if (K > 0 && (!aligned(a, 16) || !aligned(b, 16) || !aligned(sa, 4) || !aligned(sb, 4)))
+        return FP8Q_ERR_MISALIGNED;
+    return FP8Q_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8q_status fp8q_scaled_mm(const uint8_t* a, fp8q_format fa, const uint8_t* b, fp8q_format fb, int64_t M,
+                           int64_t N, int64_t K, const float* scale_a, const float* scale_b, const void* bias,
+                           fp8q_dtype yt, void* d, uint32_t* status, fp8q_stream_t stream) {
+    bool nothing = false;
+    fp8q_status st = check_scaled_mm(a, fa, b, fb, M, N, K, scale_a, scale_b, bias, yt, d, status, &nothing);
+    if (st != FP8Q_OK || nothing) return st;
+    // the per-tensor epilogue reads both scales even when K == 0
+    if (!scale_a || !scale_b) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(scale_a, 4) || !aligned(scale_b, 4)) return FP8Q_ERR_MISALIGNED;
+    return launch_scaled_mm(a, fa, b, fb, M, N, K, scale_a, 0, scale_b, 0, false, bias, yt, d, status,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp8q_status fp8q_scaled_mm_blockwise(const uint8_t* a, fp8q_format fa, const float* scale_a, const uint8_t* b,
+                                     fp8q_format fb, const float* scale_b, int64_t M, int64_t N, int64_t K,
+                                     const void* bias, fp8q_dtype yt, void* d, uint32_t* status,
+                                     fp8q_stream_t stream) {
+    bool nothing = false;
+    fp8q_status st = check_scaled_mm(a, fa, b, fb, M, N, K, scale_a, scale_b, bias, yt, d, status, &nothing);
+    if (st != FP8Q_OK || nothing) return st;
+    const int kb = static_cast<int>((K + 127) / 128);
+    return launch_scaled_mm(a, fa, b, fb, M, N, K, scale_a, kb, scale_b, kb, true, bias, yt, d, status,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

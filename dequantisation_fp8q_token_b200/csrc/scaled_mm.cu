@@ -1,0 +1,592 @@
+// scaled_mm.cu -- fp8 x fp8 matrix products on the sm_100a tensor cores.
+//
+// Two products of the same shape, D[M][N] = A[M][K] * B[N][K]^T, both
+// operands fp8 codes stored K-contiguous (A: activations, B: a weight as it
+// is stored, [out features][in features]):
+//   per-tensor scales (ColossalAI colossalai/quantization/fp8.py,
+//     _LinearFp8.forward: torch._scaled_mm with the scale_inv of each operand)
+//       D[m][n] = T(fl(acc[m][n] * fl(sa * sb)) + bias[n])
+//   fine-grained scales (DeepEP per_token_cast_to_fp8 activations, one
+//     scale_inv per 1 x 128 group: sa[M][ceil(K/128)]; a DeepSeek-V3 weight
+//     with one scale_inv per 128 x 128 block: sb[ceil(N/128)][ceil(K/128)])
+//       D[m][n] = T(sum over k-blocks kb of fl(sa[m][kb] * sb[n/128][kb]) *
+//                   acc_kb[m][n]  + bias[n])
+// where acc is the fp32 tensor-core sum of the fp8 products.
+//
+// Design (one persistent CTA per SM, warp-specialised):
+//   warp 0      TMA producer: 128 x 128-byte tiles of A and 256 x 128-byte
+//               tiles of B (128-byte swizzle) into a 4-stage shared-memory ring
+//   warp 1      allocates 512 TMEM columns; one lane issues
+//               tcgen05.mma.kind::f8f6f4 (M 128, N 256, K 32) into one of two
+//               128 x 256 fp32 TMEM accumulators and commits each stage back
+//               to the producer and each finished accumulator to the epilogue
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32 * (w % 4) .. + 31, columns of half (w - 2) / 4),
+//               scaling, bias, conversion, 32-byte stores.  With fine-grained
+//               scales the MMA warp commits every 128-deep k-block into a
+//               fresh accumulator and the epilogue folds it into registers
+//               with that block's scale, while the tensor cores fill the
+//               other accumulator.
+// Tiles are 128 x 256 of D, visited in bands of 16 row-tiles so that the
+// CTAs working at one time share A and B tiles in L2.
+//
+// Every wait on an mbarrier is bounded (a few seconds of global time).  A
+// wait that runs out sets a flag in shared memory that ends the other roles'
+// waits too, ORs a code into the caller's status word, drains the copies and
+// tensor-core operations this CTA has in flight, frees its TMEM and returns.
+#include <cuda.h>
+
+#include <cstring>
+
+#include "fp8q_device.cuh"
+#include "fp8q_internal.h"
+
+namespace fp8q {
+namespace mm {
+
+constexpr int BM = 128;         // rows of A (and of D) per tile
+constexpr int BN = 256;         // rows of B (columns of D) per tile
+constexpr int BK = 128;         // k per stage: one 128-byte swizzle row, one scale block
+constexpr int kStages = 4;
+constexpr int kAccBufs = 2;
+constexpr int kTmemCols = kAccBufs * BN;   // 512: all of TMEM
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kABytes = BM * BK;
+constexpr int kBBytes = BN * BK;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kGroupM = 16;     // row-tiles per raster band
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment slack */ + 256 /* barriers */;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+// status bits ORed into the caller's status word when a wait runs out
+enum : uint32_t { kTimeoutProducer = 1u, kTimeoutMma = 2u, kTimeoutEpilogue = 4u, kTimeoutDrain = 8u };
+
+struct Params {
+    int M, N, K;
+    int num_kb;                 // ceil(K / BK)
+    int tiles_m, tiles_n;
+    const float* sa;            // per-tensor: [1]; fine-grained: [M][sa_ld]
+    const float* sb;            // per-tensor: [1]; fine-grained: [ceil(N/128)][sb_ld]
+    int sa_ld, sb_ld;
+    const void* bias;           // [N] of the output type, or null
+    void* d;                    // [M][N]
+    int vec_store;              // D rows 32-byte aligned (base and row pitch)
+    uint32_t* status;           // optional status word
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Wait for the phase of `bar` with the given parity; false if the wait ran
+// out of time or another role of this CTA has already given up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+// the same wait, ignoring the abort flag (used to drain work in flight)
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a K-major operand tile written by TMA
+// with the 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes
+// apart (stride byte offset), leading byte offset unused (encoded 1), the
+// Blackwell descriptor version 1, layout 2 = 128-byte swizzle.  The tile
+// base is 1024-byte aligned; a k offset inside the 128-byte row moves the
+// start address only.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu)
+         | (static_cast<uint64_t>(1) << 16)
+         | (static_cast<uint64_t>(1024 >> 4) << 32)
+         | (static_cast<uint64_t>(1) << 46)
+         | (static_cast<uint64_t>(2) << 61);
+}
+// Instruction descriptor of kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B
+// formats (bits 7-9, 10-12: 0 e4m3, 1 e5m2), both K-major, N >> 3 at bit 17,
+// M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t instr_desc(int fa, int fb) {
+    return (1u << 4) | (static_cast<uint32_t>(fa) << 7) | (static_cast<uint32_t>(fb) << 10)
+         | (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// arrive on `bar` once every tcgen05 operation this thread issued so far has completed
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(bar) : "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns of TMEM into 32 registers per thread
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32"
+                 " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+                   "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+                   "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+    // the registers pass through the wait, so no use of them can be scheduled before it
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                   "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                   "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------
+// epilogue stores: 32 consecutive columns of one row of D
+// ---------------------------------------------------------------------------
+template <int YT> struct OutT;
+template <> struct OutT<kF32> { using T = float; };
+template <> struct OutT<kF16> { using T = __half; };
+template <> struct OutT<kBF16> { using T = __nv_bfloat16; };
+
+template <int YT> __device__ __forceinline__ float load_bias(const void* bias, int n) {
+    if constexpr (YT == kF32) return __ldg(static_cast<const float*>(bias) + n);
+    else if constexpr (YT == kF16) return __half2float(__ldg(static_cast<const __half*>(bias) + n));
+    else return __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(bias) + n));
+}
+
+template <int YT> __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    if constexpr (YT == kF16) {
+        __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    } else {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+}
+
+template <int YT>
+__device__ __forceinline__ void store_chunk(const Params& p, int row, int col0, const float (&v)[32]) {
+    using T = typename OutT<YT>::T;
+    T* drow = static_cast<T*>(p.d) + static_cast<int64_t>(row) * p.N;
+    if (p.vec_store && col0 + 32 <= p.N) {
+        if constexpr (YT == kF32) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(v[c * 8 + i]);
+                st_v8(drow + col0 + c * 8, w);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[i] = pack2<YT>(v[c * 16 + 2 * i], v[c * 16 + 2 * i + 1]);
+                st_v8(drow + col0 + c * 16, w);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (col0 + i < p.N) {
+                if constexpr (YT == kF32) drow[col0 + i] = v[i];
+                else if constexpr (YT == kF16) drow[col0 + i] = __float2half_rn(v[i]);
+                else drow[col0 + i] = __float2bfloat16_rn(v[i]);
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& mb, int& nb) {
+    const int band = t / (kGroupM * tiles_n);
+    const int first = band * kGroupM;
+    const int gm = min(tiles_m - first, kGroupM);
+    const int local = t - band * kGroupM * tiles_n;
+    mb = first + local % gm;
+    nb = local / gm;
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+template <int YT, bool FINE>
+__global__ void __launch_bounds__(kThreads, 1)
+scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                 const Params p, const uint32_t idesc) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ int s_abort;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kABytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kBBytes);
+    // bars: full[kStages], empty[kStages], tfull[kAccBufs], tempty[kAccBufs], drain
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 2 * kAccBufs + 1);
+    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * kStages;
+    const uint32_t tfull0 = empty0 + 8 * kStages, tempty0 = tfull0 + 8 * kAccBufs;
+    const uint32_t drain_bar = tempty0 + 8 * kAccBufs;
+    volatile int* abort = &s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int b = 0; b < kAccBufs; ++b) {
+            mbar_init(tfull0 + 8 * b, 1);
+            mbar_init(tempty0 + 8 * b, kEpiWarps);
+        }
+        mbar_init(drain_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        prefetch_tensormap(&map_a);
+        prefetch_tensormap(&map_b);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    pdl_begin();
+
+    const int tiles = p.tiles_m * p.tiles_n;
+    uint32_t fail = 0;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int64_t issued = 0;
+            for (int t = blockIdx.x; t < tiles && !fail; t += gridDim.x) {
+                int mb, nb;
+                tile_coords(t, p.tiles_m, p.tiles_n, mb, nb);
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort)) { fail = kTimeoutProducer; break; }
+                    const uint32_t fb = full0 + 8 * stage;
+                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    tma_load_2d(smem_u32(sA + stage * kABytes), &map_a, kb * BK, mb * BM, fb);
+                    tma_load_2d(smem_u32(sB + stage * kBBytes), &map_b, kb * BK, nb * BN, fb);
+                    ++issued;
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (fail) *abort = 1;
+            // every copy this thread issued has landed before the CTA exits
+            for (int s = 0; s < kStages; ++s) {
+                const bool used = s < stage || issued >= kStages;
+                if (used && !mbar_wait_drain(full0 + 8 * s, s < stage ? phase : phase ^ 1u)) fail |= kTimeoutDrain;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int t = blockIdx.x; t < tiles && !fail; t += gridDim.x) {
+                if (p.num_kb == 0) continue;
+                if (!FINE) {
+                    if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort)) { fail = kTimeoutMma; break; }
+                    tc_fence_after();
+                }
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (FINE) {
+                        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort)) { fail = kTimeoutMma; break; }
+                        tc_fence_after();
+                    }
+                    if (!mbar_wait(full0 + 8 * stage, phase, abort)) { fail = kTimeoutMma; break; }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                    const uint32_t a0 = smem_u32(sA + stage * kABytes), b0 = smem_u32(sB + stage * kBBytes);
+#pragma unroll
+                    for (int j = 0; j < BK / 32; ++j) {
+                        const uint32_t accumulate = FINE ? (j > 0) : (kb > 0 || j > 0);
+                        mma_f8f6f4(d_tmem, smem_desc_sw128(a0 + 32 * j), smem_desc_sw128(b0 + 32 * j), idesc,
+                                   accumulate);
+                    }
+                    mma_commit(empty0 + 8 * stage);
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (FINE) {
+                        mma_commit(tfull0 + 8 * acc);
+                        if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
+                    }
+                }
+                if (fail) break;
+                if (!FINE) {
+                    mma_commit(tfull0 + 8 * acc);
+                    if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
+                }
+            }
+            if (fail) *abort = 1;
+            // every tensor-core operation this thread issued has completed
+            mma_commit(drain_bar);
+            if (!mbar_wait_drain(drain_bar, 0)) fail |= kTimeoutDrain;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 2;
+        const int quarter = warp & 3;                 // TMEM lanes this warp may read
+        const int half = ew >> 2;                     // which 128 of the tile's 256 columns
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        float scale = 0.0f;
+        if (!FINE) scale = __fmul_rn(__ldg(p.sa), __ldg(p.sb));
+        for (int t = blockIdx.x; t < tiles && !fail; t += gridDim.x) {
+            int mb, nb;
+            tile_coords(t, p.tiles_m, p.tiles_n, mb, nb);
+            const int row = mb * BM + quarter * 32 + lane;
+            const int col_base = nb * BN + half * BN / 2;
+            if (!FINE) {
+                if (p.num_kb > 0) {
+                    bool ok = true;
+                    if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort);
+                    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                    if (!ok) { fail = kTimeoutEpilogue; break; }
+                    tc_fence_after();
+                }
+#pragma unroll 1
+                for (int c = 0; c < BN / 2 / 32; ++c) {
+                    float v[32];
+                    const int col0 = col_base + c * 32;
+                    if (p.num_kb > 0) {
+                        tmem_ld32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + half * BN / 2 + c * 32), v);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], scale);
+                    if (p.bias) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (col0 + i < p.N) v[i] = __fadd_rn(v[i], load_bias<YT>(p.bias, col0 + i));
+                    }
+                    if (row < p.M && col0 < p.N) store_chunk<YT>(p, row, col0, v);
+                }
+                if (p.num_kb > 0) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+                    if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
+                }
+            } else {
+                float accum[BN / 2];
+#pragma unroll
+                for (int i = 0; i < BN / 2; ++i) accum[i] = 0.0f;
+                const bool row_ok = row < p.M;
+                const bool blk_ok = col_base < p.N;
+                const float* sa_row = p.sa + static_cast<int64_t>(row_ok ? row : 0) * p.sa_ld;
+                const float* sb_row = p.sb + static_cast<int64_t>(blk_ok ? col_base / 128 : 0) * p.sb_ld;
+                float sa_next = (row_ok && p.num_kb > 0) ? __ldg(sa_row) : 0.0f;
+                float sb_next = (blk_ok && p.num_kb > 0) ? __ldg(sb_row) : 0.0f;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    const float s = __fmul_rn(sa_next, sb_next);
+                    if (kb + 1 < p.num_kb) {
+                        sa_next = row_ok ? __ldg(sa_row + kb + 1) : 0.0f;
+                        sb_next = blk_ok ? __ldg(sb_row + kb + 1) : 0.0f;
+                    }
+                    bool ok = true;
+                    if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort);
+                    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                    if (!ok) { fail = kTimeoutEpilogue; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < BN / 2 / 32; ++c) {
+                        float v[32];
+                        tmem_ld32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + half * BN / 2 + c * 32), v);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) accum[c * 32 + i] = __fmaf_rn(v[i], s, accum[c * 32 + i]);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+                    if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
+                }
+                if (fail) break;
+#pragma unroll
+                for (int c = 0; c < BN / 2 / 32; ++c) {
+                    float v[32];
+                    const int col0 = col_base + c * 32;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = accum[c * 32 + i];
+                    if (p.bias) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (col0 + i < p.N) v[i] = __fadd_rn(v[i], load_bias<YT>(p.bias, col0 + i));
+                    }
+                    if (row_ok && col0 < p.N) store_chunk<YT>(p, row, col0, v);
+                }
+            }
+        }
+        if (fail && lane == 0) *abort = 1;
+    }
+
+    if (fail && p.status && lane == 0) atomicOr(p.status, fail);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+    static EncodeTiled fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess || q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<EncodeTiled>(f);
+    }();
+    return fn;
+}
+
+// 2-D map of a [rows][K] byte matrix, boxes of box_rows x 128 bytes, 128-byte
+// swizzle; elements outside the matrix read as zero
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
+    EncodeTiled enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int YT, bool FINE>
+cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, uint32_t idesc,
+                         cudaStream_t s) {
+    auto kernel = scaled_mm_kernel<YT, FINE>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int tiles = p.tiles_m * p.tiles_n;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles < sm_count() ? tiles : sm_count()));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = FP8Q_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, p, idesc);
+}
+
+}  // namespace mm
+
+fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
+                             const float* sa, int sa_ld, const float* sb, int sb_ld, bool fine, const void* bias,
+                             int yt, void* d, uint32_t* status, cudaStream_t s) {
+    using namespace mm;
+    CUtensorMap ma, mbm;
+    memset(&ma, 0, sizeof(ma));
+    memset(&mbm, 0, sizeof(mbm));
+    if (K > 0) {
+        if (!make_map(&ma, a, M, K, BM) || !make_map(&mbm, b, N, K, BN)) return FP8Q_ERR_CUDA;
+    }
+    Params p;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.num_kb = static_cast<int>((K + BK - 1) / BK);
+    p.tiles_m = static_cast<int>((M + BM - 1) / BM);
+    p.tiles_n = static_cast<int>((N + BN - 1) / BN);
+    p.sa = sa;
+    p.sb = sb;
+    p.sa_ld = sa_ld;
+    p.sb_ld = sb_ld;
+    p.bias = bias;
+    p.d = d;
+    const int eb = yt == kF32 ? 4 : 2;
+    p.vec_store = (reinterpret_cast<uintptr_t>(d) % 32 == 0) && ((N * eb) % 32 == 0);
+    p.status = status;
+    const uint32_t idesc = instr_desc(fa, fb);
+    cudaError_t e;
+    if (fine) {
+        e = yt == kF32 ? launch_typed<kF32, true>(ma, mbm, p, idesc, s)
+          : yt == kF16 ? launch_typed<kF16, true>(ma, mbm, p, idesc, s)
+                       : launch_typed<kBF16, true>(ma, mbm, p, idesc, s);
+    } else {
+        e = yt == kF32 ? launch_typed<kF32, false>(ma, mbm, p, idesc, s)
+          : yt == kF16 ? launch_typed<kF16, false>(ma, mbm, p, idesc, s)
+                       : launch_typed<kBF16, false>(ma, mbm, p, idesc, s);
+    }
+    return cuda_status(e);
+}
+
+}  // namespace fp8q

@@ -10,6 +10,9 @@
  *                               weight_dequant / weight_dequant_kernel
  *   fp8q_cast_from_fp8          ColossalAI cast_from_fp8; DeepEP
  *                               per_token_cast_back
+ *   fp8q_scaled_mm              ColossalAI _LinearFp8.forward (torch._scaled_mm)
+ *   fp8q_scaled_mm_blockwise    DeepEP per-token activations x DeepSeek-V3
+ *                               block-scaled weight
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -334,6 +337,57 @@ fp8q_status fp8q_block_dequant_grouped(const fp8q_block_desc* descs, int count,
 fp8q_status fp8q_cast_from_fp8(const uint8_t* q, fp8q_format fmt, int64_t rows, int64_t cols,
                                const float* scale_inv, fp8q_granularity gran, int group_or_block,
                                fp8q_dtype yt, void* y, fp8q_stream_t stream);
+
+/*
+ * fp8 matrix product with per-tensor scales -- ColossalAI
+ * colossalai/quantization/fp8.py, _LinearFp8.forward: both operands cast
+ * with cast_to_fp8 (one scale_inv each), then torch._scaled_mm(x_fp8,
+ * w_fp8.t(), scale_a, scale_b, bias, out_dtype):
+ *   acc[m][n] = sum over k of float(a[m][k]) * float(b[n][k])   (tensor cores, fp32)
+ *   d[m][n]   = T(fl(fl(acc[m][n] * fl(scale_a[0] * scale_b[0])) + bias[n]))
+ * a: [M][K] fp8 codes (format fa), row-major (the activations x_fp8).
+ * b: [N][K] fp8 codes (format fb), row-major: the weight as stored
+ *    ([out features][in features]); the product uses its transpose.
+ *    e4m3fn and e5m2 mix freely (the page's backward multiplies an e5m2
+ *    gradient by an e4m3 weight).
+ * scale_a, scale_b: device fp32 [1] each (the scale_inv the casts return).
+ * bias: NULL or [N] of the output type yt (the page requires the input's dtype).
+ * d: [M][N] of type yt (bf16, fp16 or fp32), row-major (output).
+ * status: NULL or a device uint32 word.  Every internal wait of the kernel
+ *    is bounded; if one runs out (a hardware fault, never in normal use) the
+ *    kernel ORs a nonzero code into *status, leaves d incomplete and returns
+ *    instead of hanging.  The caller clears the word; the library never
+ *    reads it.
+ * The fp32 sum is the tensor cores' own (its rounding is not IEEE-sequential);
+ * tests hold it to an error bound relative to sum |a*b|, not to bit equality.
+ * Errors: K % 16 != 0 (the row pitch of a and b must be a multiple of 16
+ *   bytes), M, N or K above 2^31 - 512 -> FP8Q_ERR_BAD_SHAPE; a or b not
+ *   16-byte aligned -> FP8Q_ERR_MISALIGNED.  M == 0 or N == 0 writes
+ *   nothing; K == 0 writes the bias (or zeros).
+ */
+fp8q_status fp8q_scaled_mm(const uint8_t* a, fp8q_format fa, const uint8_t* b, fp8q_format fb,
+                           int64_t M, int64_t N, int64_t K, const float* scale_a, const float* scale_b,
+                           const void* bias, fp8q_dtype yt, void* d, uint32_t* status,
+                           fp8q_stream_t stream);
+
+/*
+ * fp8 matrix product with fine-grained scales: activations quantised by
+ * per_token_cast_to_fp8 (DeepEP "5 Utils": one scale_inv per 1 x 128 group
+ * of a row) times a weight stored with one scale_inv per 128 x 128 block
+ * (DeepSeek-V3 fp8_cast_bf16 blog, weight_dequant) -- the product of the
+ * two dequantised operands without materialising either:
+ *   acc_kb[m][n] = sum over k in [128 kb, 128 kb + 128) of float(a[m][k]) * float(b[n][k])
+ *   d[m][n]      = T(fl(sum over kb, ascending, of fl(scale_a[m][kb] * scale_b[n/128][kb]) * acc_kb[m][n])
+ *                    + bias[n])     (each step one fused multiply-add)
+ * a: [M][K] codes; scale_a: fp32 [M][ceil(K/128)] (per_token_cast_to_fp8's
+ *    second output).  b: [N][K] codes; scale_b: fp32 [ceil(N/128)][ceil(K/128)]
+ *    (the weight's scale_inv).  bias, d, status, formats and errors as
+ *    fp8q_scaled_mm.
+ */
+fp8q_status fp8q_scaled_mm_blockwise(const uint8_t* a, fp8q_format fa, const float* scale_a,
+                                     const uint8_t* b, fp8q_format fb, const float* scale_b,
+                                     int64_t M, int64_t N, int64_t K, const void* bias, fp8q_dtype yt,
+                                     void* d, uint32_t* status, fp8q_stream_t stream);
 
 #ifdef __cplusplus
 }

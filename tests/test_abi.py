@@ -127,3 +127,39 @@ def test_dequant_validation(L):
     assert L.fp8q_cast_from_fp8(P, 0, 4, 6, P, 2, 4, 2, P, None) == 4
     assert L.fp8q_cast_from_fp8(P, 0, 4, 8, P, 3, 0, 2, P, None) == 4
     assert L.fp8q_cast_from_fp8(P, 0, 4, 8, None, 1, 0, 2, P, None) == 1
+
+
+def test_scaled_mm_validation(L):
+    f = L.fp8q_scaled_mm
+    L.fp8q_scaled_mm.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                 ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    A = 0x10000   # 16-byte aligned fake pointer
+    assert f(A, 0, A, 0, 8, 8, 32, P, P, None, 7, A, None, None) == 2       # output dtype
+    assert f(A, 5, A, 0, 8, 8, 32, P, P, None, 2, A, None, None) == 3       # format of a
+    assert f(A, 0, A, 4, 8, 8, 32, P, P, None, 2, A, None, None) == 3       # format of b
+    assert f(A, 0, A, 0, 8, 8, 24, P, P, None, 2, A, None, None) == 4       # K % 16
+    assert f(A, 0, A, 0, -1, 8, 32, P, P, None, 2, A, None, None) == 4      # negative M
+    assert f(A, 0, A, 0, 8, 1 << 31, 32, P, P, None, 2, A, None, None) == 4  # N above the limit
+    assert f(None, 0, A, 0, 8, 8, 32, P, P, None, 2, A, None, None) == 1    # null a
+    assert f(A, 0, A, 0, 8, 8, 32, None, P, None, 2, A, None, None) == 1    # null scale_a
+    assert f(A, 0, A, 0, 8, 8, 32, P, P, None, 2, None, None, None) == 1    # null out
+    assert f(A + 8, 0, A, 0, 8, 8, 32, P, P, None, 2, A, None, None) == 5   # a not 16-byte aligned
+    assert f(A, 0, A, 0, 8, 8, 32, P, P, A + 1, 2, A, None, None) == 5      # bf16 bias on an odd address
+    assert f(A, 0, A, 0, 8, 8, 32, P, P, None, 2, A, A + 2, None) == 5      # status word misaligned
+    assert f(None, 0, None, 0, 0, 8, 32, None, None, None, 2, None, None, None) == 0   # M == 0: nothing
+
+
+def test_scaled_mm_blockwise_validation(L):
+    f = L.fp8q_scaled_mm_blockwise
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                  ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    A = 0x10000
+    assert f(A, 0, P, A, 0, P, 8, 8, 128, None, 9, A, None, None) == 2      # output dtype
+    assert f(A, 2, P, A, 0, P, 8, 8, 128, None, 2, A, None, None) == 3      # format
+    assert f(A, 0, P, A, 0, P, 8, 8, 136 + 1, None, 2, A, None, None) == 4  # K % 16
+    assert f(A, 0, None, A, 0, P, 8, 8, 128, None, 2, A, None, None) == 1   # null scale_a
+    assert f(A, 0, P, A, 0, None, 8, 8, 128, None, 2, A, None, None) == 1   # null scale_b
+    assert f(A, 0, P + 2, A, 0, P, 8, 8, 128, None, 2, A, None, None) == 5  # scale_a misaligned
+    assert f(A, 0, P, A, 0, P, 8, 0, 128, None, 2, None, None, None) == 0   # N == 0: nothing

@@ -1,0 +1,311 @@
+"""GPU parity of the two fp8 matrix products (tcgen05 tensor cores) with the
+CPU oracle.
+
+ColossalAI _LinearFp8.forward (torch._scaled_mm with per-tensor scales) and
+the fine-grained product of DeepEP per-token activations (1 x 128 group
+scales) with a DeepSeek-V3 block-scaled weight (128 x 128 block scales).
+
+Two kinds of comparison:
+
+* Exact-grid operands (every value a multiple of 1/8, magnitude <= 4): every
+  partial sum of the fp8 products is an fp32 number, so the tensor cores'
+  sum is exact whatever its internal order, and the output must equal the
+  oracle's single-precision rounding of the product bit for bit.  This pins
+  every index, operand, scale, bias and conversion of the data path.
+* General operands (all finite codes): the tensor cores round their fp32
+  sum.  Model: each 32-deep MMA step adds its products to the fp32
+  accumulator with one rounding of at most one fp32 ulp (2^-23 relative),
+  and the products inside a step are summed with at most one more.  Over
+  ceil(K/32) steps that bounds the sum's error by
+  (ceil(K/32) + 1) * 2^-23 * sum |a * b|; the fine-grained product adds one
+  rounding of 2^-24 per k-block for its fused multiply-adds.  The output may
+  then round to either neighbour in T: one ulp of T on top.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from gpu_util import THREADS, Guarded, dev, host
+
+pytestmark = pytest.mark.gpu
+
+E4M3FN, E5M2 = 0, 1
+F32, F16, BF16 = 0, 1, 2
+TORCH_T = {F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}
+
+
+def tdec(codes, fmt):
+    dt = torch.float8_e4m3fn if fmt == E4M3FN else torch.float8_e5m2
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(dt).to(torch.float64).numpy()
+
+
+def grid_codes(g, shape, fmt):
+    codes = workloads.finite_e4m3fn_codes() if fmt == E4M3FN else workloads.finite_e5m2_codes()
+    v = tdec(codes, fmt)
+    keep = codes[(np.abs(v) <= 4) & (v * 8 == np.round(v * 8))]
+    return keep[g.integers(0, keep.size, size=shape)].astype(np.uint8)
+
+
+def finite_codes(g, shape, fmt):
+    codes = workloads.finite_e4m3fn_codes() if fmt == E4M3FN else workloads.finite_e5m2_codes()
+    c = workloads.uniform_codes(g, shape, codes)
+    if fmt == E5M2:
+        c[(c & 0x7F) == 0x7C] = 0
+    return c
+
+
+def t_bias(g, N, yt):
+    """A bias in the output type (as the page requires) and its fp32 values."""
+    b = torch.from_numpy((g.integers(-512, 512, N) / 64.0).astype(np.float32)).to(TORCH_T[yt])
+    return b, b.to(torch.float32).numpy()
+
+
+def run(fp8q, fine, a, fa, b, fb, sa, sb, bias_t, yt, guarded=True):
+    M, K = a.shape
+    N = b.shape[0]
+    out = Guarded(M * N, TORCH_T[yt]) if guarded else None
+    o = out.t.view(M, N) if guarded else torch.empty((M, N), dtype=TORCH_T[yt], device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    A, B = dev(a), dev(b)
+    bt = None if bias_t is None else bias_t.cuda()
+    if fine:
+        fp8q.fp8q_scaled_mm_blockwise(A, dev(sa), B, dev(sb), o, bt, fa=fa, fb=fb, status=st)
+    else:
+        fp8q.fp8q_scaled_mm(A, B, dev(np.array([sa], np.float32)), dev(np.array([sb], np.float32)), o, bt,
+                            fa=fa, fb=fb, status=st)
+    if guarded:
+        out.check()
+    assert int(st.item()) == 0, "a bounded wait ran out"
+    return o
+
+
+def scales(g, M, N, K):
+    kb = -(-K // 128)
+    sa = np.exp(g.normal(-2, 0.5, (M, kb))).astype(np.float32)
+    sb = np.exp(g.normal(-2, 0.5, (-(-N // 128), kb))).astype(np.float32)
+    return sa, sb
+
+
+def oracle_rounded(orc, fine, a, fa, b, fb, sa, sb, bias, yt, rows=None):
+    if fine:
+        return orc.scaled_mm_blockwise_rounded(a, fa, sa, b, fb, sb, bias=bias, yt=yt, rows=rows, threads=THREADS)
+    return orc.scaled_mm_rounded(a, fa, b, fb, sa, sb, bias=bias, yt=yt, rows=rows, threads=THREADS)
+
+
+def bits_equal(got, want, yt):
+    if yt == F32:
+        return got.view(np.uint32) == want.view(np.uint32)
+    return got == want
+
+
+# ---------------------------------------------------------------------------
+# exact-grid operands: bit for bit
+# ---------------------------------------------------------------------------
+SMALL = [(128, 256, 128),     # one tile, one k-block
+         (1, 16, 16),         # the smallest legal product
+         (200, 300, 272),     # partial row / column tiles, a partial last k-block, no vector stores
+         (130, 512, 384)]     # two row tiles, vector stores
+FORMATS = [(E4M3FN, E4M3FN), (E5M2, E4M3FN), (E4M3FN, E5M2), (E5M2, E5M2)]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("fa,fb", FORMATS)
+@pytest.mark.parametrize("fine", [False, True], ids=["tensor", "blockwise"])
+@pytest.mark.parametrize("yt", [F32, F16, BF16])
+def test_exact_grid_bit_exact(fp8q, orc, shape, fa, fb, fine, yt):
+    M, N, K = shape
+    g = np.random.default_rng(hash((M, N, K, fa, fb, fine, yt)) % 2**32)
+    a, b = grid_codes(g, (M, K), fa), grid_codes(g, (N, K), fb)
+    sa, sb = scales(g, M, N, K) if fine else (0.0123, 3.5)
+    bias_t, bias = t_bias(g, N, yt) if (M + yt) % 2 == 0 else (None, None)
+    out = run(fp8q, fine, a, fa, b, fb, sa, sb, bias_t, yt)
+    want = oracle_rounded(orc, fine, a, fa, b, fb, sa, sb, bias, yt)
+    bad = ~bits_equal(host(out), want, yt)
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
+
+
+@pytest.mark.parametrize("fine", [False, True], ids=["tensor", "blockwise"])
+def test_exact_grid_many_tiles(fp8q, orc, fine):
+    """192 tiles on at most 148 persistent CTAs (two tiles for some CTAs, both
+    TMEM accumulators in use); rows of the first, a middle and the last row tile."""
+    M, N, K = 2048, 3000, 512
+    g = np.random.default_rng(77 + fine)
+    a, b = grid_codes(g, (M, K), E4M3FN), grid_codes(g, (N, K), E4M3FN)
+    sa, sb = scales(g, M, N, K) if fine else (0.5, 0.25)
+    bias_t, bias = t_bias(g, N, BF16)
+    got = host(run(fp8q, fine, a, E4M3FN, b, E4M3FN, sa, sb, bias_t, BF16))
+    for r0, r1 in [(0, 40), (1000, 1040), (M - 40, M)]:
+        want = oracle_rounded(orc, fine, a, E4M3FN, b, E4M3FN, sa, sb, bias, BF16, rows=(r0, r1))
+        np.testing.assert_array_equal(got[r0:r1], want[r0:r1])
+
+
+# ---------------------------------------------------------------------------
+# general operands: error bound
+# ---------------------------------------------------------------------------
+def ulp(v, yt):
+    """The spacing of T at |v| (its normal-range ulp, or the subnormal spacing)."""
+    mant, emin = {F32: (23, -126), F16: (10, -14), BF16: (7, -126)}[yt]
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** emin)))
+    return 2.0 ** (e - mant)
+
+
+def check_bound(got, exact, mag, K, yt, fine):
+    steps = -(-K // 32) + 1
+    rel = steps * 2.0 ** -23 + ((-(-K // 128)) * 2.0 ** -24 if fine else 0.0)
+    tol = rel * mag + ulp(exact, yt)
+    err = np.abs(got.astype(np.float64) - exact)
+    bad = ~(err <= tol)
+    assert not bad.any(), (f"{int(bad.sum())} of {bad.size} outside the bound; worst err/mag "
+                           f"{float((err / np.maximum(mag, 1e-300)).max()):.3g}")
+
+
+def to_f64(bits, yt):
+    if yt == F32:
+        return bits.astype(np.float64)
+    t = torch.from_numpy(bits.view(np.int16)).view(TORCH_T[yt])
+    return t.to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("fine", [False, True], ids=["tensor", "blockwise"])
+@pytest.mark.parametrize("yt", [F32, BF16])
+def test_general_operands_within_the_bound(fp8q, orc, fine, yt):
+    M, N, K = 256, 640, 7168
+    g = np.random.default_rng(5 + 2 * fine + yt)
+    a, b = finite_codes(g, (M, K), E4M3FN), finite_codes(g, (N, K), E4M3FN)
+    kb = K // 128
+    if fine:
+        sa = np.exp(g.normal(-4, 2, (M, kb))).astype(np.float32)
+        sb = np.exp(g.normal(-8, 1, (-(-N // 128), kb))).astype(np.float32)
+    else:
+        sa, sb = 0.0123, 3.5
+    got = host(run(fp8q, fine, a, E4M3FN, b, E4M3FN, sa, sb, None, yt))
+    rows = (0, 48)
+    A, W = np.abs(tdec(a[:48], E4M3FN)), np.abs(tdec(b, E4M3FN))
+    if fine:
+        exact = orc.scaled_mm_blockwise(a, E4M3FN, sa, b, E4M3FN, sb, rows=rows, threads=THREADS)[:48]
+        mag = (A * np.repeat(sa[:48], 128, 1)) @ (W * np.repeat(np.repeat(sb, 128, 0), 128, 1)[:N]).T
+    else:
+        exact = orc.scaled_mm(a, E4M3FN, b, E4M3FN, sa, sb, rows=rows, threads=THREADS)[:48]
+        mag = (A @ W.T) * float(np.float32(sa) * np.float32(sb))
+    check_bound(to_f64(got[:48], yt), exact, mag, K, yt, fine)
+
+
+def test_full_size_sampled_rows(fp8q, orc):
+    """The product bench.py times: c2's activations quantised per token
+    (4096 x 7168, by the oracle) times the 18432 x 7168 e4m3fn weight with
+    128 x 128 block scales, bf16 out, both scale modes; sampled rows."""
+    x = workloads.c2_x()
+    q, sa = orc.per_token_group_quant(x, orc.BF16, 128, E4M3FN, threads=THREADS)
+    w, sb = workloads.mm_w_s()
+    M, K = q.shape
+    N = w.shape[0]
+    A, B = dev(q), dev(w)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rows = [0, 1, 3, 7, 2047, 4095]
+    # the bound's magnitudes, in fp32 (they only scale the tolerance)
+    Aabs = np.abs(tdec(q[rows], E4M3FN)).astype(np.float32)
+    Wabs = np.abs(torch.from_numpy(w).view(torch.float8_e4m3fn).to(torch.float32).numpy())
+    # fine-grained
+    fp8q.fp8q_scaled_mm_blockwise(A, dev(sa), B, dev(sb), out, status=st)
+    got = host(out)
+    mag = ((Aabs * np.repeat(sa[rows], 128, 1)) @ (Wabs * np.repeat(np.repeat(sb, 128, 0), 128, 1)).T
+           ).astype(np.float64)
+    for i, r in enumerate(rows):
+        exact = orc.scaled_mm_blockwise(q, E4M3FN, sa, w, E4M3FN, sb, rows=(r, r + 1), threads=THREADS)[r]
+        check_bound(to_f64(got[r], BF16), exact, mag[i], K, BF16, True)
+    # per-tensor, same codes, the scales of row 0's first group and the weight's first block
+    s1, s2 = float(sa[0, 0]), float(sb[0, 0])
+    fp8q.fp8q_scaled_mm(A, B, dev(np.array([s1], np.float32)), dev(np.array([s2], np.float32)), out, status=st)
+    got = host(out)
+    mag = (Aabs @ Wabs.T).astype(np.float64) * float(np.float32(s1) * np.float32(s2))
+    for i, r in enumerate(rows):
+        exact = orc.scaled_mm(q, E4M3FN, w, E4M3FN, s1, s2, rows=(r, r + 1), threads=THREADS)[r]
+        check_bound(to_f64(got[r], BF16), exact, mag[i], K, BF16, False)
+    assert int(st.item()) == 0
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+def test_k_zero_writes_the_bias(fp8q):
+    g = np.random.default_rng(2)
+    for fine in (False, True):
+        bias_t, bias = t_bias(g, 5, BF16)
+        out = run(fp8q, fine, np.zeros((3, 0), np.uint8), E4M3FN, np.zeros((5, 0), np.uint8), E4M3FN,
+                  np.zeros((3, 0), np.float32) if fine else 1.0, np.zeros((1, 0), np.float32) if fine else 1.0,
+                  bias_t, BF16)
+        np.testing.assert_array_equal(out.float().cpu().numpy(), np.tile(bias, (3, 1)))
+        out = run(fp8q, fine, np.zeros((3, 0), np.uint8), E4M3FN, np.zeros((5, 0), np.uint8), E4M3FN,
+                  np.zeros((3, 0), np.float32) if fine else 1.0, np.zeros((1, 0), np.float32) if fine else 1.0,
+                  None, F32)
+        assert (host(out) == 0).all()
+
+
+def test_empty_rows_or_columns_write_nothing(fp8q):
+    a = dev(np.zeros((0, 32), np.uint8))
+    b = dev(np.zeros((8, 32), np.uint8))
+    s = dev(np.ones(1, np.float32))
+    out = torch.empty((0, 8), dtype=torch.bfloat16, device="cuda")
+    fp8q.fp8q_scaled_mm(a, b, s, s, out)
+    g = Guarded(0, torch.bfloat16)
+    fp8q.fp8q_scaled_mm(dev(np.zeros((4, 32), np.uint8)), dev(np.zeros((0, 32), np.uint8)), s, s,
+                        g.t.view(4, 0))
+    g.check()
+
+
+def test_nan_operand_poisons_its_row_only(fp8q):
+    g = np.random.default_rng(3)
+    a, b = grid_codes(g, (128, 256), E4M3FN), grid_codes(g, (256, 256), E4M3FN)
+    a[5, 7] = 0x7F                       # e4m3fn NaN
+    for fine in (False, True):
+        sa, sb = scales(g, 128, 256, 256) if fine else (1.0, 1.0)
+        o = host(run(fp8q, fine, a, E4M3FN, b, E4M3FN, sa, sb, None, F32))
+        assert np.isnan(o[5]).all()
+        assert not np.isnan(np.delete(o, 5, 0)).any()
+
+
+def test_repeat_calls_are_deterministic(fp8q):
+    g = np.random.default_rng(4)
+    M, N, K = 300, 520, 1024
+    a, b = finite_codes(g, (M, K), E4M3FN), finite_codes(g, (N, K), E4M3FN)
+    sa, sb = scales(g, M, N, K)
+    first = host(run(fp8q, True, a, E4M3FN, b, E4M3FN, sa, sb, None, F32))
+    second = host(run(fp8q, True, a, E4M3FN, b, E4M3FN, sa, sb, None, F32))
+    np.testing.assert_array_equal(first.view(np.uint32), second.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# the allocating helpers named after the pages' functions
+# ---------------------------------------------------------------------------
+def test_linear_fp8_matches_the_oracle_composition(fp8q, orc):
+    """ColossalAI linear_fp8 forward: per-tensor e4m3 casts of x and w, then
+    the scaled product in x's dtype, with a bias."""
+    g = np.random.default_rng(6)
+    T, Kd, Nd = 300, 1024, 384
+    x = workloads.to_bf16_bits(g.standard_normal((T, Kd), dtype=np.float32))
+    w = workloads.to_bf16_bits((g.standard_normal((Nd, Kd)) * 0.05).astype(np.float32))
+    bias_t, bias = t_bias(g, Nd, BF16)
+    y = fp8q.linear_fp8(dev(x, torch.bfloat16).view(3, 100, Kd), dev(w, torch.bfloat16), bias_t.cuda())
+    assert y.shape == (3, 100, Nd) and y.dtype == torch.bfloat16
+    qx, sx = orc.cast_per_tensor(x, orc.BF16, E4M3FN)
+    qw, sw = orc.cast_per_tensor(w, orc.BF16, E4M3FN)
+    qx, qw = qx.reshape(T, Kd), qw.reshape(Nd, Kd)
+    exact = orc.scaled_mm(qx, E4M3FN, qw, E4M3FN, float(sx[0]), float(sw[0]), bias=bias.astype(np.float64))
+    mag = (np.abs(tdec(qx, E4M3FN)) @ np.abs(tdec(qw, E4M3FN)).T) * float(sx[0] * sw[0])
+    check_bound(to_f64(host(y).reshape(T, Nd), BF16), exact, mag, Kd, BF16, False)
+
+
+def test_linear_fp8_blockwise_matches_the_oracle_composition(fp8q, orc):
+    g = np.random.default_rng(8)
+    T, Kd, Nd = 200, 512, 300
+    x = workloads.to_bf16_bits(g.standard_normal((T, Kd), dtype=np.float32))
+    w = finite_codes(g, (Nd, Kd), E4M3FN)
+    sw = workloads.lognormal_scales(g, workloads.scale_shape(Nd, Kd))
+    y = fp8q.linear_fp8_blockwise(dev(x, torch.bfloat16), dev(w).view(torch.float8_e4m3fn), dev(sw))
+    qx, sx = orc.per_token_group_quant(x, orc.BF16, 128, E4M3FN)
+    exact = orc.scaled_mm_blockwise(qx, E4M3FN, sx, w, E4M3FN, sw)
+    mag = (np.abs(tdec(qx, E4M3FN)) * np.repeat(sx, 128, 1)) @ \
+        (np.abs(tdec(w, E4M3FN)) * np.repeat(np.repeat(sw, 128, 0), 128, 1)[:Nd]).T
+    check_bound(to_f64(host(y), BF16), exact, mag, Kd, BF16, True)

@@ -26,6 +26,11 @@ Workloads (shapes and value mixes of the pages' use cases):
   64-bit indexing cases), drawn on the device by torch's seeded CUDA
   generator in chunks, because the host cannot draw them in seconds.  The
   tests copy sampled rows back for the oracle.
+* ``mm`` fp8 products: the weight W[18432, 7168] (the DeepSeek-V3 MLP gate /
+  up projection shape, [out features][in features], the transpose of c3's
+  shape) with codes uniform over the finite e4m3fn codes and 128 x 128 block
+  scales s[144, 56] = exp(N(-8, 1)); the activations are c2's x quantised
+  per token (1 x 128 groups).  Seed 20261206.
 * ``c5`` ragged MoE dequant: 64 weights [2048, 7168] then 8 weights
   [7000, 1000]; codes uniform over the finite e4m3fn codes; ceil-sized
   scales exp(N(-8, 1)).  Weight i draws from seed (20261205, i) so any
@@ -45,6 +50,7 @@ C4A_SHAPE = (8192, 8192)
 C4B_NUMEL = 64 * 1024 * 1024
 C4C_NUMEL = 1024 * 1024
 C5_SHAPES = [(2048, 7168)] * 64 + [(7000, 1000)] * 8
+MM_W_SHAPE = (18432, 7168)
 BLOCK = 128
 GROUP = 128
 
@@ -115,6 +121,14 @@ def c3_w_s():
     M, N = C3_SHAPE
     w = uniform_codes(g, (M, N), finite_e4m3fn_codes())
     s = lognormal_scales(g, scale_shape(M, N))
+    return w, s
+
+
+def mm_w_s():
+    g = rng(SEED_BASE + 6)
+    N, K = MM_W_SHAPE
+    w = uniform_codes(g, (N, K), finite_e4m3fn_codes())
+    s = lognormal_scales(g, scale_shape(N, K))
     return w, s
 
 
