@@ -25,9 +25,10 @@
 //               scaling, bias, conversion, 32-byte stores.  With fine-grained
 //               scales the MMA warp commits every 128-deep k-block into a
 //               fresh accumulator and the epilogue folds it into registers
-//               with that block's scale, while the tensor cores fill the
-//               other accumulator.
-// Tiles are 128 x 256 of D, visited in bands of 16 row-tiles so that the
+//               with that block's scale (packed fp32x2 FMAs, TMEM loads
+//               double-buffered in 16-column chunks), while the tensor
+//               cores fill the other accumulator.
+// Tiles are 128 x 256 of D, visited in bands of 32 row-tiles so that the
 // CTAs working at one time share A and B tiles in L2.
 //
 // Every wait on an mbarrier is bounded (a few seconds of global time).  A
@@ -55,7 +56,7 @@ constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kABytes = BM * BK;
 constexpr int kBBytes = BN * BK;
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kGroupM = 16;     // row-tiles per raster band
+constexpr int kGroupM = 32;     // row-tiles per raster band
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment slack */ + 256 /* barriers */;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
@@ -190,6 +191,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
                  :: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 16 consecutive columns, issued without waiting: tmem_wait16 on
+// the same registers completes it (and every other load still in flight)
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32"
+                 " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15])
+                 :: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -432,9 +451,10 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
                 }
             } else {
-                float accum[BN / 2];
+                // this warp's 128 columns of its 32 rows, as 64 fp32 pairs
+                float2 accum[BN / 4];
 #pragma unroll
-                for (int i = 0; i < BN / 2; ++i) accum[i] = 0.0f;
+                for (int i = 0; i < BN / 4; ++i) accum[i] = make_float2(0.0f, 0.0f);
                 const bool row_ok = row < p.M;
                 const bool blk_ok = col_base < p.N;
                 const float* sa_row = p.sa + static_cast<int64_t>(row_ok ? row : 0) * p.sa_ld;
@@ -452,12 +472,25 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
                     if (!ok) { fail = kTimeoutEpilogue; break; }
                     tc_fence_after();
+                    // 8 chunks of 16 columns, double-buffered: the load of chunk
+                    // c + 1 is in flight while chunk c is folded in with packed
+                    // fused multiply-adds (each lane the same as __fmaf_rn)
+                    const uint32_t col_addr = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + half * BN / 2);
+                    const float2 s2 = make_float2(s, s);
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16_async(col_addr, r0);
+                    tmem_wait16(r0);
 #pragma unroll
-                    for (int c = 0; c < BN / 2 / 32; ++c) {
-                        float v[32];
-                        tmem_ld32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + half * BN / 2 + c * 32), v);
+                    for (int c = 0; c < BN / 2 / 16; ++c) {
+                        uint32_t (&cur)[16] = (c & 1) ? r1 : r0;
+                        uint32_t (&nxt)[16] = (c & 1) ? r0 : r1;
+                        if (c + 1 < BN / 2 / 16) tmem_ld16_async(col_addr + 16 * (c + 1), nxt);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) accum[c * 32 + i] = __fmaf_rn(v[i], s, accum[c * 32 + i]);
+                        for (int i = 0; i < 8; ++i)
+                            accum[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(cur[2 * i]),
+                                                                      __uint_as_float(cur[2 * i + 1])),
+                                                          s2, accum[c * 8 + i]);
+                        if (c + 1 < BN / 2 / 16) tmem_wait16(nxt);
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -470,7 +503,10 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     float v[32];
                     const int col0 = col_base + c * 32;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = accum[c * 32 + i];
+                    for (int i = 0; i < 16; ++i) {
+                        v[2 * i] = accum[c * 16 + i].x;
+                        v[2 * i + 1] = accum[c * 16 + i].y;
+                    }
                     if (p.bias) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
