@@ -14,21 +14,22 @@
 // where acc is the fp32 tensor-core sum of the fp8 products.
 //
 // Design (one persistent CTA per SM, warp-specialised):
-//   warp 0      TMA producer: 128 x 128-byte tiles of A and 256 x 128-byte
-//               tiles of B (128-byte swizzle) into a 4-stage shared-memory ring
+//   warp 0      TMA producer: 128 x 128-byte tiles of A and BN x 128-byte
+//               tiles of B (128-byte swizzle) into a shared-memory ring
 //   warp 1      allocates 512 TMEM columns; one lane issues
-//               tcgen05.mma.kind::f8f6f4 (M 128, N 256, K 32) into one of two
-//               128 x 256 fp32 TMEM accumulators and commits each stage back
+//               tcgen05.mma.kind::f8f6f4 (M 128, N BN, K 32) into one of the
+//               128 x BN fp32 TMEM accumulators and commits each stage back
 //               to the producer and each finished accumulator to the epilogue
 //   warps 2-9   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32 * (w % 4) .. + 31, columns of half (w - 2) / 4),
+//               lanes 32 * (w % 4) .. + 31, column group (w - 2) / 4),
 //               scaling, bias, conversion, 32-byte stores.  With fine-grained
 //               scales the MMA warp commits every 128-deep k-block into a
 //               fresh accumulator and the epilogue folds it into registers
 //               with that block's scale (packed fp32x2 FMAs, TMEM loads
 //               double-buffered in 16-column chunks), while the tensor
-//               cores fill the other accumulator.
-// Tiles are 128 x 256 of D, visited in bands of 32 row-tiles so that the
+//               cores fill the other accumulators.
+// Tiles are 128 x BN of D (see Shape), visited in bands of 32 row-tiles so
+// that the
 // CTAs working at one time share A and B tiles in L2.
 //
 // Every wait on an mbarrier is bounded (a few seconds of global time).  A
@@ -46,18 +47,28 @@ namespace fp8q {
 namespace mm {
 
 constexpr int BM = 128;         // rows of A (and of D) per tile
-constexpr int BN = 256;         // rows of B (columns of D) per tile
 constexpr int BK = 128;         // k per stage: one 128-byte swizzle row, one scale block
-constexpr int kStages = 4;
-constexpr int kAccBufs = 2;
-constexpr int kTmemCols = kAccBufs * BN;   // 512: all of TMEM
+constexpr int kTmemCols = 512;  // all of TMEM, split into kAccBufs accumulators
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kABytes = BM * BK;
-constexpr int kBBytes = BN * BK;
-constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kGroupM = 32;     // row-tiles per raster band
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment slack */ + 256 /* barriers */;
+
+// Tile shape per product: 128 x 256 tiles, two TMEM accumulators (with
+// per-tensor scales one tile's epilogue overlaps the next tile's k-loop; with
+// fine-grained scales one k-block's fold overlaps the next block's MMAs), a
+// 4-stage ring.  Measured on B200: 128 x 128 tiles with four accumulators and
+// six stages lose a quarter of the fine-grained product's throughput, since
+// the narrower MMA reads twice the operand bytes per flop.
+template <bool FINE> struct Shape {
+    static constexpr int BN = 256;                          // rows of B (columns of D) per tile
+    static constexpr int kStages = 4;
+    static constexpr int kAccBufs = kTmemCols / BN;
+    static constexpr int kColsPerWarp = BN / (kEpiWarps / 4);   // tile columns one epilogue warp owns
+    static constexpr int kBBytes = BN * BK;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment slack */ + 256 /* barriers */;
+};
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
 // status bits ORed into the caller's status word when a wait runs out
@@ -153,9 +164,9 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 // Instruction descriptor of kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B
 // formats (bits 7-9, 10-12: 0 e4m3, 1 e5m2), both K-major, N >> 3 at bit 17,
 // M >> 4 at bit 24.
-__host__ __device__ constexpr uint32_t instr_desc(int fa, int fb) {
+__host__ __device__ constexpr uint32_t instr_desc(int fa, int fb, int bn) {
     return (1u << 4) | (static_cast<uint32_t>(fa) << 7) | (static_cast<uint32_t>(fb) << 10)
-         | (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+         | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
 }
 __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                            uint32_t accumulate) {
@@ -285,6 +296,12 @@ template <int YT, bool FINE>
 __global__ void __launch_bounds__(kThreads, 1)
 scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const Params p, const uint32_t idesc) {
+    constexpr int BN = Shape<FINE>::BN;
+    constexpr int kStages = Shape<FINE>::kStages;
+    constexpr int kAccBufs = Shape<FINE>::kAccBufs;
+    constexpr int kColsPerWarp = Shape<FINE>::kColsPerWarp;
+    constexpr int kBBytes = Shape<FINE>::kBBytes;
+    constexpr int kStageBytes = Shape<FINE>::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -406,7 +423,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         // ------------------------------------------------------------ epilogue
         const int ew = warp - 2;
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
-        const int half = ew >> 2;                     // which 128 of the tile's 256 columns
+        const int cgrp = ew >> 2;                     // which kColsPerWarp-wide group of the tile's columns
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -416,7 +433,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             int mb, nb;
             tile_coords(t, p.tiles_m, p.tiles_n, mb, nb);
             const int row = mb * BM + quarter * 32 + lane;
-            const int col_base = nb * BN + half * BN / 2;
+            const int col_base = nb * BN + cgrp * kColsPerWarp;
             if (!FINE) {
                 if (p.num_kb > 0) {
                     bool ok = true;
@@ -426,11 +443,11 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     tc_fence_after();
                 }
 #pragma unroll 1
-                for (int c = 0; c < BN / 2 / 32; ++c) {
+                for (int c = 0; c < kColsPerWarp / 32; ++c) {
                     float v[32];
                     const int col0 = col_base + c * 32;
                     if (p.num_kb > 0) {
-                        tmem_ld32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + half * BN / 2 + c * 32), v);
+                        tmem_ld32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + cgrp * kColsPerWarp + c * 32), v);
                     } else {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = 0.0f;
@@ -451,10 +468,10 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
                 }
             } else {
-                // this warp's 128 columns of its 32 rows, as 64 fp32 pairs
-                float2 accum[BN / 4];
+                // this warp's kColsPerWarp columns of its 32 rows, as fp32 pairs
+                float2 accum[kColsPerWarp / 2];
 #pragma unroll
-                for (int i = 0; i < BN / 4; ++i) accum[i] = make_float2(0.0f, 0.0f);
+                for (int i = 0; i < kColsPerWarp / 2; ++i) accum[i] = make_float2(0.0f, 0.0f);
                 const bool row_ok = row < p.M;
                 const bool blk_ok = col_base < p.N;
                 const float* sa_row = p.sa + static_cast<int64_t>(row_ok ? row : 0) * p.sa_ld;
@@ -475,22 +492,22 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     // 8 chunks of 16 columns, double-buffered: the load of chunk
                     // c + 1 is in flight while chunk c is folded in with packed
                     // fused multiply-adds (each lane the same as __fmaf_rn)
-                    const uint32_t col_addr = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + half * BN / 2);
+                    const uint32_t col_addr = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + cgrp * kColsPerWarp);
                     const float2 s2 = make_float2(s, s);
                     uint32_t r0[16], r1[16];
                     tmem_ld16_async(col_addr, r0);
                     tmem_wait16(r0);
 #pragma unroll
-                    for (int c = 0; c < BN / 2 / 16; ++c) {
+                    for (int c = 0; c < kColsPerWarp / 16; ++c) {
                         uint32_t (&cur)[16] = (c & 1) ? r1 : r0;
                         uint32_t (&nxt)[16] = (c & 1) ? r0 : r1;
-                        if (c + 1 < BN / 2 / 16) tmem_ld16_async(col_addr + 16 * (c + 1), nxt);
+                        if (c + 1 < kColsPerWarp / 16) tmem_ld16_async(col_addr + 16 * (c + 1), nxt);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             accum[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(cur[2 * i]),
                                                                       __uint_as_float(cur[2 * i + 1])),
                                                           s2, accum[c * 8 + i]);
-                        if (c + 1 < BN / 2 / 16) tmem_wait16(nxt);
+                        if (c + 1 < kColsPerWarp / 16) tmem_wait16(nxt);
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -499,7 +516,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 }
                 if (fail) break;
 #pragma unroll
-                for (int c = 0; c < BN / 2 / 32; ++c) {
+                for (int c = 0; c < kColsPerWarp / 32; ++c) {
                     float v[32];
                     const int col0 = col_base + c * 32;
 #pragma unroll
@@ -567,6 +584,7 @@ template <int YT, bool FINE>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, uint32_t idesc,
                          cudaStream_t s) {
     auto kernel = scaled_mm_kernel<YT, FINE>;
+    constexpr int kSmemBytes = Shape<FINE>::kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const int tiles = p.tiles_m * p.tiles_n;
@@ -589,11 +607,12 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
                              const float* sa, int sa_ld, const float* sb, int sb_ld, bool fine, const void* bias,
                              int yt, void* d, uint32_t* status, cudaStream_t s) {
     using namespace mm;
+    const int bn = fine ? Shape<true>::BN : Shape<false>::BN;
     CUtensorMap ma, mbm;
     memset(&ma, 0, sizeof(ma));
     memset(&mbm, 0, sizeof(mbm));
     if (K > 0) {
-        if (!make_map(&ma, a, M, K, BM) || !make_map(&mbm, b, N, K, BN)) return FP8Q_ERR_CUDA;
+        if (!make_map(&ma, a, M, K, BM) || !make_map(&mbm, b, N, K, bn)) return FP8Q_ERR_CUDA;
     }
     Params p;
     p.M = static_cast<int>(M);
@@ -601,7 +620,7 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     p.K = static_cast<int>(K);
     p.num_kb = static_cast<int>((K + BK - 1) / BK);
     p.tiles_m = static_cast<int>((M + BM - 1) / BM);
-    p.tiles_n = static_cast<int>((N + BN - 1) / BN);
+    p.tiles_n = static_cast<int>((N + bn - 1) / bn);
     p.sa = sa;
     p.sb = sb;
     p.sa_ld = sa_ld;
@@ -611,7 +630,7 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     const int eb = yt == kF32 ? 4 : 2;
     p.vec_store = (reinterpret_cast<uintptr_t>(d) % 32 == 0) && ((N * eb) % 32 == 0);
     p.status = status;
-    const uint32_t idesc = instr_desc(fa, fb);
+    const uint32_t idesc = instr_desc(fa, fb, bn);
     cudaError_t e;
     if (fine) {
         e = yt == kF32 ? launch_typed<kF32, true>(ma, mbm, p, idesc, s)
