@@ -18,6 +18,15 @@ the 126 MB L2, so no operation finds its inputs in L2 from the previous step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+Beside the step, rank 0 reports two more measurements that are not part of
+`value`: "isolated" times per-token quant, block dequant, the round trip, the
+per-channel and the fp32 per-tensor casts each alone, back to back over
+rotating buffer sets at least 4x the L2 size (each launch reads
+cold inputs and pays for the write-back of one launch of its own outputs);
+"matmul" times the two fp8 products on the tensor cores (TFLOP/s against the
+fp8 peak) beside torch._scaled_mm (cuBLASLt) on the same operands
+(--no-matmul skips it).
+
 With N > 1 it runs under torchrun, one rank per GPU, each rank doing the full
 step on its own copy of the inputs (independent problems, weak scaling, no
 data-path collective); the time is the max over ranks.  `--impl reference`
@@ -263,7 +272,105 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
         y = torch.empty((M, N), dtype=torch.bfloat16, device=d)
         return lambda: f.fp8q_block_dequant(w, wl.c3_s, y, 128, E4M3FN)
     run("block_dequant", dequant_set, c3_bytes, c3_bytes)
+
+    def round_trip_set(i):
+        q = wl.c2_q if i == 0 else wl.c2_q.clone()
+        s = wl.c2_s if i == 0 else wl.c2_s.clone()
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=d)
+        return lambda: f.fp8q_cast_from_fp8(q, s, y, GRAN_GROUP, 128, E4M3FN)
+    run("cast_from_fp8_group", round_trip_set, c2_bytes, c2_bytes)
+
+    R, C = wl.c4a_x.shape
+    c4a_bytes = R * C * 3 + R * 4
+
+    def per_channel_set(i):
+        x = wl.c4a_x if i == 0 else wl.c4a_x.clone()
+        q = torch.empty((R, C), dtype=torch.uint8, device=d)
+        s = torch.empty((R,), dtype=torch.float32, device=d)
+        return lambda: f.fp8q_cast_per_channel(x, q, s, E4M3FN)
+    run("cast_per_channel", per_channel_set, c4a_bytes, c4a_bytes)
+
+    n4 = wl.c4b_x.numel()
+    c4b_bytes = 2 * n4 * 4 + n4 + 4
+
+    def per_tensor_set(i):
+        x = wl.c4b_x if i == 0 else wl.c4b_x.clone()
+        q = torch.empty((n4,), dtype=torch.uint8, device=d)
+        s = torch.empty((1,), dtype=torch.float32, device=d)
+        return lambda: f.fp8q_cast_per_tensor(x, q, s, wl.ws, E5M2)
+    run("cast_per_tensor_f32_e5m2", per_tensor_set, n4 * 5 + 4, c4b_bytes)
     return out
+
+
+class MatmulWorkload:
+    """The two fp8 products on the tensor cores: c2's activations x[4096, 7168]
+    quantised per token by the library (codes and 1 x 128 scales, made once,
+    before timing) times the e4m3fn weight W[18432, 7168] with 128 x 128 block
+    scales; bf16 out [4096, 18432].  Per-tensor: the same codes with one scale
+    each (ColossalAI linear_fp8's torch._scaled_mm)."""
+
+    def __init__(self, wl: Workload):
+        f, d = wl.fp8q, wl.device
+        m, k = wl.c2_x.shape
+        self.q = torch.empty((m, k), dtype=torch.uint8, device=d)
+        self.sa = torch.empty((m, k // 128), dtype=torch.float32, device=d)
+        f.fp8q_per_token_group_quant(wl.c2_x, self.q, self.sa, 128, E4M3FN)
+        w, sb = workloads.mm_w_s()
+        self.w, self.sb = _to_dev(w, d), _to_dev(sb, d)
+        self.n = self.w.shape[0]
+        self.out = torch.empty((m, self.n), dtype=torch.bfloat16, device=d)
+        self.s1 = self.sa[:1, :1].reshape(1).clone()
+        self.s2 = self.sb[:1, :1].reshape(1).clone()
+        self.status = torch.zeros(1, dtype=torch.int32, device=d)
+        self.flops = 2.0 * m * self.n * k
+        self.shape = (m, self.n, k)
+        self.ops = {
+            "scaled_mm_blockwise": lambda: f.fp8q_scaled_mm_blockwise(self.q, self.sa, self.w, self.sb, self.out,
+                                                                      status=self.status),
+            "scaled_mm_per_tensor": lambda: f.fp8q_scaled_mm(self.q, self.w, self.s1, self.s2, self.out,
+                                                             status=self.status),
+        }
+
+    def time(self, steps: int, warmup: int, device):
+        """ms per launch of each op (CUDA events around `steps` back-to-back launches
+        after `warmup`), plus torch._scaled_mm (cuBLASLt) on the same operands."""
+        res = {}
+        ops = dict(self.ops)
+        a8 = self.q.view(torch.float8_e4m3fn)
+        b8 = self.w.view(torch.float8_e4m3fn)
+        ops["torch_scaled_mm (cuBLASLt)"] = lambda: torch._scaled_mm(a8, b8.t(), scale_a=self.s1, scale_b=self.s2,
+                                                                    out_dtype=torch.bfloat16)
+        for name, fn in ops.items():
+            try:
+                for _ in range(warmup):
+                    fn()
+                torch.cuda.synchronize(device)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with ClockSampler(device.index or 0) as clk:
+                    e0.record()
+                    for _ in range(steps):
+                        fn()
+                    e1.record()
+                    torch.cuda.synchronize(device)
+                ms = e0.elapsed_time(e1) / steps
+                res[name] = {"ms": round(ms, 4), "tflops": round(self.flops / (ms * 1e-3) / 1e12, 1),
+                             "clocks": clk.summary()}
+            except Exception as ex:      # the library baseline may be missing on some builds of torch
+                res[name] = {"unavailable": str(ex).splitlines()[0][:200]}
+        if int(self.status.item()) != 0:
+            raise RuntimeError("a bounded wait of the fp8 product ran out")
+        return res
+
+
+def fp8_tensor_peak():
+    """Dense fp8 tensor-core peak: the measured cuBLAS bf16 burst figure times
+    the nominal fp8 : bf16 ratio of 2."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return 2.0 * float(d["bf16_tflops"]), "2 x measured bf16 burst (nominal fp8:bf16 ratio)"
+    return 2.0 * 1590.0, "2 x fallback bf16 burst (nominal fp8:bf16 ratio)"
 
 
 def _to_dev(a, device, dt=None):
@@ -528,6 +635,21 @@ def run_ours(args):
     bi, bo = e2e.h2d_bytes, e2e.d2h_bytes
     del e2e
     iso = isolated_timing(wl) if rank == 0 else {}
+    mm = None
+    if rank == 0 and not args.no_matmul:
+        mmw = MatmulWorkload(wl)
+        mm_res = mmw.time(max(5, min(args.steps, 50)), max(3, args.warmup), device)
+        tpeak, tkind = fp8_tensor_peak()
+        for v in mm_res.values():
+            if "tflops" in v:
+                v["frac"] = round(v["tflops"] / tpeak, 4)
+        mm = {"workload": "fp8 products: per-token e4m3fn codes of c2 x[4096,7168] (1x128 scales) times "
+                          "e4m3fn W[18432,7168] (128x128 block scales), bf16 out; per-tensor: same codes, "
+                          "one scale each",
+              "shape_mnk": list(mmw.shape), "flops_per_launch": mmw.flops, "bound": "tensor",
+              "peak_tflops": round(tpeak, 1), "peak_kind": tkind,
+              "l2": "operands 161 MB > 126 MB L2; compute-bound, no flush", "ops": mm_res}
+        del mmw
 
     if rank != 0:
         _finish(world)
@@ -555,6 +677,7 @@ def run_ours(args):
                      "bytes_per_launch": dop.bytes, "traffic": recorded_traffic(dop.name)},
         "kernels": kernels,
         "isolated": {k: {**v, "frac": round(v["gb_s"] / peak, 4)} for k, v in iso.items()},
+        "matmul": mm,
         "clocks": clk.summary(),
         "e2e": {"value": round(world * wl.step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
@@ -657,6 +780,20 @@ def _profile_case(name, fp8q, device):
         s = torch.empty((1,), dtype=torch.float32, device=device)
         ws = torch.empty(fp8q.fp8q_cast_per_tensor_workspace_bytes(), dtype=torch.uint8, device=device)
         return (lambda: fp8q.fp8q_cast_per_tensor(x, q, s, ws, E5M2)), x.numel() * 9 + 4
+    if name in ("scaled_mm", "scaled_mm_blockwise"):
+        m, k = workloads.C2_SHAPE
+        x = _to_dev(workloads.c2_x(), device, bf16)
+        q = torch.empty((m, k), dtype=torch.uint8, device=device)
+        sa = torch.empty((m, k // 128), dtype=torch.float32, device=device)
+        fp8q.fp8q_per_token_group_quant(x, q, sa, 128, E4M3FN)
+        w, sb = workloads.mm_w_s()
+        w, sb = _to_dev(w, device), _to_dev(sb, device)
+        out = torch.empty((m, w.shape[0]), dtype=bf16, device=device)
+        s1 = torch.ones(1, dtype=torch.float32, device=device)
+        flops = 2.0 * m * w.shape[0] * k
+        if name == "scaled_mm":
+            return (lambda: fp8q.fp8q_scaled_mm(q, w, s1, s1, out)), flops
+        return (lambda: fp8q.fp8q_scaled_mm_blockwise(q, sa, w, sb, out)), flops
     if name in ("records_pack", "records_unpack"):
         # the fp8 all-gather's device work for 8 ranks of 16 Mi bf16 each
         # (32 MiB per rank): pack = each rank's per-tensor cast into its
@@ -680,7 +817,7 @@ def _profile_case(name, fp8q, device):
 
 
 PROFILE_CASES = ["per_token_4x", "cast_from_fp8_4x", "block_dequant", "grouped_16", "grouped_72", "per_channel",
-                 "per_tensor", "records_pack", "records_unpack"]
+                 "per_tensor", "records_pack", "records_unpack", "scaled_mm", "scaled_mm_blockwise"]
 
 
 def run_profile_case(name, iters):
@@ -698,6 +835,10 @@ def run_profile_case(name, iters):
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / max(iters, 1)
+    if name.startswith("scaled_mm"):
+        print(f"profile case {name}: {iters} calls, {us:.2f} us per call, "
+              f"{nbytes / (us * 1e-6) / 1e12 if iters else 0.0:.1f} TFLOP/s")
+        return
     print(f"profile case {name}: {iters} calls, {us:.2f} us per call, "
           f"{nbytes / (us * 1e-6) / 1e9 if iters else 0.0:.1f} GB/s algorithmic")
 
@@ -711,6 +852,7 @@ def main(argv=None):
     ap.add_argument("--profile", choices=PROFILE_CASES,
                     help="run one op of a fixed case --iters times for a profiler capture (no timing)")
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--no-matmul", action="store_true", help="skip the fp8 products section")
     args = ap.parse_args(argv)
     if args.profile:
         run_profile_case(args.profile, args.iters)
