@@ -95,6 +95,10 @@ def lib() -> ctypes.CDLL:
             L.orc_scaled_mm_blockwise_rounded.restype = i32
             L.orc_scaled_mm_blockwise_rounded.argtypes = [c_void, i32, c_void, c_void, i32, c_void, i64, i64, i64,
                                                           i64, c_void, i32, c_void, i64, i64]
+            L.orc_transpose_u8.restype = i32
+            L.orc_transpose_u8.argtypes = [c_void, i64, i64, c_void, i64]
+            L.orc_sum_rows.restype = i32
+            L.orc_sum_rows.argtypes = [c_void, i32, i64, i64, c_void]
             L.orc_scaled_mm_blockwise.restype = i32
             L.orc_scaled_mm_blockwise.argtypes = [c_void, i32, c_void, i64, c_void, i32, c_void, i64,
                                                   i64, i64, i64, c_void, c_void, i64, i64]
@@ -459,4 +463,24 @@ def scaled_mm_blockwise_rounded(a: np.ndarray, fa: int, sa: np.ndarray, b: np.nd
     _run(lambda x, y: _check(L.orc_scaled_mm_blockwise_rounded(_ptr(a), fa, _ptr(sa), _ptr(b), fb, _ptr(sb),
                                                                block, M, N, K, bp, yt, _ptr(out), x, y),
                              "scaled_mm_blockwise_rounded"), r0, r1, threads)
+    return out
+
+
+def transpose_u8(src: np.ndarray, ld: int = None) -> np.ndarray:
+    """ColossalAI _LinearFp8.backward's .t().contiguous() of fp8 codes: src[rows, cols]
+    -> dst[cols, ld] with dst[c, r] = src[r, c] and zeros for rows <= r < ld."""
+    src = np.ascontiguousarray(src, dtype=np.uint8)
+    rows, cols = src.shape
+    ld = rows if ld is None else ld
+    dst = np.full((cols, ld), 0xA5, np.uint8)
+    _check(lib().orc_transpose_u8(_ptr(src), rows, cols, _ptr(dst), ld), "transpose_u8")
+    return dst
+
+
+def sum_rows(x: np.ndarray, xt: int) -> np.ndarray:
+    """out_grad.sum(0) of x[rows, cols] (bit patterns of type xt), in float64."""
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    out = np.zeros((cols,), np.float64)
+    _check(lib().orc_sum_rows(_ptr(x), xt, rows, cols, _ptr(out)), "sum_rows")
     return out

@@ -219,6 +219,7 @@ static void store_elem(void* y, int yt, int64_t i, float v)
 }
 
 static int valid_fmt(int fmt) { return fmt == ORC_E4M3FN || fmt == ORC_E5M2; }
+static int valid_dtype(int t) { return t == ORC_F32 || t == ORC_F16 || t == ORC_BF16; }
 static int valid_dt(int t)    { return t == ORC_F32 || t == ORC_F16 || t == ORC_BF16; }
 
 /* max |x| over x[i0 .. i0+count), NaN-propagating like torch's max/amax:
@@ -645,5 +646,35 @@ int orc_scaled_mm_blockwise_rounded(const uint8_t* a, int fa, const float* sa, c
             if (bias) acc = acc + bias[n];
             store_elem(out, yt, m * N + n, acc);
         }
+    return 0;
+}
+
+/*
+ * [CAI] _LinearFp8.backward's data movements.
+ * orc_transpose_u8: the .t().contiguous() copy of an fp8 operand, dst[c][r] =
+ * src[r][c] for r < rows, zero for rows <= r < ld (the zero-padded pitch).
+ * orc_sum_rows: bias_grad = out_grad.sum(0), out[c] = sum over r of x[r][c],
+ * added in binary64 in ascending r (every bf16 / fp16 / fp32 value is exact
+ * in binary64, so for up to 2^24 rows of values within a few binades the sum
+ * is exact or within 2^-53 relative).
+ */
+int orc_transpose_u8(const uint8_t* src, int64_t rows, int64_t cols, uint8_t* dst, int64_t ld)
+{
+    if (rows < 0 || cols < 0 || ld < rows) return -1;
+    for (int64_t c = 0; c < cols; ++c) {
+        for (int64_t r = 0; r < rows; ++r) dst[c * ld + r] = src[r * cols + c];
+        for (int64_t r = rows; r < ld; ++r) dst[c * ld + r] = 0;
+    }
+    return 0;
+}
+
+int orc_sum_rows(const void* x, int xt, int64_t rows, int64_t cols, double* out)
+{
+    if (!valid_dtype(xt) || rows < 0 || cols < 0) return -1;
+    for (int64_t c = 0; c < cols; ++c) {
+        double acc = 0.0;
+        for (int64_t r = 0; r < rows; ++r) acc += (double)load_elem(x, xt, r * cols + c);
+        out[c] = acc;
+    }
     return 0;
 }

@@ -153,6 +153,12 @@ int orc_scaled_mm_blockwise_rounded(const uint8_t* a, int fa, const float* sa, c
                                     const float* sb, int64_t bb, int64_t M, int64_t N, int64_t K,
                                     const float* bias, int yt, void* out, int64_t r0, int64_t r1);
 
+/* [CAI] _LinearFp8.backward: the operand transpose dst[c][r] = src[r][c]
+ * (zero for rows <= r < ld) and the bias gradient out[c] = sum_r x[r][c]
+ * in binary64, ascending r. */
+int orc_transpose_u8(const uint8_t* src, int64_t rows, int64_t cols, uint8_t* dst, int64_t ld);
+int orc_sum_rows(const void* x, int xt, int64_t rows, int64_t cols, double* out);
+
 #ifdef __cplusplus
 }
 #endif

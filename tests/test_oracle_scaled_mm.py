@@ -290,3 +290,34 @@ def test_rounded_forms_stay_within_half_an_ulp_of_the_exact_product(orc):
     exact = orc.scaled_mm(a, E4M3FN, b, E4M3FN, 0.01, 3.0, bias=bias.astype(np.float64))
     mag = (np.abs(A) @ np.abs(W).T) * 0.03
     assert np.all(np.abs(got - exact) <= 2.0 ** -21 * (mag + np.abs(bias)))
+
+
+# ---------------------------------------------------------------------------
+# _LinearFp8.backward's transpose and bias gradient
+# ---------------------------------------------------------------------------
+def test_transpose_by_index(orc):
+    """Brute force on a small case: every destination byte by its index rule."""
+    g = np.random.default_rng(12)
+    rows, cols, ld = 5, 7, 16
+    src = g.integers(0, 256, (rows, cols), dtype=np.uint8)
+    dst = orc.transpose_u8(src, ld)
+    for c in range(cols):
+        for r in range(ld):
+            assert dst[c, r] == (src[r, c] if r < rows else 0)
+    big = g.integers(0, 256, (130, 333), dtype=np.uint8)
+    np.testing.assert_array_equal(orc.transpose_u8(big), big.T)
+
+
+def test_sum_rows_exact_integers(orc):
+    """Small integers are exact in bf16 and in the sum: the oracle's column
+    sums equal Python's integer sums."""
+    import torch
+    g = np.random.default_rng(13)
+    v = g.integers(-100, 101, (300, 50)).astype(np.float32)
+    bits = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    out = orc.sum_rows(bits, orc.BF16)
+    for c in range(50):
+        assert out[c] == sum(int(t) for t in v[:, c])
+    f = g.standard_normal((64, 9)).astype(np.float32)
+    np.testing.assert_allclose(orc.sum_rows(f, orc.F32), f.astype(np.float64).sum(0), rtol=1e-14, atol=1e-14)
+    assert (orc.sum_rows(np.zeros((0, 4), np.float32), orc.F32) == 0).all()
