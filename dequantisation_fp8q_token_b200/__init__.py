@@ -52,7 +52,7 @@ __all__ = [
     "RECORD_HEADER_BYTES", "record_bytes", "fp8q_record_bytes", "fp8q_pack_record", "fp8q_unpack_records",
     "exchange_records", "exchange_records_all_to_all", "exchange_payload_all_to_all", "all_gather_fp8", "all_to_all_fp8", "all_to_all_single_fp8",
     "fp8q_scaled_mm", "fp8q_scaled_mm_blockwise", "scaled_mm", "scaled_mm_blockwise", "linear_fp8",
-    "linear_fp8_blockwise",
+    "linear_fp8_blockwise", "fp8q_transpose_fp8", "fp8q_sum_rows", "transpose_fp8",
 ]
 
 E4M3FN, E5M2 = 0, 1
@@ -141,6 +141,10 @@ def lib() -> ctypes.CDLL:
             L.fp8q_unpack_records.argtypes = [p, i32, i64, i32, i32, p, p]
             L.fp8q_scaled_mm.restype = st
             L.fp8q_scaled_mm.argtypes = [p, i32, p, i32, i64, i64, i64, p, p, p, i32, p, p, p]
+            L.fp8q_transpose_fp8.restype = st
+            L.fp8q_transpose_fp8.argtypes = [p, i64, i64, p, i64, p]
+            L.fp8q_sum_rows.restype = st
+            L.fp8q_sum_rows.argtypes = [p, i32, i64, i64, p, p]
             L.fp8q_scaled_mm_blockwise.restype = st
             L.fp8q_scaled_mm_blockwise.argtypes = [p, i32, p, p, i32, p, i64, i64, i64, p, i32, p, p, p]
             _lib = L
@@ -804,19 +808,90 @@ def scaled_mm_blockwise(a: torch.Tensor, scale_a: torch.Tensor, w: torch.Tensor,
     return out
 
 
+def fp8q_transpose_fp8(src: torch.Tensor, dst: torch.Tensor, ld: Optional[int] = None, stream=None) -> None:
+    """dst[c, r] = src[r, c] (fp8 codes), zero for rows <= r < ld; dst holds [cols, ld]."""
+    if src.dim() != 2:
+        raise ValueError("src must be 2-D")
+    rows, cols = src.shape
+    ld = rows if ld is None else int(ld)
+    dev = src.device
+    _need(src, rows * cols, "src", byte=True)
+    _need(dst, cols * ld, "dst", byte=True)
+    _check(lib().fp8q_transpose_fp8(_dev_ptr(src, "src", dev), rows, cols, _dev_ptr(dst, "dst", dev), ld,
+                                    _stream(stream, dev)), "fp8q_transpose_fp8")
+
+
+def fp8q_sum_rows(x: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """out[c] = sum over rows of x[r, c] in fp32, in a fixed order, stored in x's dtype."""
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    rows, cols = x.shape
+    dev = x.device
+    _need(out, cols, "out", dtype=x.dtype)
+    _check(lib().fp8q_sum_rows(_dev_ptr(x, "x", dev), _dtype_code(x, "x"), rows, cols, _dev_ptr(out, "out", dev),
+                               _stream(stream, dev)), "fp8q_sum_rows")
+
+
+def transpose_fp8(src: torch.Tensor, pad_to: int = 1) -> torch.Tensor:
+    """The .t().contiguous() of an fp8 matrix, with the new rows zero-padded to a multiple of pad_to."""
+    rows, cols = src.shape
+    ld = -(-rows // pad_to) * pad_to
+    dst = torch.empty((cols, ld), dtype=src.dtype, device=src.device)
+    fp8q_transpose_fp8(src, dst, ld)
+    return dst
+
+
+class _LinearFp8(torch.autograd.Function):
+    """ColossalAI _LinearFp8: forward casts input and weight to e4m3 with one scale each and
+    multiplies them; backward casts the output gradient to e5m2 with one scale and takes the
+    input gradient g @ w and the weight gradient g^T @ x as two more scaled products, over
+    transposed fp8 operands (zero-padded to a row pitch of 16 bytes); the bias gradient is the
+    column sum of g.  All arithmetic runs in libfp8q.  As for torch._scaled_mm, the input's
+    last dimension (forward) and the weight's first (backward) must be multiples of 16."""
+
+    @staticmethod
+    def forward(ctx, x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor]) -> torch.Tensor:
+        if x.dtype not in (torch.bfloat16, torch.float16) or x.dtype != w.dtype:
+            raise TypeError("Only float16 and bfloat16 are allowed.")
+        if bias is not None and bias.dtype != x.dtype:
+            raise TypeError("Bias should have the same dtype as input.")
+        x = x.contiguous()
+        w = w.contiguous()
+        ctx.x_shape = x.shape
+        ctx.has_bias = bias is not None
+        x2 = x.reshape(-1, x.shape[-1])
+        x_fp8, sx = cast_to_fp8(x2, "e4m3")
+        w_fp8, sw = cast_to_fp8(w, "e4m3")
+        ctx.save_for_backward(x_fp8, w_fp8, sx, sw)
+        out = torch.empty((x2.shape[0], w.shape[0]), dtype=x.dtype, device=x.device)
+        fp8q_scaled_mm(x_fp8, w_fp8, sx, sw, out, bias)
+        return out.reshape(*x.shape[:-1], w.shape[0])
+
+    @staticmethod
+    def backward(ctx, out_grad: torch.Tensor):
+        x_fp8, w_fp8, sx, sw = ctx.saved_tensors
+        g = out_grad.contiguous().reshape(-1, out_grad.shape[-1])
+        T, N = g.shape
+        K = w_fp8.shape[1]
+        g_fp8, sg = cast_to_fp8(g, "e5m2")
+        dt = out_grad.dtype
+        # x_grad[T, K] = g[T, N] @ w[N, K]: the weight transposed to [K, N]
+        x_grad = torch.empty((T, K), dtype=dt, device=g.device)
+        fp8q_scaled_mm(g_fp8, transpose_fp8(w_fp8), sg, sw, x_grad)
+        # w_grad[N, K] = g^T[N, T] @ x[T, K]: g and x transposed, T padded to 16
+        w_grad = torch.empty((N, K), dtype=dt, device=g.device)
+        fp8q_scaled_mm(transpose_fp8(g_fp8, 16), transpose_fp8(x_fp8, 16), sg, sx, w_grad)
+        bias_grad = None
+        if ctx.has_bias:
+            bias_grad = torch.empty((N,), dtype=dt, device=g.device)
+            fp8q_sum_rows(g, bias_grad)
+        return x_grad.reshape(ctx.x_shape), w_grad, bias_grad
+
+
 def linear_fp8(input: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """ColossalAI linear_fp8 forward: per-tensor e4m3 casts of input and weight (cast_to_fp8),
-    then the scaled product with the input's dtype as output dtype."""
-    if input.dtype not in (torch.bfloat16, torch.float16) or input.dtype != weight.dtype:
-        raise TypeError("Only float16 and bfloat16 are allowed.")
-    if bias is not None and bias.dtype != input.dtype:
-        raise TypeError("Bias should have the same dtype as input.")
-    x = input.contiguous().reshape(-1, input.shape[-1])
-    x_fp8, sx = cast_to_fp8(x, "e4m3")
-    w_fp8, sw = cast_to_fp8(weight.contiguous(), "e4m3")
-    out = torch.empty((x.shape[0], weight.shape[0]), dtype=input.dtype, device=input.device)
-    fp8q_scaled_mm(x_fp8, w_fp8, sx, sw, out, bias)
-    return out.reshape(*input.shape[:-1], weight.shape[0])
+    """ColossalAI linear_fp8: per-tensor e4m3 casts of input and weight (cast_to_fp8), then the
+    scaled product with the input's dtype as output dtype; differentiable (see _LinearFp8)."""
+    return _LinearFp8.apply(input, weight, bias)
 
 
 def linear_fp8_blockwise(input: torch.Tensor, weight: torch.Tensor, weight_scale_inv: torch.Tensor,

@@ -381,3 +381,28 @@ fp8q_status fp8q_scaled_mm_blockwise(const uint8_t* a, fp8q_format fa, const flo
 }
 
 }  // extern "C"
+
+extern "C" {
+
+fp8q_status fp8q_transpose_fp8(const uint8_t* src, int64_t rows, int64_t cols, uint8_t* dst, int64_t ld,
+                               fp8q_stream_t stream) {
+    if (rows < 0 || cols < 0 || ld < rows) return FP8Q_ERR_BAD_SHAPE;
+    if (checked_mul(rows, cols) < 0 || checked_mul(cols, ld) < 0) return FP8Q_ERR_BAD_SHAPE;
+    if (checked_mul(cols, ld) == 0) return FP8Q_OK;
+    if (!dst || (rows > 0 && !src)) return FP8Q_ERR_NULL_POINTER;
+    return launch_transpose(src, rows, cols, dst, ld, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp8q_status fp8q_sum_rows(const void* x, fp8q_dtype xt, int64_t rows, int64_t cols, void* out,
+                          fp8q_stream_t stream) {
+    if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
+    if (rows < 0 || cols < 0) return FP8Q_ERR_BAD_SHAPE;
+    const int64_t numel = checked_mul(rows, cols);
+    if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
+    if (cols == 0) return FP8Q_OK;
+    if (!out || (rows > 0 && !x)) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(out, dtype_bytes(xt)) || (x && !aligned(x, dtype_bytes(xt)))) return FP8Q_ERR_MISALIGNED;
+    return launch_sum_rows(x, xt, rows, cols, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -87,6 +87,11 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
                              const float* sa, int sa_ld, const float* sb, int sb_ld, bool fine, const void* bias,
                              int yt, void* d, uint32_t* status, cudaStream_t s);
 
+// _LinearFp8.backward's data movements (linear_bwd.cu): validated shapes
+fp8q_status launch_transpose(const uint8_t* src, int64_t rows, int64_t cols, uint8_t* dst, int64_t ld,
+                             cudaStream_t s);
+fp8q_status launch_sum_rows(const void* x, int xt, int64_t rows, int64_t cols, void* out, cudaStream_t s);
+
 inline fp8q_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA; }
 
 }  // namespace fp8q

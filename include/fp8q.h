@@ -13,6 +13,8 @@
  *   fp8q_scaled_mm              ColossalAI _LinearFp8.forward (torch._scaled_mm)
  *   fp8q_scaled_mm_blockwise    DeepEP per-token activations x DeepSeek-V3
  *                               block-scaled weight
+ *   fp8q_transpose_fp8,         ColossalAI _LinearFp8.backward (the operand
+ *   fp8q_sum_rows               transposes and the bias gradient)
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -388,6 +390,33 @@ fp8q_status fp8q_scaled_mm_blockwise(const uint8_t* a, fp8q_format fa, const flo
                                      const uint8_t* b, fp8q_format fb, const float* scale_b,
                                      int64_t M, int64_t N, int64_t K, const void* bias, fp8q_dtype yt,
                                      void* d, uint32_t* status, fp8q_stream_t stream);
+
+/*
+ * Byte transpose of an fp8 matrix -- the .t().contiguous() copies that
+ * ColossalAI _LinearFp8.backward makes of its fp8 operands (the weight for
+ * the input gradient; the gradient and the input for the weight gradient):
+ *   dst[c][r] = src[r][c]   for r < rows, c < cols
+ *   dst[c][r] = 0           for rows <= r < ld  (zero padding of each dst row)
+ * src: [rows][cols] bytes, row-major.  dst: [cols][ld] bytes, ld >= rows.
+ * A pitch ld that is a multiple of 16 makes dst a legal operand of the fp8
+ * products with K = ld (the zero padding adds nothing to the sums).
+ * Errors: ld < rows or a negative size -> FP8Q_ERR_BAD_SHAPE.  rows == 0 or
+ * cols == 0 with ld == 0 writes nothing.
+ */
+fp8q_status fp8q_transpose_fp8(const uint8_t* src, int64_t rows, int64_t cols, uint8_t* dst, int64_t ld,
+                               fp8q_stream_t stream);
+
+/*
+ * Column sums -- the bias gradient of ColossalAI _LinearFp8.backward,
+ * out_grad.sum(0):
+ *   out[c] = T(sum over r of float(x[r][c]))
+ * accumulated in fp32 in a fixed order (each column's rows split into 16
+ * interleaved subsets summed in ascending row order, then the 16 partial
+ * sums added in subset order), so repeated calls give the same bits.
+ * x: [rows][cols] of type xt; out: [cols] of type xt.  rows == 0 writes zeros.
+ */
+fp8q_status fp8q_sum_rows(const void* x, fp8q_dtype xt, int64_t rows, int64_t cols, void* out,
+                          fp8q_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -163,3 +163,20 @@ def test_scaled_mm_blockwise_validation(L):
     assert f(A, 0, P, A, 0, None, 8, 8, 128, None, 2, A, None, None) == 1   # null scale_b
     assert f(A, 0, P + 2, A, 0, P, 8, 8, 128, None, 2, A, None, None) == 5  # scale_a misaligned
     assert f(A, 0, P, A, 0, P, 8, 0, 128, None, 2, None, None, None) == 0   # N == 0: nothing
+
+
+def test_transpose_and_sum_rows_validation(L):
+    f = L.fp8q_transpose_fp8
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+    assert f(P, 8, 4, P, 7, None) == 4          # ld < rows
+    assert f(P, -1, 4, P, 8, None) == 4         # negative size
+    assert f(None, 8, 4, P, 8, None) == 1       # null src
+    assert f(P, 8, 4, None, 8, None) == 1       # null dst
+    assert f(None, 0, 0, None, 0, None) == 0    # nothing to do
+    s = L.fp8q_sum_rows
+    s.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+    assert s(P, 5, 4, 4, P, None) == 2          # dtype
+    assert s(P, 2, -1, 4, P, None) == 4         # negative rows
+    assert s(P, 2, 4, 4, None, None) == 1       # null out
+    assert s(P + 1, 2, 4, 4, P, None) == 5      # bf16 input on an odd address
+    assert s(None, 2, 4, 0, None, None) == 0    # no columns
