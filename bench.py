@@ -324,6 +324,7 @@ class MatmulWorkload:
         self.status = torch.zeros(1, dtype=torch.int32, device=d)
         self.flops = 2.0 * m * self.n * k
         self.shape = (m, self.n, k)
+        self.fp8q = f
         self.ops = {
             "scaled_mm_blockwise": lambda: f.fp8q_scaled_mm_blockwise(self.q, self.sa, self.w, self.sb, self.out,
                                                                       status=self.status),
@@ -359,6 +360,42 @@ class MatmulWorkload:
                 res[name] = {"unavailable": str(ex).splitlines()[0][:200]}
         if int(self.status.item()) != 0:
             raise RuntimeError("a bounded wait of the fp8 product ran out")
+        res.update(self.time_linear(steps, warmup, device))
+        return res
+
+    def time_linear(self, steps: int, warmup: int, device):
+        """ColossalAI linear_fp8 forward + backward on bf16 x[4096, 7168], w[18432, 7168] and a bias
+        (three fp8 products of 2*M*N*K each, the casts, three operand transposes and the bias
+        gradient), and the weight transpose alone (GB/s of its 2 bytes per element)."""
+        f = self.fp8q
+        g = torch.Generator(device=device).manual_seed(20261207)
+        m, k = self.q.shape
+        x = torch.randn((m, k), generator=g, device=device).to(torch.bfloat16).requires_grad_(True)
+        w = (torch.randn((self.n, k), generator=g, device=device) * 0.02).to(torch.bfloat16).requires_grad_(True)
+        b = torch.randn((self.n,), generator=g, device=device).to(torch.bfloat16).requires_grad_(True)
+        go = (torch.randn((m, self.n), generator=g, device=device) * 1e-3).to(torch.bfloat16)
+
+        def step():
+            y = f.linear_fp8(x, w, b)
+            y.backward(go)
+
+        wt = torch.empty((k, self.n), dtype=torch.uint8, device=device)
+        res = {}
+        for name, fn, unit_work, unit in [("linear_fp8 forward+backward", step, 3 * self.flops, "tflops"),
+                                          ("transpose_fp8 (weight)", lambda: f.fp8q_transpose_fp8(self.w, wt, self.n),
+                                           2.0 * self.w.numel(), "gb_s")]:
+            for _ in range(warmup):
+                fn()
+            torch.cuda.synchronize(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize(device)
+            ms = e0.elapsed_time(e1) / steps
+            scale = 1e12 if unit == "tflops" else 1e9
+            res[name] = {"ms": round(ms, 4), unit: round(unit_work / (ms * 1e-3) / scale, 1)}
         return res
 
 
@@ -640,9 +677,12 @@ def run_ours(args):
         mmw = MatmulWorkload(wl)
         mm_res = mmw.time(max(5, min(args.steps, 50)), max(3, args.warmup), device)
         tpeak, tkind = fp8_tensor_peak()
+        hpeak, _ = measured_peaks()
         for v in mm_res.values():
             if "tflops" in v:
                 v["frac"] = round(v["tflops"] / tpeak, 4)
+            if "gb_s" in v:
+                v["frac"] = round(v["gb_s"] / hpeak, 4)
         mm = {"workload": "fp8 products: per-token e4m3fn codes of c2 x[4096,7168] (1x128 scales) times "
                           "e4m3fn W[18432,7168] (128x128 block scales), bf16 out; per-tensor: same codes, "
                           "one scale each",

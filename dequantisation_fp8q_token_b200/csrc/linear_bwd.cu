@@ -18,56 +18,86 @@ namespace fp8q {
 namespace {
 
 // ---------------------------------------------------------------------------
-// transpose: 64 x 64 byte tiles through shared memory
+// transpose: 128 x 128 byte tiles through shared memory
 // ---------------------------------------------------------------------------
-constexpr int kT = 64;                 // tile edge (bytes)
+constexpr int kT = 128;                // tile edge (bytes): full 128-byte lines on both sides
+constexpr int kTW = kT / 4;            // words per tile row
 constexpr int kTThreads = 256;
 
-// One CTA per 64 x 64 tile of the destination [cols][ld] (the padding
-// columns r in [rows, ld) are written as zeros).  Interior tiles move 4-byte
-// words when both pitches and base pointers allow it; edge tiles move bytes.
+// 4 x 4 byte transpose of four words (a[i] = row i, bytes = columns 0..3):
+// returns o[j] = column j, bytes = rows 0..3
+__device__ __forceinline__ void transpose4x4(const uint32_t (&a)[4], uint32_t (&o)[4]) {
+    const uint32_t t0 = __byte_perm(a[0], a[1], 0x5140), t1 = __byte_perm(a[0], a[1], 0x7362);
+    const uint32_t t2 = __byte_perm(a[2], a[3], 0x5140), t3 = __byte_perm(a[2], a[3], 0x7362);
+    o[0] = __byte_perm(t0, t2, 0x5410);
+    o[1] = __byte_perm(t0, t2, 0x7632);
+    o[2] = __byte_perm(t1, t3, 0x5410);
+    o[3] = __byte_perm(t1, t3, 0x7632);
+}
+
+// One CTA per 128 x 128 tile of the destination [cols][ld] (the padding
+// columns r in [rows, ld) are written as zeros).  Interior tiles with 16-byte
+// aligned pitches and bases: threads load 16 bytes of a source row at a
+// time, transpose 4 x 4 byte blocks in registers, and store 16 bytes of a
+// destination row at a time; the tile passes through shared memory as
+// words, the transposed copy with its word index XORed by (row / 4) so that
+// the block writes of a warp fall in 32 different banks.  Other tiles move
+// bytes.
 __global__ void __launch_bounds__(kTThreads)
 transpose_kernel(const uint8_t* __restrict__ src, int64_t rows, int64_t cols, uint8_t* __restrict__ dst,
-                 int64_t ld, int64_t tiles_r, int words_ok) {
-    __shared__ uint8_t tile[kT][kT + 4];
+                 int64_t ld, int64_t tiles_r, int vec_ok) {
+    __shared__ __align__(16) uint32_t ta[kT][kTW];         // source tile, rows x words
+    __shared__ uint32_t tb[kT][kTW];                       // transposed tile, swizzled words
     pdl_begin();
     const int64_t t = blockIdx.x;
     const int64_t tr = t % tiles_r;            // tile index along src rows (= dst columns)
     const int64_t tc = t / tiles_r;            // tile index along src columns (= dst rows)
     const int64_t r0 = tr * kT, c0 = tc * kT;
-    const bool full = words_ok && r0 + kT <= rows && c0 + kT <= cols;
-    if (full) {
-        // load 64 rows x 16 words
-        for (int i = threadIdx.x; i < kT * (kT / 4); i += kTThreads) {
-            const int r = i / (kT / 4), w = i % (kT / 4);
-            const uint32_t v = ld_stream_u32(src + (r0 + r) * cols + c0 + 4 * w);
-            tile[r][4 * w + 0] = static_cast<uint8_t>(v);
-            tile[r][4 * w + 1] = static_cast<uint8_t>(v >> 8);
-            tile[r][4 * w + 2] = static_cast<uint8_t>(v >> 16);
-            tile[r][4 * w + 3] = static_cast<uint8_t>(v >> 24);
+    const int tid = threadIdx.x;
+    if (vec_ok && r0 + kT <= rows && c0 + kT <= cols) {
+#pragma unroll
+        for (int k = 0; k < kT * (kT / 16) / kTThreads; ++k) {       // 128 rows x 8 chunks of 16 bytes
+            const int i = tid + k * kTThreads;
+            const int r = i >> 3, seg = i & 7;
+            const uint4 v = ld_stream_v4(src + (r0 + r) * cols + c0 + 16 * seg);
+            *reinterpret_cast<uint4*>(&ta[r][4 * seg]) = v;
         }
-    } else {
-        for (int i = threadIdx.x; i < kT * kT; i += kTThreads) {
-            const int r = i / kT, c = i % kT;
-            tile[r][c] = (r0 + r < rows && c0 + c < cols) ? src[(r0 + r) * cols + c0 + c] : 0;
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < (kT / 4) * (kT / 4) / kTThreads; ++k) {  // 32 x 32 blocks of 4 x 4 bytes
+            const int i = tid + k * kTThreads;
+            const int br = i >> 5, bc = i & 31;
+            uint32_t a[4], o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a[q] = ta[4 * br + q][bc];
+            transpose4x4(a, o);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tb[4 * bc + j][br ^ bc] = o[j];     // row 4 bc + j: swizzle (row / 4) = bc
         }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kT * (kT / 16) / kTThreads; ++k) {       // 128 dst rows x 8 chunks of 16 bytes
+            const int i = tid + k * kTThreads;
+            const int d = i >> 3, seg = i & 7;
+            const int sw = (d >> 2) & (kTW - 1);
+            uint4 v;
+            v.x = tb[d][(4 * seg + 0) ^ sw];
+            v.y = tb[d][(4 * seg + 1) ^ sw];
+            v.z = tb[d][(4 * seg + 2) ^ sw];
+            v.w = tb[d][(4 * seg + 3) ^ sw];
+            st_v4(dst + (c0 + d) * ld + r0 + 16 * seg, v);
+        }
+        return;
+    }
+    uint8_t* tile = reinterpret_cast<uint8_t*>(ta);          // bytes [kT][kT]
+    for (int i = tid; i < kT * kT; i += kTThreads) {
+        const int r = i / kT, c = i % kT;
+        tile[r * kT + c] = (r0 + r < rows && c0 + c < cols) ? src[(r0 + r) * cols + c0 + c] : 0;
     }
     __syncthreads();
-    // dst row c0 + c holds src column c0 + c; its bytes r0 .. r0 + 63 come
-    // from tile rows 0 .. 63 (zeros beyond `rows` pad the row up to ld)
-    if (full && r0 + kT <= ld) {
-        for (int i = threadIdx.x; i < kT * (kT / 4); i += kTThreads) {
-            const int c = i / (kT / 4), w = i % (kT / 4);
-            const uint32_t v = static_cast<uint32_t>(tile[4 * w + 0][c]) | (static_cast<uint32_t>(tile[4 * w + 1][c]) << 8)
-                             | (static_cast<uint32_t>(tile[4 * w + 2][c]) << 16)
-                             | (static_cast<uint32_t>(tile[4 * w + 3][c]) << 24);
-            st_u32(dst + (c0 + c) * ld + r0 + 4 * w, v);
-        }
-    } else {
-        for (int i = threadIdx.x; i < kT * kT; i += kTThreads) {
-            const int c = i / kT, r = i % kT;
-            if (c0 + c < cols && r0 + r < ld) dst[(c0 + c) * ld + r0 + r] = tile[r][c];
-        }
+    for (int i = tid; i < kT * kT; i += kTThreads) {
+        const int c = i / kT, r = i % kT;
+        if (c0 + c < cols && r0 + r < ld) dst[(c0 + c) * ld + r0 + r] = tile[r * kT + c];
     }
 }
 
@@ -121,10 +151,10 @@ fp8q_status launch_transpose(const uint8_t* src, int64_t rows, int64_t cols, uin
     const int64_t tiles_c = (cols + kT - 1) / kT;
     const int64_t tiles = tiles_r * tiles_c;
     if (tiles > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
-    const int words_ok = (cols % 4 == 0) && (ld % 4 == 0) && (reinterpret_cast<uintptr_t>(src) % 4 == 0) &&
-                         (reinterpret_cast<uintptr_t>(dst) % 4 == 0);
+    const int vec_ok = (cols % 16 == 0) && (ld % 16 == 0) && (reinterpret_cast<uintptr_t>(src) % 16 == 0) &&
+                       (reinterpret_cast<uintptr_t>(dst) % 16 == 0);
     return cuda_status(launch_kernel(transpose_kernel, dim3(static_cast<unsigned>(tiles)), dim3(kTThreads), s, src,
-                                     rows, cols, dst, ld, tiles_r, words_ok));
+                                     rows, cols, dst, ld, tiles_r, vec_ok));
 }
 
 fp8q_status launch_sum_rows(const void* x, int xt, int64_t rows, int64_t cols, void* out, cudaStream_t s) {
