@@ -54,15 +54,18 @@ constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kABytes = BM * BK;
 constexpr int kGroupM = 32;     // row-tiles per raster band
 
-// Tile shape per product: 128 x 256 tiles, two TMEM accumulators (with
+// Tile shapes.  BN = 256: 128 x 256 tiles, two TMEM accumulators (with
 // per-tensor scales one tile's epilogue overlaps the next tile's k-loop; with
 // fine-grained scales one k-block's fold overlaps the next block's MMAs), a
-// 4-stage ring.  Measured on B200: 128 x 128 tiles with four accumulators and
-// six stages lose a quarter of the fine-grained product's throughput, since
-// the narrower MMA reads twice the operand bytes per flop.
-template <bool FINE> struct Shape {
-    static constexpr int BN = 256;                          // rows of B (columns of D) per tile
-    static constexpr int kStages = 4;
+// 4-stage ring: the shape for products with enough tiles to fill the GPU.
+// BN = 128: 128 x 128 tiles, four accumulators, a 6-stage ring, for products
+// of at most 128 rows (decode-sized activations), where 256-wide tiles would
+// leave SMs without a share of the weight to stream.  Measured on B200 for
+// large products: 128 x 128 tiles lose a quarter of the fine-grained
+// throughput, since the narrower MMA reads twice the operand bytes per flop.
+template <int BN_> struct Shape {
+    static constexpr int BN = BN_;                          // rows of B (columns of D) per tile
+    static constexpr int kStages = BN_ == 256 ? 4 : 6;
     static constexpr int kAccBufs = kTmemCols / BN;
     static constexpr int kColsPerWarp = BN / (kEpiWarps / 4);   // tile columns one epilogue warp owns
     static constexpr int kBBytes = BN * BK;
@@ -84,6 +87,7 @@ struct Params {
     const void* bias;           // [N] of the output type, or null
     void* d;                    // [M][N]
     int vec_store;              // D rows 32-byte aligned (base and row pitch)
+    int stage_tx;               // bytes one stage's two TMA boxes bring
     uint32_t* status;           // optional status word
 };
 
@@ -292,16 +296,16 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int YT, bool FINE>
+template <int YT, bool FINE, int BN_>
 __global__ void __launch_bounds__(kThreads, 1)
 scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const Params p, const uint32_t idesc) {
-    constexpr int BN = Shape<FINE>::BN;
-    constexpr int kStages = Shape<FINE>::kStages;
-    constexpr int kAccBufs = Shape<FINE>::kAccBufs;
-    constexpr int kColsPerWarp = Shape<FINE>::kColsPerWarp;
-    constexpr int kBBytes = Shape<FINE>::kBBytes;
-    constexpr int kStageBytes = Shape<FINE>::kStageBytes;
+    constexpr int BN = Shape<BN_>::BN;
+    constexpr int kStages = Shape<BN_>::kStages;
+    constexpr int kAccBufs = Shape<BN_>::kAccBufs;
+    constexpr int kColsPerWarp = Shape<BN_>::kColsPerWarp;
+    constexpr int kBBytes = Shape<BN_>::kBBytes;
+    constexpr int kStageBytes = Shape<BN_>::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -359,7 +363,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 for (int kb = 0; kb < p.num_kb; ++kb) {
                     if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort)) { fail = kTimeoutProducer; break; }
                     const uint32_t fb = full0 + 8 * stage;
-                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    mbar_arrive_expect_tx(fb, static_cast<uint32_t>(p.stage_tx));
                     tma_load_2d(smem_u32(sA + stage * kABytes), &map_a, kb * BK, mb * BM, fb);
                     tma_load_2d(smem_u32(sB + stage * kBBytes), &map_b, kb * BK, nb * BN, fb);
                     ++issued;
@@ -580,11 +584,11 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int b
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int YT, bool FINE>
+template <int YT, bool FINE, int BN_>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, uint32_t idesc,
                          cudaStream_t s) {
-    auto kernel = scaled_mm_kernel<YT, FINE>;
-    constexpr int kSmemBytes = Shape<FINE>::kSmemBytes;
+    auto kernel = scaled_mm_kernel<YT, FINE, BN_>;
+    constexpr int kSmemBytes = Shape<BN_>::kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const int tiles = p.tiles_m * p.tiles_n;
@@ -601,18 +605,38 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const Par
     return cudaLaunchKernelEx(&cfg, kernel, ma, mb, p, idesc);
 }
 
+template <int BN_>
+cudaError_t launch_dtype(bool fine, int yt, const CUtensorMap& ma, const CUtensorMap& mb, const Params& p,
+                         uint32_t idesc, cudaStream_t s) {
+    if (fine) {
+        return yt == kF32 ? launch_typed<kF32, true, BN_>(ma, mb, p, idesc, s)
+             : yt == kF16 ? launch_typed<kF16, true, BN_>(ma, mb, p, idesc, s)
+                          : launch_typed<kBF16, true, BN_>(ma, mb, p, idesc, s);
+    }
+    return yt == kF32 ? launch_typed<kF32, false, BN_>(ma, mb, p, idesc, s)
+         : yt == kF16 ? launch_typed<kF16, false, BN_>(ma, mb, p, idesc, s)
+                      : launch_typed<kBF16, false, BN_>(ma, mb, p, idesc, s);
+}
+
 }  // namespace mm
 
 fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
                              const float* sa, int sa_ld, const float* sb, int sb_ld, bool fine, const void* bias,
                              int yt, void* d, uint32_t* status, cudaStream_t s) {
     using namespace mm;
-    const int bn = fine ? Shape<true>::BN : Shape<false>::BN;
+    // 128-wide tiles when a product of at most 128 rows would leave SMs idle
+    const bool narrow = M <= BM && (N + 255) / 256 < sm_count();
+    const int bn = narrow ? 128 : 256;
+    // A product of fewer than 128 rows loads only its rows, rounded up to 16:
+    // the MMA still multiplies 128 rows, and the rows past the box hold stale
+    // shared memory, but output row m depends on row m of A alone and rows
+    // at or past M are never stored.
+    const int a_rows = M >= BM ? BM : static_cast<int>((M + 15) / 16 * 16);
     CUtensorMap ma, mbm;
     memset(&ma, 0, sizeof(ma));
     memset(&mbm, 0, sizeof(mbm));
     if (K > 0) {
-        if (!make_map(&ma, a, M, K, BM) || !make_map(&mbm, b, N, K, bn)) return FP8Q_ERR_CUDA;
+        if (!make_map(&ma, a, M, K, a_rows) || !make_map(&mbm, b, N, K, bn)) return FP8Q_ERR_CUDA;
     }
     Params p;
     p.M = static_cast<int>(M);
@@ -630,17 +654,11 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     const int eb = yt == kF32 ? 4 : 2;
     p.vec_store = (reinterpret_cast<uintptr_t>(d) % 32 == 0) && ((N * eb) % 32 == 0);
     p.status = status;
+    p.stage_tx = (a_rows + bn) * BK;
     const uint32_t idesc = instr_desc(fa, fb, bn);
     cudaError_t e;
-    if (fine) {
-        e = yt == kF32 ? launch_typed<kF32, true>(ma, mbm, p, idesc, s)
-          : yt == kF16 ? launch_typed<kF16, true>(ma, mbm, p, idesc, s)
-                       : launch_typed<kBF16, true>(ma, mbm, p, idesc, s);
-    } else {
-        e = yt == kF32 ? launch_typed<kF32, false>(ma, mbm, p, idesc, s)
-          : yt == kF16 ? launch_typed<kF16, false>(ma, mbm, p, idesc, s)
-                       : launch_typed<kBF16, false>(ma, mbm, p, idesc, s);
-    }
+    if (narrow) e = launch_dtype<128>(fine, yt, ma, mbm, p, idesc, s);
+    else e = launch_dtype<256>(fine, yt, ma, mbm, p, idesc, s);
     return cuda_status(e);
 }
 

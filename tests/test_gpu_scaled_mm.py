@@ -309,3 +309,17 @@ def test_linear_fp8_blockwise_matches_the_oracle_composition(fp8q, orc):
     mag = (np.abs(tdec(qx, E4M3FN)) * np.repeat(sx, 128, 1)) @ \
         (np.abs(tdec(w, E4M3FN)) * np.repeat(np.repeat(sw, 128, 0), 128, 1)[:Nd]).T
     check_bound(to_f64(host(y), BF16), exact, mag, Kd, BF16, True)
+
+
+@pytest.mark.parametrize("fine", [False, True], ids=["tensor", "blockwise"])
+@pytest.mark.parametrize("M,N,K", [(64, 3000, 512),       # decode-sized rows: 24 tiles 128 columns wide
+                                   (1, 18432, 256),       # one token against a full weight row count
+                                   (100, 40000, 128)])    # enough columns to keep 256-wide tiles
+def test_exact_grid_small_m(fp8q, orc, fine, M, N, K):
+    g = np.random.default_rng(M + N + K + fine)
+    a, b = grid_codes(g, (M, K), E4M3FN), grid_codes(g, (N, K), E5M2)
+    sa, sb = scales(g, M, N, K) if fine else (0.25, 0.75)
+    bias_t, bias = t_bias(g, N, BF16)
+    got = host(run(fp8q, fine, a, E4M3FN, b, E5M2, sa, sb, bias_t, BF16))
+    want = oracle_rounded(orc, fine, a, E4M3FN, b, E5M2, sa, sb, bias, BF16)
+    np.testing.assert_array_equal(got, want)
