@@ -332,41 +332,81 @@ class MatmulWorkload:
                                                              status=self.status),
         }
 
+    @staticmethod
+    def _timed(fn, steps: int, warmup: int, device, min_ms: float = 20.0):
+        """ms per call of fn (CUDA events around at least `steps` back-to-back calls, and enough
+        calls to span `min_ms`, after `warmup`), with the SM clocks sampled while it runs."""
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize(device)
+        steps = max(steps, int(min_ms / max(e0.elapsed_time(e1), 1e-3)) + 1)
+        with ClockSampler(device.index or 0) as clk:
+            e0.record()
+            for _ in range(steps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / steps, clk.summary()
+
     def time(self, steps: int, warmup: int, device):
-        """ms per launch of each op (CUDA events around `steps` back-to-back launches
-        after `warmup`), plus torch._scaled_mm (cuBLASLt) on the same operands."""
-        res = {}
+        """Every entry of the section, memory-bound ones first (a long run of tensor-core work
+        leaves the SM clocks lowered by the power cap for a while)."""
+        res = self.time_decode(steps, warmup, device)
+        res.update(self.time_products(steps, warmup, device))
+        res.update(self.time_linear(steps, warmup, device))
+        if int(self.status.item()) != 0:
+            raise RuntimeError("a bounded wait of the fp8 product ran out")
+        return res
+
+    def time_products(self, steps: int, warmup: int, device):
+        """The two products on the full workload, and torch._scaled_mm (cuBLASLt) on the same
+        operands for context."""
         ops = dict(self.ops)
         a8 = self.q.view(torch.float8_e4m3fn)
         b8 = self.w.view(torch.float8_e4m3fn)
         ops["torch_scaled_mm (cuBLASLt)"] = lambda: torch._scaled_mm(a8, b8.t(), scale_a=self.s1, scale_b=self.s2,
                                                                     out_dtype=torch.bfloat16)
+        res = {}
         for name, fn in ops.items():
             try:
-                for _ in range(warmup):
-                    fn()
-                torch.cuda.synchronize(device)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                with ClockSampler(device.index or 0) as clk:
-                    e0.record()
-                    for _ in range(steps):
-                        fn()
-                    e1.record()
-                    torch.cuda.synchronize(device)
-                ms = e0.elapsed_time(e1) / steps
-                res[name] = {"ms": round(ms, 4), "tflops": round(self.flops / (ms * 1e-3) / 1e12, 1),
-                             "clocks": clk.summary()}
+                ms, clk = self._timed(fn, steps, warmup, device)
+                res[name] = {"ms": round(ms, 4), "tflops": round(self.flops / (ms * 1e-3) / 1e12, 1), "clocks": clk}
             except Exception as ex:      # the library baseline may be missing on some builds of torch
                 res[name] = {"unavailable": str(ex).splitlines()[0][:200]}
-        if int(self.status.item()) != 0:
-            raise RuntimeError("a bounded wait of the fp8 product ran out")
-        res.update(self.time_linear(steps, warmup, device))
+        return res
+
+    def time_decode(self, steps: int, warmup: int, device):
+        """The two products at decode-sized activations (M = 1 and 64 rows of the same per-token
+        codes) against the same weight: weight streaming, so GB/s of N*K + M*K + 2*M*N bytes;
+        and the weight transpose of the backward (GB/s of its 2 bytes per element)."""
+        f = self.fp8q
+        res = {}
+        for m in (1, 64):
+            q, sa = self.q[:m], self.sa[:m]
+            out = torch.empty((m, self.n), dtype=torch.bfloat16, device=device)
+            nbytes = self.w.numel() + q.numel() + 2 * out.numel()
+            for name, fn in [(f"scaled_mm_blockwise M={m}",
+                              lambda: f.fp8q_scaled_mm_blockwise(q, sa, self.w, self.sb, out, status=self.status)),
+                             (f"scaled_mm_per_tensor M={m}",
+                              lambda: f.fp8q_scaled_mm(q, self.w, self.s1, self.s2, out, status=self.status))]:
+                ms, clk = self._timed(fn, steps, warmup, device)
+                res[name] = {"ms": round(ms, 4), "gb_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "clocks": clk}
+        k = self.q.shape[1]
+        wt = torch.empty((k, self.n), dtype=torch.uint8, device=device)
+        ms, clk = self._timed(lambda: f.fp8q_transpose_fp8(self.w, wt, self.n), steps, warmup, device)
+        res["transpose_fp8 (weight)"] = {"ms": round(ms, 4), "gb_s": round(2.0 * self.w.numel() / (ms * 1e-3) / 1e9, 1),
+                                         "clocks": clk}
         return res
 
     def time_linear(self, steps: int, warmup: int, device):
         """ColossalAI linear_fp8 forward + backward on bf16 x[4096, 7168], w[18432, 7168] and a bias
         (three fp8 products of 2*M*N*K each, the casts, three operand transposes and the bias
-        gradient), and the weight transpose alone (GB/s of its 2 bytes per element)."""
+        gradient)."""
         f = self.fp8q
         g = torch.Generator(device=device).manual_seed(20261207)
         m, k = self.q.shape
@@ -378,25 +418,9 @@ class MatmulWorkload:
         def step():
             y = f.linear_fp8(x, w, b)
             y.backward(go)
-
-        wt = torch.empty((k, self.n), dtype=torch.uint8, device=device)
-        res = {}
-        for name, fn, unit_work, unit in [("linear_fp8 forward+backward", step, 3 * self.flops, "tflops"),
-                                          ("transpose_fp8 (weight)", lambda: f.fp8q_transpose_fp8(self.w, wt, self.n),
-                                           2.0 * self.w.numel(), "gb_s")]:
-            for _ in range(warmup):
-                fn()
-            torch.cuda.synchronize(device)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(steps):
-                fn()
-            e1.record()
-            torch.cuda.synchronize(device)
-            ms = e0.elapsed_time(e1) / steps
-            scale = 1e12 if unit == "tflops" else 1e9
-            res[name] = {"ms": round(ms, 4), unit: round(unit_work / (ms * 1e-3) / scale, 1)}
-        return res
+        ms, clk = self._timed(step, steps, warmup, device)
+        return {"linear_fp8 forward+backward": {"ms": round(ms, 4), "tflops": round(3 * self.flops / (ms * 1e-3) / 1e12, 1),
+                                                "clocks": clk}}
 
 
 def fp8_tensor_peak():
