@@ -844,7 +844,7 @@ def _profile_case(name, fp8q, device):
         s = torch.empty((1,), dtype=torch.float32, device=device)
         ws = torch.empty(fp8q.fp8q_cast_per_tensor_workspace_bytes(), dtype=torch.uint8, device=device)
         return (lambda: fp8q.fp8q_cast_per_tensor(x, q, s, ws, E5M2)), x.numel() * 9 + 4
-    if name in ("scaled_mm", "scaled_mm_blockwise"):
+    if name in ("scaled_mm", "scaled_mm_blockwise", "scaled_mm_blockwise_m1", "transpose_weight"):
         m, k = workloads.C2_SHAPE
         x = _to_dev(workloads.c2_x(), device, bf16)
         q = torch.empty((m, k), dtype=torch.uint8, device=device)
@@ -857,6 +857,13 @@ def _profile_case(name, fp8q, device):
         flops = 2.0 * m * w.shape[0] * k
         if name == "scaled_mm":
             return (lambda: fp8q.fp8q_scaled_mm(q, w, s1, s1, out)), flops
+        if name == "scaled_mm_blockwise_m1":
+            # one token: weight streaming, bytes moved (N*K + K + 2*N)
+            o1 = out[:1]
+            return (lambda: fp8q.fp8q_scaled_mm_blockwise(q[:1], sa[:1], w, sb, o1)), w.numel() + k + 2 * w.shape[0]
+        if name == "transpose_weight":
+            wt = torch.empty((k, w.shape[0]), dtype=torch.uint8, device=device)
+            return (lambda: fp8q.fp8q_transpose_fp8(w, wt, w.shape[0])), 2 * w.numel()
         return (lambda: fp8q.fp8q_scaled_mm_blockwise(q, sa, w, sb, out)), flops
     if name in ("records_pack", "records_unpack"):
         # the fp8 all-gather's device work for 8 ranks of 16 Mi bf16 each
@@ -881,7 +888,8 @@ def _profile_case(name, fp8q, device):
 
 
 PROFILE_CASES = ["per_token_4x", "cast_from_fp8_4x", "block_dequant", "grouped_16", "grouped_72", "per_channel",
-                 "per_tensor", "records_pack", "records_unpack", "scaled_mm", "scaled_mm_blockwise"]
+                 "per_tensor", "records_pack", "records_unpack", "scaled_mm", "scaled_mm_blockwise",
+                 "scaled_mm_blockwise_m1", "transpose_weight"]
 
 
 def run_profile_case(name, iters):
@@ -899,7 +907,7 @@ def run_profile_case(name, iters):
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / max(iters, 1)
-    if name.startswith("scaled_mm"):
+    if name in ("scaled_mm", "scaled_mm_blockwise"):
         print(f"profile case {name}: {iters} calls, {us:.2f} us per call, "
               f"{nbytes / (us * 1e-6) / 1e12 if iters else 0.0:.1f} TFLOP/s")
         return
