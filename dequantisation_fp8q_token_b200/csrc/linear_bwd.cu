@@ -35,19 +35,27 @@ __device__ __forceinline__ void transpose4x4(const uint32_t (&a)[4], uint32_t (&
     o[3] = __byte_perm(t1, t3, 0x7632);
 }
 
+// Shared-memory layouts of the two 128 x 128-byte tiles, as 32 words per row
+// in 8 chunks of 16 bytes.  Both permute whole chunks within a row, so rows
+// move in and out with 16-byte accesses:
+//   source tile:      chunk c of row r sits at chunk c ^ 2 * ((r / 4) % 4)
+//   transposed tile:  chunk c of row d sits at chunk c ^ (d / 4) % 8
+// With the block mapping of the transpose step (lane = 4 * (bc % 8) +
+// br % 4), each warp's four 4-byte reads of a block column and its four
+// 4-byte writes of the transposed words each touch 32 different banks.
+__device__ __forceinline__ int ta_word(int r, int w) { return 4 * ((w >> 2) ^ (2 * ((r >> 2) & 3))) + (w & 3); }
+__device__ __forceinline__ int tb_word(int d, int w) { return 4 * ((w >> 2) ^ ((d >> 2) & 7)) + (w & 3); }
+
 // One CTA per 128 x 128 tile of the destination [cols][ld] (the padding
 // columns r in [rows, ld) are written as zeros).  Interior tiles with 16-byte
-// aligned pitches and bases: threads load 16 bytes of a source row at a
-// time, transpose 4 x 4 byte blocks in registers, and store 16 bytes of a
-// destination row at a time; the tile passes through shared memory as
-// words, the transposed copy with its word index XORed by (row / 4) so that
-// the block writes of a warp fall in 32 different banks.  Other tiles move
-// bytes.
+// aligned pitches and bases: rows of the source tile come in with 16-byte
+// loads, 4 x 4 byte blocks are transposed in registers, and rows of the
+// destination tile go out with 16-byte stores.  Other tiles move bytes.
 __global__ void __launch_bounds__(kTThreads)
 transpose_kernel(const uint8_t* __restrict__ src, int64_t rows, int64_t cols, uint8_t* __restrict__ dst,
                  int64_t ld, int64_t tiles_r, int vec_ok) {
-    __shared__ __align__(16) uint32_t ta[kT][kTW];         // source tile, rows x words
-    __shared__ uint32_t tb[kT][kTW];                       // transposed tile, swizzled words
+    __shared__ __align__(16) uint32_t ta[kT][kTW];         // source tile, swizzled chunks
+    __shared__ __align__(16) uint32_t tb[kT][kTW];         // transposed tile, swizzled chunks
     pdl_begin();
     const int64_t t = blockIdx.x;
     const int64_t tr = t % tiles_r;            // tile index along src rows (= dst columns)
@@ -60,31 +68,28 @@ transpose_kernel(const uint8_t* __restrict__ src, int64_t rows, int64_t cols, ui
             const int i = tid + k * kTThreads;
             const int r = i >> 3, seg = i & 7;
             const uint4 v = ld_stream_v4(src + (r0 + r) * cols + c0 + 16 * seg);
-            *reinterpret_cast<uint4*>(&ta[r][4 * seg]) = v;
+            *reinterpret_cast<uint4*>(&ta[r][ta_word(r, 4 * seg)]) = v;
         }
         __syncthreads();
 #pragma unroll
         for (int k = 0; k < (kT / 4) * (kT / 4) / kTThreads; ++k) {  // 32 x 32 blocks of 4 x 4 bytes
             const int i = tid + k * kTThreads;
-            const int br = i >> 5, bc = i & 31;
+            const int lane = i & 31, wid = i >> 5;
+            const int br = 4 * (wid & 7) + (lane & 3);               // block row: source rows 4 br ..
+            const int bc = 8 * (wid >> 3) + (lane >> 2);             // block column: source columns 4 bc ..
             uint32_t a[4], o[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) a[q] = ta[4 * br + q][bc];
+            for (int q = 0; q < 4; ++q) a[q] = ta[4 * br + q][ta_word(4 * br + q, bc)];
             transpose4x4(a, o);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tb[4 * bc + j][br ^ bc] = o[j];     // row 4 bc + j: swizzle (row / 4) = bc
+            for (int j = 0; j < 4; ++j) tb[4 * bc + j][tb_word(4 * bc + j, br)] = o[j];
         }
         __syncthreads();
 #pragma unroll
         for (int k = 0; k < kT * (kT / 16) / kTThreads; ++k) {       // 128 dst rows x 8 chunks of 16 bytes
             const int i = tid + k * kTThreads;
             const int d = i >> 3, seg = i & 7;
-            const int sw = (d >> 2) & (kTW - 1);
-            uint4 v;
-            v.x = tb[d][(4 * seg + 0) ^ sw];
-            v.y = tb[d][(4 * seg + 1) ^ sw];
-            v.z = tb[d][(4 * seg + 2) ^ sw];
-            v.w = tb[d][(4 * seg + 3) ^ sw];
+            const uint4 v = *reinterpret_cast<const uint4*>(&tb[d][tb_word(d, 4 * seg)]);
             st_v4(dst + (c0 + d) * ld + r0 + 16 * seg, v);
         }
         return;
