@@ -750,6 +750,12 @@ def _mm_operands(a: torch.Tensor, b: torch.Tensor, out: torch.Tensor, bias, fa, 
     return M, N, K, fa, fb
 
 
+def _status_word(status: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    if status is not None and (status.dtype not in (torch.int32, torch.uint32) or status.numel() < 1):
+        raise TypeError("status must be a CUDA int32 or uint32 tensor of at least one element")
+    return status
+
+
 def fp8q_scaled_mm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
                    out: torch.Tensor, bias: Optional[torch.Tensor] = None, fa=None, fb=None,
                    status: Optional[torch.Tensor] = None, stream=None) -> None:
@@ -765,7 +771,7 @@ def fp8q_scaled_mm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scal
     _check(lib().fp8q_scaled_mm(
         _dev_ptr(a, "a", dev), fa, _dev_ptr(b, "b", dev), fb, M, N, K,
         _dev_ptr(scale_a, "scale_a", dev), _dev_ptr(scale_b, "scale_b", dev), _dev_ptr(bias, "bias", dev),
-        _dtype_code(out, "out"), _dev_ptr(out, "out", dev), _dev_ptr(status, "status", dev),
+        _dtype_code(out, "out"), _dev_ptr(out, "out", dev), _dev_ptr(_status_word(status), "status", dev),
         _stream(stream, dev)), "fp8q_scaled_mm")
 
 
@@ -783,7 +789,7 @@ def fp8q_scaled_mm_blockwise(a: torch.Tensor, scale_a: torch.Tensor, b: torch.Te
     _check(lib().fp8q_scaled_mm_blockwise(
         _dev_ptr(a, "a", dev), fa, _dev_ptr(scale_a, "scale_a", dev), _dev_ptr(b, "b", dev), fb,
         _dev_ptr(scale_b, "scale_b", dev), M, N, K, _dev_ptr(bias, "bias", dev), _dtype_code(out, "out"),
-        _dev_ptr(out, "out", dev), _dev_ptr(status, "status", dev), _stream(stream, dev)),
+        _dev_ptr(out, "out", dev), _dev_ptr(_status_word(status), "status", dev), _stream(stream, dev)),
         "fp8q_scaled_mm_blockwise")
 
 

@@ -29,8 +29,8 @@
 //               double-buffered in 16-column chunks), while the tensor
 //               cores fill the other accumulators.
 // Tiles are 128 x BN of D (see Shape), visited in bands of 32 row-tiles so
-// that the
-// CTAs working at one time share A and B tiles in L2.
+// that the CTAs working at one time share A and B tiles in L2.  A product of
+// fewer than 128 rows loads only its rows of A (rounded up to 16).
 //
 // Every wait on an mbarrier is bounded (a few seconds of global time).  A
 // wait that runs out sets a flag in shared memory that ends the other roles'
@@ -305,7 +305,6 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     constexpr int kAccBufs = Shape<BN_>::kAccBufs;
     constexpr int kColsPerWarp = Shape<BN_>::kColsPerWarp;
     constexpr int kBBytes = Shape<BN_>::kBBytes;
-    constexpr int kStageBytes = Shape<BN_>::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
