@@ -52,13 +52,15 @@ __all__ = [
     "RECORD_HEADER_BYTES", "record_bytes", "fp8q_record_bytes", "fp8q_pack_record", "fp8q_unpack_records",
     "exchange_records", "exchange_records_all_to_all", "exchange_payload_all_to_all", "all_gather_fp8", "all_to_all_fp8", "all_to_all_single_fp8",
     "fp8q_scaled_mm", "fp8q_scaled_mm_blockwise", "scaled_mm", "scaled_mm_blockwise", "linear_fp8",
-    "linear_fp8_blockwise", "fp8q_transpose_fp8", "fp8q_sum_rows", "transpose_fp8",
+    "linear_fp8_blockwise", "fp8q_transpose_fp8", "fp8q_sum_rows", "transpose_fp8", "fp8q_scaled_mm_ex",
+    "K_MAJOR", "MN_MAJOR",
 ]
 
 E4M3FN, E5M2 = 0, 1
 F32, F16, BF16 = 0, 1, 2
 GRAN_TENSOR, GRAN_ROW, GRAN_GROUP, GRAN_BLOCK = 0, 1, 2, 3
 SCALE_IEEE, SCALE_TORCH = 0, 1
+K_MAJOR, MN_MAJOR = 0, 1
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libfp8q.so")
@@ -141,6 +143,8 @@ def lib() -> ctypes.CDLL:
             L.fp8q_unpack_records.argtypes = [p, i32, i64, i32, i32, p, p]
             L.fp8q_scaled_mm.restype = st
             L.fp8q_scaled_mm.argtypes = [p, i32, p, i32, i64, i64, i64, p, p, p, i32, p, p, p]
+            L.fp8q_scaled_mm_ex.restype = st
+            L.fp8q_scaled_mm_ex.argtypes = [p, i32, i32, p, i32, i32, i64, i64, i64, p, p, p, i32, p, p, p]
             L.fp8q_transpose_fp8.restype = st
             L.fp8q_transpose_fp8.argtypes = [p, i64, i64, p, i64, p]
             L.fp8q_sum_rows.restype = st
@@ -814,6 +818,35 @@ def scaled_mm_blockwise(a: torch.Tensor, scale_a: torch.Tensor, w: torch.Tensor,
     return out
 
 
+def fp8q_scaled_mm_ex(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
+                      out: torch.Tensor, bias: Optional[torch.Tensor] = None, a_layout: int = K_MAJOR,
+                      b_layout: int = K_MAJOR, fa=None, fb=None, status: Optional[torch.Tensor] = None,
+                      stream=None) -> None:
+    """fp8q_scaled_mm with an operand layout each: A is stored [M, K] (K_MAJOR) or [K, M]
+    (MN_MAJOR), B is stored [N, K] (K_MAJOR) or [K, N] (MN_MAJOR); out is [M, N]."""
+    if a.dim() != 2 or b.dim() != 2:
+        raise ValueError("a and b must be 2-D")
+    M, K = (a.shape[1], a.shape[0]) if a_layout == MN_MAJOR else tuple(a.shape)
+    N, K2 = (b.shape[1], b.shape[0]) if b_layout == MN_MAJOR else tuple(b.shape)
+    if K != K2:
+        raise ValueError(f"a has K = {K} but b has K = {K2}")
+    _need(a, M * K, "a", byte=True)
+    _need(b, N * K, "b", byte=True)
+    _need(out, M * N, "out")
+    if bias is not None:
+        _need(bias, N, "bias", dtype=out.dtype)
+    _need(scale_a, 1, "scale_a", dtype=torch.float32)
+    _need(scale_b, 1, "scale_b", dtype=torch.float32)
+    fa = _fmt_of(fa) if fa is not None else _FP8_DTYPES.get(a.dtype, E4M3FN)
+    fb = _fmt_of(fb) if fb is not None else _FP8_DTYPES.get(b.dtype, E4M3FN)
+    dev = a.device
+    _check(lib().fp8q_scaled_mm_ex(
+        _dev_ptr(a, "a", dev), fa, int(a_layout), _dev_ptr(b, "b", dev), fb, int(b_layout), M, N, K,
+        _dev_ptr(scale_a, "scale_a", dev), _dev_ptr(scale_b, "scale_b", dev), _dev_ptr(bias, "bias", dev),
+        _dtype_code(out, "out"), _dev_ptr(out, "out", dev), _dev_ptr(_status_word(status), "status", dev),
+        _stream(stream, dev)), "fp8q_scaled_mm_ex")
+
+
 def fp8q_transpose_fp8(src: torch.Tensor, dst: torch.Tensor, ld: Optional[int] = None, stream=None) -> None:
     """dst[c, r] = src[r, c] (fp8 codes), zero for rows <= r < ld; dst holds [cols, ld]."""
     if src.dim() != 2:
@@ -850,10 +883,10 @@ def transpose_fp8(src: torch.Tensor, pad_to: int = 1) -> torch.Tensor:
 class _LinearFp8(torch.autograd.Function):
     """ColossalAI _LinearFp8: forward casts input and weight to e4m3 with one scale each and
     multiplies them; backward casts the output gradient to e5m2 with one scale and takes the
-    input gradient g @ w and the weight gradient g^T @ x as two more scaled products, over
-    transposed fp8 operands (zero-padded to a row pitch of 16 bytes); the bias gradient is the
-    column sum of g.  All arithmetic runs in libfp8q.  As for torch._scaled_mm, the input's
-    last dimension (forward) and the weight's first (backward) must be multiples of 16."""
+    input gradient g @ w and the weight gradient g^T @ x as two more scaled products, reading the
+    weight, g and x where they lie (MN-major operands, no transposed copies); the bias gradient is
+    the column sum of g.  All arithmetic runs in libfp8q.  As for torch._scaled_mm, the input's
+    last dimension and the weight's first must be multiples of 16."""
 
     @staticmethod
     def forward(ctx, x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor]) -> torch.Tensor:
@@ -881,12 +914,12 @@ class _LinearFp8(torch.autograd.Function):
         K = w_fp8.shape[1]
         g_fp8, sg = cast_to_fp8(g, "e5m2")
         dt = out_grad.dtype
-        # x_grad[T, K] = g[T, N] @ w[N, K]: the weight transposed to [K, N]
+        # x_grad[T, K] = g[T, N] @ w[N, K]: A = g (k = n contiguous), B = w read as [k = n][K]
         x_grad = torch.empty((T, K), dtype=dt, device=g.device)
-        fp8q_scaled_mm(g_fp8, transpose_fp8(w_fp8), sg, sw, x_grad)
-        # w_grad[N, K] = g^T[N, T] @ x[T, K]: g and x transposed, T padded to 16
+        fp8q_scaled_mm_ex(g_fp8, w_fp8, sg, sw, x_grad, a_layout=K_MAJOR, b_layout=MN_MAJOR)
+        # w_grad[N, K] = g^T[N, T] @ x[T, K]: both operands read as [k = t][.], any token count
         w_grad = torch.empty((N, K), dtype=dt, device=g.device)
-        fp8q_scaled_mm(transpose_fp8(g_fp8, 16), transpose_fp8(x_fp8, 16), sg, sx, w_grad)
+        fp8q_scaled_mm_ex(g_fp8, x_fp8, sg, sx, w_grad, a_layout=MN_MAJOR, b_layout=MN_MAJOR)
         bias_grad = None
         if ctx.has_bias:
             bias_grad = torch.empty((N,), dtype=dt, device=g.device)

@@ -329,12 +329,15 @@ namespace {
 // shared checks of the two fp8 products; returns FP8Q_OK to go on
 fp8q_status check_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
                             const float* sa, const float* sb, const void* bias, int yt, const void* d,
-                            const uint32_t* status, bool* nothing) {
+                            const uint32_t* status, bool* nothing, int a_mn = 0, int b_mn = 0) {
     *nothing = false;
     if (!dtype_ok(yt)) return FP8Q_ERR_BAD_DTYPE;
     if (!fmt_ok(fa) || !fmt_ok(fb)) return FP8Q_ERR_BAD_FORMAT;
     const int64_t lim = 0x7FFFFFFFLL - 512;
-    if (M < 0 || N < 0 || K < 0 || M > lim || N > lim || K > lim || K % 16 != 0) return FP8Q_ERR_BAD_SHAPE;
+    if (M < 0 || N < 0 || K < 0 || M > lim || N > lim || K > lim) return FP8Q_ERR_BAD_SHAPE;
+    // the row pitch of every operand is a multiple of 16 bytes (TMA)
+    if ((!(a_mn && b_mn) && K % 16 != 0) || (a_mn && M % 16 != 0) || (b_mn && N % 16 != 0))
+        return FP8Q_ERR_BAD_SHAPE;
     const int64_t mn = checked_mul(M, N);
     if (mn < 0 || checked_mul(mn, dtype_bytes(yt)) < 0 || checked_mul(M, K) < 0 || checked_mul(N, K) < 0)
         return FP8Q_ERR_BAD_SHAPE;
@@ -403,6 +406,26 @@ fp8q_status fp8q_sum_rows(const void* x, fp8q_dtype xt, int64_t rows, int64_t co
     if (!out || (rows > 0 && !x)) return FP8Q_ERR_NULL_POINTER;
     if (!aligned(out, dtype_bytes(xt)) || (x && !aligned(x, dtype_bytes(xt)))) return FP8Q_ERR_MISALIGNED;
     return launch_sum_rows(x, xt, rows, cols, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+extern "C" {
+
+fp8q_status fp8q_scaled_mm_ex(const uint8_t* a, fp8q_format fa, fp8q_layout a_layout, const uint8_t* b,
+                              fp8q_format fb, fp8q_layout b_layout, int64_t M, int64_t N, int64_t K,
+                              const float* scale_a, const float* scale_b, const void* bias, fp8q_dtype yt, void* d,
+                              uint32_t* status, fp8q_stream_t stream) {
+    if ((a_layout != FP8Q_K_MAJOR && a_layout != FP8Q_MN_MAJOR) || (b_layout != FP8Q_K_MAJOR && b_layout != FP8Q_MN_MAJOR))
+        return FP8Q_ERR_BAD_SHAPE;
+    const int a_mn = a_layout == FP8Q_MN_MAJOR, b_mn = b_layout == FP8Q_MN_MAJOR;
+    bool nothing = false;
+    fp8q_status st = check_scaled_mm(a, fa, b, fb, M, N, K, scale_a, scale_b, bias, yt, d, status, &nothing, a_mn, b_mn);
+    if (st != FP8Q_OK || nothing) return st;
+    if (!scale_a || !scale_b) return FP8Q_ERR_NULL_POINTER;
+    if (!aligned(scale_a, 4) || !aligned(scale_b, 4)) return FP8Q_ERR_MISALIGNED;
+    return launch_scaled_mm(a, fa, b, fb, M, N, K, scale_a, 0, scale_b, 0, false, bias, yt, d, status,
+                            reinterpret_cast<cudaStream_t>(stream), a_mn, b_mn);
 }
 
 }  // extern "C"

@@ -82,10 +82,11 @@ fp8q_status launch_dequant(const DequantProblem* probs, int count, int fmt, int 
 // fp8 x fp8 products on the tensor cores (scaled_mm.cu).  fine = false: sa and
 // sb are one scale each; fine = true: sa[M][sa_ld] per 1 x 128 group of A,
 // sb[ceil(N/128)][sb_ld] per 128 x 128 block of B.  Shapes validated, K % 16
-// == 0, a and b 16-byte aligned.
+// == 0 for a K-major operand, M (N) % 16 == 0 for an MN-major A (B), a and b
+// 16-byte aligned.
 fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
                              const float* sa, int sa_ld, const float* sb, int sb_ld, bool fine, const void* bias,
-                             int yt, void* d, uint32_t* status, cudaStream_t s);
+                             int yt, void* d, uint32_t* status, cudaStream_t s, int a_mn = 0, int b_mn = 0);
 
 // _LinearFp8.backward's data movements (linear_bwd.cu): validated shapes
 fp8q_status launch_transpose(const uint8_t* src, int64_t rows, int64_t cols, uint8_t* dst, int64_t ld,

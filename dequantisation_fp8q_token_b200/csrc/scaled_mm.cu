@@ -87,7 +87,8 @@ struct Params {
     const void* bias;           // [N] of the output type, or null
     void* d;                    // [M][N]
     int vec_store;              // D rows 32-byte aligned (base and row pitch)
-    int stage_tx;               // bytes one stage's two TMA boxes bring
+    int stage_tx;               // bytes one stage's TMA boxes bring
+    int a_mn, b_mn;             // operand stored MN-major ([K][M] / [K][N] row-major), else K-major
     uint32_t* status;           // optional status word
 };
 
@@ -165,11 +166,25 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
          | (static_cast<uint64_t>(1) << 46)
          | (static_cast<uint64_t>(2) << 61);
 }
+// The same for an MN-major operand tile: each 128-byte row holds 128 M (or N)
+// elements of one k, TMA writes 128 x 128-byte boxes (one per 128 M or N),
+// 8-row k groups are 1024 bytes apart (stride byte offset) and successive
+// 128-wide M or N boxes 16384 bytes apart (leading byte offset).  A k step of
+// 32 moves the start address by 32 rows, 4096 bytes.
+constexpr int kMnAtomBytes = 128 * BK;
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t addr) {
+    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu)
+         | (static_cast<uint64_t>(kMnAtomBytes >> 4) << 16)
+         | (static_cast<uint64_t>(1024 >> 4) << 32)
+         | (static_cast<uint64_t>(1) << 46)
+         | (static_cast<uint64_t>(2) << 61);
+}
 // Instruction descriptor of kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B
-// formats (bits 7-9, 10-12: 0 e4m3, 1 e5m2), both K-major, N >> 3 at bit 17,
-// M >> 4 at bit 24.
-__host__ __device__ constexpr uint32_t instr_desc(int fa, int fb, int bn) {
+// formats (bits 7-9, 10-12: 0 e4m3, 1 e5m2), A and B MN-major (bits 15, 16;
+// 0 = K-major), N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t instr_desc(int fa, int fb, int bn, int a_mn = 0, int b_mn = 0) {
     return (1u << 4) | (static_cast<uint32_t>(fa) << 7) | (static_cast<uint32_t>(fb) << 10)
+         | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16)
          | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
 }
 __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -363,8 +378,16 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort)) { fail = kTimeoutProducer; break; }
                     const uint32_t fb = full0 + 8 * stage;
                     mbar_arrive_expect_tx(fb, static_cast<uint32_t>(p.stage_tx));
-                    tma_load_2d(smem_u32(sA + stage * kABytes), &map_a, kb * BK, mb * BM, fb);
-                    tma_load_2d(smem_u32(sB + stage * kBBytes), &map_b, kb * BK, nb * BN, fb);
+                    if (p.a_mn) tma_load_2d(smem_u32(sA + stage * kABytes), &map_a, mb * BM, kb * BK, fb);
+                    else tma_load_2d(smem_u32(sA + stage * kABytes), &map_a, kb * BK, mb * BM, fb);
+                    if (p.b_mn) {
+#pragma unroll
+                        for (int h = 0; h < BN / 128; ++h)
+                            tma_load_2d(smem_u32(sB + stage * kBBytes + h * kMnAtomBytes), &map_b, nb * BN + 128 * h,
+                                        kb * BK, fb);
+                    } else {
+                        tma_load_2d(smem_u32(sB + stage * kBBytes), &map_b, kb * BK, nb * BN, fb);
+                    }
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
@@ -401,7 +424,9 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < BK / 32; ++j) {
                         const uint32_t accumulate = FINE ? (j > 0) : (kb > 0 || j > 0);
-                        mma_f8f6f4(d_tmem, smem_desc_sw128(a0 + 32 * j), smem_desc_sw128(b0 + 32 * j), idesc,
+                        const uint64_t ad = p.a_mn ? smem_desc_mn_sw128(a0 + 4096 * j) : smem_desc_sw128(a0 + 32 * j);
+                        const uint64_t bd = p.b_mn ? smem_desc_mn_sw128(b0 + 4096 * j) : smem_desc_sw128(b0 + 32 * j);
+                        mma_f8f6f4(d_tmem, ad, bd, idesc,
                                    accumulate);
                     }
                     mma_commit(empty0 + 8 * stage);
@@ -621,7 +646,7 @@ cudaError_t launch_dtype(bool fine, int yt, const CUtensorMap& ma, const CUtenso
 
 fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
                              const float* sa, int sa_ld, const float* sb, int sb_ld, bool fine, const void* bias,
-                             int yt, void* d, uint32_t* status, cudaStream_t s) {
+                             int yt, void* d, uint32_t* status, cudaStream_t s, int a_mn, int b_mn) {
     using namespace mm;
     // 128-wide tiles when a product of at most 128 rows would leave SMs idle
     const bool narrow = M <= BM && (N + 255) / 256 < sm_count();
@@ -630,12 +655,17 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     // the MMA still multiplies 128 rows, and the rows past the box hold stale
     // shared memory, but output row m depends on row m of A alone and rows
     // at or past M are never stored.
-    const int a_rows = M >= BM ? BM : static_cast<int>((M + 15) / 16 * 16);
+    // (An MN-major A keeps its 128-wide box: its rows are k, its columns m.)
+    const int a_rows = (M >= BM || a_mn) ? BM : static_cast<int>((M + 15) / 16 * 16);
     CUtensorMap ma, mbm;
     memset(&ma, 0, sizeof(ma));
     memset(&mbm, 0, sizeof(mbm));
     if (K > 0) {
-        if (!make_map(&ma, a, M, K, a_rows) || !make_map(&mbm, b, N, K, bn)) return FP8Q_ERR_CUDA;
+        // K-major: [M][K] with boxes of rows x 128 k; MN-major: [K][M] with
+        // boxes of 128 k x 128 m (B likewise, two boxes for 256 columns)
+        const bool ok_a = a_mn ? make_map(&ma, a, K, M, BK) : make_map(&ma, a, M, K, a_rows);
+        const bool ok_b = b_mn ? make_map(&mbm, b, K, N, BK) : make_map(&mbm, b, N, K, bn);
+        if (!ok_a || !ok_b) return FP8Q_ERR_CUDA;
     }
     Params p;
     p.M = static_cast<int>(M);
@@ -654,7 +684,9 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     p.vec_store = (reinterpret_cast<uintptr_t>(d) % 32 == 0) && ((N * eb) % 32 == 0);
     p.status = status;
     p.stage_tx = (a_rows + bn) * BK;
-    const uint32_t idesc = instr_desc(fa, fb, bn);
+    p.a_mn = a_mn;
+    p.b_mn = b_mn;
+    const uint32_t idesc = instr_desc(fa, fb, bn, a_mn, b_mn);
     cudaError_t e;
     if (narrow) e = launch_dtype<128>(fine, yt, ma, mbm, p, idesc, s);
     else e = launch_dtype<256>(fine, yt, ma, mbm, p, idesc, s);

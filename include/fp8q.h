@@ -373,6 +373,30 @@ fp8q_status fp8q_scaled_mm(const uint8_t* a, fp8q_format fa, const uint8_t* b, f
                            fp8q_stream_t stream);
 
 /*
+ * Operand layouts of fp8q_scaled_mm_ex.  With A the [M][K] operand and B the
+ * [N][K] operand of the product (D = A B^T):
+ *   FP8Q_K_MAJOR   stored [M][K] (resp. [N][K]) row-major: k is contiguous
+ *   FP8Q_MN_MAJOR  stored [K][M] (resp. [K][N]) row-major: m (n) is contiguous,
+ *                  i.e. the operand is the transpose of a row-major matrix
+ */
+typedef enum { FP8Q_K_MAJOR = 0, FP8Q_MN_MAJOR = 1 } fp8q_layout;
+
+/*
+ * fp8q_scaled_mm with a layout per operand, so that transposed operands
+ * need no copy -- ColossalAI _LinearFp8.backward multiplies the output
+ * gradient g [T][N] by the weight w [N][K] (input gradient: A = g K-major,
+ * B = w MN-major) and g^T by x [T][K] (weight gradient: A = g MN-major,
+ * B = x MN-major).  Same arithmetic, scales, bias, status and errors as
+ * fp8q_scaled_mm; the row pitch rule becomes: K % 16 == 0 unless both
+ * operands are MN-major, M % 16 == 0 for an MN-major A, N % 16 == 0 for an
+ * MN-major B (FP8Q_ERR_BAD_SHAPE otherwise, also for an unknown layout).
+ */
+fp8q_status fp8q_scaled_mm_ex(const uint8_t* a, fp8q_format fa, fp8q_layout a_layout, const uint8_t* b,
+                              fp8q_format fb, fp8q_layout b_layout, int64_t M, int64_t N, int64_t K,
+                              const float* scale_a, const float* scale_b, const void* bias, fp8q_dtype yt, void* d,
+                              uint32_t* status, fp8q_stream_t stream);
+
+/*
  * fp8 matrix product with fine-grained scales: activations quantised by
  * per_token_cast_to_fp8 (DeepEP "5 Utils": one scale_inv per 1 x 128 group
  * of a row) times a weight stored with one scale_inv per 128 x 128 block

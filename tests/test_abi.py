@@ -180,3 +180,16 @@ def test_transpose_and_sum_rows_validation(L):
     assert s(P, 2, 4, 4, None, None) == 1       # null out
     assert s(P + 1, 2, 4, 4, P, None) == 5      # bf16 input on an odd address
     assert s(None, 2, 4, 0, None, None) == 0    # no columns
+
+
+def test_scaled_mm_ex_validation(L):
+    f = L.fp8q_scaled_mm_ex
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    A = 0x10000
+    assert f(A, 0, 2, A, 0, 0, 32, 32, 32, P, P, None, 2, A, None, None) == 4     # unknown layout
+    assert f(A, 0, 1, A, 0, 0, 24, 32, 32, P, P, None, 2, A, None, None) == 4     # MN-major A needs M % 16
+    assert f(A, 0, 0, A, 0, 1, 32, 24, 32, P, P, None, 2, A, None, None) == 4     # MN-major B needs N % 16
+    assert f(A, 0, 0, A, 0, 1, 32, 32, 24, P, P, None, 2, A, None, None) == 4     # a K-major operand needs K % 16
+    assert f(A, 0, 1, A, 0, 1, 32, 32, 24, None, P, None, 2, A, None, None) == 1  # both MN-major: any K; null scale

@@ -323,3 +323,30 @@ def test_exact_grid_small_m(fp8q, orc, fine, M, N, K):
     got = host(run(fp8q, fine, a, E4M3FN, b, E5M2, sa, sb, bias_t, BF16))
     want = oracle_rounded(orc, fine, a, E4M3FN, b, E5M2, sa, sb, bias, BF16)
     np.testing.assert_array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------
+# operand layouts (fp8q_scaled_mm_ex): K-major or MN-major, bit for bit
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("a_mn,b_mn,M,N,K", [
+    (0, 1, 128, 256, 128), (0, 1, 200, 304, 272), (0, 1, 64, 3008, 512),
+    (1, 0, 208, 300, 272), (1, 0, 128, 256, 384),
+    (1, 1, 128, 256, 128), (1, 1, 256, 512, 300), (1, 1, 144, 3008, 37), (1, 1, 32, 16, 1),
+    (0, 0, 200, 300, 272)])
+@pytest.mark.parametrize("yt", [F32, BF16])
+def test_exact_grid_layouts(fp8q, orc, a_mn, b_mn, M, N, K, yt):
+    g = np.random.default_rng(1000 * a_mn + 100 * b_mn + M + N + K + yt)
+    a, b = grid_codes(g, (M, K), E4M3FN), grid_codes(g, (N, K), E5M2)   # logical [M, K], [N, K]
+    A = dev(np.ascontiguousarray(a.T) if a_mn else a)
+    B = dev(np.ascontiguousarray(b.T) if b_mn else b)
+    bias_t, bias = t_bias(g, N, yt)
+    out = Guarded(M * N, TORCH_T[yt])
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fp8q.fp8q_scaled_mm_ex(A, B, dev(np.array([0.0123], np.float32)), dev(np.array([3.5], np.float32)),
+                           out.t.view(M, N), bias_t.cuda(), a_layout=a_mn, b_layout=b_mn, fa=E4M3FN, fb=E5M2,
+                           status=st)
+    out.check()
+    assert int(st.item()) == 0
+    want = orc.scaled_mm_rounded(a, E4M3FN, b, E5M2, 0.0123, 3.5, bias=bias, yt=yt)
+    bad = ~bits_equal(host(out.t).reshape(M, N), want, yt)
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
