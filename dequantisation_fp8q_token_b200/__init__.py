@@ -797,15 +797,27 @@ def fp8q_scaled_mm_blockwise(a: torch.Tensor, scale_a: torch.Tensor, b: torch.Te
         "fp8q_scaled_mm_blockwise")
 
 
-def scaled_mm(a: torch.Tensor, b_t: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
+def _operand_layout(t: torch.Tensor, name: str):
+    """(storage tensor, layout) of a 2-D fp8 operand given as [rows, k]: K_MAJOR when its rows
+    are contiguous, MN_MAJOR when it is the transpose of a contiguous [k, rows] matrix."""
+    if t.is_contiguous():
+        return t, K_MAJOR
+    if t.t().is_contiguous():
+        return t.t(), MN_MAJOR
+    raise ValueError(f"{name} must be row-major or the transpose of a row-major matrix")
+
+
+def scaled_mm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
               bias: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
-    """torch._scaled_mm(a, b_t, scale_a, scale_b, bias, out_dtype) as ColossalAI calls it: b_t is the
-    transpose of a row-major weight w [N, K] (w.t()), which is what the kernel reads."""
-    w = b_t.t()
-    if not w.is_contiguous():
-        raise ValueError("b_t must be the transpose of a contiguous [N, K] weight (w.t())")
-    out = torch.empty((a.shape[0], w.shape[0]), dtype=out_dtype, device=a.device)
-    fp8q_scaled_mm(a, w, scale_a, scale_b, out, bias)
+    """torch._scaled_mm(a, b, scale_a, scale_b, bias, out_dtype): out[M, N] = a[M, K] @ b[K, N] with
+    per-tensor scales.  Each operand may be row-major or the transpose of a row-major matrix (as
+    ColossalAI passes w_fp8.t()); neither is copied."""
+    if a.dim() != 2 or b.dim() != 2:
+        raise ValueError("a and b must be 2-D")
+    A, la = _operand_layout(a, "a")                  # a as [M, K]
+    B, lb = _operand_layout(b.t(), "b")              # b^T as [N, K]
+    out = torch.empty((a.shape[0], b.shape[1]), dtype=out_dtype, device=a.device)
+    fp8q_scaled_mm_ex(A, B, scale_a, scale_b, out, bias, a_layout=la, b_layout=lb)
     return out
 
 

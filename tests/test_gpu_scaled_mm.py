@@ -350,3 +350,20 @@ def test_exact_grid_layouts(fp8q, orc, a_mn, b_mn, M, N, K, yt):
     want = orc.scaled_mm_rounded(a, E4M3FN, b, E5M2, 0.0123, 3.5, bias=bias, yt=yt)
     bad = ~bits_equal(host(out.t).reshape(M, N), want, yt)
     assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
+
+
+def test_scaled_mm_helper_takes_either_layout(fp8q, orc):
+    """torch._scaled_mm-style calls: b given as w.t() (ColossalAI) or as a row-major [K, N]
+    matrix, a row-major or transposed; the same bits either way."""
+    g = np.random.default_rng(21)
+    M, N, K = 144, 272, 256
+    a, w = grid_codes(g, (M, K), E4M3FN), grid_codes(g, (N, K), E4M3FN)
+    sa, sb = dev(np.array([0.5], np.float32)), dev(np.array([0.25], np.float32))
+    want = orc.scaled_mm_rounded(a, E4M3FN, w, E4M3FN, 0.5, 0.25, yt=BF16)
+    A = dev(a).view(torch.float8_e4m3fn)
+    W = dev(w).view(torch.float8_e4m3fn)
+    At = dev(np.ascontiguousarray(a.T)).view(torch.float8_e4m3fn).t()      # a, stored transposed
+    Wt = dev(np.ascontiguousarray(w.T)).view(torch.float8_e4m3fn)          # b = w^T, row-major [K, N]
+    for lhs in (A, At):
+        for rhs in (W.t(), Wt):
+            np.testing.assert_array_equal(host(fp8q.scaled_mm(lhs, rhs, sa, sb)), want)
