@@ -96,3 +96,48 @@ def test_c5_all_weights_row_samples(stepped, orc):
             r1 = min(M, r0 + 8)
             yo = orc.block_dequant(w, s, E4M3FN, 128, BF16, rows=(r0, r1))
             assert_out_equal(y[r0:r1], yo[r0:r1], BF16, name=f"weight {i} rows {r0}:{r1}")
+
+
+# ---------------------------------------------------------------------------
+# the fp8 products, in the launch configuration bench.py's matmul section times
+# ---------------------------------------------------------------------------
+def _mm_bound(got_bits, exact, mag, K):
+    """The accumulation bound of the fp8 products: (ceil(K/32) + 1) * 2^-23 of sum |a * b|,
+    2^-24 per k-block for the fine-grained fold, and one bf16 ulp of the output."""
+    import torch
+    got = torch.from_numpy(got_bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    rel = (-(-K // 32) + 1) * 2.0 ** -23 + (-(-K // 128)) * 2.0 ** -24
+    e = np.floor(np.log2(np.maximum(np.abs(exact), 2.0 ** -126)))
+    bad = ~(np.abs(got - exact) <= rel * mag + 2.0 ** (e - 7))
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outside the bound"
+
+
+def test_matmul_workload_sampled_rows(stepped, orc):
+    """bench.MatmulWorkload's own operands and launches: its per-token codes equal the oracle's
+    (so the oracle's product starts from its own codes), then sampled rows of both products."""
+    import torch
+    mm = bench.MatmulWorkload(stepped)
+    qo, so = orc.per_token_group_quant(stepped.host["c2_x"], BF16, 128, E4M3FN, threads=THREADS)
+    assert_codes_equal(host(mm.q), qo, E4M3FN)
+    assert_f32_equal(host(mm.sa), so)
+    w, sb = workloads.mm_w_s()
+    rows = [0, 5, 1000, 4095]
+    wabs = np.abs(torch.from_numpy(w).view(torch.float8_e4m3fn).to(torch.float32).numpy())
+    aabs = np.abs(torch.from_numpy(qo[rows]).view(torch.float8_e4m3fn).to(torch.float32).numpy())
+    K = qo.shape[1]
+    # fine-grained
+    mm.ops["scaled_mm_blockwise"]()
+    got = host(mm.out)
+    mag = ((aabs * np.repeat(so[rows], 128, 1)) @ (wabs * np.repeat(np.repeat(sb, 128, 0), 128, 1)).T).astype(np.float64)
+    for i, r in enumerate(rows):
+        exact = orc.scaled_mm_blockwise(qo, E4M3FN, so, w, E4M3FN, sb, rows=(r, r + 1), threads=THREADS)[r]
+        _mm_bound(got[r], exact, mag[i], K)
+    # per-tensor, the scales bench.py uses (the first group's and the first block's)
+    mm.ops["scaled_mm_per_tensor"]()
+    got = host(mm.out)
+    s1, s2 = float(so[0, 0]), float(sb[0, 0])
+    mag = (aabs @ wabs.T).astype(np.float64) * float(np.float32(s1) * np.float32(s2))
+    for i, r in enumerate(rows):
+        exact = orc.scaled_mm(qo, E4M3FN, w, E4M3FN, s1, s2, rows=(r, r + 1), threads=THREADS)[r]
+        _mm_bound(got[r], exact, mag[i], K)
+    assert int(mm.status.item()) == 0
