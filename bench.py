@@ -166,47 +166,100 @@ class Workload:
 
 
 class EndToEnd:
-    """The step from pinned host memory to pinned host memory.  Each op's inputs
-    go host->device on a copy-in stream, the op runs on the compute stream, its
-    outputs go device->host on a copy-out stream; events order each op's three
-    parts and keep the next step from overwriting a buffer still in use, so the
-    upload of one op overlaps the compute and download of the ones before it
-    (PCIe carries both directions at once)."""
+    """The step from pinned host memory to pinned host memory.  The step's ops
+    are cut into units -- rows or weights of an op whose rows (weights) are
+    independent, the whole op otherwise (the per-tensor casts need their
+    whole tensor) -- and each unit's inputs go host->device on a copy-in
+    stream, the unit runs on the compute stream, its outputs go device->host
+    on a copy-out stream.  Events order each unit's three parts and keep the
+    next step from overwriting a buffer still in use, so the upload of one
+    unit overlaps the compute and download of the ones before it (PCIe
+    carries both directions at once) and a large op starts downloading
+    after its first unit rather than after its last."""
 
-    def __init__(self, wl: Workload):
+    def __init__(self, wl: Workload, chunks: int = 4, weight_chunks: int = 8):
         self.wl = wl
-        self.h_in = {id(t): torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wl.inputs()}
+        f = wl.fp8q
+        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)  # noqa: E731
+        self.h = {}
         for t in wl.inputs():
-            self.h_in[id(t)].copy_(t)
-        self.h_out = {id(t): torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wl.outputs()}
+            self.h[id(t)] = pin(t)
+            self.h[id(t)].copy_(t)
+        for t in wl.outputs():
+            self.h[id(t)] = pin(t)
+        H = lambda t: self.h[id(t)]  # noqa: E731
+
+        def rows(n, k):
+            step = -(-n // k)
+            step = -(-step // 128) * 128              # whole 128-row blocks (block-scale rows)
+            return [(r, min(n, r + step)) for r in range(0, n, step)]
+
+        units = []
+        for op in wl.ops:
+            if op.name == "per_token_group_quant":
+                x, q, sc = wl.c2_x, wl.c2_q, wl.c2_s
+                for r0, r1 in rows(x.shape[0], chunks):
+                    units.append(((lambda a=x[r0:r1], b=q[r0:r1], c=sc[r0:r1]:
+                                   f.fp8q_per_token_group_quant(a, b, c, 128, E4M3FN)),
+                                  [(x[r0:r1], H(x)[r0:r1])], [(q[r0:r1], H(q)[r0:r1]), (sc[r0:r1], H(sc)[r0:r1])]))
+            elif op.name == "block_dequant":
+                w, sc, y = wl.c3_w, wl.c3_s, wl.c3_y
+                for r0, r1 in rows(w.shape[0], chunks):
+                    b0, b1 = r0 // 128, -(-r1 // 128)
+                    units.append(((lambda a=w[r0:r1], b=sc[b0:b1], c=y[r0:r1]:
+                                   f.fp8q_block_dequant(a, b, c, 128, E4M3FN)),
+                                  [(w[r0:r1], H(w)[r0:r1]), (sc[b0:b1], H(sc)[b0:b1])], [(y[r0:r1], H(y)[r0:r1])]))
+            elif op.name == "cast_from_fp8_group":
+                q, sc, y = wl.c2_q, wl.c2_s, wl.c2_y
+                for r0, r1 in rows(q.shape[0], chunks):
+                    units.append(((lambda a=q[r0:r1], b=sc[r0:r1], c=y[r0:r1]:
+                                   f.fp8q_cast_from_fp8(a, b, c, GRAN_GROUP, 128, E4M3FN)),
+                                  [], [(y[r0:r1], H(y)[r0:r1])]))
+            elif op.name == "cast_per_channel":
+                x, q, sc = wl.c4a_x, wl.c4a_q, wl.c4a_s
+                for r0, r1 in rows(x.shape[0], chunks):
+                    units.append(((lambda a=x[r0:r1], b=q[r0:r1], c=sc[r0:r1]:
+                                   f.fp8q_cast_per_channel(a, b, c, E4M3FN)),
+                                  [(x[r0:r1], H(x)[r0:r1])], [(q[r0:r1], H(q)[r0:r1]), (sc[r0:r1], H(sc)[r0:r1])]))
+            elif op.name == "block_dequant_grouped":
+                n = len(wl.c5_w)
+                step = -(-n // weight_chunks)
+                for i in range(0, n, step):
+                    ws, ss, ys = wl.c5_w[i:i + step], wl.c5_s[i:i + step], wl.c5_y[i:i + step]
+                    units.append(((lambda a=ws, b=ss, c=ys: f.fp8q_block_dequant_grouped(a, b, c, 128, E4M3FN)),
+                                  [(t, H(t)) for t in ws + ss], [(t, H(t)) for t in ys]))
+            else:
+                units.append((op.fn, [(t, H(t)) for t in op.ins], [(t, H(t)) for t in op.outs]))
+        self.units = units
         self.s_in, self.s_comp, self.s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-        n = len(wl.ops)
-        self.done_comp = [None] * n
-        self.done_out = [None] * n
+        self.done_comp = [None] * len(units)
+        self.done_out = [None] * len(units)
         self.h2d_bytes = sum(t.numel() * t.element_size() for t in wl.inputs())
         self.d2h_bytes = sum(t.numel() * t.element_size() for t in wl.outputs())
+        assert self.h2d_bytes == sum(d.numel() * d.element_size() for _, ins, _ in units for d, _ in ins)
+        assert self.d2h_bytes == sum(d.numel() * d.element_size() for _, _, outs in units for d, _ in outs)
 
     def step(self):
-        for i, op in enumerate(self.wl.ops):
+        for i, (fn, ins, outs) in enumerate(self.units):
             with torch.cuda.stream(self.s_in):
                 if self.done_comp[i] is not None:
-                    self.s_in.wait_event(self.done_comp[i])      # previous step's op i has read its inputs
-                for t in op.ins:
-                    t.copy_(self.h_in[id(t)], non_blocking=True)
+                    self.s_in.wait_event(self.done_comp[i])      # previous step's unit i has read its inputs
+                for d, hst in ins:
+                    d.copy_(hst, non_blocking=True)
                 ev_in = torch.cuda.Event()
                 ev_in.record(self.s_in)
             with torch.cuda.stream(self.s_comp):
                 self.s_comp.wait_event(ev_in)
                 if self.done_out[i] is not None:
                     self.s_comp.wait_event(self.done_out[i])     # previous step's outputs are on the host
-                op.fn()
+                fn()
                 ev_c = torch.cuda.Event()
                 ev_c.record(self.s_comp)
                 self.done_comp[i] = ev_c
             with torch.cuda.stream(self.s_out):
                 self.s_out.wait_event(ev_c)
-                for t in op.outs:
-                    self.h_out[id(t)].copy_(t, non_blocking=True)
+                for d, hst in outs:
+                    hst.copy_(d, non_blocking=True)
                 ev_o = torch.cuda.Event()
                 ev_o.record(self.s_out)
                 self.done_out[i] = ev_o
@@ -224,6 +277,49 @@ class EndToEnd:
         e1.record(self.s_out)
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / steps
+
+
+def pcie_bound(h2d_bytes: int, d2h_bytes: int, device, n: int = 1 << 30):
+    """The fastest the end-to-end step's transfers can go on this machine: pinned copies of n bytes
+    each way, alone and both at once (CUDA events), then the step's bytes moved both ways at the
+    shared rate and the remainder of the larger direction at its own rate."""
+    h1 = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    h2 = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    d1 = torch.empty(n, dtype=torch.uint8, device=device)
+    d2 = torch.empty(n, dtype=torch.uint8, device=device)
+    s1, s2 = torch.cuda.Stream(device), torch.cuda.Stream(device)
+
+    def timed(fn, reps=4):
+        fn()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / reps
+
+    def both():
+        cur = torch.cuda.current_stream(device)
+        s1.wait_stream(cur)
+        s2.wait_stream(cur)
+        with torch.cuda.stream(s1):
+            d1.copy_(h1, non_blocking=True)
+        with torch.cuda.stream(s2):
+            h2.copy_(d2, non_blocking=True)
+        cur.wait_stream(s1)
+        cur.wait_stream(s2)
+    up = n / timed(lambda: d1.copy_(h1, non_blocking=True)) / 1e6        # GB/s
+    down = n / timed(lambda: h2.copy_(d2, non_blocking=True)) / 1e6
+    shared = n / timed(both) / 1e6
+    common = min(h2d_bytes, d2h_bytes)
+    rest_up, rest_down = h2d_bytes - common, d2h_bytes - common
+    ms = common / shared / 1e6 + rest_up / up / 1e6 + rest_down / down / 1e6
+    del h1, h2, d1, d2
+    torch.cuda.empty_cache()
+    return {"h2d_gb_s": round(up, 1), "d2h_gb_s": round(down, 1), "both_gb_s_each": round(shared, 1),
+            "bound_ms_per_step": round(ms, 3)}
 
 
 def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
@@ -695,6 +791,7 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e2e.time(e2e_steps), world, device)
     bi, bo = e2e.h2d_bytes, e2e.d2h_bytes
     del e2e
+    pcie = pcie_bound(bi, bo, device) if rank == 0 else None
     iso = isolated_timing(wl) if rank == 0 else {}
     mm = None
     if rank == 0 and not args.no_matmul:
@@ -745,7 +842,8 @@ def run_ours(args):
         "clocks": clk.summary(),
         "e2e": {"value": round(world * wl.step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
-                "steps": e2e_steps},
+                "steps": e2e_steps, "pcie": pcie,
+                "frac_of_pcie_bound": round(pcie["bound_ms_per_step"] / e2e_ms, 4) if pcie else None},
         "gpu_launches": wl.launches_per_step * args.steps,
     }
     if world == 1:

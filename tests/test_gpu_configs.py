@@ -141,3 +141,16 @@ def test_matmul_workload_sampled_rows(stepped, orc):
         exact = orc.scaled_mm(qo, E4M3FN, w, E4M3FN, s1, s2, rows=(r, r + 1), threads=THREADS)[r]
         _mm_bound(got[r], exact, mag[i], K)
     assert int(mm.status.item()) == 0
+
+
+def test_end_to_end_units_give_the_device_step_bytes(stepped):
+    """bench.py's end-to-end step cuts ops into row / weight units on three streams; its host
+    outputs must equal the whole-op device step's outputs byte for byte."""
+    want = {id(t): host(t).copy() for t in stepped.outputs()}
+    e2e = bench.EndToEnd(stepped)
+    assert len(e2e.units) > len(stepped.ops)
+    e2e.step()
+    torch.cuda.synchronize()
+    for t in stepped.outputs():
+        got = e2e.h[id(t)].view(torch.uint8).numpy() if t.element_size() == 1 else host(e2e.h[id(t)])
+        np.testing.assert_array_equal(np.asarray(got).reshape(-1), want[id(t)].reshape(-1))
