@@ -63,13 +63,19 @@ constexpr int kGroupM = 32;     // row-tiles per raster band
 // leave SMs without a share of the weight to stream.  Measured on B200 for
 // large products: 128 x 128 tiles lose a quarter of the fine-grained
 // throughput, since the narrower MMA reads twice the operand bytes per flop.
-template <int BN_> struct Shape {
+// MT = 256 (per-tensor scales only): 256 x 256 tiles, two M 128 MMAs per k
+// step sharing the B tile, the two 128 x 256 accumulators filling TMEM (one
+// buffer: each tile's epilogue is not overlapped), a 3-stage ring -- a third
+// fewer operand bytes per flop than 128 x 256 tiles.
+template <int BN_, int MT_ = 128> struct Shape {
     static constexpr int BN = BN_;                          // rows of B (columns of D) per tile
-    static constexpr int kStages = BN_ == 256 ? 4 : 6;
-    static constexpr int kAccBufs = kTmemCols / BN;
+    static constexpr int MT = MT_;                          // rows of A (and of D) per tile
+    static constexpr int kATile = MT_ * BK;
+    static constexpr int kStages = MT_ == 256 ? 3 : (BN_ == 256 ? 4 : 6);
+    static constexpr int kAccBufs = MT_ == 256 ? 1 : kTmemCols / BN;
     static constexpr int kColsPerWarp = BN / (kEpiWarps / 4);   // tile columns one epilogue warp owns
     static constexpr int kBBytes = BN * BK;
-    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStageBytes = kATile + kBBytes;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment slack */ + 256 /* barriers */;
 };
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
@@ -311,20 +317,23 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int YT, bool FINE, int BN_>
+template <int YT, bool FINE, int BN_, int MT_>
 __global__ void __launch_bounds__(kThreads, 1)
 scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const Params p, const uint32_t idesc) {
-    constexpr int BN = Shape<BN_>::BN;
-    constexpr int kStages = Shape<BN_>::kStages;
-    constexpr int kAccBufs = Shape<BN_>::kAccBufs;
-    constexpr int kColsPerWarp = Shape<BN_>::kColsPerWarp;
-    constexpr int kBBytes = Shape<BN_>::kBBytes;
+    constexpr int BN = Shape<BN_, MT_>::BN;
+    constexpr int kStages = Shape<BN_, MT_>::kStages;
+    constexpr int kAccBufs = Shape<BN_, MT_>::kAccBufs;
+    constexpr int kColsPerWarp = Shape<BN_, MT_>::kColsPerWarp;
+    constexpr int kBBytes = Shape<BN_, MT_>::kBBytes;
+    constexpr int kATile = Shape<BN_, MT_>::kATile;
+    constexpr int kSub = MT_ / BM;                 // M 128 sub-tiles (MMAs per k step, accumulators per tile)
+    static_assert(!FINE || MT_ == BM, "fine-grained scales use 128-row tiles");
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + kStages * kABytes;
+    uint8_t* sB = smem + kStages * kATile;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kBBytes);
     // bars: full[kStages], empty[kStages], tfull[kAccBufs], tempty[kAccBufs], drain
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 2 * kAccBufs + 1);
@@ -378,8 +387,8 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort)) { fail = kTimeoutProducer; break; }
                     const uint32_t fb = full0 + 8 * stage;
                     mbar_arrive_expect_tx(fb, static_cast<uint32_t>(p.stage_tx));
-                    if (p.a_mn) tma_load_2d(smem_u32(sA + stage * kABytes), &map_a, mb * BM, kb * BK, fb);
-                    else tma_load_2d(smem_u32(sA + stage * kABytes), &map_a, kb * BK, mb * BM, fb);
+                    if (p.a_mn) tma_load_2d(smem_u32(sA + stage * kATile), &map_a, mb * BM, kb * BK, fb);
+                    else tma_load_2d(smem_u32(sA + stage * kATile), &map_a, kb * BK, mb * MT_, fb);
                     if (p.b_mn) {
 #pragma unroll
                         for (int h = 0; h < BN / 128; ++h)
@@ -419,15 +428,19 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     }
                     if (!mbar_wait(full0 + 8 * stage, phase, abort)) { fail = kTimeoutMma; break; }
                     tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-                    const uint32_t a0 = smem_u32(sA + stage * kABytes), b0 = smem_u32(sB + stage * kBBytes);
+                    const uint32_t a0 = smem_u32(sA + stage * kATile), b0 = smem_u32(sB + stage * kBBytes);
 #pragma unroll
                     for (int j = 0; j < BK / 32; ++j) {
                         const uint32_t accumulate = FINE ? (j > 0) : (kb > 0 || j > 0);
-                        const uint64_t ad = p.a_mn ? smem_desc_mn_sw128(a0 + 4096 * j) : smem_desc_sw128(a0 + 32 * j);
                         const uint64_t bd = p.b_mn ? smem_desc_mn_sw128(b0 + 4096 * j) : smem_desc_sw128(b0 + 32 * j);
-                        mma_f8f6f4(d_tmem, ad, bd, idesc,
-                                   accumulate);
+#pragma unroll
+                        for (int sub = 0; sub < kSub; ++sub) {
+                            // sub-tile sub: rows 128 sub .. of A (K-major when kSub > 1), its own accumulator
+                            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((acc + sub) * BN);
+                            const uint64_t ad = p.a_mn ? smem_desc_mn_sw128(a0 + 4096 * j)
+                                                       : smem_desc_sw128(a0 + sub * BM * BK + 32 * j);
+                            mma_f8f6f4(d_tmem, ad, bd, idesc, accumulate);
+                        }
                     }
                     mma_commit(empty0 + 8 * stage);
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -460,7 +473,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         for (int t = blockIdx.x; t < tiles && !fail; t += gridDim.x) {
             int mb, nb;
             tile_coords(t, p.tiles_m, p.tiles_n, mb, nb);
-            const int row = mb * BM + quarter * 32 + lane;
+            const int row = mb * MT_ + quarter * 32 + lane;
             const int col_base = nb * BN + cgrp * kColsPerWarp;
             if (!FINE) {
                 if (p.num_kb > 0) {
@@ -471,23 +484,28 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     tc_fence_after();
                 }
 #pragma unroll 1
-                for (int c = 0; c < kColsPerWarp / 32; ++c) {
-                    float v[32];
-                    const int col0 = col_base + c * 32;
-                    if (p.num_kb > 0) {
-                        tmem_ld32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + cgrp * kColsPerWarp + c * 32), v);
-                    } else {
+                for (int sub = 0; sub < kSub; ++sub) {
+                    const int srow = row + sub * BM;
+#pragma unroll 1
+                    for (int c = 0; c < kColsPerWarp / 32; ++c) {
+                        float v[32];
+                        const int col0 = col_base + c * 32;
+                        if (p.num_kb > 0) {
+                            tmem_ld32(tmem_base + lane_addr +
+                                          static_cast<uint32_t>((acc + sub) * BN + cgrp * kColsPerWarp + c * 32), v);
+                        } else {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], scale);
+                        if (p.bias) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (col0 + i < p.N) v[i] = __fadd_rn(v[i], load_bias<YT>(p.bias, col0 + i));
+                        }
+                        if (srow < p.M && col0 < p.N) store_chunk<YT>(p, srow, col0, v);
                     }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], scale);
-                    if (p.bias) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (col0 + i < p.N) v[i] = __fadd_rn(v[i], load_bias<YT>(p.bias, col0 + i));
-                    }
-                    if (row < p.M && col0 < p.N) store_chunk<YT>(p, row, col0, v);
                 }
                 if (p.num_kb > 0) {
                     tc_fence_before();
@@ -608,11 +626,11 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int b
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int YT, bool FINE, int BN_>
+template <int YT, bool FINE, int BN_, int MT_>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, uint32_t idesc,
                          cudaStream_t s) {
-    auto kernel = scaled_mm_kernel<YT, FINE, BN_>;
-    constexpr int kSmemBytes = Shape<BN_>::kSmemBytes;
+    auto kernel = scaled_mm_kernel<YT, FINE, BN_, MT_>;
+    constexpr int kSmemBytes = Shape<BN_, MT_>::kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const int tiles = p.tiles_m * p.tiles_n;
@@ -633,13 +651,21 @@ template <int BN_>
 cudaError_t launch_dtype(bool fine, int yt, const CUtensorMap& ma, const CUtensorMap& mb, const Params& p,
                          uint32_t idesc, cudaStream_t s) {
     if (fine) {
-        return yt == kF32 ? launch_typed<kF32, true, BN_>(ma, mb, p, idesc, s)
-             : yt == kF16 ? launch_typed<kF16, true, BN_>(ma, mb, p, idesc, s)
-                          : launch_typed<kBF16, true, BN_>(ma, mb, p, idesc, s);
+        return yt == kF32 ? launch_typed<kF32, true, BN_, 128>(ma, mb, p, idesc, s)
+             : yt == kF16 ? launch_typed<kF16, true, BN_, 128>(ma, mb, p, idesc, s)
+                          : launch_typed<kBF16, true, BN_, 128>(ma, mb, p, idesc, s);
     }
-    return yt == kF32 ? launch_typed<kF32, false, BN_>(ma, mb, p, idesc, s)
-         : yt == kF16 ? launch_typed<kF16, false, BN_>(ma, mb, p, idesc, s)
-                      : launch_typed<kBF16, false, BN_>(ma, mb, p, idesc, s);
+    return yt == kF32 ? launch_typed<kF32, false, BN_, 128>(ma, mb, p, idesc, s)
+         : yt == kF16 ? launch_typed<kF16, false, BN_, 128>(ma, mb, p, idesc, s)
+                      : launch_typed<kBF16, false, BN_, 128>(ma, mb, p, idesc, s);
+}
+
+// per-tensor scales, 256 x 256 tiles
+cudaError_t launch_tall(int yt, const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, uint32_t idesc,
+                        cudaStream_t s) {
+    return yt == kF32 ? launch_typed<kF32, false, 256, 256>(ma, mb, p, idesc, s)
+         : yt == kF16 ? launch_typed<kF16, false, 256, 256>(ma, mb, p, idesc, s)
+                      : launch_typed<kBF16, false, 256, 256>(ma, mb, p, idesc, s);
 }
 
 }  // namespace mm
@@ -656,7 +682,12 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     // shared memory, but output row m depends on row m of A alone and rows
     // at or past M are never stored.
     // (An MN-major A keeps its 128-wide box: its rows are k, its columns m.)
-    const int a_rows = (M >= BM || a_mn) ? BM : static_cast<int>((M + 15) / 16 * 16);
+    // Per-tensor products with a K-major A take 256 x 256 tiles (two MMAs share
+    // each B tile) when those tiles still fill nine tenths of the SMs.
+    const int64_t tall_tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256);
+    const bool tall = !fine && !narrow && !a_mn && M >= 2 * BM && tall_tiles * 10 >= 9LL * sm_count();
+    const int mt = tall ? 2 * BM : BM;
+    const int a_rows = tall ? mt : (M >= BM || a_mn) ? BM : static_cast<int>((M + 15) / 16 * 16);
     CUtensorMap ma, mbm;
     memset(&ma, 0, sizeof(ma));
     memset(&mbm, 0, sizeof(mbm));
@@ -672,7 +703,7 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     p.N = static_cast<int>(N);
     p.K = static_cast<int>(K);
     p.num_kb = static_cast<int>((K + BK - 1) / BK);
-    p.tiles_m = static_cast<int>((M + BM - 1) / BM);
+    p.tiles_m = static_cast<int>((M + mt - 1) / mt);
     p.tiles_n = static_cast<int>((N + bn - 1) / bn);
     p.sa = sa;
     p.sb = sb;
@@ -689,6 +720,7 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     const uint32_t idesc = instr_desc(fa, fb, bn, a_mn, b_mn);
     cudaError_t e;
     if (narrow) e = launch_dtype<128>(fine, yt, ma, mbm, p, idesc, s);
+    else if (tall) e = launch_tall(yt, ma, mbm, p, idesc, s);
     else e = launch_dtype<256>(fine, yt, ma, mbm, p, idesc, s);
     return cuda_status(e);
 }

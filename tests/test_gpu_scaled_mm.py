@@ -367,3 +367,17 @@ def test_scaled_mm_helper_takes_either_layout(fp8q, orc):
     for lhs in (A, At):
         for rhs in (W.t(), Wt):
             np.testing.assert_array_equal(host(fp8q.scaled_mm(lhs, rhs, sa, sb)), want)
+
+
+@pytest.mark.parametrize("M,N,K", [(257, 300, 272), (300, 512, 128), (520, 768, 384)])
+@pytest.mark.parametrize("yt", [F32, BF16])
+def test_exact_grid_tall_tiles(fp8q, orc, M, N, K, yt):
+    """Per-tensor products of at least 256 rows run 256 x 256 tiles (two MMAs per k step
+    sharing the B tile); ragged last row tiles, partial second halves, bias."""
+    g = np.random.default_rng(M * 3 + N + K + yt)
+    a, b = grid_codes(g, (M, K), E5M2), grid_codes(g, (N, K), E4M3FN)
+    bias_t, bias = t_bias(g, N, yt)
+    out = run(fp8q, False, a, E5M2, b, E4M3FN, 0.0123, 3.5, bias_t, yt)
+    want = oracle_rounded(orc, False, a, E5M2, b, E4M3FN, 0.0123, 3.5, bias, yt)
+    bad = ~bits_equal(host(out), want, yt)
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
