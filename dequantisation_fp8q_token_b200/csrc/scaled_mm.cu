@@ -51,7 +51,6 @@ constexpr int BK = 128;         // k per stage: one 128-byte swizzle row, one sc
 constexpr int kTmemCols = 512;  // all of TMEM, split into kAccBufs accumulators
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr int kABytes = BM * BK;
 constexpr int kGroupM = 32;     // row-tiles per raster band
 
 // Tile shapes.  BN = 256: 128 x 256 tiles, two TMEM accumulators (with
@@ -387,8 +386,14 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort)) { fail = kTimeoutProducer; break; }
                     const uint32_t fb = full0 + 8 * stage;
                     mbar_arrive_expect_tx(fb, static_cast<uint32_t>(p.stage_tx));
-                    if (p.a_mn) tma_load_2d(smem_u32(sA + stage * kATile), &map_a, mb * BM, kb * BK, fb);
-                    else tma_load_2d(smem_u32(sA + stage * kATile), &map_a, kb * BK, mb * MT_, fb);
+                    if (p.a_mn) {
+#pragma unroll
+                        for (int sub = 0; sub < kSub; ++sub)
+                            tma_load_2d(smem_u32(sA + stage * kATile + sub * kMnAtomBytes), &map_a,
+                                        mb * MT_ + sub * BM, kb * BK, fb);
+                    } else {
+                        tma_load_2d(smem_u32(sA + stage * kATile), &map_a, kb * BK, mb * MT_, fb);
+                    }
                     if (p.b_mn) {
 #pragma unroll
                         for (int h = 0; h < BN / 128; ++h)
@@ -435,9 +440,9 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                         const uint64_t bd = p.b_mn ? smem_desc_mn_sw128(b0 + 4096 * j) : smem_desc_sw128(b0 + 32 * j);
 #pragma unroll
                         for (int sub = 0; sub < kSub; ++sub) {
-                            // sub-tile sub: rows 128 sub .. of A (K-major when kSub > 1), its own accumulator
+                            // sub-tile sub: rows 128 sub .. of A, its own accumulator
                             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((acc + sub) * BN);
-                            const uint64_t ad = p.a_mn ? smem_desc_mn_sw128(a0 + 4096 * j)
+                            const uint64_t ad = p.a_mn ? smem_desc_mn_sw128(a0 + sub * kMnAtomBytes + 4096 * j)
                                                        : smem_desc_sw128(a0 + sub * BM * BK + 32 * j);
                             mma_f8f6f4(d_tmem, ad, bd, idesc, accumulate);
                         }
@@ -682,10 +687,10 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     // shared memory, but output row m depends on row m of A alone and rows
     // at or past M are never stored.
     // (An MN-major A keeps its 128-wide box: its rows are k, its columns m.)
-    // Per-tensor products with a K-major A take 256 x 256 tiles (two MMAs share
-    // each B tile) when those tiles still fill nine tenths of the SMs.
+    // Per-tensor products take 256 x 256 tiles (two MMAs share each B tile)
+    // when those tiles still fill nine tenths of the SMs.
     const int64_t tall_tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256);
-    const bool tall = !fine && !narrow && !a_mn && M >= 2 * BM && tall_tiles * 10 >= 9LL * sm_count();
+    const bool tall = !fine && !narrow && M >= 2 * BM && tall_tiles * 10 >= 9LL * sm_count();
     const int mt = tall ? 2 * BM : BM;
     const int a_rows = tall ? mt : (M >= BM || a_mn) ? BM : static_cast<int>((M + 15) / 16 * 16);
     CUtensorMap ma, mbm;
@@ -694,7 +699,7 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     if (K > 0) {
         // K-major: [M][K] with boxes of rows x 128 k; MN-major: [K][M] with
         // boxes of 128 k x 128 m (B likewise, two boxes for 256 columns)
-        const bool ok_a = a_mn ? make_map(&ma, a, K, M, BK) : make_map(&ma, a, M, K, a_rows);
+        const bool ok_a = a_mn ? make_map(&ma, a, K, M, BK) : make_map(&ma, a, M, K, a_rows);   // MN-major: 128-wide boxes
         const bool ok_b = b_mn ? make_map(&mbm, b, K, N, BK) : make_map(&mbm, b, N, K, bn);
         if (!ok_a || !ok_b) return FP8Q_ERR_CUDA;
     }
