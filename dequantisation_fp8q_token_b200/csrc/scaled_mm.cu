@@ -246,6 +246,29 @@ __device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
                  :: "memory");
 }
 
+// 32 lanes x 32 consecutive columns, issued without waiting (completed by
+// tmem_wait32 on the same registers)
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32"
+                 " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+                   "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+                   "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait32(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                   "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                   "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // epilogue stores: 32 consecutive columns of one row of D
 // ---------------------------------------------------------------------------
@@ -488,29 +511,40 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     if (!ok) { fail = kTimeoutEpilogue; break; }
                     tc_fence_after();
                 }
-#pragma unroll 1
-                for (int sub = 0; sub < kSub; ++sub) {
-                    const int srow = row + sub * BM;
-#pragma unroll 1
-                    for (int c = 0; c < kColsPerWarp / 32; ++c) {
-                        float v[32];
-                        const int col0 = col_base + c * 32;
-                        if (p.num_kb > 0) {
-                            tmem_ld32(tmem_base + lane_addr +
-                                          static_cast<uint32_t>((acc + sub) * BN + cgrp * kColsPerWarp + c * 32), v);
-                        } else {
+                // kSub x kColsPerWarp / 32 chunks of 32 columns, double-buffered:
+                // the load of chunk j + 1 is in flight while chunk j is scaled
+                // and stored
+                constexpr int kChunks = kSub * (kColsPerWarp / 32);
+                const uint32_t col_addr = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + cgrp * kColsPerWarp);
+                uint32_t r0[32], r1[32];
+                if (p.num_kb > 0) {
+                    tmem_ld32_async(col_addr, r0);
+                    tmem_wait32(r0);
+                } else {
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-                        }
+                    for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0u;
+                }
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], scale);
-                        if (p.bias) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (col0 + i < p.N) v[i] = __fadd_rn(v[i], load_bias<YT>(p.bias, col0 + i));
-                        }
-                        if (srow < p.M && col0 < p.N) store_chunk<YT>(p, srow, col0, v);
+                for (int j = 0; j < kChunks; ++j) {
+                    const int sub = j / (kColsPerWarp / 32), c = j % (kColsPerWarp / 32);
+                    uint32_t (&cur)[32] = (j & 1) ? r1 : r0;
+                    uint32_t (&nxt)[32] = (j & 1) ? r0 : r1;
+                    if (p.num_kb > 0 && j + 1 < kChunks) {
+                        const int sub1 = (j + 1) / (kColsPerWarp / 32), c1 = (j + 1) % (kColsPerWarp / 32);
+                        tmem_ld32_async(col_addr + static_cast<uint32_t>(sub1 * BN + c1 * 32), nxt);
                     }
+                    const int srow = row + sub * BM;
+                    const int col0 = col_base + c * 32;
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(cur[i]), scale);
+                    if (p.bias) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (col0 + i < p.N) v[i] = __fadd_rn(v[i], load_bias<YT>(p.bias, col0 + i));
+                    }
+                    if (srow < p.M && col0 < p.N) store_chunk<YT>(p, srow, col0, v);
+                    if (p.num_kb > 0 && j + 1 < kChunks) tmem_wait32(nxt);
                 }
                 if (p.num_kb > 0) {
                     tc_fence_before();
