@@ -558,6 +558,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 #pragma unroll
                 for (int i = 0; i < kColsPerWarp / 2; ++i) accum[i] = make_float2(0.0f, 0.0f);
                 const bool row_ok = row < p.M;
+                const bool warp_rows_live = row - lane < p.M;    // the warp's first row
                 const bool blk_ok = col_base < p.N;
                 const float* sa_row = p.sa + static_cast<int64_t>(row_ok ? row : 0) * p.sa_ld;
                 const float* sb_row = p.sb + static_cast<int64_t>(blk_ok ? col_base / 128 : 0) * p.sb_ld;
@@ -574,6 +575,14 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
                     if (!ok) { fail = kTimeoutEpilogue; break; }
                     tc_fence_after();
+                    if (!warp_rows_live) {
+                        // every row of this warp is past M (decode-sized
+                        // products): nothing to fold, only the handshake
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+                        if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
+                        continue;
+                    }
                     // 8 chunks of 16 columns, double-buffered: the load of chunk
                     // c + 1 is in flight while chunk c is folded in with packed
                     // fused multiply-adds (each lane the same as __fmaf_rn)

@@ -314,6 +314,8 @@ def test_linear_fp8_blockwise_matches_the_oracle_composition(fp8q, orc):
 @pytest.mark.parametrize("fine", [False, True], ids=["tensor", "blockwise"])
 @pytest.mark.parametrize("M,N,K", [(64, 3000, 512),       # decode-sized rows: 24 tiles 128 columns wide
                                    (1, 18432, 256),       # one token against a full weight row count
+                                   (33, 3000, 2560),      # a 48-row A box; 20 k-blocks wrap the 6-stage ring
+                                   (64, 1000, 1408),      # a 64-row A box, 11 k-blocks
                                    (100, 40000, 128)])    # enough columns to keep 256-wide tiles
 def test_exact_grid_small_m(fp8q, orc, fine, M, N, K):
     g = np.random.default_rng(M + N + K + fine)
