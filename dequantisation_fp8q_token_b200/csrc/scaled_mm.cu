@@ -505,9 +505,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             const int col_base = nb * BN + cgrp * kColsPerWarp;
             if (!FINE) {
                 if (p.num_kb > 0) {
-                    bool ok = true;
-                    if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort);
-                    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort));
                     if (!ok) { fail = kTimeoutEpilogue; break; }
                     tc_fence_after();
                 }
@@ -570,9 +568,8 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                         sa_next = row_ok ? __ldg(sa_row + kb + 1) : 0.0f;
                         sb_next = blk_ok ? __ldg(sb_row + kb + 1) : 0.0f;
                     }
-                    bool ok = true;
-                    if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort);
-                    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                    // every lane polls; the vote keeps the warp converged
+                    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort));
                     if (!ok) { fail = kTimeoutEpilogue; break; }
                     tc_fence_after();
                     if (!warp_rows_live) {
