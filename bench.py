@@ -504,8 +504,9 @@ class MatmulWorkload:
 
     def time_linear(self, steps: int, warmup: int, device):
         """ColossalAI linear_fp8 forward + backward on bf16 x[4096, 7168], w[18432, 7168] and a bias
-        (three fp8 products of 2*M*N*K each, the casts, three operand transposes and the bias
-        gradient)."""
+        (three fp8 products of 2*M*N*K each, the three per-tensor casts and the bias gradient).
+        The gradients are cleared before each backward, as a training step's zero_grad does, so
+        no accumulation into .grad runs in the timed region."""
         f = self.fp8q
         g = torch.Generator(device=device).manual_seed(20261207)
         m, k = self.q.shape
@@ -515,6 +516,7 @@ class MatmulWorkload:
         go = (torch.randn((m, self.n), generator=g, device=device) * 1e-3).to(torch.bfloat16)
 
         def step():
+            x.grad = w.grad = b.grad = None
             y = f.linear_fp8(x, w, b)
             y.backward(go)
         ms, clk = self._timed(step, steps, warmup, device)

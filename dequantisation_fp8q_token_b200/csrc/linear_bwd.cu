@@ -6,10 +6,11 @@
 //                      choosing, so that a token count that is not a multiple
 //                      of 16 still gives a legal row pitch to the products
 //   sum_rows_kernel    bias_grad = out_grad.sum(0): out[c] = T(sum_r x[r][c]),
-//                      summed in fp32 in a fixed order (each thread owns two
-//                      columns and walks its share of the rows in ascending
-//                      order; the 16 warps' partial sums are then added in
-//                      warp order), so the result does not depend on timing.
+//                      summed in fp32 in a fixed order (a column's rows are
+//                      split into 64 interleaved subsets, r % 64, each summed
+//                      in ascending row order; the 64 partial sums are then
+//                      added in subset order), so the result does not depend
+//                      on timing.
 // Both are streaming passes bound by HBM bandwidth.
 #include "fp8q_device.cuh"
 #include "fp8q_internal.h"
@@ -107,10 +108,14 @@ transpose_kernel(const uint8_t* __restrict__ src, int64_t rows, int64_t cols, ui
 }
 
 // ---------------------------------------------------------------------------
-// column sums: one CTA per 64 columns, 16 warps splitting the rows
+// column sums
 // ---------------------------------------------------------------------------
-constexpr int kSWarps = 16;
-constexpr int kSCols = 64;             // columns per CTA: 2 per lane
+// Rows are split into kSubsets interleaved subsets (row r belongs to subset
+// r % kSubsets); each subset is summed in ascending row order and the
+// partial sums are added in subset order.  Both kernels below keep exactly
+// this order.
+constexpr int kSubsets = 64;
+constexpr int kSThreads = 512;
 
 template <int XT> __device__ __forceinline__ float load_elem(const void* x, int64_t i) {
     if constexpr (XT == kF32) return __ldg(static_cast<const float*>(x) + i);
@@ -122,29 +127,84 @@ template <int XT> __device__ __forceinline__ void store_elem(void* y, int64_t i,
     else if constexpr (XT == kF16) static_cast<__half*>(y)[i] = __float2half_rn(v);
     else static_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(v);
 }
-
-template <int XT>
-__global__ void __launch_bounds__(32 * kSWarps)
-sum_rows_kernel(const void* __restrict__ x, int64_t rows, int64_t cols, void* __restrict__ out) {
-    __shared__ float part[kSWarps][kSCols];
-    pdl_begin();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * kSCols + 2 * lane;
-    float s0 = 0.0f, s1 = 0.0f;
-    for (int64_t r = warp; r < rows; r += kSWarps) {
-        const int64_t i = r * cols + c;
-        if (c < cols) s0 = __fadd_rn(s0, load_elem<XT>(x, i));
-        if (c + 1 < cols) s1 = __fadd_rn(s1, load_elem<XT>(x, i + 1));
-    }
-    part[warp][2 * lane] = s0;
-    part[warp][2 * lane + 1] = s1;
-    __syncthreads();
-    if (threadIdx.x < kSCols) {
-        float s = 0.0f;
+// the VEC elements of a 16-byte word, widened exactly to fp32
+template <int XT> __device__ __forceinline__ void widen16(const uint4& w, float (&v)[16 / (XT == kF32 ? 4 : 2)]) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    if constexpr (XT == kF32) {
 #pragma unroll
-        for (int w = 0; w < kSWarps; ++w) s = __fadd_rn(s, part[w][threadIdx.x]);
-        const int64_t cc = static_cast<int64_t>(blockIdx.x) * kSCols + threadIdx.x;
-        if (cc < cols) store_elem<XT>(out, cc, s);
+        for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(u[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) widen2<XT>(u[i], v[2 * i], v[2 * i + 1]);
+    }
+}
+
+// Vector path (16-byte aligned rows): a CTA owns 8 x VEC columns (64 for
+// 16-bit types, 32 for fp32); 8 threads cover one row of them with 16-byte
+// loads, so the 512 threads form 64 row lanes, one per subset.  Each lane
+// keeps kUnroll rows in flight (64 bytes per thread).
+constexpr int kUnroll = 4;
+template <int XT>
+__global__ void __launch_bounds__(kSThreads)
+sum_rows_vec_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t cols, void* __restrict__ out) {
+    constexpr int kEs = XT == kF32 ? 4 : 2;
+    constexpr int VEC = 16 / kEs;
+    constexpr int W = 8 * VEC;                          // columns per CTA
+    static_assert(kSThreads / 8 == kSubsets, "one row lane per subset");
+    __shared__ float part[kSubsets][W + 1];
+    pdl_begin();
+    const int seg = threadIdx.x & 7, lane_r = threadIdx.x >> 3;
+    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * W + seg * VEC;
+    const bool col_ok = c0 < cols;                      // cols % VEC == 0: a segment is all in or all out
+    float acc[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) acc[i] = 0.0f;
+    const int64_t pitch = cols * kEs;
+    for (int64_t r = lane_r; r < rows; r += kSubsets * kUnroll) {
+        uint4 w[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            w[u] = (col_ok && r + u * kSubsets < rows) ? ld_stream_v4(x + (r + u * kSubsets) * pitch + c0 * kEs)
+                                                        : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            if (r + u * kSubsets < rows) {
+                float v[VEC];
+                widen16<XT>(w[u], v);
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], v[i]);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) part[lane_r][seg * VEC + i] = acc[i];
+    __syncthreads();
+    if (threadIdx.x < W) {
+        float t = 0.0f;
+#pragma unroll 8
+        for (int l = 0; l < kSubsets; ++l) t = __fadd_rn(t, part[l][threadIdx.x]);
+        const int64_t cc = static_cast<int64_t>(blockIdx.x) * W + threadIdx.x;
+        if (cc < cols) store_elem<XT>(out, cc, t);
+    }
+}
+
+// Any alignment: one CTA per 8 columns, 64 row lanes x 8 columns, element loads.
+template <int XT>
+__global__ void __launch_bounds__(kSThreads)
+sum_rows_kernel(const void* __restrict__ x, int64_t rows, int64_t cols, void* __restrict__ out) {
+    __shared__ float part[kSubsets][9];
+    pdl_begin();
+    const int cl = threadIdx.x & 7, lane_r = threadIdx.x >> 3;
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * 8 + cl;
+    float acc = 0.0f;
+    if (c < cols)
+        for (int64_t r = lane_r; r < rows; r += kSubsets) acc = __fadd_rn(acc, load_elem<XT>(x, r * cols + c));
+    part[lane_r][cl] = acc;
+    __syncthreads();
+    if (threadIdx.x < 8) {
+        float t = 0.0f;
+        for (int l = 0; l < kSubsets; ++l) t = __fadd_rn(t, part[l][threadIdx.x]);
+        if (c < cols) store_elem<XT>(out, c, t);
     }
 }
 
@@ -163,13 +223,24 @@ fp8q_status launch_transpose(const uint8_t* src, int64_t rows, int64_t cols, uin
 }
 
 fp8q_status launch_sum_rows(const void* x, int xt, int64_t rows, int64_t cols, void* out, cudaStream_t s) {
-    const int64_t ctas = (cols + kSCols - 1) / kSCols;
+    const int es = xt == kF32 ? 4 : 2;
+    const int vec = 16 / es;
+    const bool vec_ok = cols % vec == 0 && reinterpret_cast<uintptr_t>(x) % 16 == 0;
+    const int64_t width = vec_ok ? 8 * vec : 8;
+    const int64_t ctas = (cols + width - 1) / width;
     if (ctas > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
-    const dim3 grid(static_cast<unsigned>(ctas)), block(32 * kSWarps);
+    const dim3 grid(static_cast<unsigned>(ctas)), block(kSThreads);
+    const uint8_t* xb = static_cast<const uint8_t*>(x);
     cudaError_t e;
-    if (xt == kF32) e = launch_kernel(sum_rows_kernel<kF32>, grid, block, s, x, rows, cols, out);
-    else if (xt == kF16) e = launch_kernel(sum_rows_kernel<kF16>, grid, block, s, x, rows, cols, out);
-    else e = launch_kernel(sum_rows_kernel<kBF16>, grid, block, s, x, rows, cols, out);
+    if (vec_ok) {
+        if (xt == kF32) e = launch_kernel(sum_rows_vec_kernel<kF32>, grid, block, s, xb, rows, cols, out);
+        else if (xt == kF16) e = launch_kernel(sum_rows_vec_kernel<kF16>, grid, block, s, xb, rows, cols, out);
+        else e = launch_kernel(sum_rows_vec_kernel<kBF16>, grid, block, s, xb, rows, cols, out);
+    } else {
+        if (xt == kF32) e = launch_kernel(sum_rows_kernel<kF32>, grid, block, s, x, rows, cols, out);
+        else if (xt == kF16) e = launch_kernel(sum_rows_kernel<kF16>, grid, block, s, x, rows, cols, out);
+        else e = launch_kernel(sum_rows_kernel<kBF16>, grid, block, s, x, rows, cols, out);
+    }
     return cuda_status(e);
 }
 

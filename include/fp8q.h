@@ -434,9 +434,10 @@ fp8q_status fp8q_transpose_fp8(const uint8_t* src, int64_t rows, int64_t cols, u
  * Column sums -- the bias gradient of ColossalAI _LinearFp8.backward,
  * out_grad.sum(0):
  *   out[c] = T(sum over r of float(x[r][c]))
- * accumulated in fp32 in a fixed order (each column's rows split into 16
- * interleaved subsets summed in ascending row order, then the 16 partial
- * sums added in subset order), so repeated calls give the same bits.
+ * accumulated in fp32 in a fixed order (each column's rows split into 64
+ * interleaved subsets, row r in subset r % 64, each summed in ascending row
+ * order, then the 64 partial sums added in subset order), so repeated calls
+ * give the same bits.
  * x: [rows][cols] of type xt; out: [cols] of type xt.  rows == 0 writes zeros.
  */
 fp8q_status fp8q_sum_rows(const void* x, fp8q_dtype xt, int64_t rows, int64_t cols, void* out,

@@ -81,7 +81,9 @@ def test_transpose_full_size_activation(fp8q, orc):
 # column sums (bias gradient)
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("yt", [F32, F16, BF16])
-@pytest.mark.parametrize("rows,cols", [(1, 1), (300, 50), (4096, 7168), (17, 130)])
+@pytest.mark.parametrize("rows,cols", [(1, 1), (300, 50), (4096, 7168), (17, 130),
+                                       (700, 72),      # 16-byte rows: a full and a partial column block
+                                       (65, 8)])       # one row past the 64 subsets
 def test_sum_rows_exact_on_integers(fp8q, orc, yt, rows, cols):
     g = np.random.default_rng(rows + cols + yt)
     x = bits_of(g.integers(-64, 65, (rows, cols)).astype(np.float32), yt)
@@ -107,6 +109,28 @@ def test_sum_rows_general_within_the_bound(fp8q, orc, yt):
     mag = np.abs(to_f64(x, yt)).sum(0)
     err = np.abs(to_f64(first, yt) - exact)
     assert np.all(err <= rows * 2.0 ** -24 * mag + ulp(exact, yt))
+
+
+@pytest.mark.parametrize("yt", [F32, BF16])
+def test_sum_rows_unaligned_base_takes_the_element_path(fp8q, orc, yt):
+    # the same rows one element into a buffer: 16-byte loads are not allowed,
+    # the element kernel keeps the same summation order
+    g = np.random.default_rng(31 + yt)
+    rows, cols = 513, 96
+    x = bits_of((g.standard_normal((rows, cols)) * 3).astype(np.float32), yt)
+    flat = np.concatenate([np.zeros(1, x.dtype), x.reshape(-1)])
+    buf = dev(flat, TORCH_T[yt]) if yt != F32 else dev(flat)
+    xa = (dev(x, TORCH_T[yt]) if yt != F32 else dev(x))
+    xu = buf[1:].view(rows, cols)
+    assert xu.data_ptr() % 16 != 0 and xa.data_ptr() % 16 == 0
+    a = torch.empty((cols,), dtype=TORCH_T[yt], device="cuda")
+    u = torch.empty((cols,), dtype=TORCH_T[yt], device="cuda")
+    fp8q.fp8q_sum_rows(xa, a)
+    fp8q.fp8q_sum_rows(xu, u)
+    np.testing.assert_array_equal(host(u), host(a))
+    exact = orc.sum_rows(x, yt)
+    mag = np.abs(to_f64(x, yt)).sum(0)
+    assert np.all(np.abs(to_f64(host(a), yt) - exact) <= rows * 2.0 ** -24 * mag + ulp(exact, yt))
 
 
 def test_sum_rows_zero_rows_writes_zeros(fp8q):
