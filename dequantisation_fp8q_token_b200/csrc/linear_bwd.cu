@@ -36,27 +36,24 @@ __device__ __forceinline__ void transpose4x4(const uint32_t (&a)[4], uint32_t (&
     o[3] = __byte_perm(t1, t3, 0x7632);
 }
 
-// Shared-memory layouts of the two 128 x 128-byte tiles, as 32 words per row
-// in 8 chunks of 16 bytes.  Both permute whole chunks within a row, so rows
-// move in and out with 16-byte accesses:
-//   source tile:      chunk c of row r sits at chunk c ^ 2 * ((r / 4) % 4)
-//   transposed tile:  chunk c of row d sits at chunk c ^ (d / 4) % 8
-// With the block mapping of the transpose step (lane = 4 * (bc % 8) +
-// br % 4), each warp's four 4-byte reads of a block column and its four
-// 4-byte writes of the transposed words each touch 32 different banks.
-__device__ __forceinline__ int ta_word(int r, int w) { return 4 * ((w >> 2) ^ (2 * ((r >> 2) & 3))) + (w & 3); }
-__device__ __forceinline__ int tb_word(int d, int w) { return 4 * ((w >> 2) ^ ((d >> 2) & 7)) + (w & 3); }
+// The transposed tile in shared memory: 128 destination rows of 32 words.
+// Word w of row d sits at word w ^ (4 * ((d / 16) % 8)): the XOR moves whole
+// groups of four words, so a row still leaves as 16-byte chunks, and the
+// word stores of the transpose step (a warp = 4 source row quads x the 8
+// chunks of a row) touch 32 different banks.
+__device__ __forceinline__ int tb_word(int d, int w) { return w ^ (4 * ((d >> 4) & 7)); }
 
 // One CTA per 128 x 128 tile of the destination [cols][ld] (the padding
 // columns r in [rows, ld) are written as zeros).  Interior tiles with 16-byte
-// aligned pitches and bases: rows of the source tile come in with 16-byte
-// loads, 4 x 4 byte blocks are transposed in registers, and rows of the
-// destination tile go out with 16-byte stores.  Other tiles move bytes.
+// aligned pitches and bases: each thread loads a 4-row x 16-byte block of the
+// source straight into registers, transposes its four 4 x 4 byte blocks there,
+// and stores the sixteen 4-byte words into the transposed tile; after one
+// barrier the destination rows leave as 16-byte stores.  Other tiles move
+// bytes.
 __global__ void __launch_bounds__(kTThreads)
 transpose_kernel(const uint8_t* __restrict__ src, int64_t rows, int64_t cols, uint8_t* __restrict__ dst,
                  int64_t ld, int64_t tiles_r, int vec_ok) {
-    __shared__ __align__(16) uint32_t ta[kT][kTW];         // source tile, swizzled chunks
-    __shared__ __align__(16) uint32_t tb[kT][kTW];         // transposed tile, swizzled chunks
+    __shared__ __align__(16) uint32_t tb[kT][kTW];         // transposed tile, swizzled words
     pdl_begin();
     const int64_t t = blockIdx.x;
     const int64_t tr = t % tiles_r;            // tile index along src rows (= dst columns)
@@ -64,38 +61,37 @@ transpose_kernel(const uint8_t* __restrict__ src, int64_t rows, int64_t cols, ui
     const int64_t r0 = tr * kT, c0 = tc * kT;
     const int tid = threadIdx.x;
     if (vec_ok && r0 + kT <= rows && c0 + kT <= cols) {
+        // thread -> (row quad q: source rows 4q..4q+3, chunk j: source bytes 16j..16j+15);
+        // a warp holds 4 row quads x the 8 chunks of a row, so each load
+        // instruction reads four whole 128-byte lines
+        const int lane = tid & 31, wid = tid >> 5;
+        const int q = 4 * wid + (lane >> 3);
+        const int j = lane & 7;
+        uint4 v[4];
 #pragma unroll
-        for (int k = 0; k < kT * (kT / 16) / kTThreads; ++k) {       // 128 rows x 8 chunks of 16 bytes
-            const int i = tid + k * kTThreads;
-            const int r = i >> 3, seg = i & 7;
-            const uint4 v = ld_stream_v4(src + (r0 + r) * cols + c0 + 16 * seg);
-            *reinterpret_cast<uint4*>(&ta[r][ta_word(r, 4 * seg)]) = v;
-        }
-        __syncthreads();
+        for (int k = 0; k < 4; ++k) v[k] = ld_stream_v4(src + (r0 + 4 * q + k) * cols + c0 + 16 * j);
 #pragma unroll
-        for (int k = 0; k < (kT / 4) * (kT / 4) / kTThreads; ++k) {  // 32 x 32 blocks of 4 x 4 bytes
-            const int i = tid + k * kTThreads;
-            const int lane = i & 31, wid = i >> 5;
-            const int br = 4 * (wid & 7) + (lane & 3);               // block row: source rows 4 br ..
-            const int bc = 8 * (wid >> 3) + (lane >> 2);             // block column: source columns 4 bc ..
-            uint32_t a[4], o[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) a[q] = ta[4 * br + q][ta_word(4 * br + q, bc)];
+        for (int w = 0; w < 4; ++w) {                            // source bytes 16j + 4w .. 16j + 4w + 3
+            const uint32_t a[4] = {(&v[0].x)[w], (&v[1].x)[w], (&v[2].x)[w], (&v[3].x)[w]};
+            uint32_t o[4];
             transpose4x4(a, o);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tb[4 * bc + j][tb_word(4 * bc + j, br)] = o[j];
+            for (int k = 0; k < 4; ++k) {
+                const int d = 16 * j + 4 * w + k;                // destination row in the tile
+                tb[d][tb_word(d, q)] = o[k];                     // bytes = source rows 4q .. 4q + 3
+            }
         }
         __syncthreads();
 #pragma unroll
         for (int k = 0; k < kT * (kT / 16) / kTThreads; ++k) {       // 128 dst rows x 8 chunks of 16 bytes
             const int i = tid + k * kTThreads;
             const int d = i >> 3, seg = i & 7;
-            const uint4 v = *reinterpret_cast<const uint4*>(&tb[d][tb_word(d, 4 * seg)]);
-            st_v4(dst + (c0 + d) * ld + r0 + 16 * seg, v);
+            const uint4 w = *reinterpret_cast<const uint4*>(&tb[d][tb_word(d, 4 * seg)]);
+            st_v4(dst + (c0 + d) * ld + r0 + 16 * seg, w);
         }
         return;
     }
-    uint8_t* tile = reinterpret_cast<uint8_t*>(ta);          // bytes [kT][kT]
+    uint8_t* tile = reinterpret_cast<uint8_t*>(tb);          // bytes [kT][kT]
     for (int i = tid; i < kT * kT; i += kTThreads) {
         const int r = i / kT, c = i % kT;
         tile[r * kT + c] = (r0 + r < rows && c0 + c < cols) ? src[(r0 + r) * cols + c0 + c] : 0;
