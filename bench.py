@@ -981,6 +981,12 @@ def _profile_case(name, fp8q, device):
             wt = torch.empty((k, w.shape[0]), dtype=torch.uint8, device=device)
             return (lambda: fp8q.fp8q_transpose_fp8(w, wt, w.shape[0])), 2 * w.numel()
         return (lambda: fp8q.fp8q_scaled_mm_blockwise(q, sa, w, sb, out)), flops
+    if name == "sum_rows":
+        # the bias gradient of linear_fp8's backward: column sums of bf16 g[4096, 18432] (151 MB)
+        m, n = workloads.C2_SHAPE[0], workloads.MM_W_SHAPE[0]
+        x = _to_dev(workloads.to_bf16_bits(g.standard_normal((m, n), dtype=np.float32)), device, bf16)
+        out = torch.empty((n,), dtype=bf16, device=device)
+        return (lambda: fp8q.fp8q_sum_rows(x, out)), x.numel() * 2 + n * 2
     if name in ("records_pack", "records_unpack"):
         # the fp8 all-gather's device work for 8 ranks of 16 Mi bf16 each
         # (32 MiB per rank): pack = each rank's per-tensor cast into its
@@ -1005,7 +1011,7 @@ def _profile_case(name, fp8q, device):
 
 PROFILE_CASES = ["per_token_4x", "cast_from_fp8_4x", "block_dequant", "grouped_16", "grouped_72", "per_channel",
                  "per_tensor", "records_pack", "records_unpack", "scaled_mm", "scaled_mm_blockwise",
-                 "scaled_mm_blockwise_m1", "transpose_weight"]
+                 "scaled_mm_blockwise_m1", "transpose_weight", "sum_rows"]
 
 
 def run_profile_case(name, iters):
