@@ -138,8 +138,8 @@ template <int XT> __device__ __forceinline__ void widen16(const uint4& w, float 
 // Vector path (16-byte aligned rows): a CTA owns 8 x VEC columns (64 for
 // 16-bit types, 32 for fp32); 8 threads cover one row of them with 16-byte
 // loads, so the 512 threads form 64 row lanes, one per subset.  Each lane
-// keeps kUnroll rows in flight (64 bytes per thread).
-constexpr int kUnroll = 4;
+// keeps kUnroll rows in flight (128 bytes per thread).
+constexpr int kUnroll = 8;
 template <int XT>
 __global__ void __launch_bounds__(kSThreads)
 sum_rows_vec_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t cols, void* __restrict__ out) {
