@@ -148,3 +148,84 @@ def test_per_tensor_and_record_above_2_32(fp8q, orc):
 def _release_memory():
     yield
     torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# the fp8 products and linear_fp8's backward helpers
+# ---------------------------------------------------------------------------
+def _grid_codes_dev(shape, gen):
+    """e4m3fn codes whose values are multiples of 1/8 with magnitude <= 4, drawn on the
+    device: every partial sum of a product of such operands over K = 32 is an fp32 number."""
+    codes = workloads.finite_e4m3fn_codes()
+    v = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    keep = torch.from_numpy(codes[(np.abs(v) <= 4) & (v * 8 == np.round(v * 8))]).cuda()
+    idx = torch.randint(0, keep.numel(), shape, generator=gen, device="cuda")
+    return keep[idx]
+
+
+@pytest.mark.parametrize("fine", [False, True], ids=["tensor", "blockwise"])
+def test_scaled_mm_output_above_2_32(fp8q, orc, fine):
+    """D [65552, 65552] bf16 (4,297,064,704 elements) from K = 32 exact-grid operands, with a
+    bias: the sampled rows (the first, those holding elements 2^31 and 2^32, the last) equal
+    the oracle's single-precision product bit for bit."""
+    M = N = 65552
+    K = 32
+    gen = torch.Generator(device="cuda").manual_seed(9107 + fine)
+    a = _grid_codes_dev((M, K), gen)
+    b = _grid_codes_dev((N, K), gen)
+    bias = (torch.randint(-512, 512, (N,), generator=gen, device="cuda") / 64.0).to(torch.bfloat16)
+    d = DevGuarded((M, N), torch.bfloat16)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if fine:
+        sa = torch.exp(torch.randn((M, 1), generator=gen, device="cuda") * 0.5 - 2.0)
+        sb = torch.exp(torch.randn((-(-N // 128), 1), generator=gen, device="cuda") * 0.5 - 2.0)
+        fp8q.fp8q_scaled_mm_blockwise(a, sa, b, sb, d.t, bias, status=st)
+    else:
+        sa = torch.tensor([0.375], device="cuda")
+        sb = torch.tensor([1.25], device="cuda")
+        fp8q.fp8q_scaled_mm(a, b, sa, sb, d.t, bias, status=st)
+    d.check()
+    assert int(st.item()) == 0
+    b_h = host(b)
+    bias_h = bias.float().cpu().numpy()
+    for r0, r1 in _sample_rows(N, M):
+        a_h = host(a[r0:r1])
+        if fine:
+            want = orc.scaled_mm_blockwise_rounded(a_h, E4M3FN, host(sa[r0:r1]), b_h, E4M3FN, host(sb),
+                                                   bias=bias_h, yt=BF16)
+        else:
+            want = orc.scaled_mm_rounded(a_h, E4M3FN, b_h, E4M3FN, 0.375, 1.25, bias=bias_h, yt=BF16)
+        np.testing.assert_array_equal(_bits(d.t[r0:r1]), want, err_msg=f"rows {r0}-{r1}")
+
+
+def test_transpose_above_2_32(fp8q, orc):
+    """uint8 [65552, 65552] (4.3 GB) transposed: the destination rows that start before 2^31,
+    past 2^31 and past 2^32 bytes, and the last ones, against the oracle's transpose of the
+    same source columns."""
+    R = C = 65552
+    gen = torch.Generator(device="cuda").manual_seed(9108)
+    src = torch.randint(0, 256, (R, C), generator=gen, device="cuda", dtype=torch.uint8)
+    dst = DevGuarded((C, R), torch.uint8)
+    fp8q.fp8q_transpose_fp8(src, dst.t, R)
+    dst.check()
+    for c0, c1 in _sample_rows(R, C):
+        cols = torch.arange(c0, c1, device="cuda")
+        want = orc.transpose_u8(host(src[:, cols]))
+        np.testing.assert_array_equal(host(dst.t[c0:c1]), want, err_msg=f"destination rows {c0}-{c1}")
+
+
+def test_sum_rows_above_2_32(fp8q, orc):
+    """bf16 [1,048,600, 4104] (4,303,454,400 elements) of integers in [-8, 8]: every partial
+    sum is an fp32 integer, so the column sums are exact in any order and equal the oracle's
+    binary64 sums rounded once to bf16; sampled columns include the partial last block."""
+    R, C = 1_048_600, 4104
+    gen = torch.Generator(device="cuda").manual_seed(9109)
+    x = torch.randint(-8, 9, (R, C), generator=gen, device="cuda", dtype=torch.int8).to(torch.bfloat16)
+    out = DevGuarded((C,), torch.bfloat16)
+    fp8q.fp8q_sum_rows(x, out.t)
+    out.check()
+    for c0, c1 in [(0, 8), (2048, 2056), (4040, 4104)]:
+        cols = torch.arange(c0, c1, device="cuda")
+        exact = orc.sum_rows(host(x[:, cols]), BF16)
+        want = torch.from_numpy(exact.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        np.testing.assert_array_equal(_bits(out.t[c0:c1]), want, err_msg=f"columns {c0}-{c1}")
