@@ -1,8 +1,10 @@
 // scaled_mm.cu -- fp8 x fp8 matrix products on the sm_100a tensor cores.
 //
 // Two products of the same shape, D[M][N] = A[M][K] * B[N][K]^T, both
-// operands fp8 codes stored K-contiguous (A: activations, B: a weight as it
-// is stored, [out features][in features]):
+// operands fp8 codes (A: activations, B: a weight as it is stored, [out
+// features][in features]), each stored K-contiguous or, for the per-tensor
+// product, MN-contiguous ([K][M] / [K][N] row-major: the transposed operands
+// of linear_fp8's backward, read where they lie):
 //   per-tensor scales (ColossalAI colossalai/quantization/fp8.py,
 //     _LinearFp8.forward: torch._scaled_mm with the scale_inv of each operand)
 //       D[m][n] = T(fl(acc[m][n] * fl(sa * sb)) + bias[n])
@@ -21,16 +23,21 @@
 //               128 x BN fp32 TMEM accumulators and commits each stage back
 //               to the producer and each finished accumulator to the epilogue
 //   warps 2-9   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32 * (w % 4) .. + 31, column group (w - 2) / 4),
-//               scaling, bias, conversion, 32-byte stores.  With fine-grained
-//               scales the MMA warp commits every 128-deep k-block into a
-//               fresh accumulator and the epilogue folds it into registers
-//               with that block's scale (packed fp32x2 FMAs, TMEM loads
-//               double-buffered in 16-column chunks), while the tensor
-//               cores fill the other accumulators.
-// Tiles are 128 x BN of D (see Shape), visited in bands of 32 row-tiles so
-// that the CTAs working at one time share A and B tiles in L2.  A product of
-// fewer than 128 rows loads only its rows of A (rounded up to 16).
+//               lanes 32 * (w % 4) .. + 31, column group (w - 2) / 4), every
+//               lane polling the accumulator's barrier; scaling, bias,
+//               conversion, 32-byte stores (TMEM loads double-buffered in
+//               32-column chunks).  With fine-grained scales the MMA warp
+//               commits every 128-deep k-block into a fresh accumulator and
+//               the epilogue folds it into registers with that block's scale
+//               (packed fp32x2 FMAs, TMEM loads double-buffered in 16-column
+//               chunks; warps whose rows all lie past M only take part in the
+//               handshake), while the tensor cores fill the other
+//               accumulator.
+// Tiles are 128 x BN of D, or 256 x 256 for large per-tensor products (two
+// M 128 MMAs per k step share the B tile; see Shape), visited in bands of 32
+// row-tiles so that the CTAs working at one time share A and B tiles in L2.
+// A product of fewer than 128 rows loads only its rows of A (rounded up to
+// 16).
 //
 // Every wait on an mbarrier is bounded (a few seconds of global time).  A
 // wait that runs out sets a flag in shared memory that ends the other roles'
