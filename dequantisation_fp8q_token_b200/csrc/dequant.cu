@@ -175,10 +175,18 @@ __device__ __forceinline__ void dequant_tile(const DqDesc& D, int gb, int gb_shi
     const int64_t cols = D.cols;
     const int64_t rows = D.rows;
     const int64_t c = ((int64_t)tc * 32 + lane) * V;  // first column of this thread's chunk
-    if (c >= cols) return;
     const int64_t r0 = tr * kRowsPerTile + warp;
     const uint8_t* q = D.q;
     const float* s = D.s;
+    if (c < cols) {
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const int64_t r = r0 + (int64_t)k * kDqWarps;
+            if (r < rows) prefetch_l2(q + r * cols + c);
+        }
+    }
+    pdl_wait();
+    if (c >= cols) return;
     Chunk codes[kUnroll];
 #pragma unroll
     for (int k = 0; k < kUnroll; ++k) {
@@ -210,7 +218,7 @@ __device__ __forceinline__ void dequant_tile(const DqDesc& D, int gb, int gb_shi
 
 template <int FMT, int YT, int GRAN, int N>
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(const __grid_constant__ DqParams<N> p) {
-    pdl_begin();
+    pdl_trigger();     // the tile's codes are prefetched into L2 before pdl_wait (in dequant_tile)
     const int64_t tile = blockIdx.x;
     int lo = 0;
     if (N > 1) {

@@ -46,6 +46,29 @@ __device__ __forceinline__ void pdl_begin() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 #endif
 }
+// The same in two halves, for kernels that warm L2 with their first input
+// lines in between (prefetch_l2 / prefetch_l2_bulk): a prefetch brings a
+// line into L2 only, and L2 is where every write lands, so the loads issued
+// after pdl_wait still see all writes of the kernel before.
+__device__ __forceinline__ void pdl_trigger() {
+#if FP8Q_PDL
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+}
+__device__ __forceinline__ void pdl_wait() {
+#if FP8Q_PDL
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+// the line holding p, into L2 (p inside a live allocation)
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
+}
+// [p, p + bytes) into L2: p 16-byte aligned, bytes a positive multiple of 16,
+// the whole range inside one live allocation
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // scale rules: rule 0 divides once (fl(FMAX / amax), fl(amax / FMAX)); rule 1

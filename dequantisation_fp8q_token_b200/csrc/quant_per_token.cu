@@ -105,15 +105,23 @@ template <int XT, int FMT, int G, int VB>
 __global__ void __launch_bounds__(kTokThreads)
 per_token_vec_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
                      float* __restrict__ sinv, int64_t ngroups, int64_t nbatch, int rule) {
-    pdl_begin();
     using C = TokCfg<XT, G, VB>;
+    pdl_trigger();
+    const int64_t b0 = (int64_t)blockIdx.x * kTokUnroll;
+    if (threadIdx.x == 0) {
+        // this CTA's groups are one contiguous range of x (G * ES bytes each,
+        // a multiple of 16, from a VB-aligned base)
+        const int64_t g0 = b0 * C::GPB;
+        const int64_t g1 = (b0 + kTokUnroll) * C::GPB < ngroups ? (b0 + kTokUnroll) * C::GPB : ngroups;
+        if (g1 > g0) prefetch_l2_bulk(x + g0 * G * C::ES, (uint32_t)((g1 - g0) * G * C::ES));
+    }
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int seg = lane / C::LANES;
     const int sl = lane % C::LANES;
     const int gw = warp * C::SEGS + seg;
     Vec<VB> v[kTokUnroll][C::VPL];
-    const int64_t b0 = (int64_t)blockIdx.x * kTokUnroll;
 #pragma unroll
     for (int u = 0; u < kTokUnroll; ++u) load_batch<XT, G, VB>(x, ngroups, b0 + u, gw, sl, v[u]);
 #pragma unroll
