@@ -70,9 +70,12 @@ template <int XT, int FMT, int K, int VB>
 __global__ void __launch_bounds__(kChThreads)
 per_channel_vec_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
                        float* __restrict__ sinv, int64_t cols, int rule) {
-    pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
     constexpr int EPV = VB / ES;
+    pdl_trigger();
+    // the row (cols * ES bytes, a multiple of VB, from a VB-aligned base) into L2
+    if (threadIdx.x == 0 && cols > 0) prefetch_l2_bulk(x + (int64_t)blockIdx.x * cols * ES, (uint32_t)(cols * ES));
+    pdl_wait();
     __shared__ uint32_t sh[kChThreads / 32];
     const int64_t row = blockIdx.x;
     const int64_t nvec = cols / EPV;
@@ -167,13 +170,20 @@ per_channel_loop_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
 template <int XT, int VB>
 __global__ void __launch_bounds__(kPtThreads)
 tensor_amax_kernel(const uint8_t* __restrict__ x, int64_t numel, uint32_t* __restrict__ partials) {
-    pdl_begin();
     constexpr int ES = ElemBytes<XT>::value;
     constexpr int EPV = VB > 0 ? VB / ES : 1;
     __shared__ uint32_t sh[kPtThreads / 32];
     const int64_t nvec = numel / EPV;
     const int64_t stride = (int64_t)gridDim.x * kPtThreads;
     int64_t i = (int64_t)blockIdx.x * kPtThreads + threadIdx.x;
+    pdl_trigger();
+    if constexpr (VB > 0) {
+        // the vectors of this thread's first unrolled step into L2
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (i + u * stride < nvec) prefetch_l2(x + (i + u * stride) * VB);
+    }
+    pdl_wait();
     uint32_t bits;
     if constexpr (VB > 0) {
         // vectors from keep_from on stay in L2 for pass 2
