@@ -53,7 +53,7 @@ __all__ = [
     "exchange_records", "exchange_records_all_to_all", "exchange_payload_all_to_all", "all_gather_fp8", "all_to_all_fp8", "all_to_all_single_fp8",
     "fp8q_scaled_mm", "fp8q_scaled_mm_blockwise", "scaled_mm", "scaled_mm_blockwise", "linear_fp8",
     "linear_fp8_blockwise", "fp8q_transpose_fp8", "fp8q_sum_rows", "transpose_fp8", "fp8q_scaled_mm_ex",
-    "K_MAJOR", "MN_MAJOR",
+    "K_MAJOR", "MN_MAJOR", "fp8q_scaled_mm_wait_test",
 ]
 
 E4M3FN, E5M2 = 0, 1
@@ -143,6 +143,8 @@ def lib() -> ctypes.CDLL:
             L.fp8q_unpack_records.argtypes = [p, i32, i64, i32, i32, p, p]
             L.fp8q_scaled_mm.restype = st
             L.fp8q_scaled_mm.argtypes = [p, i32, p, i32, i64, i64, i64, p, p, p, i32, p, p, p]
+            L.fp8q_scaled_mm_wait_test.restype = st
+            L.fp8q_scaled_mm_wait_test.argtypes = [p, p, i64, i64, i64, p, p, p, p, ctypes.c_uint64, i32, p]
             L.fp8q_scaled_mm_ex.restype = st
             L.fp8q_scaled_mm_ex.argtypes = [p, i32, i32, p, i32, i32, i64, i64, i64, p, p, p, i32, p, p, p]
             L.fp8q_transpose_fp8.restype = st
@@ -777,6 +779,30 @@ def fp8q_scaled_mm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scal
         _dev_ptr(scale_a, "scale_a", dev), _dev_ptr(scale_b, "scale_b", dev), _dev_ptr(bias, "bias", dev),
         _dtype_code(out, "out"), _dev_ptr(out, "out", dev), _dev_ptr(_status_word(status), "status", dev),
         _stream(stream, dev)), "fp8q_scaled_mm")
+
+
+WAIT_PRODUCER, WAIT_MMA, WAIT_EPILOGUE, WAIT_DRAIN = 1, 2, 4, 8      # status bits of the products
+
+
+def fp8q_scaled_mm_wait_test(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
+                             out: torch.Tensor, status: torch.Tensor, wait_limit_ns: int, stall_kb: int = -1,
+                             stream=None) -> None:
+    """Test of the products' bounded waits: fp8q_scaled_mm (e4m3fn operands, bf16 out, no bias)
+    with every internal wait bounded by wait_limit_ns; stall_kb >= 0 leaves out the copies of that
+    k-block of each CTA's first tile, so that its waits run out and WAIT_* bits land in `status`."""
+    M, N, K, _, _ = _mm_operands(a, b, out, None, E4M3FN, E4M3FN)
+    dev = a.device
+    _need(scale_a, 1, "scale_a", dtype=torch.float32)
+    _need(scale_b, 1, "scale_b", dtype=torch.float32)
+    if out.dtype != torch.bfloat16:
+        raise TypeError("out must be bf16")
+    if status is None:
+        raise TypeError("status is required")
+    _check(lib().fp8q_scaled_mm_wait_test(
+        _dev_ptr(a, "a", dev), _dev_ptr(b, "b", dev), M, N, K,
+        _dev_ptr(scale_a, "scale_a", dev), _dev_ptr(scale_b, "scale_b", dev), _dev_ptr(out, "out", dev),
+        _dev_ptr(_status_word(status), "status", dev), int(wait_limit_ns), int(stall_kb),
+        _stream(stream, dev)), "fp8q_scaled_mm_wait_test")
 
 
 def fp8q_scaled_mm_blockwise(a: torch.Tensor, scale_a: torch.Tensor, b: torch.Tensor, scale_b: torch.Tensor,

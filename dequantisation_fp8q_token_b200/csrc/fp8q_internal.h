@@ -83,10 +83,13 @@ fp8q_status launch_dequant(const DequantProblem* probs, int count, int fmt, int 
 // sb are one scale each; fine = true: sa[M][sa_ld] per 1 x 128 group of A,
 // sb[ceil(N/128)][sb_ld] per 128 x 128 block of B.  Shapes validated, K % 16
 // == 0 for a K-major operand, M (N) % 16 == 0 for an MN-major A (B), a and b
-// 16-byte aligned.
+// 16-byte aligned.  wait_limit_ns: bound of every wait inside the kernel (0:
+// the default of a few seconds); stall_kb >= 0 leaves out the copies of that
+// k-block of each CTA's first tile (the test of the bounded waits).
 fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
                              const float* sa, int sa_ld, const float* sb, int sb_ld, bool fine, const void* bias,
-                             int yt, void* d, uint32_t* status, cudaStream_t s, int a_mn = 0, int b_mn = 0);
+                             int yt, void* d, uint32_t* status, cudaStream_t s, int a_mn = 0, int b_mn = 0,
+                             uint64_t wait_limit_ns = 0, int stall_kb = -1);
 
 // _LinearFp8.backward's data movements (linear_bwd.cu): validated shapes
 fp8q_status launch_transpose(const uint8_t* src, int64_t rows, int64_t cols, uint8_t* dst, int64_t ld,

@@ -84,10 +84,12 @@ template <int BN_, int MT_ = 128> struct Shape {
     static constexpr int kStageBytes = kATile + kBBytes;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment slack */ + 256 /* barriers */;
 };
-constexpr uint64_t kWaitLimitNs = 4000000000ull;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;   // every wait's default limit
 
 // status bits ORed into the caller's status word when a wait runs out
 enum : uint32_t { kTimeoutProducer = 1u, kTimeoutMma = 2u, kTimeoutEpilogue = 4u, kTimeoutDrain = 8u };
+static_assert(kTimeoutProducer == FP8Q_WAIT_PRODUCER && kTimeoutMma == FP8Q_WAIT_MMA &&
+              kTimeoutEpilogue == FP8Q_WAIT_EPILOGUE && kTimeoutDrain == FP8Q_WAIT_DRAIN, "status bits");
 
 struct Params {
     int M, N, K;
@@ -102,6 +104,8 @@ struct Params {
     int stage_tx;               // bytes one stage's TMA boxes bring
     int a_mn, b_mn;             // operand stored MN-major ([K][M] / [K][N] row-major), else K-major
     uint32_t* status;           // optional status word
+    uint64_t wait_limit_ns;     // bound of every wait (kWaitLimitNs unless a test sets it)
+    int stall_kb;               // test hook: k-block of each CTA's first tile whose copies are left out (-1: none)
 };
 
 // ---------------------------------------------------------------------------
@@ -134,22 +138,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 // Wait for the phase of `bar` with the given parity; false if the wait ran
 // out of time or another role of this CTA has already given up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (global_ns() - t0 > kWaitLimitNs) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
 }
 // the same wait, ignoring the abort flag (used to drain work in flight)
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > kWaitLimitNs) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
 }
 
@@ -413,9 +417,16 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 int mb, nb;
                 tile_coords(t, p.tiles_m, p.tiles_n, mb, nb);
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort)) { fail = kTimeoutProducer; break; }
+                    if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort, p.wait_limit_ns)) { fail = kTimeoutProducer; break; }
                     const uint32_t fb = full0 + 8 * stage;
                     mbar_arrive_expect_tx(fb, static_cast<uint32_t>(p.stage_tx));
+                    if (kb == p.stall_kb && t == static_cast<int>(blockIdx.x)) {
+                        // test hook: this stage's bytes never arrive, so every
+                        // wait that depends on them runs out
+                        ++issued;
+                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                        continue;
+                    }
                     if (p.a_mn) {
 #pragma unroll
                         for (int sub = 0; sub < kSub; ++sub)
@@ -440,7 +451,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             // every copy this thread issued has landed before the CTA exits
             for (int s = 0; s < kStages; ++s) {
                 const bool used = s < stage || issued >= kStages;
-                if (used && !mbar_wait_drain(full0 + 8 * s, s < stage ? phase : phase ^ 1u)) fail |= kTimeoutDrain;
+                if (used && !mbar_wait_drain(full0 + 8 * s, s < stage ? phase : phase ^ 1u, p.wait_limit_ns)) fail |= kTimeoutDrain;
             }
         }
     } else if (warp == 1) {
@@ -453,15 +464,15 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             for (int t = blockIdx.x; t < tiles && !fail; t += gridDim.x) {
                 if (p.num_kb == 0) continue;
                 if (!FINE) {
-                    if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort)) { fail = kTimeoutMma; break; }
+                    if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort, p.wait_limit_ns)) { fail = kTimeoutMma; break; }
                     tc_fence_after();
                 }
                 for (int kb = 0; kb < p.num_kb; ++kb) {
                     if (FINE) {
-                        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort)) { fail = kTimeoutMma; break; }
+                        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort, p.wait_limit_ns)) { fail = kTimeoutMma; break; }
                         tc_fence_after();
                     }
-                    if (!mbar_wait(full0 + 8 * stage, phase, abort)) { fail = kTimeoutMma; break; }
+                    if (!mbar_wait(full0 + 8 * stage, phase, abort, p.wait_limit_ns)) { fail = kTimeoutMma; break; }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sA + stage * kATile), b0 = smem_u32(sB + stage * kBBytes);
 #pragma unroll
@@ -493,7 +504,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             if (fail) *abort = 1;
             // every tensor-core operation this thread issued has completed
             mma_commit(drain_bar);
-            if (!mbar_wait_drain(drain_bar, 0)) fail |= kTimeoutDrain;
+            if (!mbar_wait_drain(drain_bar, 0, p.wait_limit_ns)) fail |= kTimeoutDrain;
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -512,7 +523,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             const int col_base = nb * BN + cgrp * kColsPerWarp;
             if (!FINE) {
                 if (p.num_kb > 0) {
-                    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort));
+                    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort, p.wait_limit_ns));
                     if (!ok) { fail = kTimeoutEpilogue; break; }
                     tc_fence_after();
                 }
@@ -576,7 +587,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                         sb_next = blk_ok ? __ldg(sb_row + kb + 1) : 0.0f;
                     }
                     // every lane polls; the vote keeps the warp converged
-                    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort));
+                    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort, p.wait_limit_ns));
                     if (!ok) { fail = kTimeoutEpilogue; break; }
                     tc_fence_after();
                     if (!warp_rows_live) {
@@ -724,7 +735,8 @@ cudaError_t launch_tall(int yt, const CUtensorMap& ma, const CUtensorMap& mb, co
 
 fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
                              const float* sa, int sa_ld, const float* sb, int sb_ld, bool fine, const void* bias,
-                             int yt, void* d, uint32_t* status, cudaStream_t s, int a_mn, int b_mn) {
+                             int yt, void* d, uint32_t* status, cudaStream_t s, int a_mn, int b_mn,
+                             uint64_t wait_limit_ns, int stall_kb) {
     using namespace mm;
     // 128-wide tiles when a product of at most 128 rows would leave SMs idle
     const bool narrow = M <= BM && (N + 255) / 256 < sm_count();
@@ -769,6 +781,8 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     p.stage_tx = (a_rows + bn) * BK;
     p.a_mn = a_mn;
     p.b_mn = b_mn;
+    p.wait_limit_ns = wait_limit_ns > 0 ? wait_limit_ns : kWaitLimitNs;
+    p.stall_kb = stall_kb;
     const uint32_t idesc = instr_desc(fa, fb, bn, a_mn, b_mn);
     cudaError_t e;
     if (narrow) e = launch_dtype<128>(fine, yt, ma, mbm, p, idesc, s);

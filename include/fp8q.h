@@ -372,6 +372,33 @@ fp8q_status fp8q_scaled_mm(const uint8_t* a, fp8q_format fa, const uint8_t* b, f
                            const void* bias, fp8q_dtype yt, void* d, uint32_t* status,
                            fp8q_stream_t stream);
 
+/* Bits that a product kernel ORs into its status word when a wait runs out:
+ * the copy producer, the tensor-core issuer, the epilogue (each of these
+ * also stops the others), and the final wait for work still in flight. */
+#define FP8Q_WAIT_PRODUCER 1u
+#define FP8Q_WAIT_MMA      2u
+#define FP8Q_WAIT_EPILOGUE 4u
+#define FP8Q_WAIT_DRAIN    8u
+
+/*
+ * Test of the bounded waits (not for production use): fp8q_scaled_mm with
+ * e4m3fn operands, no bias and bf16 output, run with every internal wait
+ * bounded by wait_limit_ns (1 ns .. 4 s) instead of the default of a few
+ * seconds.  stall_kb >= 0 leaves out the shared-memory copies of k-block
+ * stall_kb of each CTA's first tile, so the barrier those copies would
+ * complete never does: the waits that depend on it run out, the kernel ORs
+ * FP8Q_WAIT_* bits into *status, waits (again bounded) for its own copies
+ * and tensor-core work in flight, frees its tensor memory and returns, with
+ * d left incomplete.  Every access stays inside the operands.  stall_kb = -1
+ * runs the product normally under the given limit.
+ * status: a device uint32 word, required.
+ * Errors: as fp8q_scaled_mm; also K == 0, M or N == 0, wait_limit_ns outside
+ *   1 .. 4e9 or stall_kb outside -1 .. ceil(K / 128) - 1 -> FP8Q_ERR_BAD_SHAPE.
+ */
+fp8q_status fp8q_scaled_mm_wait_test(const uint8_t* a, const uint8_t* b, int64_t M, int64_t N, int64_t K,
+                                     const float* scale_a, const float* scale_b, void* d, uint32_t* status,
+                                     uint64_t wait_limit_ns, int stall_kb, fp8q_stream_t stream);
+
 /*
  * Operand layouts of fp8q_scaled_mm_ex.  With A the [M][K] operand and B the
  * [N][K] operand of the product (D = A B^T):

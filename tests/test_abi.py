@@ -165,6 +165,22 @@ def test_scaled_mm_blockwise_validation(L):
     assert f(A, 0, P, A, 0, P, 8, 0, 128, None, 2, None, None, None) == 0   # N == 0: nothing
 
 
+def test_scaled_mm_wait_test_validation(L):
+    f = L.fp8q_scaled_mm_wait_test
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p]
+    A = 0x10000
+    assert f(A, A, 8, 8, 24, P, P, A, A, 1000, 0, None) == 4                # K % 16
+    assert f(A, A, 8, 8, 0, P, P, A, A, 1000, -1, None) == 4                # K == 0
+    assert f(A, A, 8, 8, 128, P, P, A, A, 0, 0, None) == 4                  # no wait limit
+    assert f(A, A, 8, 8, 128, P, P, A, A, 5_000_000_000, 0, None) == 4      # limit above 4 s
+    assert f(A, A, 8, 8, 128, P, P, A, A, 1000, 1, None) == 4               # stall past the last k-block
+    assert f(A, A, 8, 8, 128, P, P, A, A, 1000, -2, None) == 4
+    assert f(A, A, 8, 8, 128, P, P, A, None, 1000, 0, None) == 1            # the status word is required
+    assert f(A, A, 8, 8, 128, None, P, A, A, 1000, 0, None) == 1            # null scale_a
+    assert f(A, A, 8, 8, 128, P, P, A, A + 2, 1000, 0, None) == 5           # status word misaligned
+
+
 def test_transpose_and_sum_rows_validation(L):
     f = L.fp8q_transpose_fp8
     f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]

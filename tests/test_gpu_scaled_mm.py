@@ -384,3 +384,45 @@ def test_exact_grid_tall_tiles(fp8q, orc, M, N, K, yt):
     want = oracle_rounded(orc, False, a, E5M2, b, E4M3FN, 0.0123, 3.5, bias, yt)
     bad = ~bits_equal(host(out), want, yt)
     assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
+
+
+# ---------------------------------------------------------------------------
+# bounded waits: a wait that runs out is reported, and the context stays usable
+# ---------------------------------------------------------------------------
+def test_bounded_waits_run_out_report_and_return(fp8q, orc):
+    """The copies of k-block 2 of each CTA's first tile are left out, so the barrier they would
+    complete never does: with a 20 ms limit every wait that depends on it runs out, the kernel sets
+    its WAIT_* bits, writes nothing outside d, frees its tensor memory and returns.  The same
+    product then runs normally on the same stream, under the same short limit and without it, and
+    both equal the oracle bit for bit."""
+    import time
+    M, N, K = 256, 512, 1024                     # two 128 x 256 tiles, 8 k-blocks (the ring wraps)
+    g = np.random.default_rng(404)
+    a, b = grid_codes(g, (M, K), E4M3FN), grid_codes(g, (N, K), E4M3FN)
+    A, B = dev(a), dev(b)
+    sa, sb = dev(np.array([0.5], np.float32)), dev(np.array([0.25], np.float32))
+    want = oracle_rounded(orc, False, a, E4M3FN, b, E4M3FN, 0.5, 0.25, None, BF16)
+
+    out = Guarded(M * N, torch.bfloat16)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    fp8q.fp8q_scaled_mm_wait_test(A, B, sa, sb, out.t.view(M, N), st, 20_000_000, 2)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    out.check()
+    bits = int(st.item())
+    assert bits & fp8q.WAIT_MMA and bits & fp8q.WAIT_DRAIN, f"status {bits:#x}"
+    assert bits & ~0xF == 0, f"status {bits:#x}"
+    assert dt < 2.0, f"the stalled kernel took {dt:.2f} s"
+
+    for limit in (20_000_000, 4_000_000_000):
+        out2 = Guarded(M * N, torch.bfloat16)
+        st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+        fp8q.fp8q_scaled_mm_wait_test(A, B, sa, sb, out2.t.view(M, N), st2, limit, -1)
+        out2.check()
+        assert int(st2.item()) == 0
+        np.testing.assert_array_equal(host(out2.t.view(M, N)), want)
+    out3 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    fp8q.fp8q_scaled_mm(A, B, sa, sb, out3)
+    np.testing.assert_array_equal(host(out3), want)
