@@ -32,7 +32,7 @@ constexpr int kDqWarps = kDqThreads / 32;
 #define FP8Q_DQ_V32 1  // 32-code chunks with 256-bit loads / stores where aligned
 #endif
 constexpr int kUnroll = FP8Q_DQ_UNROLL;  // rows per thread per tile
-constexpr int kRowsPerTile = kDqWarps * kUnroll;  // 32
+constexpr int kRowsPerTile = kDqWarps * kUnroll;  // 16 with the default unroll
 constexpr int kMaxGroupedDescs = 96;
 
 struct DqDesc {
