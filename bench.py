@@ -640,12 +640,19 @@ OP_SOURCES = {
 
 
 def source_fingerprint(files) -> str:
+    """Hash of the kernel sources' code: comments and whitespace are removed first, so an edit
+    to a comment keeps a capture's record valid and any change to the code voids it."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dequantisation_fp8q_token_b200", "csrc")
     for fn in sorted(files):
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(fn.encode() + f.read())
+        with open(os.path.join(csrc, fn), encoding="utf-8") as f:
+            code = f.read()
+        code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
+        code = re.sub(r"//[^\n]*", " ", code)
+        code = re.sub(r"\s+", " ", code).strip()
+        h.update(fn.encode() + b"\0" + code.encode())
     return h.hexdigest()[:16]
 
 
