@@ -69,9 +69,10 @@ class Op:
     """One call of the step: `ins` are the tensors it reads that come from the
     host in an end-to-end run, `outs` the tensors it writes."""
 
-    def __init__(self, name, fn, bytes_, launches, kernel, ins=(), outs=()):
+    def __init__(self, name, fn, bytes_, launches, kernel, ins=(), outs=(), elems=0):
         self.name, self.fn, self.bytes, self.launches, self.kernel = name, fn, bytes_, launches, kernel
         self.ins, self.outs = list(ins), list(outs)
+        self.elems = elems          # elements the op converts
 
 
 class Workload:
@@ -130,21 +131,23 @@ class Workload:
         # the per-token quant.  The step total does not depend on the order.
         self.ops = [
             Op("cast_per_tensor_f16_zero", lambda: f.fp8q_cast_per_tensor(self.c4c_x, self.c4c_q, self.c4c_s, self.ws, E4M3FN),
-               c4c_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel", [self.c4c_x], [self.c4c_q, self.c4c_s]),
+               c4c_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel", [self.c4c_x], [self.c4c_q, self.c4c_s],
+               workloads.C4C_NUMEL),
             Op("per_token_group_quant", lambda: f.fp8q_per_token_group_quant(self.c2_x, self.c2_q, self.c2_s, 128, E4M3FN),
-               c2_bytes, 1, "per_token_vec_kernel", [self.c2_x], [self.c2_q, self.c2_s]),
+               c2_bytes, 1, "per_token_vec_kernel", [self.c2_x], [self.c2_q, self.c2_s], c2_el),
             Op("block_dequant", lambda: f.fp8q_block_dequant(self.c3_w, self.c3_s, self.c3_y, 128, E4M3FN),
-               c3_bytes, 1, "dequant_kernel", [self.c3_w, self.c3_s], [self.c3_y]),
+               c3_bytes, 1, "dequant_kernel", [self.c3_w, self.c3_s], [self.c3_y], c3_el),
             # the round trip reads q after the block dequant has streamed ~400 MB
             # through L2, so it finds no q bytes left in L2
             Op("cast_from_fp8_group", lambda: f.fp8q_cast_from_fp8(self.c2_q, self.c2_s, self.c2_y, GRAN_GROUP, 128, E4M3FN),
-               c2_bytes, 1, "dequant_kernel", [], [self.c2_y]),
+               c2_bytes, 1, "dequant_kernel", [], [self.c2_y], c2_el),
             Op("cast_per_channel", lambda: f.fp8q_cast_per_channel(self.c4a_x, self.c4a_q, self.c4a_s, E4M3FN),
-               c4a_bytes, 1, "per_channel_vec_kernel", [self.c4a_x], [self.c4a_q, self.c4a_s]),
+               c4a_bytes, 1, "per_channel_vec_kernel", [self.c4a_x], [self.c4a_q, self.c4a_s], R * C),
             Op("cast_per_tensor_f32_e5m2", lambda: f.fp8q_cast_per_tensor(self.c4b_x, self.c4b_q, self.c4b_s, self.ws, E5M2),
-               c4b_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel", [self.c4b_x], [self.c4b_q, self.c4b_s]),
+               c4b_bytes, 2, "tensor_amax_kernel+tensor_cast_kernel", [self.c4b_x], [self.c4b_q, self.c4b_s],
+               workloads.C4B_NUMEL),
             Op("block_dequant_grouped", lambda: f.fp8q_block_dequant_grouped(self.c5_w, self.c5_s, self.c5_y, 128, E4M3FN),
-               c5_bytes, 1, "dequant_kernel", [*self.c5_w, *self.c5_s], self.c5_y),
+               c5_bytes, 1, "dequant_kernel", [*self.c5_w, *self.c5_s], self.c5_y, c5_el),
         ]
         self.step_bytes = sum(o.bytes for o in self.ops)
         self.launches_per_step = sum(o.launches for o in self.ops)
@@ -788,8 +791,9 @@ def run_ours(args):
     for k in range(split_steps):
         wl.step(events[k])
     torch.cuda.synchronize()
-    per_op_ms = [statistics.mean(events[k][i][0].elapsed_time(events[k][i][1]) for k in range(split_steps))
-                 for i in range(nops)]
+    per_op_samples = [sorted(events[k][i][0].elapsed_time(events[k][i][1]) for k in range(split_steps))
+                      for i in range(nops)]
+    per_op_ms = [statistics.median(v) for v in per_op_samples]
     dom = max(range(nops), key=lambda i: per_op_ms[i])
     dom_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
@@ -842,10 +846,15 @@ def run_ours(args):
         return
     peak, peak_kind = measured_peaks()
     kernels = {}
-    for op, ms in zip(wl.ops, per_op_ms):
+    def pct(v, q):
+        return v[min(len(v) - 1, int(round(q * (len(v) - 1))))]
+    for op, ms, v in zip(wl.ops, per_op_ms, per_op_samples):
         gbs = op.bytes / (ms * 1e-3) / 1e9
-        kernels[op.name] = {"us": round(ms * 1e3, 2), "bytes": op.bytes, "gb_s": round(gbs, 1),
-                            "frac": round(gbs / peak, 4), "launches": op.launches}
+        kernels[op.name] = {"us": round(ms * 1e3, 2), "us_mean": round(statistics.mean(v) * 1e3, 2),
+                            "bytes": op.bytes, "gb_s": round(gbs, 1),
+                            "frac": round(gbs / peak, 4), "launches": op.launches, "elements": op.elems,
+                            "gelem_s": round(op.elems / (ms * 1e-3) / 1e9, 2),
+                            "us_p10_p50_p90": [round(pct(v, q) * 1e3, 2) for q in (0.1, 0.5, 0.9)]}
     dop = wl.ops[dom]
     dgbs = dop.bytes / (dom_ms * 1e-3) / 1e9      # CUDA events around it in every timed step
     value = world * wl.step_bytes / (ms_step * 1e-3) / 1e9
@@ -855,6 +864,7 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp32 -> fp8 (u8)",
         "data": "synthetic (seeded generators; shapes and value mixes of the pages' workloads)",
         "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "pct_of_nominal_8tbs": round(100.0 * value / world / 8000.0, 2),
         "config": {"workload": WORKLOAD, "step_bytes": wl.step_bytes, "parallelism": f"replicas x{world}",
                    "l2": "no flush: each step streams ~4.4 GB through the 126 MB L2, so every op's inputs are cold"},
         "roofline": {"bound": "hbm", "kernel": dop.kernel, "op": dop.name, "achieved": round(dgbs, 1),
