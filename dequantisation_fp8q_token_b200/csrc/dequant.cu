@@ -3,14 +3,16 @@
 // covering DeepSeek-V3 weight_dequant (B x B blocks, bf16 out) and ColossalAI
 // cast_from_fp8 / DeepEP per_token_cast_back (tensor, row and 1 x G groups).
 //
-// Work decomposition: each problem is cut into tiles of kRowsPerTile rows by
+// Work decomposition: each problem is cut into tiles of 8 * U rows by
 // 32 chunks of V consecutive elements (V = 32, 16, 8, 4, 2 or 1, the widest
 // that the row length, granule edge and pointer alignment allow).  A CTA of 8
 // warps owns one tile: warp w handles rows w, w + 8, ..., lane l the l-th
 // chunk, so at V = 32 every warp-wide load is one 256-bit access per lane
 // (1 KiB of contiguous codes) and each lane writes its 32 bf16 outputs with
-// two 256-bit stores.  Each thread issues its kUnroll row loads before
-// converting any of them.  Problems of one launch (a checkpoint's weights, a
+// two 256-bit stores.  Each thread issues its U row loads before converting
+// any of them.  U (rows per thread: 4, 2 or 1) is the largest that still
+// gives the launch at least four waves of resident CTAs: large problems
+// take long tiles, and a problem of a few waves keeps the last one short.  Problems of one launch (a checkpoint's weights, a
 // mixture-of-experts layer) share the grid through a descriptor table in
 // kernel-parameter space; a CTA finds its problem by binary search over the
 // first-tile prefix, so heterogeneous shapes need no device-side metadata.
@@ -25,14 +27,10 @@ namespace {
 
 constexpr int kDqThreads = 256;
 constexpr int kDqWarps = kDqThreads / 32;
-#ifndef FP8Q_DQ_UNROLL
-#define FP8Q_DQ_UNROLL 2
-#endif
 #ifndef FP8Q_DQ_V32
 #define FP8Q_DQ_V32 1  // 32-code chunks with 256-bit loads / stores where aligned
 #endif
-constexpr int kUnroll = FP8Q_DQ_UNROLL;  // rows per thread per tile
-constexpr int kRowsPerTile = kDqWarps * kUnroll;  // 16 with the default unroll
+constexpr int kMinWaves = 4;            // waves of resident CTAs a launch should have at least
 constexpr int kMaxGroupedDescs = 96;
 
 struct DqDesc {
@@ -168,28 +166,28 @@ __device__ __forceinline__ void convert_store(const Chunk& c, float sc, void* y,
     }
 }
 
-template <int FMT, int YT, int GRAN, int V>
+template <int FMT, int YT, int GRAN, int V, int U>
 __device__ __forceinline__ void dequant_tile(const DqDesc& D, int gb, int gb_shift, int64_t tr, int tc) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int64_t cols = D.cols;
     const int64_t rows = D.rows;
     const int64_t c = ((int64_t)tc * 32 + lane) * V;  // first column of this thread's chunk
-    const int64_t r0 = tr * kRowsPerTile + warp;
+    const int64_t r0 = tr * (kDqWarps * U) + warp;
     const uint8_t* q = D.q;
     const float* s = D.s;
     if (c < cols) {
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k) {
+        for (int k = 0; k < U; ++k) {
             const int64_t r = r0 + (int64_t)k * kDqWarps;
             if (r < rows) prefetch_l2(q + r * cols + c);
         }
     }
     pdl_wait();
     if (c >= cols) return;
-    Chunk codes[kUnroll];
+    Chunk codes[U];
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
+    for (int k = 0; k < U; ++k) {
         const int64_t r = r0 + (int64_t)k * kDqWarps;
         if (r < rows) codes[k] = load_codes<V>(q + r * cols + c);
     }
@@ -203,7 +201,7 @@ __device__ __forceinline__ void dequant_tile(const DqDesc& D, int gb, int gb_shi
         s_col = div_gb((uint32_t)c, gb, gb_shift);
     }
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
+    for (int k = 0; k < U; ++k) {
         const int64_t r = r0 + (int64_t)k * kDqWarps;
         if (r < rows) {
             float sc;
@@ -216,7 +214,7 @@ __device__ __forceinline__ void dequant_tile(const DqDesc& D, int gb, int gb_shi
     }
 }
 
-template <int FMT, int YT, int GRAN, int N>
+template <int FMT, int YT, int GRAN, int N, int U>
 __global__ void __launch_bounds__(kDqThreads) dequant_kernel(const __grid_constant__ DqParams<N> p) {
     pdl_trigger();     // the tile's codes are prefetched into L2 before pdl_wait (in dequant_tile)
     const int64_t tile = blockIdx.x;
@@ -235,13 +233,13 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(const __grid_consta
     const int tc = (int)(t - tr * D.tiles_per_row);
     switch (D.vshift) {
 #if FP8Q_DQ_V32
-    case 5: dequant_tile<FMT, YT, GRAN, 32>(D, p.gb, p.gb_shift, tr, tc); break;
+    case 5: dequant_tile<FMT, YT, GRAN, 32, U>(D, p.gb, p.gb_shift, tr, tc); break;
 #endif
-    case 4: dequant_tile<FMT, YT, GRAN, 16>(D, p.gb, p.gb_shift, tr, tc); break;
-    case 3: dequant_tile<FMT, YT, GRAN, 8>(D, p.gb, p.gb_shift, tr, tc); break;
-    case 2: dequant_tile<FMT, YT, GRAN, 4>(D, p.gb, p.gb_shift, tr, tc); break;
-    case 1: dequant_tile<FMT, YT, GRAN, 2>(D, p.gb, p.gb_shift, tr, tc); break;
-    default: dequant_tile<FMT, YT, GRAN, 1>(D, p.gb, p.gb_shift, tr, tc); break;
+    case 4: dequant_tile<FMT, YT, GRAN, 16, U>(D, p.gb, p.gb_shift, tr, tc); break;
+    case 3: dequant_tile<FMT, YT, GRAN, 8, U>(D, p.gb, p.gb_shift, tr, tc); break;
+    case 2: dequant_tile<FMT, YT, GRAN, 4, U>(D, p.gb, p.gb_shift, tr, tc); break;
+    case 1: dequant_tile<FMT, YT, GRAN, 2, U>(D, p.gb, p.gb_shift, tr, tc); break;
+    default: dequant_tile<FMT, YT, GRAN, 1, U>(D, p.gb, p.gb_shift, tr, tc); break;
     }
 }
 
@@ -261,6 +259,32 @@ int choose_vshift(const DequantProblem& P, int gran, int gb, int ybytes) {
     return 0;
 }
 
+// resident CTAs of one instantiation across the GPU (cached)
+template <int FMT, int YT, int GRAN, int N, int U>
+int64_t resident_ctas() {
+    static const int64_t n = [] {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dequant_kernel<FMT, YT, GRAN, N, U>, kDqThreads,
+                                                          0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        return (int64_t)per_sm * sm_count();
+    }();
+    return n;
+}
+
+template <int FMT, int YT, int GRAN, int N, int U>
+// each problem's first tile with U rows per thread (8 * U rows per tile)
+cudaError_t assign_tiles(DqParams<N>& p, int64_t& tiles) {
+    tiles = 0;
+    for (int i = 0; i < p.count; ++i) {
+        DqDesc& D = p.d[i];
+        D.tile_begin = tiles;
+        tiles += ((D.rows + kDqWarps * U - 1) / (kDqWarps * U)) * D.tiles_per_row;
+    }
+    if (tiles > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+    return cudaSuccess;
+}
+
 template <int FMT, int YT, int GRAN, int N>
 fp8q_status run_batch(const DequantProblem* probs, int count, int gb, cudaStream_t s) {
     DqParams<N> p;
@@ -271,7 +295,6 @@ fp8q_status run_batch(const DequantProblem* probs, int count, int gb, cudaStream
         p.gb_shift = 0;
         while ((1 << p.gb_shift) < gb) ++p.gb_shift;
     }
-    int64_t tiles = 0;
     const int ybytes = YT == kF32 ? 4 : 2;
     for (int i = 0; i < count; ++i) {
         const DequantProblem& P = probs[i];
@@ -286,12 +309,22 @@ fp8q_status run_batch(const DequantProblem* probs, int count, int gb, cudaStream
         D.vshift = choose_vshift(P, GRAN, gb, ybytes);
         const int64_t span = (int64_t)32 << D.vshift;
         D.tiles_per_row = (int32_t)((P.cols + span - 1) / span);
-        D.tile_begin = tiles;
-        tiles += ((P.rows + kRowsPerTile - 1) / kRowsPerTile) * D.tiles_per_row;
     }
     if (p.count == 0) return FP8Q_OK;
-    if (tiles > 0x7FFFFFFFLL) return FP8Q_ERR_BAD_SHAPE;
-    const cudaError_t err = launch_kernel(dequant_kernel<FMT, YT, GRAN, N>, dim3((unsigned)tiles), dim3(kDqThreads), s, p);
+    // rows per thread: the largest of 4, 2, 1 that leaves at least kMinWaves
+    // waves of resident CTAs
+    int64_t tiles = 0;
+    cudaError_t err;
+    if (assign_tiles<FMT, YT, GRAN, N, 4>(p, tiles) == cudaSuccess &&
+        tiles >= kMinWaves * resident_ctas<FMT, YT, GRAN, N, 4>()) {
+        err = launch_kernel(dequant_kernel<FMT, YT, GRAN, N, 4>, dim3((unsigned)tiles), dim3(kDqThreads), s, p);
+    } else if (assign_tiles<FMT, YT, GRAN, N, 2>(p, tiles) == cudaSuccess &&
+               tiles >= kMinWaves * resident_ctas<FMT, YT, GRAN, N, 2>()) {
+        err = launch_kernel(dequant_kernel<FMT, YT, GRAN, N, 2>, dim3((unsigned)tiles), dim3(kDqThreads), s, p);
+    } else {
+        if (assign_tiles<FMT, YT, GRAN, N, 1>(p, tiles) != cudaSuccess) return FP8Q_ERR_BAD_SHAPE;
+        err = launch_kernel(dequant_kernel<FMT, YT, GRAN, N, 1>, dim3((unsigned)tiles), dim3(kDqThreads), s, p);
+    }
     return cuda_status(err);
 }
 
