@@ -12,10 +12,11 @@
 // two 256-bit stores.  Each thread issues its U row loads before converting
 // any of them.  U (rows per thread: 4, 2 or 1) is the largest that still
 // gives the launch at least four waves of resident CTAs: large problems
-// take long tiles, and a problem of a few waves keeps the last one short.  Problems of one launch (a checkpoint's weights, a
-// mixture-of-experts layer) share the grid through a descriptor table in
-// kernel-parameter space; a CTA finds its problem by binary search over the
-// first-tile prefix, so heterogeneous shapes need no device-side metadata.
+// take long tiles, and a problem of a few waves keeps the last one short.
+// Problems of one launch (a checkpoint's weights, a mixture-of-experts
+// layer) share the grid through a descriptor table in kernel-parameter
+// space; a CTA finds its problem by binary search over the first-tile
+// prefix, so heterogeneous shapes need no device-side metadata.
 //
 // Arithmetic: two codes -> f16x2 (exact), widened to fp32, one fp32 multiply
 // each, then one round-to-nearest-even into the output type.
