@@ -731,9 +731,32 @@ def cpu_baseline(h, budget_s: float = 15.0):
         dt = time.perf_counter() - t0
     what = (f"{reps} passes over the whole step" if reps > 1 else
             f"the first {frac:.5f} of the rows / elements of every op of the step")
+    # one thread, on a sample grown until one pass takes an eighth of the budget or more
+    f1 = 1.0 / 4096
+    while True:
+        t0 = time.perf_counter()
+        b1 = oracle_sample_pass(orc, h, f1, 1)
+        d1 = time.perf_counter() - t0
+        if d1 >= budget_s / 8 or f1 >= 1.0:
+            break
+        f1 = min(1.0, f1 * min(8.0, max(1.5, (budget_s / 4) / max(d1, 1e-3))))
     return {"value": round(b / dt / 1e9, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{what} ({b / 1e6:.1f} MB algorithmic), plain C oracle on {threads} threads",
-            "seconds": round(dt, 2)}
+            "seconds": round(dt, 2), "cpu_model": cpu_model(),
+            "one_thread": {"value": round(b1 / d1 / 1e9, 4), "unit": UNIT, "seconds": round(d1, 2),
+                           "sample": f"the first {f1:.5f} of every op of the step ({b1 / 1e6:.1f} MB algorithmic)"}}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 # ---------------------------------------------------------------------------
