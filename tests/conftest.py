@@ -19,7 +19,16 @@ def pytest_configure(config):
 
 @pytest.fixture(scope="session")
 def orc():
-    import oracle
+    alt = os.environ.get("FP8Q_ORACLE_DIR")
+    if alt:
+        # a copy of the oracle with one planted mistake (tests/test_oracle_mutations.py)
+        import importlib.util
+        spec = importlib.util.spec_from_file_location("oracle_under_test", os.path.join(alt, "__init__.py"),
+                                                      submodule_search_locations=[alt])
+        oracle = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(oracle)
+    else:
+        import oracle
     oracle.build()
     oracle.lib()
     return oracle
