@@ -818,8 +818,11 @@ def run_ours(args):
                       for i in range(nops)]
     per_op_ms = [statistics.median(v) for v in per_op_samples]
     dom = max(range(nops), key=lambda i: per_op_ms[i])
-    dom_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
+    # the dominant op's event pair rides on every `every`-th timed step only (about 20
+    # samples): a pair on every step cost the step about 1.5% on B200
+    every = max(1, args.steps // 20)
+    dom_events = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for k in range(0, args.steps, every)}
 
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -827,14 +830,17 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         t_start.record()
         for k in range(args.steps):
-            wl.step(dom_events[k], only=dom)
+            if k in dom_events:
+                wl.step(dom_events[k], only=dom)
+            else:
+                wl.step()
         t_end.record()
         torch.cuda.synchronize()
     barrier(world)
     ms_local = t_start.elapsed_time(t_end)
     ms_total = max_over_ranks(ms_local, world, device)
     ms_step = ms_total / args.steps
-    dom_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in dom_events)
+    dom_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in dom_events.values())
 
     # end to end: pinned host inputs -> device, the step, outputs -> pinned host
     e2e = EndToEnd(wl)
@@ -879,7 +885,7 @@ def run_ours(args):
                             "gelem_s": round(op.elems / (ms * 1e-3) / 1e9, 2),
                             "us_p10_p50_p90": [round(pct(v, q) * 1e3, 2) for q in (0.1, 0.5, 0.9)]}
     dop = wl.ops[dom]
-    dgbs = dop.bytes / (dom_ms * 1e-3) / 1e9      # CUDA events around it in every timed step
+    dgbs = dop.bytes / (dom_ms * 1e-3) / 1e9      # CUDA events around it in sampled timed steps
     value = world * wl.step_bytes / (ms_step * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
@@ -891,6 +897,7 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "step_bytes": wl.step_bytes, "parallelism": f"replicas x{world}",
                    "l2": "no flush: each step streams ~4.4 GB through the 126 MB L2, so every op's inputs are cold"},
         "roofline": {"bound": "hbm", "kernel": dop.kernel, "op": dop.name, "achieved": round(dgbs, 1),
+                     "timed_launches": len(dom_events),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dgbs / peak, 4),
                      "bytes_per_launch": dop.bytes, "traffic": recorded_traffic(dop.name)},
         "kernels": kernels,
