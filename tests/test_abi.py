@@ -209,3 +209,28 @@ def test_scaled_mm_ex_validation(L):
     assert f(A, 0, 0, A, 0, 1, 32, 24, 32, P, P, None, 2, A, None, None) == 4     # MN-major B needs N % 16
     assert f(A, 0, 0, A, 0, 1, 32, 32, 24, P, P, None, 2, A, None, None) == 4     # a K-major operand needs K % 16
     assert f(A, 0, 1, A, 0, 1, 32, 32, 24, None, P, None, 2, A, None, None) == 1  # both MN-major: any K; null scale
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """With no libfp8q.so every entry point raises: there is no CPU fallback.  Run in a fresh
+    interpreter, pointed at a path where no library exists."""
+    import subprocess
+    import sys
+    code = (
+        "import sys, torch\n"
+        f"sys.path.insert(0, {ROOT!r})\n"
+        "import dequantisation_fp8q_token_b200 as f\n"
+        f"f._LIB_PATH = {str(tmp_path / 'libfp8q.so')!r}\n"
+        "for call in (lambda: f.lib(),\n"
+        "             lambda: f.fp8q_version(),\n"
+        "             lambda: f.per_token_cast_to_fp8(torch.zeros(4, 128, dtype=torch.bfloat16))):\n"
+        "    try:\n"
+        "        call()\n"
+        "        print('returned')\n"
+        "    except Exception as e:\n"
+        "        print('raised', type(e).__name__)\n")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = r.stdout.strip().splitlines()
+    assert lines[0] == "raised ImportError"
+    assert all(line.startswith("raised") for line in lines), r.stdout
