@@ -210,6 +210,13 @@ fp8q_status fp8q_pack_record(const void* x, fp8q_dtype xt, int64_t numel, fp8q_f
     if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
     if (!record) return FP8Q_ERR_NULL_POINTER;
     if (!aligned(record, 16)) return FP8Q_ERR_MISALIGNED;
+    // every check of the cast below, before the header memsets are enqueued
+    if (numel > 0) {
+        if (!x) return FP8Q_ERR_NULL_POINTER;
+        if (!aligned(x, dtype_bytes(xt))) return FP8Q_ERR_MISALIGNED;
+        if (!workspace || workspace_bytes < kPerTensorWorkspaceBytes || !aligned(workspace, 16))
+            return FP8Q_ERR_WORKSPACE;
+    }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // header padding and the payload's last partial 16-byte block start at zero
     if (cudaMemsetAsync(record, 0, 16, s) != cudaSuccess) return FP8Q_ERR_CUDA;

@@ -234,3 +234,98 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
     lines = r.stdout.strip().splitlines()
     assert lines[0] == "raised ImportError"
     assert all(line.startswith("raised") for line in lines), r.stdout
+
+
+def test_sharded_pipeline_and_record_validation(L):
+    """Host-side checks of the sharded per-tensor cast, the pipeline cast and the all-gather
+    records: every case below stops at a check, before any CUDA call."""
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    A = 0x10000
+    WS = L.fp8q_cast_per_tensor_workspace_bytes
+    WS.restype, WS.argtypes = sz, []
+    ws = WS()
+    assert ws >= 4 and ws % 4 == 0
+
+    f = L.fp8q_tensor_amax
+    f.argtypes = [vp, i32, i64, vp, vp, sz, vp]
+    assert f(A, 9, 8, A, A, ws, None) == 2                  # dtype
+    assert f(A, 0, -1, A, A, ws, None) == 4                 # negative numel
+    assert f(A, 0, 8, None, A, ws, None) == 1               # null amax word
+    assert f(A, 0, 8, A + 2, A, ws, None) == 5              # misaligned amax word
+    assert f(None, 0, 8, A, A, ws, None) == 1               # null x
+    assert f(A + 2, 0, 8, A, A, ws, None) == 5              # fp32 x on a 2-byte boundary
+    assert f(A, 0, 8, A, None, ws, None) == 6               # no workspace
+    assert f(A, 0, 8, A, A, ws - 4, None) == 6              # workspace too small
+    assert f(A, 0, 8, A, A + 4, ws, None) == 6              # workspace not 16-byte aligned
+
+    f = L.fp8q_cast_per_tensor_with_amax
+    f.argtypes = [vp, i32, i64, i32, vp, vp, vp, i32, vp]
+    assert f(A, 9, 8, 0, A, A, A, 0, None) == 2             # dtype
+    assert f(A, 0, 8, 0, A, A, A, 7, None) == 10            # scale rule
+    assert f(A, 0, 8, 5, A, A, A, 0, None) == 3             # format
+    assert f(A, 0, -8, 0, A, A, A, 0, None) == 4            # negative numel
+    assert f(A, 0, 8, 0, None, A, A, 0, None) == 1          # null amax word
+    assert f(A, 0, 8, 0, A, A, None, 0, None) == 1          # null scale_inv
+    assert f(A, 0, 8, 0, A + 1, A, A, 0, None) == 5         # misaligned amax word
+    assert f(None, 0, 8, 0, A, A, A, 0, None) == 1          # null x of a non-empty shard
+    assert f(A, 0, 8, 0, A, None, A, 0, None) == 1          # null q of a non-empty shard
+
+    f = L.fp8q_cast_pipeline
+    f.argtypes = [vp, i32, i64, vp, vp, vp, vp, sz, i32, vp]
+    assert f(A, 9, 8, A, A, A, A, ws, 0, None) == 2         # dtype
+    assert f(A, 0, 8, A, A, A, A, ws, 3, None) == 10        # scale rule
+    assert f(A, 0, -1, A, A, A, A, ws, 0, None) == 4        # negative numel
+    assert f(A, 0, 8, A, None, A, A, ws, 0, None) == 1      # null scale_inv
+    assert f(A, 0, 8, A, A, None, A, ws, 0, None) == 1      # null format tag
+    assert f(A, 0, 8, A, A, A + 2, A, ws, 0, None) == 5     # misaligned format tag
+    assert f(A, 0, 8, None, A, A, A, ws, 0, None) == 1      # null q
+    assert f(A, 0, 8, A, A, A, None, ws, 0, None) == 6      # no workspace
+
+    f = L.fp8q_cast_from_pipeline
+    f.argtypes = [vp, i64, vp, vp, i32, vp, vp]
+    assert f(A, 8, A, A, 9, A, None) == 2                   # dtype
+    assert f(A, -8, A, A, 2, A, None) == 4                  # negative numel
+    assert f(None, 0, None, None, 2, None, None) == 0       # empty: nothing to do
+    assert f(A, 8, A, None, 2, A, None) == 1                # null format tag
+    assert f(A, 8, A, A, 2, A + 1, None) == 5               # bf16 output on an odd address
+
+    rb = L.fp8q_record_bytes
+    rb.restype, rb.argtypes = sz, [i64]
+    assert [rb(n) for n in (0, 1, 16, 17, 4096)] == [16, 32, 32, 48, 4112]
+    assert rb(-1) == 0
+
+    f = L.fp8q_pack_record
+    f.argtypes = [vp, i32, i64, i32, vp, vp, sz, i32, vp]
+    assert f(A, 9, 8, 0, A, A, ws, 0, None) == 2            # dtype
+    assert f(A, 0, 8, 0, A, A, ws, 5, None) == 10           # scale rule
+    assert f(A, 0, 8, 4, A, A, ws, 0, None) == 3            # format
+    assert f(A, 0, -8, 0, A, A, ws, 0, None) == 4           # negative numel
+    assert f(A, 0, 8, 0, None, A, ws, 0, None) == 1         # null record
+    assert f(A, 0, 8, 0, A + 8, A, ws, 0, None) == 5        # record not 16-byte aligned
+    # the cast's own checks come before the header is zeroed, so none of these enqueues anything
+    assert f(None, 0, 8, 0, A, A, ws, 0, None) == 1         # null x
+    assert f(A + 2, 0, 8, 0, A, A, ws, 0, None) == 5        # fp32 x on a 2-byte boundary
+    assert f(A, 0, 8, 0, A, None, ws, 0, None) == 6         # no workspace
+
+    f = L.fp8q_unpack_records
+    f.argtypes = [vp, i32, i64, i32, i32, vp, vp]
+    assert f(A, 2, 8, 7, 2, A, None) == 3                   # format
+    assert f(A, 2, 8, 0, 9, A, None) == 2                   # dtype
+    assert f(A, -1, 8, 0, 2, A, None) == 9                  # negative count
+    assert f(A, 2, -8, 0, 2, A, None) == 4                  # negative numel
+    assert f(None, 0, 8, 0, 2, None, None) == 0             # no records: nothing to do
+    assert f(None, 2, 8, 0, 2, A, None) == 1                # null records
+    assert f(A + 8, 2, 8, 0, 2, A, None) == 5               # records not 16-byte aligned
+
+
+def test_status_strings_and_version(L):
+    L.fp8q_status_string.restype = ctypes.c_char_p
+    L.fp8q_status_string.argtypes = [ctypes.c_int]
+    names = [L.fp8q_status_string(i).decode() for i in range(11)]
+    assert names[0] == "FP8Q_OK"
+    assert all(n.startswith("FP8Q_ERR_") for n in names[1:])
+    assert len(set(names)) == 11
+    assert L.fp8q_status_string(99).decode() == "FP8Q_ERR_UNKNOWN"
+    L.fp8q_version.restype = ctypes.c_int
+    v = L.fp8q_version()
+    assert v >= 10000 and v % 100 < 100
