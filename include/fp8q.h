@@ -11,10 +11,20 @@
  *   fp8q_cast_from_fp8          ColossalAI cast_from_fp8; DeepEP
  *                               per_token_cast_back
  *   fp8q_scaled_mm              ColossalAI _LinearFp8.forward (torch._scaled_mm)
+ *   fp8q_scaled_mm_ex           the same with either operand stored MN-major
+ *                               (_LinearFp8.backward's transposed operands)
  *   fp8q_scaled_mm_blockwise    DeepEP per-token activations x DeepSeek-V3
  *                               block-scaled weight
  *   fp8q_transpose_fp8,         ColossalAI _LinearFp8.backward (the operand
  *   fp8q_sum_rows               transposes and the bias gradient)
+ *   fp8q_tensor_amax,           the per-tensor cast of a tensor sharded over
+ *   fp8q_cast_per_tensor_with_amax  ranks (ColossalAI FSDP params hook)
+ *   fp8q_cast_pipeline(_from)   ColossalAI cast_to_fp8_pipeline /
+ *                               cast_from_fp8_pipeline
+ *   fp8q_pack_record,           ColossalAI all_gather_fp8: the [scale |
+ *   fp8q_unpack_records         payload] records
+ *   fp8q_*_ex                   torch's rounding of the scale expressions
+ *   fp8q_scaled_mm_wait_test    a test of the products' bounded waits
  *
  * Conventions shared by every entry point
  * ---------------------------------------
