@@ -19,8 +19,8 @@
  *   fp8q_sum_rows               transposes and the bias gradient)
  *   fp8q_tensor_amax,           the per-tensor cast of a tensor sharded over
  *   fp8q_cast_per_tensor_with_amax  ranks (ColossalAI FSDP params hook)
- *   fp8q_cast_pipeline(_from)   ColossalAI cast_to_fp8_pipeline /
- *                               cast_from_fp8_pipeline
+ *   fp8q_cast_pipeline,         ColossalAI cast_to_fp8_pipeline /
+ *   fp8q_cast_from_pipeline     cast_from_fp8_pipeline
  *   fp8q_pack_record,           ColossalAI all_gather_fp8: the [scale |
  *   fp8q_unpack_records         payload] records
  *   fp8q_*_ex                   torch's rounding of the scale expressions
