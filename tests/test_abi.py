@@ -329,3 +329,64 @@ def test_status_strings_and_version(L):
     L.fp8q_version.restype = ctypes.c_int
     v = L.fp8q_version()
     assert v >= 10000 and v % 100 < 100
+
+
+def test_every_python_entry_point_refuses_host_tensors(L):
+    """No CPU fallback anywhere in the binding: given host tensors, every public helper raises
+    because its tensors are not CUDA tensors, before the C library is called."""
+    import torch
+    import dequantisation_fp8q_token_b200 as f
+    bf, u8, f32, i32 = torch.bfloat16, torch.uint8, torch.float32, torch.int32
+    x = torch.zeros(4, 256, dtype=bf)
+    q = torch.zeros(4, 256, dtype=u8)
+    s2 = torch.ones(4, 2, dtype=f32)
+    s1 = torch.ones(1, dtype=f32)
+    sr = torch.ones(4, dtype=f32)
+    ws = torch.zeros(f.fp8q_cast_per_tensor_workspace_bytes(), dtype=u8)
+    y = torch.zeros(4, 256, dtype=bf)
+    w = torch.zeros(256, 256, dtype=u8)
+    sw = torch.ones(2, 2, dtype=f32)
+    yw = torch.zeros(256, 256, dtype=bf)
+    a8 = torch.zeros(16, 256, dtype=torch.float8_e4m3fn)
+    b8 = torch.zeros(32, 256, dtype=torch.float8_e4m3fn)
+    out = torch.zeros(16, 32, dtype=bf)
+    tag = torch.zeros(1, dtype=i32)
+    rec = torch.zeros(f.record_bytes(x.numel()), dtype=u8)
+    calls = {
+        "fp8q_per_token_group_quant": lambda: f.fp8q_per_token_group_quant(x, q, s2, 128),
+        "per_token_cast_to_fp8": lambda: f.per_token_cast_to_fp8(x),
+        "per_token_cast_back": lambda: f.per_token_cast_back(q.view(torch.float8_e4m3fn), s2),
+        "fp8q_cast_per_channel": lambda: f.fp8q_cast_per_channel(x, q, sr),
+        "fp8q_cast_per_tensor": lambda: f.fp8q_cast_per_tensor(x, q, s1, ws),
+        "fp8q_cast_per_tensor_noalloc": lambda: f.fp8q_cast_per_tensor_noalloc(x, q, s1),
+        "fp8q_tensor_amax": lambda: f.fp8q_tensor_amax(x, tag, ws),
+        "fp8q_cast_per_tensor_with_amax": lambda: f.fp8q_cast_per_tensor_with_amax(x, tag, q, s1),
+        "cast_to_fp8": lambda: f.cast_to_fp8(x),
+        "cast_from_fp8": lambda: f.cast_from_fp8(q.view(torch.float8_e4m3fn), s1, bf),
+        "fp8q_cast_pipeline": lambda: f.fp8q_cast_pipeline(x, q, s1, tag, ws),
+        "fp8q_cast_from_pipeline": lambda: f.fp8q_cast_from_pipeline(q, s1, tag, y),
+        "fp8q_block_dequant": lambda: f.fp8q_block_dequant(w, sw, yw, 128),
+        "fp8q_block_dequant_grouped": lambda: f.fp8q_block_dequant_grouped([w], [sw], [yw], 128),
+        "weight_dequant": lambda: f.weight_dequant(w.view(torch.float8_e4m3fn), sw),
+        "fp8q_cast_from_fp8": lambda: f.fp8q_cast_from_fp8(q, s2, y, f.GRAN_GROUP, 128),
+        "fp8q_pack_record": lambda: f.fp8q_pack_record(x, rec, ws),
+        "fp8q_unpack_records": lambda: f.fp8q_unpack_records(rec, 1, x.numel(), y),
+        "fp8q_scaled_mm": lambda: f.fp8q_scaled_mm(a8, b8, s1, s1, out),
+        "fp8q_scaled_mm_ex": lambda: f.fp8q_scaled_mm_ex(a8, b8, s1, s1, out),
+        "fp8q_scaled_mm_blockwise": lambda: f.fp8q_scaled_mm_blockwise(
+            a8, torch.ones(16, 2, dtype=f32), b8, torch.ones(1, 2, dtype=f32), out),
+        "scaled_mm": lambda: f.scaled_mm(a8, b8.t(), s1, s1),
+        "fp8q_transpose_fp8": lambda: f.fp8q_transpose_fp8(w, torch.zeros(256, 256, dtype=u8)),
+        "transpose_fp8": lambda: f.transpose_fp8(w),
+        "fp8q_sum_rows": lambda: f.fp8q_sum_rows(y, torch.zeros(256, dtype=bf)),
+        "linear_fp8": lambda: f.linear_fp8(torch.zeros(16, 256, dtype=bf), torch.zeros(32, 256, dtype=bf)),
+    }
+    did_not_refuse = {}
+    for name, call in calls.items():
+        try:
+            call()
+            did_not_refuse[name] = "returned"
+        except Exception as e:   # the refusal is a ValueError naming the CUDA requirement
+            if "CUDA" not in str(e):
+                did_not_refuse[name] = f"{type(e).__name__}: {e}"
+    assert not did_not_refuse, did_not_refuse
