@@ -26,6 +26,12 @@ MUTATIONS = [
     ("per-token clamp dropped (DeepEP 5 Utils: amax.clamp(1e-4))", CASTS,
      "            if (amax < clampmin)\n                amax = clampmin;",
      "            (void)clampmin;"),
+    ("e4m3fn encode saturates at 448 instead of giving NaN (torch's .to(float8_e4m3fn))", CODECS,
+     "return (uint8_t)((c > 0x7Eu ? 0x7Fu : c) | sign);",
+     "return (uint8_t)((c > 0x7Eu ? 0x7Eu : c) | sign);"),
+    ("per-token groups start one element apart instead of one group apart", CASTS,
+     "            int64_t base = r * n + g * group;",
+     "            int64_t base = r * n + g;"),
     ("fp8 encode rounds ties away from zero instead of to even", CODECS,
      "if (rem > half || (rem == half && (kept & 1u)))",
      "if (rem >= half)"),
