@@ -42,3 +42,21 @@ def test_step_bytes_match_the_derivation():
     assert bi == 58_720_256 + 132_120_576 + 32_256 + 134_217_728 + 268_435_456 + 2_097_152 + 995_524_096 + 243_456
     assert bo == (29_360_128 + 917_504 + 58_720_256 + 264_241_152 + 67_108_864 + 32_768 + 67_108_864 + 4
                   + 1_048_576 + 4 + 995_524_096 * 2)
+
+
+def test_traffic_fingerprint_ignores_comments_only(tmp_path, monkeypatch):
+    """The DRAM-traffic record stays valid across comment and whitespace edits of the kernel
+    sources, and any change to their code voids it."""
+    import bench
+    csrc = tmp_path / "dequantisation_fp8q_token_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+
+    def fp(text):
+        (csrc / "k.cu").write_text(text)
+        return bench.source_fingerprint(["k.cu"])
+
+    base = fp("int f(int x) {\n    return x + 1;  // one more\n}\n")
+    assert fp("/* a header */\nint f(int x) {\n  return x + 1;   // one more, said differently\n}\n") == base
+    assert fp("int f(int x) {\n    return x + 2;  // one more\n}\n") != base
+    assert fp("int f(int y) {\n    return y + 1;\n}\n") != base
