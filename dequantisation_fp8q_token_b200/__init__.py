@@ -191,6 +191,14 @@ def _dev_ptr(t: Optional[torch.Tensor], name: str, device=None) -> Optional[int]
 
 
 def _stream(stream, device) -> int:
+    """The raw stream handle for a call on `device`.  The library sizes its launches (and picks
+    the allocation-free cast's scratch) from the CURRENT device, so a tensor on any other device
+    is refused before anything is enqueued."""
+    if device is not None and device.type == "cuda":
+        cur = torch.cuda.current_device()
+        if device.index is not None and device.index != cur:
+            raise ValueError(f"tensors are on {device} but the current device is cuda:{cur}; "
+                             f"call under torch.cuda.device({device.index})")
     if stream is None:
         return torch.cuda.current_stream(device).cuda_stream
     if isinstance(stream, torch.cuda.Stream):

@@ -13,6 +13,9 @@
 // In host code the array's name is only a host-side stand-in, never a device
 // address; its device address is fetched with cudaGetSymbolAddress, once per
 // device, with that device current, on the first call made on that device.
+// The cached address belongs to the device's primary context: after
+// cudaDeviceReset the context is rebuilt and the array may sit elsewhere, so
+// this entry point must not be called again in that process.
 #include <mutex>
 
 #include "fp8q.h"
@@ -21,8 +24,11 @@
 namespace fp8q {
 namespace {
 
-// room for kMaxPartials per-CTA maxima: 2048 x 4 bytes = 8 KiB per GPU
+// room for kMaxPartials per-CTA maxima: 2048 x 4 bytes = 8 KiB per GPU.  The
+// amax pass clamps its grid to kMaxPartials CTAs (one partial each), so every
+// launch fits the array whatever the tensor's size or the device's SM count.
 constexpr int kNoAllocPartials = kMaxPartials;
+static_assert(kNoAllocPartials >= kMaxPartials, "the amax pass may write kMaxPartials partials");
 static __device__ __align__(256) uint32_t g_noalloc_partials[kNoAllocPartials];
 
 constexpr int kMaxDevices = 128;
@@ -67,11 +73,6 @@ extern "C" fp8q_status fp8q_cast_per_tensor_noalloc(const void* x, fp8q_dtype xt
     if (numel == 0) return launch_fill(scale_inv, 1, 1.0f, s);
     if (!x || !q) return FP8Q_ERR_NULL_POINTER;
     if ((uintptr_t)x % es) return FP8Q_ERR_MISALIGNED;
-    // The amax pass launches at most min(8 x SMs, kMaxPartials) CTAs, one
-    // partial each; refuse a device whose launch would need more slots than
-    // the static array has (none on B200: 148 SMs -> 1184 partials).
-    const int64_t needed = (int64_t)sm_count() * 8 < kMaxPartials ? (int64_t)sm_count() * 8 : kMaxPartials;
-    if (needed > kNoAllocPartials) return FP8Q_ERR_WORKSPACE;
     uint32_t* scratch = nullptr;
     const fp8q_status st = scratch_on_current_device(&scratch);
     if (st != FP8Q_OK) return st;

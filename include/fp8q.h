@@ -35,7 +35,9 @@
  *   no state between calls and enqueues all work on the given stream (NULL =
  *   the legacy default stream).  Calls on different streams are independent.
  *   Calls return as soon as the work is enqueued; outputs are valid once the
- *   stream reaches that point.
+ *   stream reaches that point.  The stream must belong to the current device
+ *   and the tensors must live on it: launch shapes are sized from the
+ *   current device's SM count.
  * - Arithmetic is IEEE binary32 with round-to-nearest-even: scales are
  *   computed with true division (fl(FMAX / amax)), products are single
  *   fp32 multiplies, narrowing to fp8 / bf16 / fp16 rounds to nearest-even.
@@ -196,12 +198,16 @@ fp8q_status fp8q_cast_per_tensor_ex(const void* x, fp8q_dtype xt, int64_t numel,
  * cudaMalloc because that call may synchronise the device.  The scratch for
  * the amax pass lives in a file-scope __device__ array inside the library:
  * 8 KiB (2048 per-CTA partial maxima), present on every GPU that loads the
- * library until the process exits.  Every tensor size fits, because the
- * amax pass never uses more than 2048 CTAs; a launch that would need more
- * slots than the array holds is refused with FP8Q_ERR_WORKSPACE.
+ * library until the process exits.  Every tensor size fits: the amax pass
+ * clamps its grid to 2048 CTAs, one partial maximum each, so no size is
+ * refused for want of scratch (FP8Q_ERR_WORKSPACE is never returned).
  * - The call allocates nothing (no cudaMalloc / cudaFree).  The first call on
  *   a device looks up the array's device address on that device (with it
  *   current) and caches it; make that first call before any stream capture.
+ *   The cached address is the primary context's: after cudaDeviceReset do
+ *   not call this entry point again in the same process.
+ * - `stream` must belong to the current device, and x, q and scale_inv must
+ *   live on it (the scratch used is the current device's).
  * - All calls share the one array per device, and it keeps the last call's
  *   contents; nothing needs clearing, since each call writes every slot it
  *   reads.  Calls whose work overlaps on the GPU (different streams, no

@@ -390,3 +390,21 @@ def test_every_python_entry_point_refuses_host_tensors(L):
             if "CUDA" not in str(e):
                 did_not_refuse[name] = f"{type(e).__name__}: {e}"
     assert not did_not_refuse, did_not_refuse
+
+
+def test_binding_refuses_a_device_other_than_the_current_one(monkeypatch):
+    """The library sizes launches (and picks the allocation-free cast's static scratch) from the
+    current device, so the binding refuses tensors on any other device before calling it.  Every
+    call into the library takes its stream from the one helper that checks this."""
+    import inspect
+    import torch
+    import dequantisation_fp8q_token_b200 as f
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="current device"):
+        f._stream(None, torch.device("cuda", 1))
+    src = inspect.getsource(f)
+    calls = re.findall(r"lib\(\)\.fp8q_\w+\(|\bf\(_dev_ptr", src)
+    streams = re.findall(r"_stream\(stream, dev\)\)", src)
+    assert len(calls) > 0 and len(streams) >= len(calls) - sum(
+        1 for n in ("fp8q_status_string", "fp8q_version", "fp8q_cast_per_tensor_workspace_bytes",
+                    "fp8q_record_bytes") if f"lib().{n}(" in src)

@@ -62,6 +62,31 @@ def test_noalloc_matches_workspace_entry_point_twice(fp8q):
         assert _same(_noalloc(lib, x, xt, fmt), _reference(fp8q, x, fmt))
 
 
+def test_noalloc_allocates_no_device_memory(fp8q):
+    """The point of the entry point: repeated calls leave the device's free memory unchanged.
+    Every tensor is allocated and one warm-up call made (it loads the kernels and looks up the
+    scratch address) before the free bytes are read."""
+    lib = fp8q.lib()
+    f = _c_noalloc(lib)
+    x = torch.randn(3_000_000, device="cuda")
+    q = torch.empty(x.numel(), dtype=torch.uint8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def call():
+        st = f(x.data_ptr(), F32, x.numel(), E4M3FN, q.data_ptr(), s.data_ptr(), stream)
+        assert st == 0, lib.fp8q_status_string(st)
+
+    call()
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    for _ in range(8):
+        call()
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before
+
+
 def test_noalloc_binding_and_errors(fp8q):
     x = torch.ones(1000, dtype=torch.float16, device="cuda")
     x[17] = -7.0
