@@ -22,24 +22,17 @@
 //               tcgen05.mma.kind::f8f6f4 (M 128, N BN, K 32) into one of the
 //               128 x BN fp32 TMEM accumulators and commits each stage back
 //               to the producer and each finished accumulator to the epilogue
-//   warps 2..   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32 * (w % 4) .. + 31 and one column group of the
-//               tile), every lane polling the accumulator's barrier.
-//     per-tensor scales: eight warps, 128 columns each; scaling, bias,
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32 * (w % 4) .. + 31, column group (w - 2) / 4), every
+//               lane polling the accumulator's barrier; scaling, bias,
 //               conversion, 32-byte stores (TMEM loads double-buffered in
-//               32-column chunks).
-//     fine-grained scales: the MMA warp commits every 128-deep k-block into
-//               a fresh accumulator and the epilogue folds it into registers
-//               with that block's scale (packed fp32x2 FMAs) while the tensor
-//               cores fill the other accumulator.  128 x 256 tiles: sixteen
-//               warps (four per lane quarter), 64 columns each, 16-column
-//               loads one at a time; 128 x 128 tiles: eight warps, 64 columns
-//               each, 16-column loads double-buffered.  Warps whose rows all
-//               lie past M only take part in the handshake.
-//               Measured on B200: the fold's TMEM reads compete with the
-//               tensor cores' own accumulator traffic, so each k-block's MMAs
-//               run 40-60% longer than alone; sixteen warps finish the fold
-//               sooner than eight and gained 4-5%.
+//               32-column chunks).  With fine-grained scales the MMA warp
+//               commits every 128-deep k-block into a fresh accumulator and
+//               the epilogue folds it into registers with that block's scale
+//               (packed fp32x2 FMAs, TMEM loads double-buffered in 16-column
+//               chunks; warps whose rows all lie past M only take part in the
+//               handshake), while the tensor cores fill the other
+//               accumulator.
 // Tiles are 128 x BN of D, or 256 x 256 for large per-tensor products (two
 // M 128 MMAs per k step share the B tile; see Shape), visited in bands of 32
 // row-tiles so that the CTAs working at one time share A and B tiles in L2.
@@ -63,18 +56,9 @@ namespace mm {
 constexpr int BM = 128;         // rows of A (and of D) per tile
 constexpr int BK = 128;         // k per stage: one 128-byte swizzle row, one scale block
 constexpr int kTmemCols = 512;  // all of TMEM, split into kAccBufs accumulators
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kGroupM = 32;     // row-tiles per raster band
-
-// The fine-grained product's fold on 128 x 256 tiles: FP8Q_FINE_EW epilogue
-// warps (16: four per TMEM lane quarter, 64 columns each, 16-column loads one
-// at a time; 8: 128 columns each, 16-column loads double-buffered), each
-// loading FP8Q_FINE_FL accumulator columns per tcgen05.ld.
-#ifndef FP8Q_FINE_EW
-#define FP8Q_FINE_EW 16
-#endif
-#ifndef FP8Q_FINE_FL
-#define FP8Q_FINE_FL 16
-#endif
 
 // Tile shapes.  BN = 256: 128 x 256 tiles, two TMEM accumulators (with
 // per-tensor scales one tile's epilogue overlaps the next tile's k-loop; with
@@ -89,16 +73,13 @@ constexpr int kGroupM = 32;     // row-tiles per raster band
 // step sharing the B tile, the two 128 x 256 accumulators filling TMEM (one
 // buffer: each tile's epilogue is not overlapped), a 3-stage ring -- a third
 // fewer operand bytes per flop than 128 x 256 tiles.
-template <int BN_, int MT_ = 128, int EW_ = 8> struct Shape {
+template <int BN_, int MT_ = 128> struct Shape {
     static constexpr int BN = BN_;                          // rows of B (columns of D) per tile
     static constexpr int MT = MT_;                          // rows of A (and of D) per tile
-    static constexpr int kEpiWarps = EW_;                   // epilogue warps, a multiple of 4
-    static constexpr int kCtrlWarps = 2;                   // warp 0 TMA producer, warp 1 MMA issuer
-    static constexpr int kThreads = 32 * (kCtrlWarps + EW_);
     static constexpr int kATile = MT_ * BK;
     static constexpr int kStages = MT_ == 256 ? 3 : (BN_ == 256 ? 4 : 6);
     static constexpr int kAccBufs = MT_ == 256 ? 1 : kTmemCols / BN;
-    static constexpr int kColsPerWarp = BN / (EW_ / 4);         // tile columns one epilogue warp owns
+    static constexpr int kColsPerWarp = BN / (kEpiWarps / 4);   // tile columns one epilogue warp owns
     static constexpr int kBBytes = BN * BK;
     static constexpr int kStageBytes = kATile + kBBytes;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment slack */ + 256 /* barriers */;
@@ -357,45 +338,6 @@ __device__ __forceinline__ void store_chunk(const Params& p, int row, int col0, 
     }
 }
 
-// 16 consecutive columns of one row of D, the bias added first: one or two
-// 32-byte stores when the row allows, else element by element
-template <int YT>
-__device__ __forceinline__ void store_group16(const Params& p, int row, int col0, float (&v)[16]) {
-    using T = typename OutT<YT>::T;
-    T* drow = static_cast<T*>(p.d) + static_cast<int64_t>(row) * p.N;
-    if (p.vec_store && col0 + 16 <= p.N) {
-        if (p.bias) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = __fadd_rn(v[i], load_bias<YT>(p.bias, col0 + i));
-        }
-        if constexpr (YT == kF32) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t w[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(v[c * 8 + i]);
-                st_v8(drow + col0 + c * 8, w);
-            }
-        } else {
-            uint32_t w[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = pack2<YT>(v[2 * i], v[2 * i + 1]);
-            st_v8(drow + col0, w);
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (col0 + i < p.N) {
-                float x = v[i];
-                if (p.bias) x = __fadd_rn(x, load_bias<YT>(p.bias, col0 + i));
-                if constexpr (YT == kF32) drow[col0 + i] = x;
-                else if constexpr (YT == kF16) drow[col0 + i] = __float2half_rn(x);
-                else drow[col0 + i] = __float2bfloat16_rn(x);
-            }
-        }
-    }
-}
-
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& mb, int& nb) {
     const int band = t / (kGroupM * tiles_n);
     const int first = band * kGroupM;
@@ -408,21 +350,16 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int YT, bool FINE, int BN_, int MT_, int EW_, int FL_>
-__global__ void __launch_bounds__(Shape<BN_, MT_, EW_>::kThreads, 1)
+template <int YT, bool FINE, int BN_, int MT_>
+__global__ void __launch_bounds__(kThreads, 1)
 scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const Params p, const uint32_t idesc) {
-    using S = Shape<BN_, MT_, EW_>;
-    constexpr int BN = S::BN;
-    constexpr int kStages = S::kStages;
-    constexpr int kAccBufs = S::kAccBufs;
-    constexpr int kColsPerWarp = S::kColsPerWarp;
-    constexpr int kBBytes = S::kBBytes;
-    constexpr int kATile = S::kATile;
-    constexpr int kEpiWarps = S::kEpiWarps;
-    constexpr int kCtrlWarps = S::kCtrlWarps;
-    static_assert(FL_ == 16 || FL_ == 32, "fold loads of 16 or 32 columns");
-    static_assert(kColsPerWarp % FL_ == 0 && kColsPerWarp % 32 == 0, "whole chunks per warp");
+    constexpr int BN = Shape<BN_, MT_>::BN;
+    constexpr int kStages = Shape<BN_, MT_>::kStages;
+    constexpr int kAccBufs = Shape<BN_, MT_>::kAccBufs;
+    constexpr int kColsPerWarp = Shape<BN_, MT_>::kColsPerWarp;
+    constexpr int kBBytes = Shape<BN_, MT_>::kBBytes;
+    constexpr int kATile = Shape<BN_, MT_>::kATile;
     constexpr int kSub = MT_ / BM;                 // M 128 sub-tiles (MMAs per k step, accumulators per tile)
     static_assert(!FINE || MT_ == BM, "fine-grained scales use 128-row tiles");
     extern __shared__ uint8_t smem_raw[];
@@ -569,9 +506,9 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             mma_commit(drain_bar);
             if (!mbar_wait_drain(drain_bar, 0, p.wait_limit_ns)) fail |= kTimeoutDrain;
         }
-    } else if (warp >= kCtrlWarps) {
+    } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - kCtrlWarps;
+        const int ew = warp - 2;
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
         const int cgrp = ew >> 2;                     // which kColsPerWarp-wide group of the tile's columns
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
@@ -590,11 +527,11 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     if (!ok) { fail = kTimeoutEpilogue; break; }
                     tc_fence_after();
                 }
-                const uint32_t col_addr = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + cgrp * kColsPerWarp);
                 // kSub x kColsPerWarp / 32 chunks of 32 columns, double-buffered:
                 // the load of chunk j + 1 is in flight while chunk j is scaled
                 // and stored
                 constexpr int kChunks = kSub * (kColsPerWarp / 32);
+                const uint32_t col_addr = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + cgrp * kColsPerWarp);
                 uint32_t r0[32], r1[32];
                 if (p.num_kb > 0) {
                     tmem_ld32_async(col_addr, r0);
@@ -639,10 +576,16 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 const bool row_ok = row < p.M;
                 const bool warp_rows_live = row - lane < p.M;    // the warp's first row
                 const bool blk_ok = col_base < p.N;
+                const float* sa_row = p.sa + static_cast<int64_t>(row_ok ? row : 0) * p.sa_ld;
+                const float* sb_row = p.sb + static_cast<int64_t>(blk_ok ? col_base / 128 : 0) * p.sb_ld;
+                float sa_next = (row_ok && p.num_kb > 0) ? __ldg(sa_row) : 0.0f;
+                float sb_next = (blk_ok && p.num_kb > 0) ? __ldg(sb_row) : 0.0f;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    // this k-block's two scales, loaded while the accumulator is awaited
-                    const float sa = row_ok ? __ldg(p.sa + static_cast<int64_t>(row) * p.sa_ld + kb) : 0.0f;
-                    const float sb = blk_ok ? __ldg(p.sb + static_cast<int64_t>(col_base / 128) * p.sb_ld + kb) : 0.0f;
+                    const float s = __fmul_rn(sa_next, sb_next);
+                    if (kb + 1 < p.num_kb) {
+                        sa_next = row_ok ? __ldg(sa_row + kb + 1) : 0.0f;
+                        sb_next = blk_ok ? __ldg(sb_row + kb + 1) : 0.0f;
+                    }
                     // every lane polls; the vote keeps the warp converged
                     const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort, p.wait_limit_ns));
                     if (!ok) { fail = kTimeoutEpilogue; break; }
@@ -655,54 +598,25 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                         if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
                         continue;
                     }
-                    const float s = __fmul_rn(sa, sb);
-                    // kColsPerWarp / FL_ chunks of FL_ columns folded in with packed
-                    // fused multiply-adds (each lane the same as __fmaf_rn).  FL_ 16:
-                    // double-buffered, the load of chunk c + 1 in flight while chunk
-                    // c is folded; FL_ 32: one load in flight, the other warps of the
-                    // lane quarter keep TMEM busy meanwhile.
+                    // 8 chunks of 16 columns, double-buffered: the load of chunk
+                    // c + 1 is in flight while chunk c is folded in with packed
+                    // fused multiply-adds (each lane the same as __fmaf_rn)
                     const uint32_t col_addr = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + cgrp * kColsPerWarp);
                     const float2 s2 = make_float2(s, s);
-                    if constexpr (FL_ == 16 && kEpiWarps > 8) {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16_async(col_addr, r0);
+                    tmem_wait16(r0);
 #pragma unroll
-                        for (int c = 0; c < kColsPerWarp / 16; ++c) {
-                            uint32_t r[16];
-                            tmem_ld16_async(col_addr + 16 * c, r);
-                            tmem_wait16(r);
+                    for (int c = 0; c < kColsPerWarp / 16; ++c) {
+                        uint32_t (&cur)[16] = (c & 1) ? r1 : r0;
+                        uint32_t (&nxt)[16] = (c & 1) ? r0 : r1;
+                        if (c + 1 < kColsPerWarp / 16) tmem_ld16_async(col_addr + 16 * (c + 1), nxt);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                accum[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(r[2 * i]),
-                                                                          __uint_as_float(r[2 * i + 1])),
-                                                              s2, accum[c * 8 + i]);
-                        }
-                    } else if constexpr (FL_ == 16) {
-                        uint32_t r0[16], r1[16];
-                        tmem_ld16_async(col_addr, r0);
-                        tmem_wait16(r0);
-#pragma unroll
-                        for (int c = 0; c < kColsPerWarp / 16; ++c) {
-                            uint32_t (&cur)[16] = (c & 1) ? r1 : r0;
-                            uint32_t (&nxt)[16] = (c & 1) ? r0 : r1;
-                            if (c + 1 < kColsPerWarp / 16) tmem_ld16_async(col_addr + 16 * (c + 1), nxt);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                accum[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(cur[2 * i]),
-                                                                          __uint_as_float(cur[2 * i + 1])),
-                                                              s2, accum[c * 8 + i]);
-                            if (c + 1 < kColsPerWarp / 16) tmem_wait16(nxt);
-                        }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < kColsPerWarp / 32; ++c) {
-                            uint32_t r[32];
-                            tmem_ld32_async(col_addr + 32 * c, r);
-                            tmem_wait32(r);
-#pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                accum[c * 16 + i] = __ffma2_rn(make_float2(__uint_as_float(r[2 * i]),
-                                                                           __uint_as_float(r[2 * i + 1])),
-                                                               s2, accum[c * 16 + i]);
-                        }
+                        for (int i = 0; i < 8; ++i)
+                            accum[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(cur[2 * i]),
+                                                                      __uint_as_float(cur[2 * i + 1])),
+                                                          s2, accum[c * 8 + i]);
+                        if (c + 1 < kColsPerWarp / 16) tmem_wait16(nxt);
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -710,18 +624,21 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
                 }
                 if (fail) break;
-                if (row_ok) {
 #pragma unroll
-                    for (int c = 0; c < kColsPerWarp / 16; ++c) {
-                        const int col0 = col_base + c * 16;
-                        float v[16];
+                for (int c = 0; c < kColsPerWarp / 32; ++c) {
+                    float v[32];
+                    const int col0 = col_base + c * 32;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            v[2 * i] = accum[c * 8 + i].x;
-                            v[2 * i + 1] = accum[c * 8 + i].y;
-                        }
-                        if (col0 < p.N) store_group16<YT>(p, row, col0, v);
+                    for (int i = 0; i < 16; ++i) {
+                        v[2 * i] = accum[c * 16 + i].x;
+                        v[2 * i + 1] = accum[c * 16 + i].y;
                     }
+                    if (p.bias) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (col0 + i < p.N) v[i] = __fadd_rn(v[i], load_bias<YT>(p.bias, col0 + i));
+                    }
+                    if (row_ok && col0 < p.N) store_chunk<YT>(p, row, col0, v);
                 }
             }
         }
@@ -772,18 +689,18 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int b
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int YT, bool FINE, int BN_, int MT_, int EW_ = 8, int FL_ = 16>
+template <int YT, bool FINE, int BN_, int MT_>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, uint32_t idesc,
                          cudaStream_t s) {
-    using S = Shape<BN_, MT_, EW_>;
-    auto kernel = scaled_mm_kernel<YT, FINE, BN_, MT_, EW_, FL_>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+    auto kernel = scaled_mm_kernel<YT, FINE, BN_, MT_>;
+    constexpr int kSmemBytes = Shape<BN_, MT_>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const int tiles = p.tiles_m * p.tiles_n;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles < sm_count() ? tiles : sm_count()));
-    cfg.blockDim = dim3(S::kThreads);
-    cfg.dynamicSmemBytes = S::kSmemBytes;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -797,13 +714,9 @@ template <int BN_>
 cudaError_t launch_dtype(bool fine, int yt, const CUtensorMap& ma, const CUtensorMap& mb, const Params& p,
                          uint32_t idesc, cudaStream_t s) {
     if (fine) {
-        // 128 x 256 tiles: the fold's warp count and load width as configured;
-        // 128 x 128 tiles (decode-sized products): eight warps, 16-column loads
-        constexpr int EW = BN_ == 256 ? FP8Q_FINE_EW : 8;
-        constexpr int FL = BN_ == 256 ? FP8Q_FINE_FL : 16;
-        return yt == kF32 ? launch_typed<kF32, true, BN_, 128, EW, FL>(ma, mb, p, idesc, s)
-             : yt == kF16 ? launch_typed<kF16, true, BN_, 128, EW, FL>(ma, mb, p, idesc, s)
-                          : launch_typed<kBF16, true, BN_, 128, EW, FL>(ma, mb, p, idesc, s);
+        return yt == kF32 ? launch_typed<kF32, true, BN_, 128>(ma, mb, p, idesc, s)
+             : yt == kF16 ? launch_typed<kF16, true, BN_, 128>(ma, mb, p, idesc, s)
+                          : launch_typed<kBF16, true, BN_, 128>(ma, mb, p, idesc, s);
     }
     return yt == kF32 ? launch_typed<kF32, false, BN_, 128>(ma, mb, p, idesc, s)
          : yt == kF16 ? launch_typed<kF16, false, BN_, 128>(ma, mb, p, idesc, s)
