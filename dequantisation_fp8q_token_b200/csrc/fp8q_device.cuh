@@ -262,13 +262,18 @@ template <int XT> __device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32
 }
 
 // non-saturating semantics for one value given the hardware code c:
-//   NaN -> NaN code (sign kept); e4m3fn: |v| > 464 (incl. Inf) -> NaN;
-//   e5m2: |v| >= 61440 (incl. Inf) -> Inf.
+//   NaN -> 0x7F, the positive NaN code of either format; e4m3fn: |v| > 464
+//   (incl. Inf) -> NaN with v's sign; e5m2: |v| >= 61440 (incl. Inf) -> Inf
+//   with v's sign.
+// IEEE 754 leaves the sign of a NaN produced by arithmetic unspecified.  GPU
+// arithmetic returns the canonical positive NaN, so on a CUDA device the
+// pages' torch expressions (x * scale, then .to(float8_*)) give 0x7F for
+// every NaN; writing 0x7F here keeps that whatever sign the product had.
 template <int FMT> __device__ __forceinline__ uint32_t fix_code(float v, uint32_t c) {
     uint32_t u = __float_as_uint(v);
     uint32_t a = u & 0x7FFFFFFFu;
     uint32_t s = (u >> 24) & 0x80u;
-    if (a > 0x7F800000u) return 0x7Fu | s;
+    if (a > 0x7F800000u) return 0x7Fu;
     if (FMT == kE4M3) {
         if (a > 0x43E80000u) return 0x7Fu | s;
     } else {
