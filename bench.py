@@ -18,19 +18,27 @@ the 126 MB L2, so no operation finds its inputs in L2 from the previous step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Beside the step, rank 0 reports two more measurements that are not part of
-`value`: "isolated" times per-token quant, block dequant, the round trip, the
-per-channel and the fp32 per-tensor casts each alone, back to back over
-rotating buffer sets at least 4x the L2 size (each launch reads
-cold inputs and pays for the write-back of one launch of its own outputs);
-"matmul" times the two fp8 products on the tensor cores (TFLOP/s against the
-fp8 peak) beside torch._scaled_mm (cuBLASLt) on the same operands
-(--no-matmul skips it).
+Beside the step, rank 0 reports measurements that are not part of `value`:
+"isolated" times per-token quant, block dequant, the round trip, the
+per-channel and the fp32 per-tensor casts each alone, over rotating buffer
+sets at least 4x the L2 size (each launch reads cold inputs and pays for the
+write-back of one launch of its own outputs), as the median and p10 / p90 of
+blocks of back-to-back launches; "matmul" times the two fp8 products on the
+tensor cores (TFLOP/s against the fp8 peak) beside the library products on
+the same operands (torch._scaled_mm / cuBLASLt for per-tensor scales; torch's
+blockwise scaled_mm and vLLM's CUTLASS blockwise product for the per-token x
+128 x 128-block scales), then each product back to back for two seconds
+under the board's power cap (--no-matmul skips the section).
 
 With N > 1 it runs under torchrun, one rank per GPU, each rank doing the full
 step on its own copy of the inputs (independent problems, weak scaling, no
-data-path collective); the time is the max over ranks.  `--impl reference`
-times the CPU oracle on a bounded sample of the same workload instead.
+data-path collective); the time is the max over ranks.  Beside it, every
+rank then runs the method's two exchange steps ("sharded": the per-tensor
+cast of a tensor split over the ranks with its 4-byte int32 MAX all-reduce,
+and the fp8 all-gather beside a bf16 NCCL all-gather); --sharded runs them
+at N = 1 too.  `--marginal` prints each op's marginal cost inside the live
+step instead.  `--impl reference` times the CPU oracle on a bounded sample
+of the same workload.
 """
 from __future__ import annotations
 
@@ -285,6 +293,136 @@ class EndToEnd:
         return e0.elapsed_time(e1) / steps
 
 
+def shard_range(numel: int, world: int, rank: int, align: int = 8):
+    """[start, stop) of `rank`'s shard of a flat tensor: equal shards, each a multiple of
+    `align` elements (32-byte aligned for fp32), the last one shorter or empty."""
+    per = -(-numel // world)
+    per = -(-per // align) * align
+    start = min(numel, rank * per)
+    return start, min(numel, start + per)
+
+
+class LegKernels:
+    """The device work of the sharded leg, through libfp8q's binding."""
+
+    def __init__(self, fp8q):
+        self.f = fp8q
+
+    def tensor_amax(self, x, amax_bits, ws):
+        self.f.fp8q_tensor_amax(x, amax_bits, ws)
+
+    def cast_with_amax(self, x, amax_bits, q, scale_inv):
+        self.f.fp8q_cast_per_tensor_with_amax(x, amax_bits, q, scale_inv, E5M2)
+
+    def all_gather_fp8(self, out, x, group):
+        self.f.all_gather_fp8(out, x, group, "e5m2")
+
+
+class ShardedLeg:
+    """The method's two exchange steps across the ranks of a torchrun job, timed beside the
+    replicas headline (they are not part of `value`):
+
+      cast_to_fp8_sharded  the per-tensor e5m2 cast of the fp32 v[64 Mi] tensor split over the
+                           ranks: each rank's amax pass over its shard, an int32 MAX all-reduce
+                           of the 4-byte amax bits, then each rank's cast pass with the global
+                           amax (ColossalAI fp8_compress_fsdp_params_comm_hook's all_reduce(MAX))
+      all_gather_fp8       each rank's bf16 shard of `gather_elems` elements cast with its own
+                           scale into a record, one NCCL all-gather of the records, every record
+                           dequantised (ColossalAI all_gather_fp8), beside a plain bf16 NCCL
+                           all_gather_into_tensor of the same shards
+
+    Times are per call, CUDA events on the current stream, the max over ranks.  `kernels` and
+    `timer` are the device work and the clock; tests pass host stand-ins to run the rest of
+    the leg (sharding, buffers, exchanges, byte counts) on gloo ranks."""
+
+    def __init__(self, device, rank, world, v_host, gather_elems=1 << 24, group=None, kernels=None,
+                 timer=None, ws_bytes=8192, seed=20261208):
+        self.device, self.rank, self.world, self.group = device, rank, world, group
+        self.k = kernels
+        self.timer = timer or _device_timer
+        self.numel = int(v_host.size)
+        s0, s1 = shard_range(self.numel, world, rank)
+        self.shard = (s0, s1)
+        self.x = _to_dev(np.ascontiguousarray(v_host[s0:s1]), device)
+        self.q = torch.empty((s1 - s0,), dtype=torch.uint8, device=device)
+        self.sinv = torch.empty((1,), dtype=torch.float32, device=device)
+        self.amax = torch.zeros((1,), dtype=torch.int32, device=device)
+        self.ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=device)
+        g = np.random.default_rng(seed + rank)
+        self.gather_elems = int(gather_elems)
+        self.g = _to_dev(workloads.to_bf16_bits(g.standard_normal(self.gather_elems, dtype=np.float32)),
+                         device, torch.bfloat16)
+        self.out = torch.empty((world * self.gather_elems,), dtype=torch.bfloat16, device=device)
+
+    def cast_sharded(self):
+        import dequantisation_fp8q_token_b200 as fp8q
+        self.k.tensor_amax(self.x, self.amax, self.ws)
+        fp8q.allreduce_amax_bits(self.amax, self.group)
+        self.k.cast_with_amax(self.x, self.amax, self.q, self.sinv)
+
+    def gather_fp8(self):
+        self.k.all_gather_fp8(self.out, self.g, self.group)
+
+    def gather_bf16(self):
+        import torch.distributed as dist
+        dist.all_gather_into_tensor(self.out, self.g, group=self.group)
+
+    def _time(self, fn, reps, warmup):
+        for _ in range(warmup):
+            fn()
+        barrier(self.world)
+        return max_over_ranks(self.timer(fn, reps, self.device), self.world, self.device)
+
+    def run(self, reps: int = 20, warmup: int = 3):
+        import dequantisation_fp8q_token_b200 as fp8q
+        import torch.distributed as dist
+        res = {}
+        ms = self._time(self.cast_sharded, reps, warmup)
+        # every rank must hold the one scale_inv that the global amax gives
+        same = True
+        if self.world > 1:
+            allsinv = torch.empty((self.world,), dtype=torch.float32, device=self.device)
+            dist.all_gather_into_tensor(allsinv, self.sinv, group=self.group)
+            bits = allsinv.view(torch.int32).cpu()
+            same = bool((bits == bits[0]).all())
+        nbytes = 2 * self.numel * 4 + self.numel + 4
+        res["cast_to_fp8_sharded"] = {
+            "what": "per-tensor e5m2 cast of fp32 v[64 Mi] split over the ranks: amax pass, int32 MAX "
+                    "all-reduce of 4 bytes, cast pass",
+            "elements_total": self.numel, "elements_this_rank": self.shard[1] - self.shard[0],
+            "us": round(ms * 1e3, 2), "bytes_total": nbytes, "gb_s_total": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "allreduce_bytes": 4, "scale_inv_identical_on_all_ranks": same}
+        R = fp8q.record_bytes(self.gather_elems)
+        ms8 = self._time(self.gather_fp8, reps, warmup)
+        gathered = self.world * self.gather_elems * 2          # bf16 bytes every rank ends up with
+        e = {"what": "each rank's bf16 shard cast into a [scale | e5m2 codes] record, one NCCL all-gather "
+                     "of the records, every record dequantised to bf16",
+             "elements_per_rank": self.gather_elems, "record_bytes": R,
+             "wire_bytes_received_per_rank": (self.world - 1) * R,
+             "bf16_wire_bytes_received_per_rank": (self.world - 1) * 2 * self.gather_elems,
+             "us": round(ms8 * 1e3, 2), "bf16_gb_s_gathered": round(gathered / (ms8 * 1e-3) / 1e9, 1)}
+        if self.world > 1:
+            ms16 = self._time(self.gather_bf16, reps, warmup)
+            e["nccl_bf16_all_gather_us"] = round(ms16 * 1e3, 2)
+            e["nccl_bf16_gb_s_gathered"] = round(gathered / (ms16 * 1e-3) / 1e9, 1)
+            e["speedup_vs_bf16"] = round(ms16 / ms8, 3)
+        res["all_gather_fp8"] = e
+        res["ranks"] = self.world
+        return res
+
+
+def _device_timer(fn, reps, device):
+    """Milliseconds per call of fn: CUDA events around `reps` calls on the current stream."""
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize(device)
+    return e0.elapsed_time(e1) / reps
+
+
 def pcie_bound(h2d_bytes: int, d2h_bytes: int, device, n: int = 1 << 30):
     """The fastest the end-to-end step's transfers can go on this machine: pinned copies of n bytes
     each way, alone and both at once (CUDA events), then the step's bytes moved both ways at the
@@ -328,16 +466,31 @@ def pcie_bound(h2d_bytes: int, d2h_bytes: int, device, n: int = 1 << 30):
             "bound_ms_per_step": round(ms, 3)}
 
 
+def _quantile(v, q):
+    """The q-quantile of a sorted list (nearest rank)."""
+    return v[min(len(v) - 1, int(round(q * (len(v) - 1))))]
+
+
 def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
     """Each op the metric names, timed alone in a steady state: the op runs
-    back to back over `sets` copies of its buffers, rotating, with the sets
-    together at least 4x the L2 size, so every launch reads cold inputs and
-    pays for the write-back of exactly one launch's outputs (its own kind).
-    Returns {op name: {"us", "gb_s", "sets"}} (mean over `launches`)."""
+    over `sets` copies of its buffers, rotating, with the sets together at
+    least 4x the L2 size, so every launch reads cold inputs and pays for the
+    write-back of exactly one launch's outputs (its own kind).
+
+    `us` and its p10 / p50 / p90 come from `blocks` blocks of launches run
+    back to back, one event pair per block (the per-launch mean of each
+    block is one sample).  An event pair around every single launch is
+    reported too (`us_event_per_launch`), but it overstates a short kernel:
+    an event between two kernels serialises them and exposes the launch
+    latency that back-to-back launches hide under programmatic dependent
+    launch (measured on B200: 19.6 us against 13.6 us for the 89 MB
+    per-token quant)."""
     f = wl.fp8q
     d = wl.device
     l2 = torch.cuda.get_device_properties(d).L2_cache_size
     need = max(4 * l2, min_footprint)
+    blocks = 10
+    per_block = max(1, launches // blocks)
     out = {}
 
     def run(name, make_set, footprint, nbytes):
@@ -345,14 +498,30 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
         for fn in sets:
             fn()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for k in range(launches):
-            sets[k % len(sets)]()
-        e1.record()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(blocks)]
+        k = 0
+        for b in range(blocks):
+            evs[b][0].record()
+            for _ in range(per_block):
+                sets[k % len(sets)]()
+                k += 1
+            evs[b][1].record()
         torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / launches
-        out[name] = {"us": round(us, 2), "gb_s": round(nbytes / (us * 1e-6) / 1e9, 1), "sets": len(sets)}
+        blk = sorted(a.elapsed_time(e) * 1e3 / per_block for a, e in evs)
+        one = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+        for j in range(launches):
+            one[j][0].record()
+            sets[j % len(sets)]()
+            one[j][1].record()
+        torch.cuda.synchronize()
+        durs = sorted(a.elapsed_time(e) * 1e3 for a, e in one)
+        us = statistics.median(blk)
+        out[name] = {"us": round(us, 2), "gb_s": round(nbytes / (us * 1e-6) / 1e9, 1),
+                     "us_p10_p50_p90": [round(_quantile(blk, q), 2) for q in (0.1, 0.5, 0.9)],
+                     "launches": blocks * per_block, "blocks": blocks,
+                     "us_event_per_launch": round(statistics.median(durs), 2),
+                     "us_event_per_launch_p10_p50_p90": [round(_quantile(durs, q), 2) for q in (0.1, 0.5, 0.9)],
+                     "sets": len(sets)}
         del sets
         torch.cuda.empty_cache()
 
@@ -402,6 +571,13 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
         return lambda: f.fp8q_cast_per_tensor(x, q, s, wl.ws, E5M2)
     run("cast_per_tensor_f32_e5m2", per_tensor_set, n4 * 5 + 4, c4b_bytes)
     return out
+
+
+def _raiser(msg: str):
+    """A stand-in for a library call that is unavailable here: raises with the reason."""
+    def fn():
+        raise RuntimeError(msg)
+    return fn
 
 
 class MatmulWorkload:
@@ -461,25 +637,97 @@ class MatmulWorkload:
         res = self.time_decode(steps, warmup, device)
         res.update(self.time_products(steps, warmup, device))
         res.update(self.time_linear(steps, warmup, device))
+        res["sustained 2 s"] = self.time_sustained(device)
         if int(self.status.item()) != 0:
             raise RuntimeError("a bounded wait of the fp8 product ran out")
         return res
 
-    def time_products(self, steps: int, warmup: int, device):
-        """The two products on the full workload, and torch._scaled_mm (cuBLASLt) on the same
-        operands for context."""
-        ops = dict(self.ops)
+    def library_ops(self):
+        """Library products on the same operands, for context: torch._scaled_mm (cuBLASLt) with
+        per-tensor scales; for the fine-grained scales, torch's blockwise scaled_mm (1 x 128 and
+        128 x 128, which this torch build serves on sm_90 only) and vLLM's CUTLASS blockwise
+        product (cutlass_scaled_mm: activation scales M-major, the weight and its block scales
+        passed transposed, as vLLM's own block-fp8 linear passes them)."""
         a8 = self.q.view(torch.float8_e4m3fn)
         b8 = self.w.view(torch.float8_e4m3fn)
-        ops["torch_scaled_mm (cuBLASLt)"] = lambda: torch._scaled_mm(a8, b8.t(), scale_a=self.s1, scale_b=self.s2,
-                                                                    out_dtype=torch.bfloat16)
+        ops = {"torch_scaled_mm (cuBLASLt)": lambda: torch._scaled_mm(a8, b8.t(), scale_a=self.s1, scale_b=self.s2,
+                                                                      out_dtype=torch.bfloat16)}
+
+        def torch_blockwise():
+            import torch.nn.functional as F
+            st = F.ScalingType
+            return F.scaled_mm(a8, b8.t(), self.sa, st.BlockWise1x128, self.sb, st.BlockWise128x128,
+                               output_dtype=torch.bfloat16)
+        ops["torch scaled_mm blockwise (1x128, 128x128)"] = torch_blockwise
+        try:
+            import vllm._custom_ops as vops
+            sa_mn = self.sa.t().contiguous().t()
+            sb_t = self.sb.t()
+            out = torch.empty_like(self.out)
+            ops["vllm cutlass_scaled_mm blockwise (CUTLASS sm100)"] = (
+                lambda: torch.ops._C.cutlass_scaled_mm(out, a8, b8.t(), sa_mn, sb_t, None) or out)
+            major, minor = torch.cuda.get_device_capability()
+            if not vops.cutlass_scaled_mm_supports_block_fp8(major * 10 + minor):
+                raise RuntimeError("vLLM reports no block-fp8 CUTLASS product for this device")
+        except Exception as ex:     # vLLM or its compiled ops missing on this box
+            msg = str(ex).splitlines()[0][:200] if str(ex) else type(ex).__name__
+            ops["vllm cutlass_scaled_mm blockwise (CUTLASS sm100)"] = _raiser(msg)
+        return ops
+
+    def time_products(self, steps: int, warmup: int, device):
+        """The two products on the full workload, and the library products (library_ops) on the
+        same operands for context; each library output is compared with libfp8q's once."""
+        ops = dict(self.ops)
+        lib_ops = self.library_ops()
+        ops.update(lib_ops)
+        ref = {}
+        for name, fn in self.ops.items():
+            fn()
+            ref[name] = self.out.float().clone()
         res = {}
         for name, fn in ops.items():
             try:
                 ms, clk = self._timed(fn, steps, warmup, device)
                 res[name] = {"ms": round(ms, 4), "tflops": round(self.flops / (ms * 1e-3) / 1e12, 1), "clocks": clk}
-            except Exception as ex:      # the library baseline may be missing on some builds of torch
-                res[name] = {"unavailable": str(ex).splitlines()[0][:200]}
+                if name in lib_ops:
+                    y = fn().float()
+                    r = ref["scaled_mm_blockwise" if "blockwise" in name else "scaled_mm_per_tensor"]
+                    res[name]["max_abs_diff_over_max_abs_vs_libfp8q"] = float((y - r).abs().max() / r.abs().max())
+            except Exception as ex:      # the library baseline may be missing on some builds
+                res[name] = {"unavailable": str(ex).splitlines()[0][:200] if str(ex) else type(ex).__name__}
+        del ref
+        return res
+
+    def time_sustained(self, device, seconds: float = 2.0):
+        """Each product back to back for `seconds` (CUDA events around the run, NVML clocks and
+        power sampled during it): under the board's 1000 W cap a dense product settles at lowered
+        SM clocks after the first tens of milliseconds, which the short timings above precede."""
+        ops = dict(self.ops)
+        lib = self.library_ops()
+        for k in ("torch_scaled_mm (cuBLASLt)", "vllm cutlass_scaled_mm blockwise (CUTLASS sm100)"):
+            ops[k] = lib[k]
+        res = {}
+        for name, fn in ops.items():
+            try:
+                fn()
+                torch.cuda.synchronize(device)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                n = 0
+                with ClockSampler(device.index or 0, period_s=0.02, power=True) as clk:
+                    t0 = time.perf_counter()
+                    e0.record()
+                    while time.perf_counter() - t0 < seconds:
+                        for _ in range(10):
+                            fn()
+                        n += 10
+                        torch.cuda.synchronize(device)
+                    e1.record()
+                    torch.cuda.synchronize(device)
+                ms = e0.elapsed_time(e1) / n
+                res[name] = {"ms": round(ms, 4), "tflops": round(self.flops / (ms * 1e-3) / 1e12, 1), "launches": n,
+                             "clocks": clk.summary()}
+            except Exception as ex:
+                res[name] = {"unavailable": str(ex).splitlines()[0][:200] if str(ex) else type(ex).__name__}
         return res
 
     def time_decode(self, steps: int, warmup: int, device):
@@ -527,15 +775,18 @@ class MatmulWorkload:
                                                 "clocks": clk}}
 
 
-def fp8_tensor_peak():
-    """Dense fp8 tensor-core peak: the measured cuBLAS bf16 burst figure times
-    the nominal fp8 : bf16 ratio of 2."""
+def fp8_tensor_peak(sustained: bool = False):
+    """Dense fp8 tensor-core peak: the measured cuBLAS bf16 figure (burst, or the seconds-long
+    loop under the power cap) times the nominal fp8 : bf16 ratio of 2."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    kind = "sustained" if sustained else "burst"
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return 2.0 * float(d["bf16_tflops"]), "2 x measured bf16 burst (nominal fp8:bf16 ratio)"
-    return 2.0 * 1590.0, "2 x fallback bf16 burst (nominal fp8:bf16 ratio)"
+        if key in d:
+            return 2.0 * float(d[key]), f"2 x measured bf16 {kind} (nominal fp8:bf16 ratio)"
+    return 2.0 * (1400.0 if sustained else 1590.0), f"2 x fallback bf16 {kind} (nominal fp8:bf16 ratio)"
 
 
 def _to_dev(a, device, dt=None):
@@ -565,9 +816,10 @@ class ClockSampler:
     REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, index: int, period_s: float = 0.005):
-        self.index, self.period = index, period_s
+    def __init__(self, index: int, period_s: float = 0.005, power: bool = False):
+        self.index, self.period, self.power = index, period_s, power
         self.samples, self.reasons, self.max_mhz, self.ok = [], set(), None, False
+        self.watts = []
         self._stop = threading.Event()
         try:
             import pynvml
@@ -582,6 +834,8 @@ class ClockSampler:
     def _sample(self):
         nv = self.nv
         self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        if self.power:
+            self.watts.append(nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
         r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
         for k, bit in self.REASONS.items():
             if r & bit:
@@ -614,8 +868,11 @@ class ClockSampler:
     def summary(self):
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        d = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+             "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        if self.power and self.watts:
+            d["power_w_median"] = round(statistics.median(self.watts), 1)
+        return d
 
 
 # ---------------------------------------------------------------------------
@@ -770,7 +1027,7 @@ def dist_setup(ngpus):
         import datetime
         import torch.distributed as dist
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     return world, rank, local
 
@@ -849,6 +1106,13 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e2e.time(e2e_steps), world, device)
     bi, bo = e2e.h2d_bytes, e2e.d2h_bytes
     del e2e
+    sharded = None
+    if world > 1 or args.sharded:
+        leg = ShardedLeg(device, rank, world, h["c4b_v"], kernels=LegKernels(fp8q),
+                         ws_bytes=fp8q.fp8q_cast_per_tensor_workspace_bytes())
+        sharded = leg.run()
+        del leg
+        torch.cuda.empty_cache()
     pcie = pcie_bound(bi, bo, device) if rank == 0 else None
     iso = isolated_timing(wl) if rank == 0 else {}
     mm = None
@@ -856,8 +1120,14 @@ def run_ours(args):
         mmw = MatmulWorkload(wl)
         mm_res = mmw.time(max(5, min(args.steps, 50)), max(3, args.warmup), device)
         tpeak, tkind = fp8_tensor_peak()
+        tpeak_s, tkind_s = fp8_tensor_peak(sustained=True)
         hpeak, _ = measured_peaks()
-        for v in mm_res.values():
+        for name, v in mm_res.items():
+            if name.startswith("sustained"):
+                for e in v.values():
+                    if "tflops" in e:
+                        e["frac_of_sustained_peak"] = round(e["tflops"] / tpeak_s, 4)
+                continue
             if "tflops" in v:
                 v["frac"] = round(v["tflops"] / tpeak, 4)
             if "gb_s" in v:
@@ -867,6 +1137,7 @@ def run_ours(args):
                           "one scale each",
               "shape_mnk": list(mmw.shape), "flops_per_launch": mmw.flops, "bound": "tensor",
               "peak_tflops": round(tpeak, 1), "peak_kind": tkind,
+              "sustained_peak_tflops": round(tpeak_s, 1), "sustained_peak_kind": tkind_s,
               "l2": "operands 161 MB > 126 MB L2; compute-bound, no flush", "ops": mm_res}
         del mmw
 
@@ -875,8 +1146,7 @@ def run_ours(args):
         return
     peak, peak_kind = measured_peaks()
     kernels = {}
-    def pct(v, q):
-        return v[min(len(v) - 1, int(round(q * (len(v) - 1))))]
+    pct = _quantile
     for op, ms, v in zip(wl.ops, per_op_ms, per_op_samples):
         gbs = op.bytes / (ms * 1e-3) / 1e9
         kernels[op.name] = {"us": round(ms * 1e3, 2), "us_mean": round(statistics.mean(v) * 1e3, 2),
@@ -902,7 +1172,8 @@ def run_ours(args):
                      "bytes_per_launch": dop.bytes, "traffic": recorded_traffic(dop.name)},
         "kernels": kernels,
         "kernels_from": f"{split_steps} instrumented steps before the timed ones (events around every op)",
-        "isolated": {k: {**v, "frac": round(v["gb_s"] / peak, 4)} for k, v in iso.items()},
+        "isolated": {k: {**v, "frac": round(v["gb_s"] / peak, 4),
+                         "pct_of_nominal_8tbs": round(100.0 * v["gb_s"] / 8000.0, 2)} for k, v in iso.items()},
         "matmul": mm,
         "clocks": clk.summary(),
         "e2e": {"value": round(world * wl.step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
@@ -911,10 +1182,58 @@ def run_ours(args):
                 "frac_of_pcie_bound": round(pcie["bound_ms_per_step"] / e2e_ms, 4) if pcie else None},
         "gpu_launches": wl.launches_per_step * args.steps,
     }
+    if sharded is not None:
+        line["sharded"] = sharded
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(h)
     print(json.dumps(line), flush=True)
     _finish(world)
+
+
+def run_marginal(args):
+    """Each op's marginal cost inside the live step, measured by adding work, never by skipping
+    it: the step with one more instance of op i appended at its end (after the 3 GB grouped
+    dequant, so the extra instance's inputs are cold and the op before it leaves dirty L2
+    lines, as in the step), minus the plain step.  Rounds alternate the plain step and each
+    extended step; the medians over rounds are reported.  Prints one JSON line."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    import dequantisation_fp8q_token_b200 as fp8q
+    fp8q.lib()
+    wl = Workload(device, fp8q, make_host_inputs())
+    steps, rounds = max(5, args.steps // 10), 5
+
+    def timed(extra):
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            wl.step()
+            if extra is not None:
+                extra.fn()
+        e1.record()
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / steps
+
+    for _ in range(max(3, args.warmup)):
+        wl.step()
+    base, extra = [], {op.name: [] for op in wl.ops}
+    with ClockSampler(0) as clk:
+        for _ in range(rounds):
+            base.append(timed(None))
+            for op in wl.ops:
+                extra[op.name].append(timed(op))
+    peak, peak_kind = measured_peaks()
+    b = statistics.median(base)
+    res = {}
+    for op in wl.ops:
+        us = (statistics.median(extra[op.name]) - b) * 1e3
+        res[op.name] = {"marginal_us": round(us, 2), "bytes": op.bytes,
+                        "gb_s": round(op.bytes / (us * 1e-6) / 1e9, 1) if us > 0 else None,
+                        "frac": round(op.bytes / (us * 1e-6) / 1e9 / peak, 4) if us > 0 else None}
+    print(json.dumps({"marginal": res, "step_us_median": round(b * 1e3, 2), "steps_per_timing": steps,
+                      "rounds": rounds, "peak_gb_s": peak, "peak_kind": peak_kind, "clocks": clk.summary(),
+                      "sum_of_marginals_us": round(sum(v["marginal_us"] for v in res.values()), 2)}), flush=True)
 
 
 def _finish(world):
@@ -1094,9 +1413,16 @@ def main(argv=None):
                     help="run one op of a fixed case --iters times for a profiler capture (no timing)")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--no-matmul", action="store_true", help="skip the fp8 products section")
+    ap.add_argument("--marginal", action="store_true",
+                    help="print each op's marginal cost inside the live step (one JSON line) and exit")
+    ap.add_argument("--sharded", action="store_true",
+                    help="run the sharded exchange leg at N = 1 too (it always runs when N > 1)")
     args = ap.parse_args(argv)
     if args.profile:
         run_profile_case(args.profile, args.iters)
+        return
+    if args.marginal:
+        run_marginal(args)
         return
     args.warmup = max(3, args.warmup)   # the timing rules want at least 3 untimed steps
     args.steps = max(1, args.steps)
