@@ -50,6 +50,7 @@ __all__ = [
     "per_token_cast_to_fp8", "per_token_cast_back", "cast_to_fp8", "cast_from_fp8", "weight_dequant",
     "cast_to_fp8_pipeline", "cast_from_fp8_pipeline",
     "RECORD_HEADER_BYTES", "record_bytes", "fp8q_record_bytes", "fp8q_pack_record", "fp8q_unpack_records",
+    "RECORD_PACKED4", "RECORD_ALIGNED16", "fp8q_record_bytes_ex", "fp8q_pack_record_ex", "fp8q_unpack_records_ex",
     "exchange_records", "exchange_records_all_to_all", "exchange_payload_all_to_all", "all_gather_fp8", "all_to_all_fp8", "all_to_all_single_fp8",
     "fp8q_scaled_mm", "fp8q_scaled_mm_blockwise", "scaled_mm", "scaled_mm_blockwise", "linear_fp8",
     "linear_fp8_blockwise", "fp8q_transpose_fp8", "fp8q_sum_rows", "transpose_fp8", "fp8q_scaled_mm_ex",
@@ -61,6 +62,7 @@ F32, F16, BF16 = 0, 1, 2
 GRAN_TENSOR, GRAN_ROW, GRAN_GROUP, GRAN_BLOCK = 0, 1, 2, 3
 SCALE_IEEE, SCALE_TORCH = 0, 1
 K_MAJOR, MN_MAJOR = 0, 1
+RECORD_PACKED4, RECORD_ALIGNED16 = 4, 16     # fp8q_record_layout: the page's 4-byte header / 16-byte aligned
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libfp8q.so")
@@ -141,6 +143,12 @@ def lib() -> ctypes.CDLL:
             L.fp8q_pack_record.argtypes = [p, i32, i64, i32, p, p, ctypes.c_size_t, i32, p]
             L.fp8q_unpack_records.restype = st
             L.fp8q_unpack_records.argtypes = [p, i32, i64, i32, i32, p, p]
+            L.fp8q_record_bytes_ex.restype = ctypes.c_size_t
+            L.fp8q_record_bytes_ex.argtypes = [i64, i32]
+            L.fp8q_pack_record_ex.restype = st
+            L.fp8q_pack_record_ex.argtypes = [p, i32, i64, i32, p, p, ctypes.c_size_t, i32, i32, p]
+            L.fp8q_unpack_records_ex.restype = st
+            L.fp8q_unpack_records_ex.argtypes = [p, i32, i64, i32, i32, p, i32, p]
             L.fp8q_scaled_mm.restype = st
             L.fp8q_scaled_mm.argtypes = [p, i32, p, i32, i64, i64, i64, p, p, p, i32, p, p, p]
             L.fp8q_scaled_mm_wait_test.restype = st
@@ -573,13 +581,22 @@ def cast_from_fp8_pipeline(q: torch.Tensor, scale_inv: torch.Tensor, fmt_tag: to
 RECORD_HEADER_BYTES = 16
 
 
-def record_bytes(numel: int) -> int:
-    """Size of one record: a 16-byte header (fp32 scale_inv, then zeros) and
-    the fp8 payload padded with zeros to a multiple of 16 bytes.  The same
-    arithmetic as fp8q_record_bytes, on the host, so that buffers can be sized
-    without loading the library."""
+def _layout_of(layout) -> int:
+    if layout not in (RECORD_PACKED4, RECORD_ALIGNED16):
+        raise ValueError("record layout must be RECORD_PACKED4 (4) or RECORD_ALIGNED16 (16)")
+    return int(layout)
+
+
+def record_bytes(numel: int, layout: int = RECORD_ALIGNED16) -> int:
+    """Size of one record: RECORD_ALIGNED16, a 16-byte header (fp32 scale_inv,
+    then zeros) and the fp8 payload padded with zeros to a multiple of 16
+    bytes; RECORD_PACKED4, the page's own layout, the 4-byte scale then the
+    codes.  The same arithmetic as fp8q_record_bytes_ex, on the host, so that
+    buffers can be sized without loading the library."""
     if numel < 0:
         raise ValueError("numel must be >= 0")
+    if _layout_of(layout) == RECORD_PACKED4:
+        return 4 + numel
     return RECORD_HEADER_BYTES + -(-numel // 16) * 16
 
 
@@ -587,27 +604,44 @@ def fp8q_record_bytes(numel: int) -> int:
     return int(lib().fp8q_record_bytes(int(numel)))
 
 
+def fp8q_record_bytes_ex(numel: int, layout: int = RECORD_ALIGNED16) -> int:
+    return int(lib().fp8q_record_bytes_ex(int(numel), int(layout)))
+
+
 def fp8q_pack_record(x: torch.Tensor, record: torch.Tensor, workspace: torch.Tensor, fmt=E5M2,
                      rule=SCALE_IEEE, stream=None) -> None:
     """Per-tensor cast of x into one record (uint8, record_bytes(x.numel()) bytes)."""
+    fp8q_pack_record_ex(x, record, workspace, fmt, rule, RECORD_ALIGNED16, stream)
+
+
+def fp8q_pack_record_ex(x: torch.Tensor, record: torch.Tensor, workspace: torch.Tensor, fmt=E5M2,
+                        rule=SCALE_IEEE, layout: int = RECORD_ALIGNED16, stream=None) -> None:
+    """Per-tensor cast of x into one record of the given layout (uint8, record_bytes(numel, layout))."""
     dev = x.device
     n = x.numel()
-    _need(record, record_bytes(n), "record", byte=True)
+    _need(record, record_bytes(n, layout), "record", byte=True)
     wbytes = workspace.numel() * workspace.element_size()
-    _check(lib().fp8q_pack_record(
+    _check(lib().fp8q_pack_record_ex(
         _dev_ptr(x, "x"), _dtype_code(x, "x"), n, _fmt_of(fmt), _dev_ptr(record, "record", dev),
-        _dev_ptr(workspace, "workspace", dev), wbytes, _rule_of(rule), _stream(stream, dev)), "fp8q_pack_record")
+        _dev_ptr(workspace, "workspace", dev), wbytes, _rule_of(rule), _layout_of(layout), _stream(stream, dev)),
+        "fp8q_pack_record_ex")
 
 
 def fp8q_unpack_records(records: torch.Tensor, count: int, numel: int, y: torch.Tensor, fmt=E5M2,
                         stream=None) -> None:
     """Dequantise `count` back-to-back records of `numel` codes into y[count * numel] (dtype of y)."""
+    fp8q_unpack_records_ex(records, count, numel, y, fmt, RECORD_ALIGNED16, stream)
+
+
+def fp8q_unpack_records_ex(records: torch.Tensor, count: int, numel: int, y: torch.Tensor, fmt=E5M2,
+                           layout: int = RECORD_ALIGNED16, stream=None) -> None:
+    """Dequantise `count` back-to-back records of the given layout into y[count * numel]."""
     dev = records.device
-    _need(records, count * record_bytes(numel), "records", byte=True)
+    _need(records, count * record_bytes(numel, layout), "records", byte=True)
     _need(y, count * numel, "y")
-    _check(lib().fp8q_unpack_records(
+    _check(lib().fp8q_unpack_records_ex(
         _dev_ptr(records, "records"), int(count), int(numel), _fmt_of(fmt), _dtype_code(y, "y"),
-        _dev_ptr(y, "y", dev), _stream(stream, dev)), "fp8q_unpack_records")
+        _dev_ptr(y, "y", dev), _layout_of(layout), _stream(stream, dev)), "fp8q_unpack_records_ex")
 
 
 def exchange_records(combined: torch.Tensor, group=None) -> None:
@@ -652,29 +686,31 @@ def _world_rank(group):
 
 
 def all_gather_fp8(output_list, input_: torch.Tensor, group=None, fp8_format: str = "e5m2",
-                   rule=SCALE_IEEE) -> None:
+                   rule=SCALE_IEEE, layout: int = RECORD_ALIGNED16) -> None:
     """ColossalAI all_gather_fp8 (and all_gather_fp8_lagacy): every rank casts
     its tensor with its own per-tensor scale into a record, one all-gather
     moves the records, and each output_list[r] receives rank r's tensor
     dequantised with rank r's scale, in input_'s dtype.  output_list may
-    also be one contiguous tensor [world, *input_.shape]."""
+    also be one contiguous tensor [world, *input_.shape].  layout
+    RECORD_PACKED4 puts the page's own bytes on the wire (4-byte scale, then
+    the codes; numel a multiple of 4 when there is more than one rank)."""
     world, rank = _world_rank(group)
     dev = input_.device
     n = input_.numel()
     f = _fmt_of(fp8_format)
-    R = record_bytes(n)
+    R = record_bytes(n, layout)
     combined = torch.empty(world * R, dtype=torch.uint8, device=dev)
-    fp8q_pack_record(input_, combined[rank * R:(rank + 1) * R], _workspace(dev), f, rule)
+    fp8q_pack_record_ex(input_, combined[rank * R:(rank + 1) * R], _workspace(dev), f, rule, layout)
     exchange_records(combined, group)
     if isinstance(output_list, torch.Tensor):
         if output_list.numel() != world * n or not output_list.is_contiguous():
             raise ValueError("the output tensor must be contiguous with world * input_.numel() elements")
-        fp8q_unpack_records(combined, world, n, output_list, f)
+        fp8q_unpack_records_ex(combined, world, n, output_list, f, layout)
         return
     if len(output_list) != world:
         raise ValueError(f"output_list has {len(output_list)} tensors, the group has {world} ranks")
     for r, out in enumerate(output_list):
-        fp8q_unpack_records(combined[r * R:(r + 1) * R], 1, n, out, f)
+        fp8q_unpack_records_ex(combined[r * R:(r + 1) * R], 1, n, out, f, layout)
 
 
 def all_to_all_fp8(output_list, input_list, group=None, fp8_format: str = "e5m2", rule=SCALE_IEEE) -> None:

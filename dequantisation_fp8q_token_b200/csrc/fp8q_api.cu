@@ -197,19 +197,26 @@ fp8q_status fp8q_cast_from_pipeline(const uint8_t* q, int64_t numel, const float
     return launch_cast_from_pipeline(q, numel, scale_inv, fmt_tag, yt, y, reinterpret_cast<cudaStream_t>(stream));
 }
 
-size_t fp8q_record_bytes(int64_t numel) {
-    if (numel < 0) return 0;
+static bool layout_ok(int layout) { return layout == FP8Q_RECORD_PACKED4 || layout == FP8Q_RECORD_ALIGNED16; }
+
+size_t fp8q_record_bytes_ex(int64_t numel, fp8q_record_layout layout) {
+    if (numel < 0 || !layout_ok(layout)) return 0;
+    if (layout == FP8Q_RECORD_PACKED4) return (size_t)(4 + numel);
     return (size_t)(16 + ((numel + 15) / 16) * 16);
 }
 
-fp8q_status fp8q_pack_record(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt, uint8_t* record,
-                             void* workspace, size_t workspace_bytes, fp8q_scale_rule rule, fp8q_stream_t stream) {
+size_t fp8q_record_bytes(int64_t numel) { return fp8q_record_bytes_ex(numel, FP8Q_RECORD_ALIGNED16); }
+
+fp8q_status fp8q_pack_record_ex(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt, uint8_t* record,
+                                void* workspace, size_t workspace_bytes, fp8q_scale_rule rule,
+                                fp8q_record_layout layout, fp8q_stream_t stream) {
     if (!dtype_ok(xt)) return FP8Q_ERR_BAD_DTYPE;
     if (!rule_ok(rule)) return FP8Q_ERR_BAD_RULE;
     if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
+    if (!layout_ok(layout)) return FP8Q_ERR_BAD_SHAPE;
     if (numel < 0 || checked_mul(numel, dtype_bytes(xt)) < 0) return FP8Q_ERR_BAD_SHAPE;
     if (!record) return FP8Q_ERR_NULL_POINTER;
-    if (!aligned(record, 16)) return FP8Q_ERR_MISALIGNED;
+    if (!aligned(record, layout == FP8Q_RECORD_PACKED4 ? 4 : 16)) return FP8Q_ERR_MISALIGNED;
     // every check of the cast below, before the header memsets are enqueued
     if (numel > 0) {
         if (!x) return FP8Q_ERR_NULL_POINTER;
@@ -218,29 +225,42 @@ fp8q_status fp8q_pack_record(const void* x, fp8q_dtype xt, int64_t numel, fp8q_f
             return FP8Q_ERR_WORKSPACE;
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // header padding and the payload's last partial 16-byte block start at zero
-    if (cudaMemsetAsync(record, 0, 16, s) != cudaSuccess) return FP8Q_ERR_CUDA;
-    if (numel % 16 && cudaMemsetAsync(record + 16 + (numel / 16) * 16, 0, 16, s) != cudaSuccess)
-        return FP8Q_ERR_CUDA;
-    return fp8q_cast_per_tensor_ex(x, xt, numel, fmt, record + 16, reinterpret_cast<float*>(record), workspace,
+    const int head = layout == FP8Q_RECORD_PACKED4 ? 4 : 16;
+    if (layout == FP8Q_RECORD_ALIGNED16) {
+        // header padding and the payload's last partial 16-byte block start at zero
+        if (cudaMemsetAsync(record, 0, 16, s) != cudaSuccess) return FP8Q_ERR_CUDA;
+        if (numel % 16 && cudaMemsetAsync(record + 16 + (numel / 16) * 16, 0, 16, s) != cudaSuccess)
+            return FP8Q_ERR_CUDA;
+    }
+    return fp8q_cast_per_tensor_ex(x, xt, numel, fmt, record + head, reinterpret_cast<float*>(record), workspace,
                                    workspace_bytes, rule, stream);
 }
 
-fp8q_status fp8q_unpack_records(const uint8_t* records, int count, int64_t numel, fp8q_format fmt, fp8q_dtype yt,
-                                void* y, fp8q_stream_t stream) {
+fp8q_status fp8q_pack_record(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt, uint8_t* record,
+                             void* workspace, size_t workspace_bytes, fp8q_scale_rule rule, fp8q_stream_t stream) {
+    return fp8q_pack_record_ex(x, xt, numel, fmt, record, workspace, workspace_bytes, rule, FP8Q_RECORD_ALIGNED16,
+                               stream);
+}
+
+fp8q_status fp8q_unpack_records_ex(const uint8_t* records, int count, int64_t numel, fp8q_format fmt,
+                                   fp8q_dtype yt, void* y, fp8q_record_layout layout, fp8q_stream_t stream) {
     if (!fmt_ok(fmt)) return FP8Q_ERR_BAD_FORMAT;
     if (!dtype_ok(yt)) return FP8Q_ERR_BAD_DTYPE;
+    if (!layout_ok(layout)) return FP8Q_ERR_BAD_SHAPE;
     if (count < 0) return FP8Q_ERR_TOO_MANY;
     if (numel < 0 || checked_mul(checked_mul(numel, count), dtype_bytes(yt)) < 0) return FP8Q_ERR_BAD_SHAPE;
     if (count == 0 || numel == 0) return FP8Q_OK;
     if (!records || !y) return FP8Q_ERR_NULL_POINTER;
-    if (!aligned(records, 16) || !aligned(y, dtype_bytes(yt))) return FP8Q_ERR_MISALIGNED;
+    const bool packed = layout == FP8Q_RECORD_PACKED4;
+    if (!aligned(records, packed ? 4 : 16) || !aligned(y, dtype_bytes(yt))) return FP8Q_ERR_MISALIGNED;
+    if (packed && count > 1 && numel % 4) return FP8Q_ERR_MISALIGNED;   // record r's scale at r * (4 + numel)
     // each record's payload as a [numel / 4096][4096] matrix plus a one-row
     // tail, both with the header's single scale: a block edge above any size
     // makes every element's scale index 0
     constexpr int64_t kCols = 4096;
     const int64_t body_rows = numel / kCols, tail = numel % kCols;
-    const size_t rec = fp8q_record_bytes(numel);
+    const size_t rec = fp8q_record_bytes_ex(numel, layout);
+    const int head = packed ? 4 : 16;
     const int yb = dtype_bytes(yt);
     // up to 48 records (96 problems) per launch; nothing is allocated
     constexpr int kBatch = 96;
@@ -250,8 +270,8 @@ fp8q_status fp8q_unpack_records(const uint8_t* records, int count, int64_t numel
         const uint8_t* base = records + (size_t)r * rec;
         const float* sc = reinterpret_cast<const float*>(base);
         uint8_t* yr = static_cast<uint8_t*>(y) + (size_t)r * numel * yb;
-        if (body_rows) probs[n++] = DequantProblem{base + 16, sc, yr, body_rows, kCols};
-        if (tail) probs[n++] = DequantProblem{base + 16 + body_rows * kCols, sc, yr + body_rows * kCols * yb, 1, tail};
+        if (body_rows) probs[n++] = DequantProblem{base + head, sc, yr, body_rows, kCols};
+        if (tail) probs[n++] = DequantProblem{base + head + body_rows * kCols, sc, yr + body_rows * kCols * yb, 1, tail};
         if (n > kBatch - 2 || r == count - 1) {
             const fp8q_status st = launch_dequant(probs, n, fmt, kGranBlock, 1 << 30, yt,
                                                   reinterpret_cast<cudaStream_t>(stream));
@@ -260,6 +280,11 @@ fp8q_status fp8q_unpack_records(const uint8_t* records, int count, int64_t numel
         }
     }
     return FP8Q_OK;
+}
+
+fp8q_status fp8q_unpack_records(const uint8_t* records, int count, int64_t numel, fp8q_format fmt, fp8q_dtype yt,
+                                void* y, fp8q_stream_t stream) {
+    return fp8q_unpack_records_ex(records, count, numel, fmt, yt, y, FP8Q_RECORD_ALIGNED16, stream);
 }
 
 fp8q_status fp8q_block_dequant(const uint8_t* w, fp8q_format fmt, int64_t M, int64_t N,

@@ -21,8 +21,9 @@
  *   fp8q_cast_per_tensor_with_amax  ranks (ColossalAI FSDP params hook)
  *   fp8q_cast_pipeline,         ColossalAI cast_to_fp8_pipeline /
  *   fp8q_cast_from_pipeline     cast_from_fp8_pipeline
- *   fp8q_pack_record,           ColossalAI all_gather_fp8: the [scale |
- *   fp8q_unpack_records         payload] records
+ *   fp8q_pack_record(_ex),      ColossalAI all_gather_fp8: the [scale |
+ *   fp8q_unpack_records(_ex)    payload] records (_ex: the page's packed
+ *                               4-byte-header layout as well)
  *   fp8q_*_ex                   torch's rounding of the scale expressions
  *   fp8q_scaled_mm_wait_test    a test of the products' bounded waits
  *
@@ -284,7 +285,8 @@ fp8q_status fp8q_cast_from_pipeline(const uint8_t* q, int64_t numel, const float
  *   bytes [0, 4)            fp32 scale_inv (fl(1 / scale) of the per-tensor cast)
  *   bytes [4, 16)           zero
  *   bytes [16, 16 + numel)  fp8 codes, then zero padding to a multiple of 16
- * (the page uses a 4-byte header; 16 keeps the payload 16-byte aligned), so
+ * (the page uses a 4-byte header, offered by the _ex calls below; 16 keeps
+ * the payload 16-byte aligned), so
  * records of equal numel can be gathered back to back by any byte-level
  * all-gather (NCCL all_gather_into_tensor on uint8).
  *   fp8q_record_bytes:   the record size for numel codes.
@@ -305,6 +307,32 @@ fp8q_status fp8q_pack_record(const void* x, fp8q_dtype xt, int64_t numel, fp8q_f
                              fp8q_stream_t stream);
 fp8q_status fp8q_unpack_records(const uint8_t* records, int count, int64_t numel, fp8q_format fmt,
                                 fp8q_dtype yt, void* y, fp8q_stream_t stream);
+
+/*
+ * The same records in either layout:
+ *   FP8Q_RECORD_PACKED4    the page's own layout (ColossalAI
+ *                          all_gather_fp8_lagacy, SCALE_BYTES = 4): bytes
+ *                          [0, 4) the fp32 scale_inv, bytes [4, 4 + numel)
+ *                          the codes, no padding; record r of a gathered
+ *                          buffer starts at r * (4 + numel).
+ *   FP8Q_RECORD_ALIGNED16  the layout above (16-byte header, payload padded
+ *                          to a multiple of 16); the calls without _ex.
+ * A packed record's scale is read and written as an fp32, so it must be
+ * 4-byte aligned: pack wants `record` 4-byte aligned, and unpack wants
+ * `records` 4-byte aligned and, when count > 1, numel a multiple of 4 (so
+ * that every record's scale is); otherwise FP8Q_ERR_MISALIGNED.  Its payload
+ * starts 4 bytes in and takes the narrower accesses of an unaligned tensor.
+ * fp8q_record_bytes_ex returns 0 for numel < 0 or an unknown layout; the
+ * other two return FP8Q_ERR_BAD_SHAPE for an unknown layout.  Everything
+ * else as fp8q_pack_record / fp8q_unpack_records.
+ */
+typedef enum { FP8Q_RECORD_PACKED4 = 4, FP8Q_RECORD_ALIGNED16 = 16 } fp8q_record_layout;
+size_t fp8q_record_bytes_ex(int64_t numel, fp8q_record_layout layout);
+fp8q_status fp8q_pack_record_ex(const void* x, fp8q_dtype xt, int64_t numel, fp8q_format fmt, uint8_t* record,
+                                void* workspace, size_t workspace_bytes, fp8q_scale_rule rule,
+                                fp8q_record_layout layout, fp8q_stream_t stream);
+fp8q_status fp8q_unpack_records_ex(const uint8_t* records, int count, int64_t numel, fp8q_format fmt,
+                                   fp8q_dtype yt, void* y, fp8q_record_layout layout, fp8q_stream_t stream);
 
 /*
  * Block dequantisation -- DeepSeek-V3 weight_dequant / weight_dequant_kernel:

@@ -300,35 +300,41 @@ def cast_from_fp8(q: np.ndarray, scale_inv: np.ndarray, gran: int, fmt: int = E4
 # are plain Python lists here.  The record is the sender's
 # [fp32 scale_inv | fp8 codes] buffer of all_gather_fp8_lagacy, with a
 # 16-byte header (scale_inv in bytes 0..3, zeros after) and the payload
-# zero-padded to a multiple of 16 bytes.
+# zero-padded to a multiple of 16 bytes, or (header 4) exactly the page's
+# 4-byte scale followed by the codes.
 # ---------------------------------------------------------------------------
 RECORD_HEADER = 16
 
 
-def record_size(numel: int) -> int:
+def record_size(numel: int, header: int = RECORD_HEADER) -> int:
+    """Bytes of one record.  header 16: 16-byte header, payload padded to a
+    multiple of 16.  header 4: the page's own layout (all_gather_fp8_lagacy,
+    SCALE_BYTES = 4), the scale then the codes, no padding."""
+    if header == 4:
+        return 4 + numel
     return RECORD_HEADER + ((numel + 15) // 16) * 16
 
 
-def record(x: np.ndarray, xt: int, fmt: int, rule: int = RULE_IEEE) -> np.ndarray:
+def record(x: np.ndarray, xt: int, fmt: int, rule: int = RULE_IEEE, header: int = RECORD_HEADER) -> np.ndarray:
     """The sender's record for tensor x: its per-tensor cast, header first."""
     q, s = cast_per_tensor(x, xt, fmt, rule=rule)
-    r = np.zeros((record_size(q.size),), np.uint8)
+    r = np.zeros((record_size(q.size, header),), np.uint8)
     r[0:4] = np.frombuffer(s.astype("<f4").tobytes(), np.uint8)
-    r[RECORD_HEADER:RECORD_HEADER + q.size] = q
+    r[header:header + q.size] = q
     return r
 
 
-def record_decode(r: np.ndarray, numel: int, fmt: int, yt: int) -> np.ndarray:
+def record_decode(r: np.ndarray, numel: int, fmt: int, yt: int, header: int = RECORD_HEADER) -> np.ndarray:
     """The receiver's step: cast_from_fp8 of the payload with the header's scale_inv."""
     s = np.frombuffer(r[0:4].tobytes(), "<f4").astype(np.float32)
-    q = r[RECORD_HEADER:RECORD_HEADER + numel].reshape(1, numel)
+    q = r[header:header + numel].reshape(1, numel)
     return cast_from_fp8(q, s, GRAN_TENSOR, fmt, yt=yt).reshape(-1)
 
 
-def all_gather_fp8(xs, xt: int, fmt: int, rule: int = RULE_IEEE):
+def all_gather_fp8(xs, xt: int, fmt: int, rule: int = RULE_IEEE, header: int = RECORD_HEADER):
     """xs[r] = rank r's tensor; returns out[r], which every rank receives:
     rank r's tensor cast with rank r's own scale and cast back to xt."""
-    return [record_decode(record(x, xt, fmt, rule), np.asarray(x).size, fmt, xt) for x in xs]
+    return [record_decode(record(x, xt, fmt, rule, header), np.asarray(x).size, fmt, xt, header) for x in xs]
 
 
 def all_to_all_fp8(inputs, xt: int, fmt: int, rule: int = RULE_IEEE):

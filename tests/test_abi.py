@@ -45,7 +45,8 @@ def test_enum_values_match_the_binding():
                       ("FP8Q_E4M3FN", fp8q.E4M3FN), ("FP8Q_E5M2", fp8q.E5M2), ("FP8Q_F32", fp8q.F32),
                       ("FP8Q_F16", fp8q.F16), ("FP8Q_BF16", fp8q.BF16), ("FP8Q_GRAN_TENSOR", fp8q.GRAN_TENSOR),
                       ("FP8Q_GRAN_ROW", fp8q.GRAN_ROW), ("FP8Q_GRAN_GROUP", fp8q.GRAN_GROUP),
-                      ("FP8Q_GRAN_BLOCK", fp8q.GRAN_BLOCK)]:
+                      ("FP8Q_GRAN_BLOCK", fp8q.GRAN_BLOCK), ("FP8Q_RECORD_PACKED4", fp8q.RECORD_PACKED4),
+                      ("FP8Q_RECORD_ALIGNED16", fp8q.RECORD_ALIGNED16)]:
         assert re.search(rf"\b{name}\s*=\s*{val}\b", src), name
 
 
@@ -317,6 +318,27 @@ def test_sharded_pipeline_and_record_validation(L):
     assert f(None, 2, 8, 0, 2, A, None) == 1                # null records
     assert f(A + 8, 2, 8, 0, 2, A, None) == 5               # records not 16-byte aligned
 
+    # the two record layouts (4: the page's packed [scale | codes]; 16: aligned)
+    rb = L.fp8q_record_bytes_ex
+    rb.restype, rb.argtypes = sz, [i64, i32]
+    assert [rb(n, 4) for n in (0, 1, 16, 17)] == [4, 5, 20, 21]
+    assert [rb(n, 16) for n in (0, 1, 16, 17)] == [16, 32, 32, 48]
+    assert rb(8, 8) == 0 and rb(-1, 4) == 0                 # unknown layout, negative numel
+
+    f = L.fp8q_pack_record_ex
+    f.argtypes = [vp, i32, i64, i32, vp, vp, sz, i32, i32, vp]
+    assert f(A, 0, 8, 0, A, A, ws, 0, 8, None) == 4         # unknown layout
+    assert f(A, 0, 8, 0, A + 2, A, ws, 0, 4, None) == 5     # packed record: its scale must be 4-byte aligned
+    assert f(A, 0, 8, 0, A + 4, A, ws, 0, 16, None) == 5    # aligned record: 16-byte aligned
+    assert f(None, 0, 8, 0, A + 4, A, ws, 0, 4, None) == 1  # packed, 4-byte aligned: on to the cast's checks
+
+    f = L.fp8q_unpack_records_ex
+    f.argtypes = [vp, i32, i64, i32, i32, vp, i32, vp]
+    assert f(A, 2, 8, 0, 2, A, 8, None) == 4                # unknown layout
+    assert f(A + 2, 2, 8, 0, 2, A, 4, None) == 5            # packed records not 4-byte aligned
+    assert f(A, 2, 6, 0, 2, A, 4, None) == 5                # record 1's scale at 4 + 6 bytes
+    assert f(None, 2, 8, 0, 2, A, 4, None) == 1             # null records
+
 
 def test_status_strings_and_version(L):
     L.fp8q_status_string.restype = ctypes.c_char_p
@@ -371,6 +393,8 @@ def test_every_python_entry_point_refuses_host_tensors(L):
         "fp8q_cast_from_fp8": lambda: f.fp8q_cast_from_fp8(q, s2, y, f.GRAN_GROUP, 128),
         "fp8q_pack_record": lambda: f.fp8q_pack_record(x, rec, ws),
         "fp8q_unpack_records": lambda: f.fp8q_unpack_records(rec, 1, x.numel(), y),
+        "fp8q_pack_record_ex": lambda: f.fp8q_pack_record_ex(x, rec, ws, layout=f.RECORD_PACKED4),
+        "fp8q_unpack_records_ex": lambda: f.fp8q_unpack_records_ex(rec, 1, x.numel(), y, layout=f.RECORD_PACKED4),
         "fp8q_scaled_mm": lambda: f.fp8q_scaled_mm(a8, b8, s1, s1, out),
         "fp8q_scaled_mm_ex": lambda: f.fp8q_scaled_mm_ex(a8, b8, s1, s1, out),
         "fp8q_scaled_mm_blockwise": lambda: f.fp8q_scaled_mm_blockwise(
@@ -403,8 +427,17 @@ def test_binding_refuses_a_device_other_than_the_current_one(monkeypatch):
     with pytest.raises(ValueError, match="current device"):
         f._stream(None, torch.device("cuda", 1))
     src = inspect.getsource(f)
-    calls = re.findall(r"lib\(\)\.fp8q_\w+\(|\bf\(_dev_ptr", src)
-    streams = re.findall(r"_stream\(stream, dev\)\)", src)
-    assert len(calls) > 0 and len(streams) >= len(calls) - sum(
-        1 for n in ("fp8q_status_string", "fp8q_version", "fp8q_cast_per_tensor_workspace_bytes",
-                    "fp8q_record_bytes") if f"lib().{n}(" in src)
+    no_stream = {"fp8q_status_string", "fp8q_version", "fp8q_cast_per_tensor_workspace_bytes",
+                 "fp8q_record_bytes", "fp8q_record_bytes_ex"}
+    checked = 0
+    for m in re.finditer(r"lib\(\)\.(fp8q_\w+)\(", src):
+        name = m.group(1)
+        depth, i = 1, m.end()
+        while depth:                       # the call's argument list, to its matching parenthesis
+            depth += {"(": 1, ")": -1}.get(src[i], 0)
+            i += 1
+        args = src[m.end():i]
+        if name not in no_stream:
+            assert "_stream(stream, dev)" in args, name
+            checked += 1
+    assert checked >= 15

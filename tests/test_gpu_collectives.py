@@ -45,13 +45,14 @@ def _to_dev(x, xt):
     return dev(x, TORCH_DT[xt]) if xt != F32 else dev(x)
 
 
-def _compare_records(got, want, n, fmt):
-    """Header scale_inv (NaN as a class), header zeros, codes, padding zeros."""
+def _compare_records(got, want, n, fmt, head=16):
+    """Header scale_inv (NaN as a class), header zeros, codes, padding zeros (head 16); the
+    scale then the codes (head 4, the page's packed layout)."""
     assert got.size == want.size
-    assert_f32_equal(got[:4].view(np.float32), want[:4].view(np.float32), name="scale_inv")
-    np.testing.assert_array_equal(got[4:16], want[4:16])
-    assert_codes_equal(got[16:16 + n], want[16:16 + n], fmt)
-    np.testing.assert_array_equal(got[16 + n:], want[16 + n:])
+    assert_f32_equal(got[:4].copy().view(np.float32), want[:4].copy().view(np.float32), name="scale_inv")
+    np.testing.assert_array_equal(got[4:head], want[4:head])
+    assert_codes_equal(got[head:head + n], want[head:head + n], fmt)
+    np.testing.assert_array_equal(got[head + n:], want[head + n:])
 
 
 def _compare_values(got, want, xt):
@@ -181,6 +182,9 @@ def test_collectives_one_rank_nccl(fp8q, orc):
         flat = torch.empty((1, xd.numel()), dtype=torch.bfloat16, device="cuda")
         fp8q.all_gather_fp8(flat, xd, fp8_format="e4m3")
         _compare_values(host(flat).reshape(-1), orc.all_gather_fp8([x], BF16, E4M3FN)[0], BF16)
+        # the page's own wire layout (4-byte scale, then the codes)
+        fp8q.all_gather_fp8(flat, xd, fp8_format="e5m2", layout=fp8q.RECORD_PACKED4)
+        _compare_values(host(flat).reshape(-1), orc.all_gather_fp8([x], BF16, E5M2, header=4)[0], BF16)
         # all_to_all_fp8: one tensor for the one rank
         y = [torch.empty_like(xd)]
         fp8q.all_to_all_fp8(y, [xd], fp8_format="e4m3")
@@ -191,3 +195,63 @@ def test_collectives_one_rank_nccl(fp8q, orc):
         out = torch.empty_like(vd)
         fp8q.all_to_all_single_fp8(out, vd, fp8_format="e5m2")
         _compare_values(host(out).reshape(-1), orc.all_to_all_single_fp8([v.reshape(-1)], F32, E5M2)[0], F32)
+
+
+def _emulated_all_gather_packed4(fp8q, orc, xs, xt, fmt, rule):
+    """The page's own wire layout (all_gather_fp8_lagacy, SCALE_BYTES = 4): each rank's record
+    is its 4-byte scale then its codes, back to back; compared byte for byte with the oracle's
+    records of that layout, and the decoded values bit for bit."""
+    W, n = len(xs), np.asarray(xs[0]).size
+    R = fp8q.record_bytes(n, fp8q.RECORD_PACKED4)
+    assert R == 4 + n == fp8q.fp8q_record_bytes_ex(n, fp8q.RECORD_PACKED4)
+    combined = Guarded(W * R, torch.uint8)
+    ws = torch.empty(fp8q.fp8q_cast_per_tensor_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    for r, x in enumerate(xs):
+        fp8q.fp8q_pack_record_ex(_to_dev(x, xt), combined.t[r * R:(r + 1) * R], ws, fmt, rule, fp8q.RECORD_PACKED4)
+    combined.check()
+    got = host(combined.t)
+    for r, x in enumerate(xs):
+        want = orc.record(x, xt, fmt, rule, header=4)
+        assert want.size == R
+        _compare_records(got[r * R:(r + 1) * R], want, n, fmt, head=4)
+    y = Guarded(W * n, TORCH_DT[xt] if xt != F32 else torch.float32)
+    fp8q.fp8q_unpack_records_ex(combined.t, W, n, y.t, fmt, fp8q.RECORD_PACKED4)
+    y.check()
+    ys = host(y.t)
+    want = orc.all_gather_fp8(xs, xt, fmt, rule, header=4)
+    for r in range(W):
+        _compare_values(ys[r * n:(r + 1) * n], want[r], xt)
+
+
+@pytest.mark.parametrize("n", [4, 16, 20, 4096, 4100, 3 * 4096 + 20, 1_000_004])
+@pytest.mark.parametrize("fmt", [E4M3FN, E5M2])
+def test_records_packed4_emulated_ranks(fp8q, orc, n, fmt):
+    g = np.random.default_rng(n * 11 + fmt)
+    for xt in (F32, BF16):
+        xs = [_input(g, n, xt, "normal") for _ in range(3)]
+        _emulated_all_gather_packed4(fp8q, orc, xs, xt, fmt, 0)
+
+
+@pytest.mark.parametrize("n", [1, 3, 4097])
+def test_records_packed4_one_record_any_numel(fp8q, orc, n):
+    """A single packed record takes any numel: its scale sits at the (4-byte aligned) start."""
+    g = np.random.default_rng(n)
+    _emulated_all_gather_packed4(fp8q, orc, [_input(g, n, F32, "nonfinite")], F32, E5M2, 1)
+
+
+def test_records_packed4_arguments_checked(fp8q):
+    x = torch.zeros(6, dtype=torch.float32, device="cuda")
+    buf = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(fp8q.fp8q_cast_per_tensor_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    y = torch.empty(12, dtype=torch.float32, device="cuda")
+    P4 = fp8q.RECORD_PACKED4
+    with pytest.raises(fp8q.Fp8qError, match="align"):            # the scale would be unaligned
+        fp8q.fp8q_pack_record_ex(x, buf[2:12], ws, E4M3FN, 0, P4)
+    with pytest.raises(fp8q.Fp8qError, match="align"):            # record 1's scale at 4 + 6 = 10
+        fp8q.fp8q_unpack_records_ex(buf[:20], 2, 6, y, E4M3FN, P4)
+    fp8q.fp8q_pack_record_ex(x, buf[4:14], ws, E4M3FN, 0, P4)     # 4-byte aligned: accepted
+    fp8q.fp8q_unpack_records_ex(buf[4:14], 1, 6, y[:6], E4M3FN, P4)
+    assert (host(y[:6]) == 0).all()
+    assert host(buf[4:8]).view(np.float32)[0] == np.float32(1.0) / np.float32(448.0)
+    with pytest.raises(ValueError):
+        fp8q.record_bytes(6, 8)

@@ -39,6 +39,25 @@ def test_record_golden(orc):
 def test_record_size():
     from oracle import record_size
     assert [record_size(n) for n in (0, 1, 15, 16, 17, 4096)] == [16, 32, 32, 32, 48, 4112]
+    assert [record_size(n, 4) for n in (0, 1, 15, 16, 17, 4096)] == [4, 5, 19, 20, 21, 4100]
+
+
+def test_record_golden_packed4(orc):
+    """The page's own record layout (all_gather_fp8_lagacy, SCALE_BYTES = 4): the fp32 scale
+    then the codes, no padding; the same hand-worked values as the 16-byte layout."""
+    g = load_golden("record_small.txt")
+    x = hex_list(g["x_f32_bits"], np.uint32).view(np.float32)
+    for fmt, key in ((E4M3FN, "record_e4m3_packed4"), (E5M2, "record_e5m2_packed4")):
+        want = hex_list(g[key], np.uint8)
+        got = orc.record(x, F32, fmt, header=4)
+        assert got.size == 7 == orc.record_size(3, 4)
+        np.testing.assert_array_equal(got, want)
+        y = orc.record_decode(got, 3, fmt, F32, header=4)
+        np.testing.assert_array_equal(y.view(np.uint32), hex_list(g["y_f32_bits"], np.uint32))
+        # the two layouts carry the same scale and codes
+        r16 = orc.record(x, F32, fmt)
+        np.testing.assert_array_equal(r16[:4], got[:4])
+        np.testing.assert_array_equal(r16[16:19], got[4:7])
 
 
 def _exact_tensor(g, n, fmt, k):
