@@ -1184,6 +1184,12 @@ def run_ours(args):
     }
     if sharded is not None:
         line["sharded"] = sharded
+    # the two ops the metric names, each timed alone (isolated) and inside the step (marginal
+    # cost is printed by --marginal; `kernels` holds the instrumented split)
+    line["headline_ops"] = {k: {"us": iso[k]["us"], "gb_s": iso[k]["gb_s"], "frac": round(iso[k]["gb_s"] / peak, 4),
+                                "pct_of_nominal_8tbs": round(100.0 * iso[k]["gb_s"] / 8000.0, 2),
+                                "us_p10_p50_p90": iso[k]["us_p10_p50_p90"]}
+                            for k in ("per_token_group_quant", "block_dequant") if k in iso}
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(h)
     print(json.dumps(line), flush=True)
