@@ -85,6 +85,9 @@ template <int BN_, int MT_ = 128> struct Shape {
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment slack */ + 256 /* barriers */;
 };
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // every wait's default limit
+#ifndef FP8Q_PAIRS
+#define FP8Q_PAIRS 1
+#endif
 
 // status bits ORed into the caller's status word when a wait runs out
 enum : uint32_t { kTimeoutProducer = 1u, kTimeoutMma = 2u, kTimeoutEpilogue = 4u, kTimeoutDrain = 8u };
@@ -662,6 +665,257 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 }
 
 // ---------------------------------------------------------------------------
+// CTA pairs (per-tensor scales, both operands K-major): the two CTAs of a
+// cluster compute one 256 x 256 tile with tcgen05.mma.cta_group::2 (M 256,
+// N 256, K 32).  Each CTA loads its own 128 rows of A and its own 128 rows of
+// B (half of the tile's N) into its shared memory, so a CTA reads a quarter
+// fewer operand bytes per flop than a 128 x 256 tile on one SM; each CTA's
+// TMEM holds its 128 rows x 256 columns of the tile, two buffers of it, so one
+// tile's epilogue overlaps the next tile's k-loop.  The even CTA of the pair
+// (the leader) expects both CTAs' bytes on its stage barriers and issues the
+// MMAs; its commits release the stages and hand over finished accumulators
+// in both CTAs at once (commit with .multicast::cluster); both CTAs' epilogue
+// warps hand their accumulator back on the leader's barrier.  No load uses
+// multicast: every CTA fetches its own tiles.
+// ---------------------------------------------------------------------------
+namespace pair {
+
+constexpr int kStages = 6;
+constexpr int BN = 256;                         // columns of D per tile (B rows, both CTAs together)
+constexpr int kHalfB = BN / 2;                  // B rows one CTA loads
+constexpr int kATile = BM * BK;                 // 16 KB: this CTA's 128 rows of A
+constexpr int kBTile = kHalfB * BK;             // 16 KB: this CTA's half of B
+constexpr int kAccBufs = 2;
+constexpr int kTmemCols = 512;
+constexpr int kColsPerWarp = BN / (kEpiWarps / 4);
+constexpr int kSmemBytes = kStages * (kATile + kBTile) + 1024 + 256;
+// clears the CTA-rank bit of a shared::cluster address: the same offset in the even CTA
+constexpr uint32_t kLeaderMask = 0xFEFFFFFFu;
+
+__device__ __forceinline__ uint32_t cta_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// a 2-D box into this CTA's shared memory, its bytes counted on the leader's barrier
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile("cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar & kLeaderMask)
+                 : "memory");
+}
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// arrive on `bar` in both CTAs of the pair once this thread's MMAs so far have completed
+__device__ __forceinline__ void commit_both(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 :: "r"(bar), "h"(static_cast<uint16_t>(3)) : "memory");
+}
+__device__ __forceinline__ void commit_local(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+}
+// arrive on the leader's barrier at the offset of `bar`
+__device__ __forceinline__ void arrive_leader(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" :: "r"(bar & kLeaderMask) : "memory");
+}
+
+template <int YT>
+__global__ void __launch_bounds__(kThreads, 1)
+scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                      const Params p, const uint32_t idesc) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ int s_abort;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kATile;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kBTile);
+    // bars: full[kStages], empty[kStages], tfull[kAccBufs], tempty[kAccBufs], drain
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 2 * kAccBufs + 1);
+    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * kStages;
+    const uint32_t tfull0 = empty0 + 8 * kStages, tempty0 = tfull0 + 8 * kAccBufs;
+    const uint32_t drain_bar = tempty0 + 8 * kAccBufs;
+    volatile int* abort = &s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cta_rank();
+    const bool leader = rank == 0;
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full0 + 8 * s, 1);           // the leader's expect-tx arrival, bytes of both CTAs
+            mbar_init(empty0 + 8 * s, 1);          // the leader's commit
+        }
+        for (int b = 0; b < kAccBufs; ++b) {
+            mbar_init(tfull0 + 8 * b, 1);          // the leader's commit
+            mbar_init(tempty0 + 8 * b, 2 * kEpiWarps);   // every epilogue warp of both CTAs (leader's copy)
+        }
+        mbar_init(drain_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        prefetch_tensormap(&map_a);
+        prefetch_tensormap(&map_b);
+    }
+    // the peer's barriers exist before anything signals them
+    cluster_sync();
+    if (warp == 1) {
+        // both CTAs allocate, from the same warp, into the same slot offset
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    pdl_begin();
+
+    const int tiles = p.tiles_m * p.tiles_n;          // 256 x 256 tiles
+    const int pair_id = blockIdx.x >> 1, pairs = gridDim.x >> 1;
+    uint32_t fail = 0;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int64_t issued = 0;
+            for (int t = pair_id; t < tiles && !fail; t += pairs) {
+                int mb, nb;
+                tile_coords(t, p.tiles_m, p.tiles_n, mb, nb);
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort, p.wait_limit_ns)) { fail = kTimeoutProducer; break; }
+                    const uint32_t fb = full0 + 8 * stage;
+                    if (leader) mbar_arrive_expect_tx(fb, static_cast<uint32_t>(2 * (kATile + kBTile)));
+                    tma_load_2d_pair(smem_u32(sA + stage * kATile), &map_a, kb * BK, mb * 2 * BM + rank * BM, fb);
+                    tma_load_2d_pair(smem_u32(sB + stage * kBTile), &map_b, kb * BK, nb * BN + rank * kHalfB, fb);
+                    ++issued;
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (fail) *abort = 1;
+            // every stage this CTA filled has been consumed by the pair's MMAs
+            // (so its copies have landed) before the CTA moves on
+            for (int s = 0; s < kStages; ++s) {
+                const bool used = s < stage || issued >= kStages;
+                // (a stage refilled in this lap waits for the release of that fill, parity
+                // `phase`; one last filled in the previous lap, parity `phase ^ 1`)
+                if (used && !mbar_wait_drain(empty0 + 8 * s, s < stage ? phase : phase ^ 1u, p.wait_limit_ns))
+                    fail |= kTimeoutDrain;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (lane == 0 && leader) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int t = pair_id; t < tiles && !fail; t += pairs) {
+                if (p.num_kb == 0) continue;
+                if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort, p.wait_limit_ns)) { fail = kTimeoutMma; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait(full0 + 8 * stage, phase, abort, p.wait_limit_ns)) { fail = kTimeoutMma; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * kATile), b0 = smem_u32(sB + stage * kBTile);
+#pragma unroll
+                    for (int j = 0; j < BK / 32; ++j)
+                        mma_pair(tmem_base + static_cast<uint32_t>(acc * BN), smem_desc_sw128(a0 + 32 * j),
+                                 smem_desc_sw128(b0 + 32 * j), idesc, (kb > 0 || j > 0));
+                    commit_both(empty0 + 8 * stage);
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+                if (fail) break;
+                commit_both(tfull0 + 8 * acc);
+                if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
+            }
+            if (fail) *abort = 1;
+            // every tensor-core operation issued has completed
+            commit_local(drain_bar);
+            if (!mbar_wait_drain(drain_bar, 0, p.wait_limit_ns)) fail |= kTimeoutDrain;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int ew = warp - 2;
+        const int quarter = warp & 3;
+        const int cgrp = ew >> 2;
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        const float scale = __fmul_rn(__ldg(p.sa), __ldg(p.sb));
+        for (int t = pair_id; t < tiles && !fail; t += pairs) {
+            int mb, nb;
+            tile_coords(t, p.tiles_m, p.tiles_n, mb, nb);
+            const int row = mb * 2 * BM + static_cast<int>(rank) * BM + quarter * 32 + lane;
+            const int col_base = nb * BN + cgrp * kColsPerWarp;
+            if (p.num_kb > 0) {
+                const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort, p.wait_limit_ns));
+                if (!ok) { fail = kTimeoutEpilogue; break; }
+                tc_fence_after();
+            }
+            constexpr int kChunks = kColsPerWarp / 32;
+            const uint32_t col_addr = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + cgrp * kColsPerWarp);
+            uint32_t r0[32], r1[32];
+            if (p.num_kb > 0) {
+                tmem_ld32_async(col_addr, r0);
+                tmem_wait32(r0);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0u;
+            }
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+                uint32_t (&cur)[32] = (c & 1) ? r1 : r0;
+                uint32_t (&nxt)[32] = (c & 1) ? r0 : r1;
+                if (p.num_kb > 0 && c + 1 < kChunks) tmem_ld32_async(col_addr + static_cast<uint32_t>(32 * (c + 1)), nxt);
+                const int col0 = col_base + c * 32;
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(cur[i]), scale);
+                if (p.bias) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (col0 + i < p.N) v[i] = __fadd_rn(v[i], load_bias<YT>(p.bias, col0 + i));
+                }
+                if (row < p.M && col0 < p.N) store_chunk<YT>(p, row, col0, v);
+                if (p.num_kb > 0 && c + 1 < kChunks) tmem_wait32(nxt);
+            }
+            if (p.num_kb > 0) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive_leader(tempty0 + 8 * acc);
+                if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
+            }
+        }
+        if (fail && lane == 0) *abort = 1;
+    }
+
+    if (fail && p.status && lane == 0) atomicOr(p.status, fail);
+    // neither CTA leaves (or frees TMEM) while the other may still signal its
+    // barriers or the pair's MMAs may still write its TMEM
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace pair
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -736,6 +990,43 @@ cudaError_t launch_tall(int yt, const CUtensorMap& ma, const CUtensorMap& mb, co
                       : launch_typed<kBF16, false, 256, 256>(ma, mb, p, idesc, s);
 }
 
+// per-tensor scales, 256 x 256 tiles on CTA pairs: the grid is the pairs that
+// fit at once (at most one per tile), two CTAs each
+template <int YT>
+cudaError_t launch_pair_typed(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, uint32_t idesc,
+                              cudaStream_t s) {
+    auto kernel = pair::scaled_mm_pair_kernel<YT>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pair::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pair::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = FP8Q_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cfg.gridDim = dim3(2);
+    int fit = 0;
+    if (cudaOccupancyMaxActiveClusters(&fit, kernel, &cfg) != cudaSuccess || fit < 1) fit = sm_count() / 2;
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int pairs = tiles < fit ? tiles : fit;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, p, idesc);
+}
+
+cudaError_t launch_pair(int yt, const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, uint32_t idesc,
+                        cudaStream_t s) {
+    return yt == kF32 ? launch_pair_typed<kF32>(ma, mb, p, idesc, s)
+         : yt == kF16 ? launch_pair_typed<kF16>(ma, mb, p, idesc, s)
+                      : launch_pair_typed<kBF16>(ma, mb, p, idesc, s);
+}
+
 }  // namespace mm
 
 fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb, int64_t M, int64_t N, int64_t K,
@@ -755,12 +1046,17 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     // when those tiles still fill nine tenths of the SMs.
     const int64_t tall_tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256);
     const bool tall = !fine && !narrow && M >= 2 * BM && tall_tiles * 10 >= 9LL * sm_count();
+    // the same tiles on CTA pairs when both operands are K-major (the forward product)
+    const bool pairs = FP8Q_PAIRS && tall && !a_mn && !b_mn && stall_kb < 0;
     const int mt = tall ? 2 * BM : BM;
     const int a_rows = tall ? mt : (M >= BM || a_mn) ? BM : static_cast<int>((M + 15) / 16 * 16);
     CUtensorMap ma, mbm;
     memset(&ma, 0, sizeof(ma));
     memset(&mbm, 0, sizeof(mbm));
-    if (K > 0) {
+    if (K > 0 && pairs) {
+        // each CTA of a pair loads 128 rows of A and 128 rows of B
+        if (!make_map(&ma, a, M, K, BM) || !make_map(&mbm, b, N, K, pair::kHalfB)) return FP8Q_ERR_CUDA;
+    } else if (K > 0) {
         // K-major: [M][K] with boxes of rows x 128 k; MN-major: [K][M] with
         // boxes of 128 k x 128 m (B likewise, two boxes for 256 columns)
         const bool ok_a = a_mn ? make_map(&ma, a, K, M, BK) : make_map(&ma, a, M, K, a_rows);   // MN-major: 128-wide boxes
@@ -790,7 +1086,12 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     p.stall_kb = stall_kb;
     const uint32_t idesc = instr_desc(fa, fb, bn, a_mn, b_mn);
     cudaError_t e;
-    if (narrow) e = launch_dtype<128>(fine, yt, ma, mbm, p, idesc, s);
+    if (pairs) {
+        // M 256 (128 rows per CTA), N 256
+        const uint32_t pair_idesc = (1u << 4) | (static_cast<uint32_t>(fa) << 7) | (static_cast<uint32_t>(fb) << 10)
+                                  | (static_cast<uint32_t>(256 >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
+        e = launch_pair(yt, ma, mbm, p, pair_idesc, s);
+    } else if (narrow) e = launch_dtype<128>(fine, yt, ma, mbm, p, idesc, s);
     else if (tall) e = launch_tall(yt, ma, mbm, p, idesc, s);
     else e = launch_dtype<256>(fine, yt, ma, mbm, p, idesc, s);
     return cuda_status(e);

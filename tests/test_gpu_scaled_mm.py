@@ -386,6 +386,23 @@ def test_exact_grid_tall_tiles(fp8q, orc, M, N, K, yt):
     assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
 
 
+@pytest.mark.parametrize("M,N,K,fa,fb,yt,with_bias", [
+    (2000, 4100, 1008, E4M3FN, E4M3FN, BF16, True),     # 8 x 17 tiles: ragged rows in the second CTA, 4 ragged columns, a partial k-block
+    (4096, 2304, 256, E4M3FN, E5M2, F32, False),        # 16 x 9 tiles
+    (2304, 4352, 384, E5M2, E4M3FN, F16, True)])        # 9 x 17 tiles: an odd row-tile count
+def test_exact_grid_cta_pairs(fp8q, orc, M, N, K, fa, fb, yt, with_bias):
+    """Per-tensor products with enough 256 x 256 tiles to fill the GPU and both operands K-major
+    run on CTA pairs (tcgen05.mma.cta_group::2: each CTA loads 128 rows of A and 128 rows of B
+    and holds its 128 rows of the tile in TMEM).  Every output is compared bit for bit."""
+    g = np.random.default_rng(M + N + K + yt)
+    a, b = grid_codes(g, (M, K), fa), grid_codes(g, (N, K), fb)
+    bias_t, bias = t_bias(g, N, yt) if with_bias else (None, None)
+    out = run(fp8q, False, a, fa, b, fb, 0.375, 1.75, bias_t, yt)
+    want = oracle_rounded(orc, False, a, fa, b, fb, 0.375, 1.75, bias, yt)
+    bad = ~bits_equal(host(out), want, yt)
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
+
+
 # ---------------------------------------------------------------------------
 # bounded waits: a wait that runs out is reported, and the context stays usable
 # ---------------------------------------------------------------------------
