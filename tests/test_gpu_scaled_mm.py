@@ -403,6 +403,21 @@ def test_exact_grid_cta_pairs(fp8q, orc, M, N, K, fa, fb, yt, with_bias):
     assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
 
 
+@pytest.mark.parametrize("M,N,K,yt", [(2000, 4100, 1008, BF16), (2304, 4352, 384, F32)])
+def test_exact_grid_fine_wide_products(fp8q, orc, M, N, K, yt):
+    """Fine-grained products with enough 256 x 256 tiles to fill the GPU (on CTA pairs where the
+    build takes them for these scales): ragged rows and columns, a partial last k-block, per-token
+    and block scales, bias; every output bit for bit against the oracle's rounding."""
+    g = np.random.default_rng(M * 7 + N + K)
+    a, b = grid_codes(g, (M, K), E4M3FN), grid_codes(g, (N, K), E4M3FN)
+    sa, sb = scales(g, M, N, K)
+    bias_t, bias = t_bias(g, N, yt)
+    out = run(fp8q, True, a, E4M3FN, b, E4M3FN, sa, sb, bias_t, yt)
+    want = oracle_rounded(orc, True, a, E4M3FN, b, E4M3FN, sa, sb, bias, yt)
+    bad = ~bits_equal(host(out), want, yt)
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
+
+
 # ---------------------------------------------------------------------------
 # bounded waits: a wait that runs out is reported, and the context stays usable
 # ---------------------------------------------------------------------------
