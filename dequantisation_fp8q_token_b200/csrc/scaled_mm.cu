@@ -665,7 +665,7 @@ scaled_mm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 }
 
 // ---------------------------------------------------------------------------
-// CTA pairs (per-tensor scales, both operands K-major): the two CTAs of a
+// CTA pairs (per-tensor scales, either operand K- or MN-major): the two CTAs of a
 // cluster compute one 256 x 256 tile with tcgen05.mma.cta_group::2 (M 256,
 // N 256, K 32).  Each CTA loads its own 128 rows of A and its own 128 rows of
 // B (half of the tile's N) into its shared memory, so a CTA reads a quarter
@@ -795,8 +795,13 @@ scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                     if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort, p.wait_limit_ns)) { fail = kTimeoutProducer; break; }
                     const uint32_t fb = full0 + 8 * stage;
                     if (leader) mbar_arrive_expect_tx(fb, static_cast<uint32_t>(2 * (kATile + kBTile)));
-                    tma_load_2d_pair(smem_u32(sA + stage * kATile), &map_a, kb * BK, mb * 2 * BM + rank * BM, fb);
-                    tma_load_2d_pair(smem_u32(sB + stage * kBTile), &map_b, kb * BK, nb * BN + rank * kHalfB, fb);
+                    // K-major: boxes of 128 rows x 128 k; MN-major: 128 k x 128 rows
+                    const int m0 = mb * 2 * BM + static_cast<int>(rank) * BM;
+                    const int n0 = nb * BN + static_cast<int>(rank) * kHalfB;
+                    if (p.a_mn) tma_load_2d_pair(smem_u32(sA + stage * kATile), &map_a, m0, kb * BK, fb);
+                    else tma_load_2d_pair(smem_u32(sA + stage * kATile), &map_a, kb * BK, m0, fb);
+                    if (p.b_mn) tma_load_2d_pair(smem_u32(sB + stage * kBTile), &map_b, n0, kb * BK, fb);
+                    else tma_load_2d_pair(smem_u32(sB + stage * kBTile), &map_b, kb * BK, n0, fb);
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
@@ -828,9 +833,13 @@ scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sA + stage * kATile), b0 = smem_u32(sB + stage * kBTile);
 #pragma unroll
-                    for (int j = 0; j < BK / 32; ++j)
-                        mma_pair(tmem_base + static_cast<uint32_t>(acc * BN), smem_desc_sw128(a0 + 32 * j),
-                                 smem_desc_sw128(b0 + 32 * j), idesc, (kb > 0 || j > 0));
+                    for (int j = 0; j < BK / 32; ++j) {
+                        // a k step of 32 moves a K-major tile's start by 32 bytes, an MN-major
+                        // tile's by 32 rows of 128 bytes
+                        const uint64_t ad = p.a_mn ? smem_desc_mn_sw128(a0 + 4096 * j) : smem_desc_sw128(a0 + 32 * j);
+                        const uint64_t bd = p.b_mn ? smem_desc_mn_sw128(b0 + 4096 * j) : smem_desc_sw128(b0 + 32 * j);
+                        mma_pair(tmem_base + static_cast<uint32_t>(acc * BN), ad, bd, idesc, (kb > 0 || j > 0));
+                    }
                     commit_both(empty0 + 8 * stage);
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
@@ -1046,16 +1055,21 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     // when those tiles still fill nine tenths of the SMs.
     const int64_t tall_tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256);
     const bool tall = !fine && !narrow && M >= 2 * BM && tall_tiles * 10 >= 9LL * sm_count();
-    // the same tiles on CTA pairs when both operands are K-major (the forward product)
-    const bool pairs = FP8Q_PAIRS && tall && !a_mn && !b_mn && stall_kb < 0;
-    const int mt = tall ? 2 * BM : BM;
+    // 256 x 256 tiles on CTA pairs when those tiles give two CTAs each to nine
+    // tenths of the SMs (the same tiles on one CTA each need twice as many)
+    const bool pairs = FP8Q_PAIRS && !fine && !narrow && M >= 2 * BM && tall_tiles * 20 >= 9LL * sm_count() &&
+                       stall_kb < 0;
+    const int mt = (tall || pairs) ? 2 * BM : BM;
     const int a_rows = tall ? mt : (M >= BM || a_mn) ? BM : static_cast<int>((M + 15) / 16 * 16);
     CUtensorMap ma, mbm;
     memset(&ma, 0, sizeof(ma));
     memset(&mbm, 0, sizeof(mbm));
     if (K > 0 && pairs) {
-        // each CTA of a pair loads 128 rows of A and 128 rows of B
-        if (!make_map(&ma, a, M, K, BM) || !make_map(&mbm, b, N, K, pair::kHalfB)) return FP8Q_ERR_CUDA;
+        // each CTA of a pair loads 128 rows of A and 128 rows of B (MN-major: one
+        // 128 k x 128-row box each)
+        const bool ok_a = a_mn ? make_map(&ma, a, K, M, BK) : make_map(&ma, a, M, K, BM);
+        const bool ok_b = b_mn ? make_map(&mbm, b, K, N, BK) : make_map(&mbm, b, N, K, pair::kHalfB);
+        if (!ok_a || !ok_b) return FP8Q_ERR_CUDA;
     } else if (K > 0) {
         // K-major: [M][K] with boxes of rows x 128 k; MN-major: [K][M] with
         // boxes of 128 k x 128 m (B likewise, two boxes for 256 columns)
@@ -1089,6 +1103,7 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     if (pairs) {
         // M 256 (128 rows per CTA), N 256
         const uint32_t pair_idesc = (1u << 4) | (static_cast<uint32_t>(fa) << 7) | (static_cast<uint32_t>(fb) << 10)
+                                  | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16)
                                   | (static_cast<uint32_t>(256 >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
         e = launch_pair(yt, ma, mbm, p, pair_idesc, s);
     } else if (narrow) e = launch_dtype<128>(fine, yt, ma, mbm, p, idesc, s);

@@ -335,7 +335,8 @@ def test_exact_grid_small_m(fp8q, orc, fine, M, N, K):
     (1, 0, 208, 300, 272), (1, 0, 128, 256, 384),
     (1, 1, 128, 256, 128), (1, 1, 256, 512, 300), (1, 1, 144, 3008, 37), (1, 1, 32, 16, 1),
     (0, 0, 200, 300, 272),
-    (1, 1, 512, 17008, 100), (1, 0, 512, 17008, 64), (0, 1, 512, 17008, 64)])   # enough tiles for 256-row tiles
+    (1, 1, 512, 17008, 100), (1, 0, 512, 17008, 64), (0, 1, 512, 17008, 64),    # enough tiles for 256-row tiles
+    (0, 0, 256, 17008, 256), (1, 1, 256, 17408, 128)])   # one row of 256 x 256 tiles, one CTA pair per tile
 @pytest.mark.parametrize("yt", [F32, BF16])
 def test_exact_grid_layouts(fp8q, orc, a_mn, b_mn, M, N, K, yt):
     g = np.random.default_rng(1000 * a_mn + 100 * b_mn + M + N + K + yt)
