@@ -495,8 +495,14 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
 
     def run(name, make_set, footprint, nbytes):
         sets = [make_set(i) for i in range(max(1, -(-need // footprint)))]
-        for fn in sets:
-            fn()
+        # warm up for at least 10 ms of launches, so the clocks have settled before timing
+        t0 = time.perf_counter()
+        k = 0
+        while k < len(sets) or time.perf_counter() - t0 < 0.01:
+            sets[k % len(sets)]()
+            k += 1
+            if k % 32 == 0:
+                torch.cuda.synchronize()
         torch.cuda.synchronize()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(blocks)]
         k = 0
@@ -611,9 +617,15 @@ class MatmulWorkload:
         }
 
     @staticmethod
-    def _timed(fn, steps: int, warmup: int, device, min_ms: float = 20.0):
+    def _timed(fn, steps: int, warmup: int, device, min_ms: float = 20.0, rest_s: float = 0.0):
         """ms per call of fn (CUDA events around at least `steps` back-to-back calls, and enough
-        calls to span `min_ms`, after `warmup`), with the SM clocks sampled while it runs."""
+        calls to span `min_ms`, after `warmup`), with the SM clocks sampled while it runs.
+        rest_s: an idle pause first, so that products timed one after another each start from
+        the same power state (a dense product drives the board to its power cap within tens of
+        milliseconds, and the clocks it leaves lowered would otherwise fall on the next entry)."""
+        if rest_s > 0:
+            torch.cuda.synchronize(device)
+            time.sleep(rest_s)
         for _ in range(warmup):
             fn()
         torch.cuda.synchronize(device)
@@ -687,8 +699,9 @@ class MatmulWorkload:
         res = {}
         for name, fn in ops.items():
             try:
-                ms, clk = self._timed(fn, steps, warmup, device)
-                res[name] = {"ms": round(ms, 4), "tflops": round(self.flops / (ms * 1e-3) / 1e12, 1), "clocks": clk}
+                ms, clk = self._timed(fn, steps, warmup, device, rest_s=1.0)
+                res[name] = {"ms": round(ms, 4), "tflops": round(self.flops / (ms * 1e-3) / 1e12, 1), "clocks": clk,
+                             "rest_before_s": 1.0}
                 if name in lib_ops:
                     y = fn().float()
                     r = ref["scaled_mm_blockwise" if "blockwise" in name else "scaled_mm_per_tensor"]
