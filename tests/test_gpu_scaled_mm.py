@@ -328,6 +328,62 @@ def test_exact_grid_small_m(fp8q, orc, fine, M, N, K):
 
 
 # ---------------------------------------------------------------------------
+# decode-sized products (at most 128 rows): 128 x 128 tiles, A boxes of M rows
+# rounded up to 16, one tile of 128 weight rows per CTA
+# ---------------------------------------------------------------------------
+DECODE = [(1, 3000, 1024),     # one row, 24 tiles, 8 k-blocks: the 6-stage ring wraps
+          (2, 1000, 144),      # a partial second k-block, a partial last tile
+          (16, 384, 272),      # a 16-row A box; a partial last k-block
+          (17, 2000, 400),     # a 32-row A box
+          (32, 640, 16),       # one 16-deep k-block
+          (33, 1280, 2000),    # a 48-row A box, 16 k-blocks
+          (64, 3000, 1168),
+          (65, 1000, 384),     # an 80-row A box: rows in three TMEM lane quarters
+          (128, 2048, 640),    # a whole 128-row tile
+          (5, 30000, 384)]     # 235 tiles: two for some CTAs
+
+
+@pytest.mark.parametrize("M,N,K", DECODE, ids=lambda v: str(v))
+@pytest.mark.parametrize("fine", [False, True], ids=["tensor", "blockwise"])
+def test_exact_grid_decode_sized(fp8q, orc, M, N, K, fine):
+    i = DECODE.index((M, N, K))
+    fa, fb = FORMATS[i % 4]
+    yt = (F32, F16, BF16)[i % 3]
+    g = np.random.default_rng(9000 + 7 * i + fine)
+    a, b = grid_codes(g, (M, K), fa), grid_codes(g, (N, K), fb)
+    sa, sb = scales(g, M, N, K) if fine else (0.375, 1.25)
+    bias_t, bias = t_bias(g, N, yt) if i % 2 == 0 else (None, None)
+    got = host(run(fp8q, fine, a, fa, b, fb, sa, sb, bias_t, yt))
+    want = oracle_rounded(orc, fine, a, fa, b, fb, sa, sb, bias, yt)
+    bad = ~bits_equal(got, want, yt)
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ, first at {np.argwhere(bad)[:4].tolist()}"
+
+
+@pytest.mark.parametrize("M", [1, 64])
+@pytest.mark.parametrize("fine", [False, True], ids=["tensor", "blockwise"])
+def test_general_operands_decode_sized(fp8q, orc, M, fine):
+    """All finite codes, K = 7168: within the same bound as the large products."""
+    N, K = 640, 7168
+    g = np.random.default_rng(31 + M + fine)
+    a, b = finite_codes(g, (M, K), E4M3FN), finite_codes(g, (N, K), E4M3FN)
+    kb = K // 128
+    if fine:
+        sa = np.exp(g.normal(-4, 2, (M, kb))).astype(np.float32)
+        sb = np.exp(g.normal(-8, 1, (-(-N // 128), kb))).astype(np.float32)
+    else:
+        sa, sb = 0.0123, 3.5
+    got = host(run(fp8q, fine, a, E4M3FN, b, E4M3FN, sa, sb, None, BF16))
+    A, W = np.abs(tdec(a, E4M3FN)), np.abs(tdec(b, E4M3FN))
+    if fine:
+        exact = orc.scaled_mm_blockwise(a, E4M3FN, sa, b, E4M3FN, sb, threads=THREADS)
+        mag = (A * np.repeat(sa, 128, 1)) @ (W * np.repeat(np.repeat(sb, 128, 0), 128, 1)[:N]).T
+    else:
+        exact = orc.scaled_mm(a, E4M3FN, b, E4M3FN, sa, sb, threads=THREADS)
+        mag = (A @ W.T) * float(np.float32(sa) * np.float32(sb))
+    check_bound(to_f64(got, BF16), exact, mag, K, BF16, fine)
+
+
+# ---------------------------------------------------------------------------
 # operand layouts (fp8q_scaled_mm_ex): K-major or MN-major, bit for bit
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("a_mn,b_mn,M,N,K", [
@@ -459,3 +515,34 @@ def test_bounded_waits_run_out_report_and_return(fp8q, orc):
     out3 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     fp8q.fp8q_scaled_mm(A, B, sa, sb, out3)
     np.testing.assert_array_equal(host(out3), want)
+
+
+def test_bounded_waits_run_out_decode_sized(fp8q, orc):
+    """The same for a one-row product (128 x 128 tiles, a 16-row A box): k-block 2 of each CTA's
+    tile never arrives, every wait that depends on it runs out and is reported, and the same
+    product then runs normally on the same stream."""
+    import time
+    M, N, K = 1, 3000, 1024                      # 24 tiles of 128 weight rows, 8 k-blocks
+    g = np.random.default_rng(405)
+    a, b = grid_codes(g, (M, K), E4M3FN), grid_codes(g, (N, K), E4M3FN)
+    A, B = dev(a), dev(b)
+    sa, sb = dev(np.array([0.5], np.float32)), dev(np.array([0.25], np.float32))
+    want = oracle_rounded(orc, False, a, E4M3FN, b, E4M3FN, 0.5, 0.25, None, BF16)
+    out = Guarded(M * N, torch.bfloat16)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    fp8q.fp8q_scaled_mm_wait_test(A, B, sa, sb, out.t.view(M, N), st, 20_000_000, 2)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    out.check()
+    bits = int(st.item())
+    assert bits & fp8q.WAIT_MMA and bits & fp8q.WAIT_DRAIN, f"status {bits:#x}"
+    assert bits & ~0xF == 0, f"status {bits:#x}"
+    assert dt < 2.0, f"the stalled kernel took {dt:.2f} s"
+    out2 = Guarded(M * N, torch.bfloat16)
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fp8q.fp8q_scaled_mm_wait_test(A, B, sa, sb, out2.t.view(M, N), st2, 20_000_000, -1)
+    out2.check()
+    assert int(st2.item()) == 0
+    np.testing.assert_array_equal(host(out2.t.view(M, N)), want)
