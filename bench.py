@@ -477,14 +477,18 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
     least 4x the L2 size, so every launch reads cold inputs and pays for the
     write-back of exactly one launch's outputs (its own kind).
 
-    `us` and its p10 / p50 / p90 come from `blocks` blocks of launches run
-    back to back, one event pair per block (the per-launch mean of each
-    block is one sample).  An event pair around every single launch is
-    reported too (`us_event_per_launch`), but it overstates a short kernel:
-    an event between two kernels serialises them and exposes the launch
-    latency that back-to-back launches hide under programmatic dependent
-    launch (measured on B200: 19.6 us against 13.6 us for the 89 MB
-    per-token quant)."""
+    `us` and its p10 / p50 / p90: the op's launches over every set, captured
+    once in a CUDA graph (the same kernels with the same arguments; the
+    launches keep their programmatic-dependent-launch attribute) and replayed
+    `blocks` times, one event pair per replay (the per-launch mean of each
+    replay is one sample).  Launched one by one from Python instead, a short
+    op is bound by the binding's host cost (~10-12 us a call, `host_us_per_call`):
+    the 89 MB per-token quant reads 14.4-14.9 us that way against 13.2 us from
+    the graph on B200, so that figure (`us_stream`, blocks of back-to-back
+    launches) is reported beside it, not as the op's time.  An event pair
+    around every single launch (`us_event_per_launch`) overstates a short
+    kernel further: an event between two kernels serialises them and exposes
+    the launch latency that back-to-back launches hide."""
     f = wl.fp8q
     d = wl.device
     l2 = torch.cuda.get_device_properties(d).L2_cache_size
@@ -504,6 +508,13 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
             if k % 32 == 0:
                 torch.cuda.synchronize()
         torch.cuda.synchronize()
+        # the binding's host cost per call (no synchronisation inside)
+        t0 = time.perf_counter()
+        for j in range(4 * len(sets)):
+            sets[j % len(sets)]()
+        host_us = (time.perf_counter() - t0) / (4 * len(sets)) * 1e6
+        torch.cuda.synchronize()
+        # launched one by one from Python: blocks of back-to-back launches
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(blocks)]
         k = 0
         for b in range(blocks):
@@ -514,6 +525,30 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
             evs[b][1].record()
         torch.cuda.synchronize()
         blk = sorted(a.elapsed_time(e) * 1e3 / per_block for a, e in evs)
+        # the same launches replayed from a CUDA graph: per_block launches of every set
+        nl = per_block * len(sets)
+        side = torch.cuda.Stream(d)
+        side.wait_stream(torch.cuda.current_stream(d))
+        with torch.cuda.stream(side):
+            for j in range(nl):
+                sets[j % len(sets)]()
+        torch.cuda.current_stream(d).wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for j in range(nl):
+                sets[j % len(sets)]()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(blocks)]
+        for b in range(blocks):
+            gev[b][0].record()
+            graph.replay()
+            gev[b][1].record()
+        torch.cuda.synchronize()
+        rep = sorted(a.elapsed_time(e) * 1e3 / nl for a, e in gev)
+        del graph
         one = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
         for j in range(launches):
             one[j][0].record()
@@ -521,10 +556,14 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
             one[j][1].record()
         torch.cuda.synchronize()
         durs = sorted(a.elapsed_time(e) * 1e3 for a, e in one)
-        us = statistics.median(blk)
+        us = statistics.median(rep)
+        us_stream = statistics.median(blk)
         out[name] = {"us": round(us, 2), "gb_s": round(nbytes / (us * 1e-6) / 1e9, 1),
-                     "us_p10_p50_p90": [round(_quantile(blk, q), 2) for q in (0.1, 0.5, 0.9)],
-                     "launches": blocks * per_block, "blocks": blocks,
+                     "us_p10_p50_p90": [round(_quantile(rep, q), 2) for q in (0.1, 0.5, 0.9)],
+                     "launches": blocks * nl, "replays": blocks, "timing": "cuda_graph_replay",
+                     "us_stream": round(us_stream, 2), "gb_s_stream": round(nbytes / (us_stream * 1e-6) / 1e9, 1),
+                     "us_stream_p10_p50_p90": [round(_quantile(blk, q), 2) for q in (0.1, 0.5, 0.9)],
+                     "host_us_per_call": round(host_us, 1),
                      "us_event_per_launch": round(statistics.median(durs), 2),
                      "us_event_per_launch_p10_p50_p90": [round(_quantile(durs, q), 2) for q in (0.1, 0.5, 0.9)],
                      "sets": len(sets)}
@@ -1201,7 +1240,10 @@ def run_ours(args):
     # cost is printed by --marginal; `kernels` holds the instrumented split)
     line["headline_ops"] = {k: {"us": iso[k]["us"], "gb_s": iso[k]["gb_s"], "frac": round(iso[k]["gb_s"] / peak, 4),
                                 "pct_of_nominal_8tbs": round(100.0 * iso[k]["gb_s"] / 8000.0, 2),
-                                "us_p10_p50_p90": iso[k]["us_p10_p50_p90"]}
+                                "us_p10_p50_p90": iso[k]["us_p10_p50_p90"], "timing": iso[k]["timing"],
+                                "us_stream": iso[k]["us_stream"],
+                                "frac_stream": round(iso[k]["gb_s_stream"] / peak, 4),
+                                "host_us_per_call": iso[k]["host_us_per_call"]}
                             for k in ("per_token_group_quant", "block_dequant") if k in iso}
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(h)
