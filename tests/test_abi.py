@@ -423,7 +423,7 @@ def test_binding_refuses_a_device_other_than_the_current_one(monkeypatch):
     import inspect
     import torch
     import dequantisation_fp8q_token_b200 as f
-    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    monkeypatch.setattr(f, "_current_device", lambda: 0)      # the helper the binding reads it with
     with pytest.raises(ValueError, match="current device"):
         f._stream(None, torch.device("cuda", 1))
     src = inspect.getsource(f)
