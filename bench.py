@@ -682,6 +682,35 @@ class MatmulWorkload:
             torch.cuda.synchronize(device)
         return e0.elapsed_time(e1) / steps, clk.summary()
 
+    @staticmethod
+    def _timed_graph(fn, per_graph: int, replays: int, device):
+        """ms per call of fn replayed from a CUDA graph of `per_graph` back-to-back calls (the same
+        kernels and arguments, without the host's launch path between them): the median over
+        `replays` replays, with the SM clocks sampled while they run."""
+        side = torch.cuda.Stream(device)
+        side.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(side):
+            for _ in range(per_graph):
+                fn()
+        torch.cuda.current_stream(device).wait_stream(side)
+        torch.cuda.synchronize(device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(per_graph):
+                fn()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize(device)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+        with ClockSampler(device.index or 0) as clk:
+            for a, e in evs:
+                a.record()
+                graph.replay()
+                e.record()
+            torch.cuda.synchronize(device)
+        del graph
+        return statistics.median(a.elapsed_time(e) / per_graph for a, e in evs), clk.summary()
+
     def time(self, steps: int, warmup: int, device):
         """Every entry of the section, memory-bound ones first (a long run of tensor-core work
         leaves the SM clocks lowered by the power cap for a while)."""
@@ -796,8 +825,13 @@ class MatmulWorkload:
                               lambda: f.fp8q_scaled_mm_blockwise(q, sa, self.w, self.sb, out, status=self.status)),
                              (f"scaled_mm_per_tensor M={m}",
                               lambda: f.fp8q_scaled_mm(q, self.w, self.s1, self.s2, out, status=self.status))]:
-                ms, clk = self._timed(fn, steps, warmup, device)
-                res[name] = {"ms": round(ms, 4), "gb_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "clocks": clk}
+                # launched one by one from Python, then the same calls replayed from a CUDA
+                # graph (a ~25 us product is close enough to the launch path's cost for it to show)
+                ms_stream, _ = self._timed(fn, steps, warmup, device)
+                ms, clk = self._timed_graph(fn, 40, 10, device)
+                res[name] = {"ms": round(ms, 4), "gb_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "clocks": clk,
+                             "timing": "cuda_graph_replay", "ms_stream": round(ms_stream, 4),
+                             "gb_s_stream": round(nbytes / (ms_stream * 1e-3) / 1e9, 1)}
         k = self.q.shape[1]
         wt = torch.empty((k, self.n), dtype=torch.uint8, device=device)
         ms, clk = self._timed(lambda: f.fp8q_transpose_fp8(self.w, wt, self.n), steps, warmup, device)
