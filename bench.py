@@ -497,7 +497,7 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
     per_block = max(1, launches // blocks)
     out = {}
 
-    def run(name, make_set, footprint, nbytes):
+    def run(name, make_set, footprint, nbytes, elems):
         sets = [make_set(i) for i in range(max(1, -(-need // footprint)))]
         # warm up for at least 10 ms of launches, so the clocks have settled before timing
         t0 = time.perf_counter()
@@ -559,6 +559,7 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
         us = statistics.median(rep)
         us_stream = statistics.median(blk)
         out[name] = {"us": round(us, 2), "gb_s": round(nbytes / (us * 1e-6) / 1e9, 1),
+                     "gelem_s": round(elems / (us * 1e-6) / 1e9, 2),
                      "us_p10_p50_p90": [round(_quantile(rep, q), 2) for q in (0.1, 0.5, 0.9)],
                      "launches": blocks * nl, "replays": blocks, "timing": "cuda_graph_replay",
                      "us_stream": round(us_stream, 2), "gb_s_stream": round(nbytes / (us_stream * 1e-6) / 1e9, 1),
@@ -578,7 +579,7 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
         q = torch.empty((m, n), dtype=torch.uint8, device=d)
         s = torch.empty((m, n // 128), dtype=torch.float32, device=d)
         return lambda: f.fp8q_per_token_group_quant(x, q, s, 128, E4M3FN)
-    run("per_token_group_quant", per_token_set, c2_bytes, c2_bytes)
+    run("per_token_group_quant", per_token_set, c2_bytes, c2_bytes, m * n)
 
     M, N = wl.c3_w.shape
     c3_bytes = M * N * 3 + wl.c3_s.numel() * 4
@@ -587,14 +588,14 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
         w = wl.c3_w if i == 0 else wl.c3_w.clone()
         y = torch.empty((M, N), dtype=torch.bfloat16, device=d)
         return lambda: f.fp8q_block_dequant(w, wl.c3_s, y, 128, E4M3FN)
-    run("block_dequant", dequant_set, c3_bytes, c3_bytes)
+    run("block_dequant", dequant_set, c3_bytes, c3_bytes, M * N)
 
     def round_trip_set(i):
         q = wl.c2_q if i == 0 else wl.c2_q.clone()
         s = wl.c2_s if i == 0 else wl.c2_s.clone()
         y = torch.empty((m, n), dtype=torch.bfloat16, device=d)
         return lambda: f.fp8q_cast_from_fp8(q, s, y, GRAN_GROUP, 128, E4M3FN)
-    run("cast_from_fp8_group", round_trip_set, c2_bytes, c2_bytes)
+    run("cast_from_fp8_group", round_trip_set, c2_bytes, c2_bytes, m * n)
 
     R, C = wl.c4a_x.shape
     c4a_bytes = R * C * 3 + R * 4
@@ -604,7 +605,7 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
         q = torch.empty((R, C), dtype=torch.uint8, device=d)
         s = torch.empty((R,), dtype=torch.float32, device=d)
         return lambda: f.fp8q_cast_per_channel(x, q, s, E4M3FN)
-    run("cast_per_channel", per_channel_set, c4a_bytes, c4a_bytes)
+    run("cast_per_channel", per_channel_set, c4a_bytes, c4a_bytes, R * C)
 
     n4 = wl.c4b_x.numel()
     c4b_bytes = 2 * n4 * 4 + n4 + 4
@@ -614,7 +615,7 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
         q = torch.empty((n4,), dtype=torch.uint8, device=d)
         s = torch.empty((1,), dtype=torch.float32, device=d)
         return lambda: f.fp8q_cast_per_tensor(x, q, s, wl.ws, E5M2)
-    run("cast_per_tensor_f32_e5m2", per_tensor_set, n4 * 5 + 4, c4b_bytes)
+    run("cast_per_tensor_f32_e5m2", per_tensor_set, n4 * 5 + 4, c4b_bytes, n4)
     return out
 
 
@@ -1272,7 +1273,8 @@ def run_ours(args):
         line["sharded"] = sharded
     # the two ops the metric names, each timed alone (isolated) and inside the step (marginal
     # cost is printed by --marginal; `kernels` holds the instrumented split)
-    line["headline_ops"] = {k: {"us": iso[k]["us"], "gb_s": iso[k]["gb_s"], "frac": round(iso[k]["gb_s"] / peak, 4),
+    line["headline_ops"] = {k: {"us": iso[k]["us"], "gb_s": iso[k]["gb_s"], "gelem_s": iso[k]["gelem_s"],
+                                "frac": round(iso[k]["gb_s"] / peak, 4),
                                 "pct_of_nominal_8tbs": round(100.0 * iso[k]["gb_s"] / 8000.0, 2),
                                 "us_p10_p50_p90": iso[k]["us_p10_p50_p90"], "timing": iso[k]["timing"],
                                 "us_stream": iso[k]["us_stream"],
