@@ -535,7 +535,9 @@ def isolated_timing(wl: Workload, launches: int = 60, min_footprint: int = 0):
         torch.cuda.current_stream(d).wait_stream(side)
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        # thread-local capture: other threads (a process group's watchdog under torchrun) keep
+        # making CUDA calls while this thread captures
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             for j in range(nl):
                 sets[j % len(sets)]()
         for _ in range(3):
@@ -696,7 +698,7 @@ class MatmulWorkload:
         torch.cuda.current_stream(device).wait_stream(side)
         torch.cuda.synchronize(device)
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             for _ in range(per_graph):
                 fn()
         for _ in range(3):
