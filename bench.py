@@ -1164,9 +1164,11 @@ def run_ours(args):
                       for i in range(nops)]
     per_op_ms = [statistics.median(v) for v in per_op_samples]
     dom = max(range(nops), key=lambda i: per_op_ms[i])
-    # the dominant op's event pair rides on every `every`-th timed step only (about 20
-    # samples): a pair on every step cost the step about 1.5% on B200
-    every = max(1, args.steps // 20)
+    # the dominant op's event pair rides on every `every`-th timed step only (about 5
+    # samples, the first on step 0): the pair keeps the op from overlapping its neighbours
+    # under programmatic dependent launch, which cost the step about 1.5% with a pair on every
+    # step on B200 (20 timed steps: 6439 against 6630 GB/s with 200)
+    every = max(1, args.steps // 5)
     dom_events = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for k in range(0, args.steps, every)}
 
