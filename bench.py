@@ -1146,6 +1146,9 @@ def run_ours(args):
     wl = Workload(device, fp8q, h)
     torch.cuda.synchronize()
 
+    # NVML is set up before the warm-up: its initialisation takes milliseconds, and a GPU left
+    # idle that long just before the timed steps ran the first of them measurably slower
+    clk = ClockSampler(local)
     nops = len(wl.ops)
     for _ in range(args.warmup):
         wl.step()
@@ -1165,17 +1168,19 @@ def run_ours(args):
     per_op_ms = [statistics.median(v) for v in per_op_samples]
     dom = max(range(nops), key=lambda i: per_op_ms[i])
     # the dominant op's event pair rides on every `every`-th timed step only (about 5
-    # samples, the first on step 0): the pair keeps the op from overlapping its neighbours
-    # under programmatic dependent launch, which cost the step about 1.5% with a pair on every
-    # step on B200 (20 timed steps: 6439 against 6630 GB/s with 200)
+    # samples): the pair keeps the op from overlapping its neighbours under programmatic
+    # dependent launch, which cost the step about 1.5% with a pair on every step on B200
+    # (20 timed steps: 6439 against 6630 GB/s with 200).  The samples end each group of
+    # `every` steps, so none falls on the first timed step, which starts on an idle GPU
+    # (its dominant op measured up to a quarter slower there).
     every = max(1, args.steps // 5)
     dom_events = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for k in range(0, args.steps, every)}
+                  for k in range(max(every - 1, 1) if args.steps > 1 else 0, args.steps, every)}
 
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with clk:
         t_start.record()
         for k in range(args.steps):
             if k in dom_events:
