@@ -1136,6 +1136,13 @@ def max_over_ranks(v: float, world: int, device) -> float:
     return float(t.item())
 
 
+def dominant_sample_steps(steps: int, samples: int = 5):
+    """The timed steps that carry the dominant op's event pair: the last step of each of about
+    `samples` equal groups, never step 0 unless it is the only one."""
+    every = max(1, steps // samples)
+    return list(range(max(every - 1, 1) if steps > 1 else 0, steps, every))
+
+
 def run_ours(args):
     world, rank, local = dist_setup(args.gpus)
     device = torch.device("cuda", local)
@@ -1173,9 +1180,8 @@ def run_ours(args):
     # (20 timed steps: 6439 against 6630 GB/s with 200).  The samples end each group of
     # `every` steps, so none falls on the first timed step, which starts on an idle GPU
     # (its dominant op measured up to a quarter slower there).
-    every = max(1, args.steps // 5)
     dom_events = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for k in range(max(every - 1, 1) if args.steps > 1 else 0, args.steps, every)}
+                  for k in dominant_sample_steps(args.steps)}
 
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)

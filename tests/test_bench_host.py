@@ -60,3 +60,17 @@ def test_traffic_fingerprint_ignores_comments_only(tmp_path, monkeypatch):
     assert fp("/* a header */\nint f(int x) {\n  return x + 1;   // one more, said differently\n}\n") == base
     assert fp("int f(int x) {\n    return x + 2;  // one more\n}\n") != base
     assert fp("int f(int y) {\n    return y + 1;\n}\n") != base
+
+
+def test_dominant_sample_steps():
+    """The dominant op's event pairs in the timed region: about five, spread over the steps,
+    never on the first timed step (which starts on an idle GPU) unless it is the only one."""
+    import bench
+    assert bench.dominant_sample_steps(1) == [0]
+    assert bench.dominant_sample_steps(2) == [1]
+    assert bench.dominant_sample_steps(5) == [1, 2, 3, 4]
+    assert bench.dominant_sample_steps(20) == [3, 7, 11, 15, 19]
+    assert bench.dominant_sample_steps(200) == [39, 79, 119, 159, 199]
+    for k in range(2, 400):
+        got = bench.dominant_sample_steps(k)
+        assert 0 not in got and got and all(0 < s < k for s in got) and len(got) <= 9
