@@ -1,7 +1,8 @@
 """bench.py's algorithmic byte counts, checked against the figures derived
 independently from the workload shapes (input read once per pass the method
 needs, output written once), without a GPU: the Workload is built on torch's
-meta device from zero-filled host arrays of the right shapes."""
+meta device from zero-filled host arrays of the right shapes.  Also the choice of the timed
+steps that carry the dominant op's event pair."""
 import numpy as np
 import torch
 
