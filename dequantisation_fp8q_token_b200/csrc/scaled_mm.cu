@@ -795,6 +795,13 @@ scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                     if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort, p.wait_limit_ns)) { fail = kTimeoutProducer; break; }
                     const uint32_t fb = full0 + 8 * stage;
                     if (leader) mbar_arrive_expect_tx(fb, static_cast<uint32_t>(2 * (kATile + kBTile)));
+                    if (leader && kb == p.stall_kb && t == pair_id) {
+                        // test hook: the leader's half of this stage never arrives, so the
+                        // stage never completes and every wait that depends on it runs out
+                        ++issued;
+                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                        continue;
+                    }
                     // K-major: boxes of 128 rows x 128 k; MN-major: 128 k x 128 rows
                     const int m0 = mb * 2 * BM + static_cast<int>(rank) * BM;
                     const int n0 = nb * BN + static_cast<int>(rank) * kHalfB;
@@ -1057,8 +1064,7 @@ fp8q_status launch_scaled_mm(const uint8_t* a, int fa, const uint8_t* b, int fb,
     const bool tall = !fine && !narrow && M >= 2 * BM && tall_tiles * 10 >= 9LL * sm_count();
     // 256 x 256 tiles on CTA pairs when those tiles give two CTAs each to nine
     // tenths of the SMs (the same tiles on one CTA each need twice as many)
-    const bool pairs = FP8Q_PAIRS && !fine && !narrow && M >= 2 * BM && tall_tiles * 20 >= 9LL * sm_count() &&
-                       stall_kb < 0;
+    const bool pairs = FP8Q_PAIRS && !fine && !narrow && M >= 2 * BM && tall_tiles * 20 >= 9LL * sm_count();
     const int mt = (tall || pairs) ? 2 * BM : BM;
     const int a_rows = tall ? mt : (M >= BM || a_mn) ? BM : static_cast<int>((M + 15) / 16 * 16);
     CUtensorMap ma, mbm;

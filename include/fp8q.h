@@ -429,8 +429,9 @@ fp8q_status fp8q_scaled_mm(const uint8_t* a, fp8q_format fa, const uint8_t* b, f
  * e4m3fn operands, no bias and bf16 output, run with every internal wait
  * bounded by wait_limit_ns (1 ns .. 4 s) instead of the default of a few
  * seconds.  stall_kb >= 0 leaves out the shared-memory copies of k-block
- * stall_kb of each CTA's first tile, so the barrier those copies would
- * complete never does: the waits that depend on it run out, the kernel ORs
+ * stall_kb of each CTA's first tile (on CTA pairs: the leading CTA's half of
+ * its pair's first tile), so the barrier those copies would complete never
+ * does: the waits that depend on it run out, the kernel ORs
  * FP8Q_WAIT_* bits into *status, waits (again bounded) for its own copies
  * and tensor-core work in flight, frees its tensor memory and returns, with
  * d left incomplete.  Every access stays inside the operands.  stall_kb = -1

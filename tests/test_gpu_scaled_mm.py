@@ -517,6 +517,38 @@ def test_bounded_waits_run_out_report_and_return(fp8q, orc):
     np.testing.assert_array_equal(host(out3), want)
 
 
+
+def test_bounded_waits_run_out_cta_pairs(fp8q, orc):
+    """The same for a product on CTA pairs (256 x 256 tiles, tcgen05.mma.cta_group::2): the
+    leader CTA leaves out its half of k-block 2 of its pair's tile, so that stage never completes;
+    the leader's MMA wait runs out, the follower's epilogue and both CTAs' drains run out on their
+    own limits, both CTAs meet at the final cluster barrier, free TMEM and return."""
+    import time
+    M, N, K = 512, 8704, 512                     # 68 tiles of 256 x 256: CTA pairs; 4 k-blocks
+    g = np.random.default_rng(406)
+    a, b = grid_codes(g, (M, K), E4M3FN), grid_codes(g, (N, K), E4M3FN)
+    A, B = dev(a), dev(b)
+    sa, sb = dev(np.array([0.5], np.float32)), dev(np.array([0.125], np.float32))
+    want = oracle_rounded(orc, False, a, E4M3FN, b, E4M3FN, 0.5, 0.125, None, BF16)
+    out = Guarded(M * N, torch.bfloat16)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    fp8q.fp8q_scaled_mm_wait_test(A, B, sa, sb, out.t.view(M, N), st, 20_000_000, 2)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    out.check()
+    bits = int(st.item())
+    assert bits & fp8q.WAIT_MMA and bits & fp8q.WAIT_DRAIN, f"status {bits:#x}"
+    assert bits & ~0xF == 0, f"status {bits:#x}"
+    assert dt < 2.0, f"the stalled kernel took {dt:.2f} s"
+    out2 = Guarded(M * N, torch.bfloat16)
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fp8q.fp8q_scaled_mm_wait_test(A, B, sa, sb, out2.t.view(M, N), st2, 20_000_000, -1)
+    out2.check()
+    assert int(st2.item()) == 0
+    np.testing.assert_array_equal(host(out2.t.view(M, N)), want)
+
 def test_bounded_waits_run_out_decode_sized(fp8q, orc):
     """The same for a one-row product (128 x 128 tiles, a 16-row A box): k-block 2 of each CTA's
     tile never arrives, every wait that depends on it runs out and is reported, and the same
