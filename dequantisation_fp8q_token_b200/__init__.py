@@ -155,6 +155,8 @@ def lib() -> ctypes.CDLL:
             L.fp8q_scaled_mm.argtypes = [p, i32, p, i32, i64, i64, i64, p, p, p, i32, p, p, p]
             L.fp8q_scaled_mm_wait_test.restype = st
             L.fp8q_scaled_mm_wait_test.argtypes = [p, p, i64, i64, i64, p, p, p, p, ctypes.c_uint64, i32, p]
+            L.fp8q_scaled_mm_blockwise_wait_test.restype = st
+            L.fp8q_scaled_mm_blockwise_wait_test.argtypes = [p, p, p, p, i64, i64, i64, p, p, ctypes.c_uint64, i32, p]
             L.fp8q_scaled_mm_ex.restype = st
             L.fp8q_scaled_mm_ex.argtypes = [p, i32, i32, p, i32, i32, i64, i64, i64, p, p, p, i32, p, p, p]
             L.fp8q_transpose_fp8.restype = st
@@ -859,6 +861,28 @@ def fp8q_scaled_mm_wait_test(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Te
         _dev_ptr(scale_a, "scale_a", dev), _dev_ptr(scale_b, "scale_b", dev), _dev_ptr(out, "out", dev),
         _dev_ptr(_status_word(status), "status", dev), int(wait_limit_ns), int(stall_kb),
         _stream(stream, dev)), "fp8q_scaled_mm_wait_test")
+
+
+def fp8q_scaled_mm_blockwise_wait_test(a: torch.Tensor, scale_a: torch.Tensor, b: torch.Tensor,
+                                       scale_b: torch.Tensor, out: torch.Tensor, status: torch.Tensor,
+                                       wait_limit_ns: int, stall_kb: int = -1, stream=None) -> None:
+    """The bounded-wait test of the fine-grained product: fp8q_scaled_mm_blockwise (e4m3fn operands,
+    bf16 out, no bias) with every internal wait bounded by wait_limit_ns; stall_kb >= 0 leaves out
+    the copies of that k-block of each CTA's first tile."""
+    M, N, K, _, _ = _mm_operands(a, b, out, None, E4M3FN, E4M3FN)
+    dev = a.device
+    kb = -(-K // 128)
+    _need(scale_a, M * kb, "scale_a", dtype=torch.float32)
+    _need(scale_b, -(-N // 128) * kb, "scale_b", dtype=torch.float32)
+    if out.dtype != torch.bfloat16:
+        raise TypeError("out must be bf16")
+    if status is None:
+        raise TypeError("status is required")
+    _check(lib().fp8q_scaled_mm_blockwise_wait_test(
+        _dev_ptr(a, "a", dev), _dev_ptr(scale_a, "scale_a", dev), _dev_ptr(b, "b", dev),
+        _dev_ptr(scale_b, "scale_b", dev), M, N, K, _dev_ptr(out, "out", dev),
+        _dev_ptr(_status_word(status), "status", dev), int(wait_limit_ns), int(stall_kb),
+        _stream(stream, dev)), "fp8q_scaled_mm_blockwise_wait_test")
 
 
 def fp8q_scaled_mm_blockwise(a: torch.Tensor, scale_a: torch.Tensor, b: torch.Tensor, scale_b: torch.Tensor,

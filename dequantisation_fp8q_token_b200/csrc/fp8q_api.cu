@@ -419,6 +419,23 @@ fp8q_status fp8q_scaled_mm_wait_test(const uint8_t* a, const uint8_t* b, int64_t
                             d, status, reinterpret_cast<cudaStream_t>(stream), 0, 0, wait_limit_ns, stall_kb);
 }
 
+fp8q_status fp8q_scaled_mm_blockwise_wait_test(const uint8_t* a, const float* scale_a, const uint8_t* b,
+                                               const float* scale_b, int64_t M, int64_t N, int64_t K, void* d,
+                                               uint32_t* status, uint64_t wait_limit_ns, int stall_kb,
+                                               fp8q_stream_t stream) {
+    bool nothing = false;
+    fp8q_status st = check_scaled_mm(a, FP8Q_E4M3FN, b, FP8Q_E4M3FN, M, N, K, scale_a, scale_b, nullptr, FP8Q_BF16, d,
+                                     status, &nothing);
+    if (st != FP8Q_OK) return st;
+    if (nothing || K == 0 || wait_limit_ns == 0 || wait_limit_ns > 4000000000ull || stall_kb < -1 ||
+        stall_kb >= (K + 127) / 128)
+        return FP8Q_ERR_BAD_SHAPE;
+    if (!status) return FP8Q_ERR_NULL_POINTER;
+    const int kb = static_cast<int>((K + 127) / 128);
+    return launch_scaled_mm(a, FP8Q_E4M3FN, b, FP8Q_E4M3FN, M, N, K, scale_a, kb, scale_b, kb, true, nullptr, FP8Q_BF16,
+                            d, status, reinterpret_cast<cudaStream_t>(stream), 0, 0, wait_limit_ns, stall_kb);
+}
+
 fp8q_status fp8q_scaled_mm_blockwise(const uint8_t* a, fp8q_format fa, const float* scale_a, const uint8_t* b,
                                      fp8q_format fb, const float* scale_b, int64_t M, int64_t N, int64_t K,
                                      const void* bias, fp8q_dtype yt, void* d, uint32_t* status,

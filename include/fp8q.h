@@ -25,7 +25,8 @@
  *   fp8q_unpack_records(_ex)    payload] records (_ex: the page's packed
  *                               4-byte-header layout as well)
  *   fp8q_*_ex                   torch's rounding of the scale expressions
- *   fp8q_scaled_mm_wait_test    a test of the products' bounded waits
+ *   fp8q_scaled_mm_wait_test,   tests of the products' bounded waits
+ *   fp8q_scaled_mm_blockwise_wait_test
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -443,6 +444,14 @@ fp8q_status fp8q_scaled_mm(const uint8_t* a, fp8q_format fa, const uint8_t* b, f
 fp8q_status fp8q_scaled_mm_wait_test(const uint8_t* a, const uint8_t* b, int64_t M, int64_t N, int64_t K,
                                      const float* scale_a, const float* scale_b, void* d, uint32_t* status,
                                      uint64_t wait_limit_ns, int stall_kb, fp8q_stream_t stream);
+/* The same test for the fine-grained product: fp8q_scaled_mm_blockwise with
+ * e4m3fn operands, no bias and bf16 output (scale_a [M][ceil(K/128)],
+ * scale_b [ceil(N/128)][ceil(K/128)]), every wait bounded by wait_limit_ns,
+ * stall_kb as above.  Errors as fp8q_scaled_mm_blockwise and as above. */
+fp8q_status fp8q_scaled_mm_blockwise_wait_test(const uint8_t* a, const float* scale_a, const uint8_t* b,
+                                               const float* scale_b, int64_t M, int64_t N, int64_t K, void* d,
+                                               uint32_t* status, uint64_t wait_limit_ns, int stall_kb,
+                                               fp8q_stream_t stream);
 
 /*
  * Operand layouts of fp8q_scaled_mm_ex.  With A the [M][K] operand and B the

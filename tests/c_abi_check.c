@@ -32,7 +32,8 @@ int main(void) {
         (any_fn)fp8q_cast_pipeline, (any_fn)fp8q_pack_record, (any_fn)fp8q_pack_record_ex,
         (any_fn)fp8q_per_token_group_quant, (any_fn)fp8q_per_token_group_quant_ex, (any_fn)fp8q_record_bytes,
         (any_fn)fp8q_record_bytes_ex, (any_fn)fp8q_scaled_mm, (any_fn)fp8q_scaled_mm_blockwise,
-        (any_fn)fp8q_scaled_mm_ex, (any_fn)fp8q_scaled_mm_wait_test, (any_fn)fp8q_status_string,
+        (any_fn)fp8q_scaled_mm_ex, (any_fn)fp8q_scaled_mm_wait_test, (any_fn)fp8q_scaled_mm_blockwise_wait_test,
+        (any_fn)fp8q_status_string,
         (any_fn)fp8q_sum_rows, (any_fn)fp8q_tensor_amax, (any_fn)fp8q_transpose_fp8,
         (any_fn)fp8q_unpack_records, (any_fn)fp8q_unpack_records_ex, (any_fn)fp8q_version};
     const size_t n_entry = sizeof(entry_points) / sizeof(entry_points[0]);

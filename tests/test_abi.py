@@ -181,6 +181,16 @@ def test_scaled_mm_wait_test_validation(L):
     assert f(A, A, 8, 8, 128, None, P, A, A, 1000, 0, None) == 1            # null scale_a
     assert f(A, A, 8, 8, 128, P, P, A, A + 2, 1000, 0, None) == 5           # status word misaligned
 
+    g = L.fp8q_scaled_mm_blockwise_wait_test
+    g.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                  ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p]
+    assert g(A, P, A, P, 8, 8, 24, A, A, 1000, 0, None) == 4                # K % 16
+    assert g(A, P, A, P, 8, 8, 0, A, A, 1000, -1, None) == 4                # K == 0
+    assert g(A, P, A, P, 8, 8, 128, A, A, 0, 0, None) == 4                  # no wait limit
+    assert g(A, P, A, P, 8, 8, 256, A, A, 1000, 2, None) == 4               # stall past the last k-block
+    assert g(A, P, A, P, 8, 8, 128, A, None, 1000, 0, None) == 1            # the status word is required
+    assert g(A, None, A, P, 8, 8, 128, A, A, 1000, 0, None) == 1            # null scale_a
+    assert g(A, P, A, P + 2, 8, 8, 128, A, A, 1000, 0, None) == 5           # scale_b misaligned
 
 def test_transpose_and_sum_rows_validation(L):
     f = L.fp8q_transpose_fp8

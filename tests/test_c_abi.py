@@ -26,4 +26,4 @@ def test_a_c99_caller_compiles_links_and_runs(tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr + r.stdout
-    assert r.stdout.startswith("ok: 29 entry points"), r.stdout
+    assert r.stdout.startswith("ok: 30 entry points"), r.stdout

@@ -518,6 +518,39 @@ def test_bounded_waits_run_out_report_and_return(fp8q, orc):
 
 
 
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 1024),     # two 128 x 256 tiles, 8 k-blocks
+                                   (1, 3000, 1024)],     # decode-sized 128 x 128 tiles
+                         ids=["tiles", "decode"])
+def test_bounded_waits_run_out_fine_grained(fp8q, orc, M, N, K):
+    """The fine-grained product (one accumulator per k-block, folded by the epilogue warps) with
+    k-block 2 of each CTA's first tile left out: the MMA's wait runs out, the fold's and the drains'
+    waits end, the status bits are reported, and the same product then runs normally."""
+    import time
+    g = np.random.default_rng(407 + M)
+    a, b = grid_codes(g, (M, K), E4M3FN), grid_codes(g, (N, K), E4M3FN)
+    sa, sb = scales(g, M, N, K)
+    A, B, SA, SB = dev(a), dev(b), dev(sa), dev(sb)
+    want = oracle_rounded(orc, True, a, E4M3FN, b, E4M3FN, sa, sb, None, BF16)
+    out = Guarded(M * N, torch.bfloat16)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    fp8q.fp8q_scaled_mm_blockwise_wait_test(A, SA, B, SB, out.t.view(M, N), st, 20_000_000, 2)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    out.check()
+    bits = int(st.item())
+    assert bits & fp8q.WAIT_MMA and bits & fp8q.WAIT_DRAIN, f"status {bits:#x}"
+    assert bits & ~0xF == 0, f"status {bits:#x}"
+    assert dt < 2.0, f"the stalled kernel took {dt:.2f} s"
+    out2 = Guarded(M * N, torch.bfloat16)
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fp8q.fp8q_scaled_mm_blockwise_wait_test(A, SA, B, SB, out2.t.view(M, N), st2, 20_000_000, -1)
+    out2.check()
+    assert int(st2.item()) == 0
+    np.testing.assert_array_equal(host(out2.t.view(M, N)), want)
+
 def test_bounded_waits_run_out_cta_pairs(fp8q, orc):
     """The same for a product on CTA pairs (256 x 256 tiles, tcgen05.mma.cta_group::2): the
     leader CTA leaves out its half of k-block 2 of its pair's tile, so that stage never completes;
