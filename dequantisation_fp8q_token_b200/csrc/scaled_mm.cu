@@ -33,11 +33,14 @@
 //               chunks; warps whose rows all lie past M only take part in the
 //               handshake), while the tensor cores fill the other
 //               accumulator.
-// Tiles are 128 x BN of D, or 256 x 256 for large per-tensor products (two
-// M 128 MMAs per k step share the B tile; see Shape), visited in bands of 32
-// row-tiles so that the CTAs working at one time share A and B tiles in L2.
-// A product of fewer than 128 rows loads only its rows of A (rounded up to
-// 16).
+// Tiles are 128 x BN of D, visited in bands of 32 row-tiles so that the CTAs
+// working at one time share A and B tiles in L2.  Per-tensor products with
+// enough rows take 256 x 256 tiles on CTA pairs instead (namespace pair below:
+// one tcgen05.mma.cta_group::2 per k step across two SMs) when those tiles
+// give two CTAs each to nine tenths of the SMs.  A one-CTA 256 x 256 variant
+// (two M 128 MMAs per k step share the B tile; see Shape) serves builds
+// without pairs (FP8Q_PAIRS=0).  A product of fewer than 128 rows loads only
+// its rows of A (rounded up to 16).
 //
 // Every wait on an mbarrier is bounded (a few seconds of global time).  A
 // wait that runs out sets a flag in shared memory that ends the other roles'
